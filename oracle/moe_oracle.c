@@ -1,0 +1,385 @@
+/*
+ * moe_oracle.c -- plain, slow fp64 CPU oracle of the routed MoE FFN.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only tests/, __graft_entry__.smoke() and
+ * bench.py's cpu_baseline / reference leg may load this library.  It shares no
+ * code, header, table or constant with the CUDA library (it includes nothing
+ * but the C standard library) and the CUDA library never calls it.
+ *
+ * What it computes, for every token t (x[t] in R^H, logits[t] in R^E):
+ *
+ *   p          = softmax(logits[t])                                  (route)
+ *   ids[t, :]  = the K experts of largest p, descending, ties -> lower id
+ *   w[t, j]    = p[ids[t,j]] / sum_j' p[ids[t,j']]                   (renormalise)
+ *   W[n, k]    = e4m3fn(q[n, k]) * s[n/128, k/128]                    (block-scaled FP8)
+ *   FFN_e(x)   = Wd_e (silu(Wg_e x) * (Wu_e x)),  silu(z) = z / (1 + e^-z)
+ *   out[t]     = sum_j w[t,j] FFN_{ids[t,j]}(x[t]) + FFN_shared(x[t])
+ *
+ * Sources (page title, section):
+ *  - dstair/gated-deltanet-nki-trainium, "FP8 MoE decode kernel
+ *    (moe_fused_w8_35b)": the fused expert chain gate/up GEMM -> SwiGLU ->
+ *    down GEMM -> affinity scale -> expert-sum with E4M3FN weights and 128x128
+ *    block scales; "Serving contract": router softmax -> top-8 -> norm, shared
+ *    expert added after the routed sum.
+ *  - nemo_automodel ... qwen3_5.layers, `_silu_mul`: SwiGLU is silu(gate) * up.
+ *  - spark_model/layers/nemotron_moe.rs, module doc and `prefill` step 5: sort
+ *    tokens by expert, grouped GEMM over each expert's rows, unpermute-reduce.
+ *  - ROCm/aiter PR #5988 description: the sorted pipeline with an inverse
+ *    route map and an FP32 route reduction; "10 routed experts plus one shared
+ *    expert".
+ *  - NKI Library kernel reference, MoE kernels: Router Top-K, Permute Routed
+ *    Tokens (sort by expert), Top-K Reduce.
+ *
+ * Precision: fp64 throughout (exp, silu, every product and sum).  Inputs are
+ * bf16 / fp32 / E4M3FN bit patterns and are widened exactly.  The one place
+ * where floating point decides an integer is the top-K choice; it compares the
+ * fp32 logits themselves.  Softmax is strictly increasing in the logit, so the
+ * K largest logits are the K largest probabilities; comparing the fp32 inputs
+ * takes that decision exactly, in the same precision as the kernel.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define ORACLE_BLOCK 128
+
+/* ---------------------------------------------------------------- threads */
+
+static int g_threads = 1;
+
+int oracle_set_threads(int n) {
+#ifdef _OPENMP
+    if (n < 1) n = 1;
+    g_threads = n;
+    return n;
+#else
+    (void)n;
+    g_threads = 1;
+    return 1;
+#endif
+}
+
+int oracle_get_threads(void) { return g_threads; }
+
+/* ---------------------------------------------------------------- formats */
+
+/* OCP FP8 E4M3FN (the "official E4M3FN" weights of the decode kernel page):
+ * 1 sign bit, 4 exponent bits with bias 7, 3 mantissa bits.
+ * exponent 0: subnormal, value (m/8) * 2^-6.  exponent 1..15: (1 + m/8) * 2^(e-7).
+ * S.1111.111 is NaN; there is no infinity (so S.1111.110 = 448 is the maximum). */
+double oracle_e4m3fn_value(uint8_t code) {
+    int sign = (code >> 7) & 1;
+    int e = (code >> 3) & 0xF;
+    int m = code & 0x7;
+    double v;
+    if (e == 0xF && m == 0x7) return NAN;
+    if (e == 0)
+        v = ldexp((double)m / 8.0, -6);
+    else
+        v = ldexp(1.0 + (double)m / 8.0, e - 7);
+    return sign ? -v : v;
+}
+
+/* bfloat16: the upper 16 bits of an IEEE binary32. */
+double oracle_bf16_value(uint16_t bits) {
+    uint32_t u = (uint32_t)bits << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* One weight element of a block-scaled FP8 matrix [rows, cols] (cols contiguous):
+ * W[n, k] = e4m3fn(q[n, k]) * s[n / 128, k / 128]. */
+static double weight(const uint8_t* q, const float* s, int cols, int n, int k) {
+    int ncb = cols / ORACLE_BLOCK;
+    return oracle_e4m3fn_value(q[(size_t)n * cols + k]) *
+           (double)s[(size_t)(n / ORACLE_BLOCK) * ncb + (k / ORACLE_BLOCK)];
+}
+
+/* ---------------------------------------------------------------- route */
+
+/* Router of the decode kernel page's serving contract: softmax over the E
+ * logits, the top-K experts, then their probabilities renormalised to sum 1.
+ * Slot j holds the j-th largest; equal logits go to the lower expert id.
+ * zero_mask (nullable, [T, K]): a nonzero entry forces w[t, j] = 0 after the
+ * renormalisation, with no second renormalisation (the "zero routing weights"
+ * replay case of the aiter prefill PR). */
+void oracle_route(const float* logits, int T, int E, int K, const uint8_t* zero_mask,
+                  int32_t* ids, double* w) {
+#pragma omp parallel for num_threads(g_threads) schedule(static)
+    for (int t = 0; t < T; ++t) {
+        const float* l = logits + (size_t)t * E;
+        double* p = (double*)malloc(sizeof(double) * (size_t)E);
+        unsigned char* taken = (unsigned char*)calloc((size_t)E, 1);
+        double lmax = -INFINITY, z = 0.0;
+        for (int e = 0; e < E; ++e)
+            if ((double)l[e] > lmax) lmax = (double)l[e];
+        for (int e = 0; e < E; ++e) {
+            p[e] = exp((double)l[e] - lmax);
+            z += p[e];
+        }
+        for (int e = 0; e < E; ++e) p[e] /= z;
+
+        double sel = 0.0;
+        for (int j = 0; j < K; ++j) {
+            int best = -1;
+            for (int e = 0; e < E; ++e) {
+                if (taken[e]) continue;
+                if (best < 0 || l[e] > l[best]) best = e; /* strict >: ties keep the lower id */
+            }
+            taken[best] = 1;
+            ids[(size_t)t * K + j] = best;
+            sel += p[best];
+        }
+        for (int j = 0; j < K; ++j) {
+            double v = p[ids[(size_t)t * K + j]] / sel;
+            if (zero_mask && zero_mask[(size_t)t * K + j]) v = 0.0;
+            w[(size_t)t * K + j] = v;
+        }
+        free(p);
+        free(taken);
+    }
+}
+
+/* ---------------------------------------------------------------- sort */
+
+/* Sort the R = T*K routes (route r = t*K + j carries expert ids[r]) by expert,
+ * keeping route order within an expert (a stable counting sort: count, exclusive
+ * scan, scatter in route order).  This is the "sort tokens by expert" step of the
+ * Nemotron prefill path and the NKI "Permute Routed Tokens" kernel.
+ *   offsets[e]       = number of valid routes with id < e; offsets[E] = valid routes
+ *   sorted_route[p]  = the route at sorted position p (p < offsets[E]); -1 after
+ *   inv_route[r]     = the sorted position of route r; -1 for an id outside [0, E)
+ * Returns the number of routes whose id is outside [0, E) (they are skipped). */
+int oracle_sort(const int32_t* ids, int T, int K, int E, int32_t* offsets,
+                int32_t* sorted_route, int32_t* inv_route) {
+    long R = (long)T * K;
+    int bad = 0;
+    int32_t* count = (int32_t*)calloc((size_t)E + 1, sizeof(int32_t));
+    for (long r = 0; r < R; ++r) {
+        int e = ids[r];
+        if (e < 0 || e >= E) { bad++; continue; }
+        count[e]++;
+    }
+    offsets[0] = 0;
+    for (int e = 0; e < E; ++e) offsets[e + 1] = offsets[e] + count[e];
+    int32_t* cursor = count;
+    for (int e = 0; e < E; ++e) cursor[e] = offsets[e];
+    for (long p = 0; p < R; ++p) sorted_route[p] = -1;
+    for (long r = 0; r < R; ++r) {
+        int e = ids[r];
+        if (e < 0 || e >= E) { inv_route[r] = -1; continue; }
+        int32_t pos = cursor[e]++;
+        sorted_route[pos] = (int32_t)r;
+        inv_route[r] = pos;
+    }
+    free(count);
+    return bad;
+}
+
+/* ---------------------------------------------------------------- expert FFN */
+
+/* One expert applied to one row: y = Wd (silu(Wg x) * (Wu x)).
+ * Wg, Wu: [I, H] codes with [I/128, H/128] scales; Wd: [H, I] with [H/128, I/128].
+ * SwiGLU as `_silu_mul` of the qwen3_5.layers page: silu(gate) * up. */
+static void expert_row(const double* x, int H, int I,
+                       const uint8_t* wg, const float* sg, const uint8_t* wu, const float* su,
+                       const uint8_t* wd, const float* sd, double* h, double* y) {
+    for (int i = 0; i < I; ++i) {
+        double g = 0.0, u = 0.0;
+        for (int k = 0; k < H; ++k) {
+            g += weight(wg, sg, H, i, k) * x[k];
+            u += weight(wu, su, H, i, k) * x[k];
+        }
+        h[i] = (g / (1.0 + exp(-g))) * u;
+    }
+    for (int n = 0; n < H; ++n) {
+        double acc = 0.0;
+        for (int i = 0; i < I; ++i) acc += weight(wd, sd, I, n, i) * h[i];
+        y[n] = acc;
+    }
+}
+
+/* Expert tensors, expert-major as the CUDA library also takes them. */
+typedef struct {
+    const uint8_t* w_gate; const float* s_gate;
+    const uint8_t* w_up;   const float* s_up;
+    const uint8_t* w_down; const float* s_down;
+    int n_experts; int inter;
+} oracle_experts;
+
+static void expert_ptrs(const oracle_experts* ex, int e, int H,
+                        const uint8_t** wg, const float** sg, const uint8_t** wu,
+                        const float** su, const uint8_t** wd, const float** sd) {
+    size_t I = (size_t)ex->inter;
+    size_t nw = I * (size_t)H, ns = (I / ORACLE_BLOCK) * ((size_t)H / ORACLE_BLOCK);
+    *wg = ex->w_gate + (size_t)e * nw; *sg = ex->s_gate + (size_t)e * ns;
+    *wu = ex->w_up + (size_t)e * nw;   *su = ex->s_up + (size_t)e * ns;
+    *wd = ex->w_down + (size_t)e * nw; *sd = ex->s_down + (size_t)e * ns;
+}
+
+static void load_row(const uint16_t* x, int H, int t, double* xr) {
+    for (int k = 0; k < H; ++k) xr[k] = oracle_bf16_value(x[(size_t)t * H + k]);
+}
+
+/* Grouped expert FFN over the sorted routes (the "sorted grouped GEMM" of the
+ * Nemotron prefill path): for each expert e and each sorted position p in
+ * [offsets[e], offsets[e+1]), route r = sorted_route[p], token t = r / K:
+ *     y_sorted[p] = w[r] * FFN_e(x[t])
+ * (the affinity scale of the decode kernel page's chain, applied per route). */
+void oracle_ffn_sorted(const uint16_t* x, int T, int H, int K, const oracle_experts* ex,
+                       const int32_t* offsets, const int32_t* sorted_route, const double* w,
+                       double* y_sorted) {
+    (void)T;
+    int E = ex->n_experts, I = ex->inter;
+    for (int e = 0; e < E; ++e) {
+        const uint8_t *wg, *wu, *wd; const float *sg, *su, *sd;
+        expert_ptrs(ex, e, H, &wg, &sg, &wu, &su, &wd, &sd);
+        int p0 = offsets[e], p1 = offsets[e + 1];
+#pragma omp parallel for num_threads(g_threads) schedule(dynamic, 1)
+        for (int p = p0; p < p1; ++p) {
+            double* xr = (double*)malloc(sizeof(double) * (size_t)H);
+            double* h = (double*)malloc(sizeof(double) * (size_t)I);
+            int r = sorted_route[p];
+            load_row(x, H, r / K, xr);
+            double* y = y_sorted + (size_t)p * H;
+            expert_row(xr, H, I, wg, sg, wu, su, wd, sd, h, y);
+            for (int n = 0; n < H; ++n) y[n] *= w[r];
+            free(xr);
+            free(h);
+        }
+    }
+}
+
+/* The always-on shared expert (weight 1, every token): y_shared[t] = FFN_s(x[t]). */
+void oracle_ffn_shared(const uint16_t* x, int T, int H, const oracle_experts* sh,
+                       double* y_shared) {
+    const uint8_t *wg, *wu, *wd; const float *sg, *su, *sd;
+    expert_ptrs(sh, 0, H, &wg, &sg, &wu, &su, &wd, &sd);
+    int I = sh->inter;
+#pragma omp parallel for num_threads(g_threads) schedule(dynamic, 1)
+    for (int t = 0; t < T; ++t) {
+        double* xr = (double*)malloc(sizeof(double) * (size_t)H);
+        double* h = (double*)malloc(sizeof(double) * (size_t)I);
+        load_row(x, H, t, xr);
+        expert_row(xr, H, I, wg, sg, wu, su, wd, sd, h, y_shared + (size_t)t * H);
+        free(xr);
+        free(h);
+    }
+}
+
+/* Top-K reduce through the inverse route map (Nemotron's unpermute-reduce, the
+ * aiter FP32 route reduction, NKI Top-K Reduce): out[t] = sum over slots j of
+ * y_sorted[inv_route[t*K + j]] (+ y_shared[t]); routes with inv_route -1 add 0. */
+void oracle_combine(const double* y_sorted, const int32_t* inv_route, const double* y_shared,
+                    int T, int K, int H, double* out) {
+#pragma omp parallel for num_threads(g_threads) schedule(static)
+    for (int t = 0; t < T; ++t) {
+        double* o = out + (size_t)t * H;
+        for (int n = 0; n < H; ++n) o[n] = y_shared ? y_shared[(size_t)t * H + n] : 0.0;
+        for (int j = 0; j < K; ++j) {
+            int32_t p = inv_route[(size_t)t * K + j];
+            if (p < 0) continue;
+            const double* y = y_sorted + (size_t)p * H;
+            for (int n = 0; n < H; ++n) o[n] += y[n];
+        }
+    }
+}
+
+/* The same reduction over bf16 operands (for checking the combine step alone). */
+void oracle_combine_bf16(const uint16_t* y_sorted, const int32_t* inv_route,
+                         const uint16_t* y_shared, int T, int K, int H, double* out) {
+#pragma omp parallel for num_threads(g_threads) schedule(static)
+    for (int t = 0; t < T; ++t) {
+        double* o = out + (size_t)t * H;
+        for (int n = 0; n < H; ++n)
+            o[n] = y_shared ? oracle_bf16_value(y_shared[(size_t)t * H + n]) : 0.0;
+        for (int j = 0; j < K; ++j) {
+            int32_t p = inv_route[(size_t)t * K + j];
+            if (p < 0) continue;
+            for (int n = 0; n < H; ++n) o[n] += oracle_bf16_value(y_sorted[(size_t)p * H + n]);
+        }
+    }
+}
+
+/* ---------------------------------------------------------------- whole path */
+
+/* Structured form: route -> sort -> grouped FFN -> shared -> combine, returning
+ * every intermediate.  y_sorted is [T*K, H]; y_shared may be NULL when sh is NULL. */
+int oracle_moe(const uint16_t* x, const float* logits, int T, int H, int E, int K,
+               const uint8_t* zero_mask, const oracle_experts* routed, const oracle_experts* sh,
+               int32_t* ids, double* w, int32_t* offsets, int32_t* sorted_route,
+               int32_t* inv_route, double* y_sorted, double* y_shared, double* out) {
+    oracle_route(logits, T, E, K, zero_mask, ids, w);
+    int bad = oracle_sort(ids, T, K, E, offsets, sorted_route, inv_route);
+    oracle_ffn_sorted(x, T, H, K, routed, offsets, sorted_route, w, y_sorted);
+    if (sh) oracle_ffn_shared(x, T, H, sh, y_shared);
+    oracle_combine(y_sorted, inv_route, sh ? y_shared : NULL, T, K, H, out);
+    return bad;
+}
+
+/* Brute-force form, straight from the per-token definition, for a list of tokens
+ * (tokens == NULL: all T in order): out[i] = sum_j w[t,j] FFN_{ids[t,j]}(x[t]) + FFN_s(x[t])
+ * with t = tokens[i].  No sort, no inverse map. */
+void oracle_moe_tokens(const uint16_t* x, const float* logits, int T, int H, int E, int K,
+                       const uint8_t* zero_mask, const oracle_experts* routed,
+                       const oracle_experts* sh, const int32_t* tokens, int n_tokens,
+                       double* out) {
+    (void)T;
+    int I = routed->inter;
+    int Is = sh ? sh->inter : 0;
+    int Imax = I > Is ? I : Is;
+#pragma omp parallel for num_threads(g_threads) schedule(dynamic, 1)
+    for (int i = 0; i < n_tokens; ++i) {
+        int t = tokens ? tokens[i] : i;
+        double* xr = (double*)malloc(sizeof(double) * (size_t)H);
+        double* h = (double*)malloc(sizeof(double) * (size_t)Imax);
+        double* y = (double*)malloc(sizeof(double) * (size_t)H);
+        int32_t* tid = (int32_t*)malloc(sizeof(int32_t) * (size_t)K);
+        double* tw = (double*)malloc(sizeof(double) * (size_t)K);
+        double* o = out + (size_t)i * H;
+        load_row(x, H, t, xr);
+        oracle_route(logits + (size_t)t * E, 1, E, K, zero_mask ? zero_mask + (size_t)t * K : NULL,
+                     tid, tw);
+        for (int n = 0; n < H; ++n) o[n] = 0.0;
+        for (int j = 0; j < K; ++j) {
+            const uint8_t *wg, *wu, *wd; const float *sg, *su, *sd;
+            expert_ptrs(routed, tid[j], H, &wg, &sg, &wu, &su, &wd, &sd);
+            expert_row(xr, H, I, wg, sg, wu, su, wd, sd, h, y);
+            for (int n = 0; n < H; ++n) o[n] += tw[j] * y[n];
+        }
+        if (sh) {
+            const uint8_t *wg, *wu, *wd; const float *sg, *su, *sd;
+            expert_ptrs(sh, 0, H, &wg, &sg, &wu, &su, &wd, &sd);
+            expert_row(xr, H, Is, wg, sg, wu, su, wd, sd, h, y);
+            for (int n = 0; n < H; ++n) o[n] += y[n];
+        }
+        free(xr); free(h); free(y); free(tid); free(tw);
+    }
+}
+
+/* One expert FFN on explicit rows (no routing): y[i] = FFN_e(x[rows[i]]). */
+void oracle_expert_rows(const uint16_t* x, int H, const oracle_experts* ex, int e,
+                        const int32_t* rows, int n_rows, double* y) {
+    const uint8_t *wg, *wu, *wd; const float *sg, *su, *sd;
+    expert_ptrs(ex, e, H, &wg, &sg, &wu, &su, &wd, &sd);
+    int I = ex->inter;
+#pragma omp parallel for num_threads(g_threads) schedule(dynamic, 1)
+    for (int i = 0; i < n_rows; ++i) {
+        double* xr = (double*)malloc(sizeof(double) * (size_t)H);
+        double* h = (double*)malloc(sizeof(double) * (size_t)I);
+        load_row(x, H, rows[i], xr);
+        expert_row(xr, H, I, wg, sg, wu, su, wd, sd, h, y + (size_t)i * H);
+        free(xr);
+        free(h);
+    }
+}
+
+/* SwiGLU alone, for pinning: h[i] = silu(g[i]) * u[i]. */
+void oracle_swiglu(const double* g, const double* u, int n, double* h) {
+    for (int i = 0; i < n; ++i) h[i] = (g[i] / (1.0 + exp(-g[i]))) * u[i];
+}

@@ -1,0 +1,341 @@
+"""Pins of the CPU oracle to things other than itself (CPU only).
+
+Each test checks one oracle function against a library routine (torch's FP8
+and bf16 casts, torch.nn.functional, numpy's stable argsort, scipy's softmax,
+Python's sorted), a closed form, an invariant of the method, or brute force on
+tiny inputs.  The mistakes they are chosen to catch are named in each test.
+"""
+import numpy as np
+import pytest
+import scipy.special
+import torch
+import torch.nn.functional as F
+
+import oracle
+from mixture_experts_ffn_sort_b200 import workloads as wl
+
+
+def _fp8_dense(codes: np.ndarray, scales: np.ndarray) -> torch.Tensor:
+    """Library decode: torch's E4M3FN -> float64, times the block scale expanded
+    with a Kronecker product (rows and cols of one block share one scale)."""
+    v = torch.from_numpy(np.ascontiguousarray(codes)).view(torch.float8_e4m3fn).to(torch.float64)
+    s = torch.from_numpy(np.kron(scales.astype(np.float64), np.ones((128, 128))))
+    return v * s
+
+
+def _torch_mlp(x64: torch.Tensor, ex, e: int) -> torch.Tensor:
+    """The eager SwiGLU MLP (down(silu(gate(x)) * up(x))) with torch Linear ops."""
+    wg = _fp8_dense(ex.w_gate[e], ex.s_gate[e])
+    wu = _fp8_dense(ex.w_up[e], ex.s_up[e])
+    wd = _fp8_dense(ex.w_down[e], ex.s_down[e])
+    return F.linear(F.silu(F.linear(x64, wg)) * F.linear(x64, wu), wd)
+
+
+def _x64(x_bits: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(x_bits.view(np.int16).copy()).view(torch.bfloat16).to(torch.float64)
+
+
+# ------------------------------------------------------------------ formats
+
+def test_e4m3fn_every_code_matches_torch_cast():
+    """All 256 codes against torch's float8_e4m3fn -> float32 conversion
+    (catches a wrong bias, a subnormal rule or a sign slip)."""
+    codes = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    ref = codes.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = np.array([oracle.e4m3fn_value(c) for c in range(256)])
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan], ref[~nan])
+    assert np.array_equal(np.signbit(got[~nan]), np.signbit(ref[~nan]))
+
+
+def test_e4m3fn_closed_forms():
+    """Values fixed by the E4M3FN definition (bias 7, 3 mantissa bits, no inf)."""
+    assert oracle.e4m3fn_value(0x00) == 0.0
+    assert oracle.e4m3fn_value(0x01) == 2.0 ** -9          # smallest subnormal
+    assert oracle.e4m3fn_value(0x07) == 7 * 2.0 ** -9      # largest subnormal
+    assert oracle.e4m3fn_value(0x08) == 2.0 ** -6          # smallest normal
+    assert oracle.e4m3fn_value(0x38) == 1.0
+    assert oracle.e4m3fn_value(0x3C) == 1.5
+    assert oracle.e4m3fn_value(0x7E) == 448.0              # largest finite
+    assert oracle.e4m3fn_value(0xFE) == -448.0
+    assert np.isnan(oracle.e4m3fn_value(0x7F)) and np.isnan(oracle.e4m3fn_value(0xFF))
+    assert np.signbit(oracle.e4m3fn_value(0x80))
+
+
+def test_bf16_matches_torch_cast():
+    rng = np.random.default_rng(1)
+    bits = rng.integers(0, 1 << 16, size=2000, dtype=np.uint32).astype(np.uint16)
+    bits[:4] = [0x3F80, 0xC000, 0x0001, 0x7F7F]
+    ref = torch.from_numpy(bits.view(np.int16).copy()).view(torch.bfloat16).to(torch.float64).numpy()
+    got = np.array([oracle.bf16_value(int(b)) for b in bits])
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan], ref[~nan])
+    assert got[0] == 1.0 and got[1] == -2.0 and got[2] == 2.0 ** -133
+
+
+# ------------------------------------------------------------------ route
+
+def _sorted_topk(l: np.ndarray, K: int):
+    return [e for _, e in sorted((-float(v), e) for e, v in enumerate(l))][:K]
+
+
+@pytest.mark.parametrize("T,E,K,levels", [(40, 8, 2, None), (30, 256, 8, None),
+                                          (50, 6, 3, 2), (50, 33, 7, 3), (5, 16, 16, None)])
+def test_route_ids_match_python_sorted(T, E, K, levels):
+    """Top-K, descending, ties to the lower id: against Python's sorted on
+    (-logit, id) (catches ascending order, a wrong tie rule, repeated picks)."""
+    lg = (wl.tie_logits(T, E, seed=T, levels=levels) if levels
+          else np.random.default_rng(T).standard_normal((T, E)).astype(np.float32))
+    ids, w = oracle.route(lg, K)
+    for t in range(T):
+        assert list(ids[t]) == _sorted_topk(lg[t], K)
+
+
+def test_route_ranking_equals_probability_ranking():
+    """Ranking by logit equals ranking the fp64 softmax (scipy) probabilities."""
+    lg = np.random.default_rng(7).standard_normal((200, 64)).astype(np.float32) * 3
+    ids, _ = oracle.route(lg, 10)
+    p = scipy.special.softmax(lg.astype(np.float64), axis=1)
+    ref = np.argsort(-p, axis=1, kind="stable")[:, :10]
+    assert np.array_equal(ids, ref)
+
+
+def test_route_weights_full_k_is_softmax():
+    """With K = E the renormalisation is a no-op: w equals scipy's softmax."""
+    lg = np.random.default_rng(3).standard_normal((20, 12)).astype(np.float32) * 2
+    ids, w = oracle.route(lg, 12)
+    p = scipy.special.softmax(lg.astype(np.float64), axis=1)
+    np.testing.assert_allclose(w, np.take_along_axis(p, ids, axis=1), rtol=1e-13, atol=0)
+
+
+def test_route_weight_closed_forms():
+    """Renormalised weights sum to 1, and w_i / w_j = exp(l_i - l_j) (softmax
+    ratio); adding a constant to a token's logits changes nothing."""
+    lg = np.random.default_rng(4).standard_normal((64, 40)).astype(np.float32)
+    ids, w = oracle.route(lg, 6)
+    np.testing.assert_allclose(w.sum(1), 1.0, rtol=0, atol=1e-14)
+    l_sel = np.take_along_axis(lg.astype(np.float64), ids, axis=1)
+    np.testing.assert_allclose(w[:, 1:] / w[:, :1], np.exp(l_sel[:, 1:] - l_sel[:, :1]), rtol=1e-12)
+    ids2, w2 = oracle.route(lg + np.float32(8.0), 6)
+    assert np.array_equal(ids, ids2)
+    np.testing.assert_allclose(w2, w, rtol=1e-5)   # the shifted fp32 logits round
+
+
+def test_route_zero_mask_forces_zero_without_renormalising():
+    lg = np.random.default_rng(5).standard_normal((30, 16)).astype(np.float32)
+    mask = np.zeros((30, 4), np.uint8)
+    mask[::3, 1] = 1
+    ids0, w0 = oracle.route(lg, 4)
+    ids1, w1 = oracle.route(lg, 4, mask)
+    assert np.array_equal(ids0, ids1)
+    assert np.all(w1[mask == 1] == 0.0)
+    assert np.array_equal(w1[mask == 0], w0[mask == 0])
+
+
+# ------------------------------------------------------------------ sort
+
+@pytest.mark.parametrize("T,K,E,distinct", [(0, 4, 8, True), (1, 1, 1, True), (37, 3, 5, True),
+                                            (200, 8, 64, True), (100, 5, 7, False),
+                                            (513, 10, 512, True)])
+def test_sort_matches_numpy_stable_argsort(T, K, E, distinct):
+    ids = wl.random_ids(T, K, E, seed=T + K, distinct=distinct) if T else np.zeros((0, K), np.int32)
+    off, sr, inv, bad = oracle.sort(ids, E)
+    flat = ids.ravel()
+    assert bad == 0
+    assert np.array_equal(sr, np.argsort(flat, kind="stable"))
+    assert np.array_equal(off, np.concatenate([[0], np.cumsum(np.bincount(flat, minlength=E))]))
+    assert np.array_equal(inv[sr], np.arange(T * K))
+
+
+def test_sort_all_routes_on_one_expert():
+    ids = np.full((50, 1), 3, np.int32)
+    off, sr, inv, bad = oracle.sort(ids, 8)
+    assert list(off) == [0, 0, 0, 0, 50, 50, 50, 50, 50]
+    assert np.array_equal(sr, np.arange(50)) and np.array_equal(inv, np.arange(50))
+
+
+def test_sort_skips_out_of_range_ids():
+    ids = np.array([[0, 9], [-1, 2], [2, 0]], np.int32)
+    off, sr, inv, bad = oracle.sort(ids, 4)
+    assert bad == 2
+    assert list(off) == [0, 2, 2, 4, 4]
+    assert list(sr) == [0, 5, 3, 4, -1, -1]
+    assert list(inv) == [0, -1, -1, 2, 3, 1]
+
+
+# ------------------------------------------------------------------ FFN
+
+def test_swiglu_matches_torch_silu():
+    """silu(gate) * up against torch.nn.functional.silu (catches a swapped
+    gate/up, sigmoid(g)*u, or a sign error in the exponent)."""
+    rng = np.random.default_rng(6)
+    g = rng.standard_normal(1000) * 6
+    u = rng.standard_normal(1000) * 3
+    ref = (F.silu(torch.from_numpy(g)) * torch.from_numpy(u)).numpy()
+    np.testing.assert_allclose(oracle.swiglu(g, u), ref, rtol=1e-14, atol=1e-300)
+    h = oracle.swiglu(np.array([0.0, 1.0, 2.0, -50.0]), np.array([5.0, 2.0, 1.0, 1.0]))
+    assert h[0] == 0.0
+    assert abs(h[1] - 2.0 / (1.0 + np.exp(-1.0))) < 1e-15       # silu(1) * 2
+    assert abs(h[2] - 2.0 / (1.0 + np.exp(-2.0))) < 1e-15       # silu(2) * 1
+    assert abs(h[3]) < 1e-20
+
+
+@pytest.mark.parametrize("H,I", [(256, 384), (384, 128)])
+def test_expert_ffn_matches_torch_mlp(H, I):
+    """One expert against the eager torch MLP built from torch-decoded weights.
+    H != I and per-block random scales catch transposed operands, a transposed
+    scale grid, or a scale applied to the wrong block."""
+    ex = wl.draw_experts(seed=11, tag=99, n=2, I=I, H=H, std=0.05, threads=1)
+    for e in range(2):
+        ex.s_gate[e] *= np.exp2(np.random.default_rng(e).integers(-3, 4, ex.s_gate[e].shape))
+        ex.s_down[e] *= np.exp2(np.random.default_rng(9 + e).integers(-3, 4, ex.s_down[e].shape))
+    x = wl.random_rows_bf16(5, H, seed=2)
+    for e in range(2):
+        got = oracle.expert_rows(x, ex, e, np.arange(5))
+        ref = _torch_mlp(_x64(x), ex, e).numpy()
+        np.testing.assert_allclose(got, ref, rtol=1e-10, atol=1e-12 * np.abs(ref).max())
+
+
+def test_expert_ffn_subnormal_and_all_codes():
+    """Blocks of E4M3FN subnormals only, and blocks using every finite code."""
+    for ex in (wl.subnormal_experts(1, 128, 256), wl.all_code_experts(1, 128, 256)):
+        x = wl.random_rows_bf16(3, 256, seed=5)
+        got = oracle.expert_rows(x, ex, 0, np.arange(3))
+        ref = _torch_mlp(_x64(x), ex, 0).numpy()
+        np.testing.assert_allclose(got, ref, rtol=1e-10, atol=1e-12 * np.abs(ref).max())
+
+
+# ------------------------------------------------------------------ whole path
+
+@pytest.fixture(scope="module")
+def tiny():
+    return wl.make_workload("tiny", threads=1)
+
+
+def test_structured_equals_brute_force(tiny):
+    """Route -> sort -> grouped FFN -> combine equals the per-token definition."""
+    o = oracle.workload(tiny)
+    b = oracle.moe_tokens(tiny.x, tiny.logits, tiny.shape.K, tiny.routed)
+    np.testing.assert_allclose(o["out"], b, rtol=1e-12, atol=1e-14)
+    assert o["bad"] == 0
+
+
+def test_brute_force_tiny_against_library_chain():
+    """The whole chain on tiny inputs from library pieces: Python sorted for the
+    top-K, scipy softmax, torch Linear/SiLU for each expert."""
+    T, H, I, E, K = 4, 128, 128, 5, 2
+    ex = wl.draw_experts(seed=4, tag=98, n=E, I=I, H=H, std=0.05, threads=1)
+    x = wl.random_rows_bf16(T, H, seed=8)
+    lg = np.random.default_rng(12).standard_normal((T, E)).astype(np.float32)
+    got = oracle.moe_tokens(x, lg, K, ex)
+    x64 = _x64(x)
+    for t in range(T):
+        p = scipy.special.softmax(lg[t].astype(np.float64))
+        sel = _sorted_topk(lg[t], K)
+        ref = sum(p[e] / p[sel].sum() * _torch_mlp(x64[t:t + 1], ex, e)[0].numpy() for e in sel)
+        np.testing.assert_allclose(got[t], ref, rtol=1e-10, atol=1e-13)
+
+
+def test_full_topk_equals_softmax_mixture():
+    """K = E: the routed sum is the full softmax mixture sum_e p_e FFN_e(x)."""
+    T, H, I, E = 3, 128, 128, 4
+    ex = wl.draw_experts(seed=5, tag=97, n=E, I=I, H=H, std=0.05, threads=1)
+    x = wl.random_rows_bf16(T, H, seed=9)
+    lg = np.random.default_rng(13).standard_normal((T, E)).astype(np.float32)
+    got = oracle.moe_tokens(x, lg, E, ex)
+    p = scipy.special.softmax(lg.astype(np.float64), axis=1)
+    ref = sum(p[:, e:e + 1] * oracle.expert_rows(x, ex, e, np.arange(T)) for e in range(E))
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-14)
+
+
+def test_zero_weight_route_contributes_nothing(tiny):
+    """A masked route adds exactly 0: replacing its expert's weights by other
+    finite values leaves the output bit-identical."""
+    T, K = tiny.shape.T, tiny.shape.K
+    ids, _ = oracle.route(tiny.logits, K)
+    mask = np.zeros((T, K), np.uint8)
+    mask[:, 0] = 1
+    hot = ids[:, 0]
+    # Every slot-0 expert is masked everywhere; only experts never used unmasked change.
+    used_unmasked = set(ids[:, 1:].ravel().tolist())
+    victims = [e for e in set(hot.tolist()) if e not in used_unmasked]
+    assert victims
+    a = oracle.moe(tiny.x, tiny.logits, K, tiny.routed, zero_mask=mask)["out"]
+    ex2 = wl.FP8Experts(*(np.copy(v) for v in (tiny.routed.w_gate, tiny.routed.s_gate,
+                                                tiny.routed.w_up, tiny.routed.s_up,
+                                                tiny.routed.w_down, tiny.routed.s_down)))
+    for e in victims:
+        ex2.w_down[e] = 0x7E                  # 448: large but finite
+        ex2.s_down[e] = 3.0
+    b = oracle.moe(tiny.x, tiny.logits, K, ex2, zero_mask=mask)["out"]
+    assert np.array_equal(a, b)
+
+
+def test_token_permutation_permutes_rows(tiny):
+    perm = np.random.default_rng(1).permutation(tiny.shape.T)
+    a = oracle.moe(tiny.x, tiny.logits, tiny.shape.K, tiny.routed)["out"]
+    b = oracle.moe(tiny.x[perm], tiny.logits[perm], tiny.shape.K, tiny.routed)["out"]
+    assert np.array_equal(a[perm], b)
+
+
+def test_shared_expert_is_added_with_weight_one():
+    T, H, I, E, K = 6, 128, 128, 4, 2
+    ex = wl.draw_experts(seed=6, tag=96, n=E, I=I, H=H, std=0.05, threads=1)
+    sh = wl.draw_experts(seed=6, tag=95, n=1, I=256, H=H, std=0.05, threads=1)
+    x = wl.random_rows_bf16(T, H, seed=10)
+    lg = np.random.default_rng(14).standard_normal((T, E)).astype(np.float32)
+    with_s = oracle.moe(x, lg, K, ex, sh)
+    without = oracle.moe(x, lg, K, ex)
+    ref = _torch_mlp(_x64(x), sh, 0).numpy()
+    np.testing.assert_allclose(with_s["out"] - without["out"], ref, rtol=1e-9, atol=1e-12)
+    np.testing.assert_allclose(with_s["y_shared"], ref, rtol=1e-10, atol=1e-13)
+
+
+def test_combine_closed_form():
+    """y for route r, column n = (r+1)(n+1): out[t, n] = (n+1) * sum_j (tK+j+1)
+    exactly (catches a dropped or doubled slot and a wrong inverse lookup)."""
+    T, K, E, H = 9, 3, 5, 16
+    ids = wl.random_ids(T, K, E, seed=3)
+    off, sr, inv, _ = oracle.sort(ids, E)
+    y = np.empty((T * K, H))
+    for p in range(T * K):
+        y[p] = (sr[p] + 1) * (np.arange(H) + 1.0)
+    out = oracle.combine(y, inv, None, T, K)
+    for t in range(T):
+        s = sum(t * K + j + 1 for j in range(K))
+        assert np.array_equal(out[t], s * (np.arange(H) + 1.0))
+    sh = np.full((T, H), 0.5)
+    assert np.array_equal(oracle.combine(y, inv, sh, T, K), out + 0.5)
+
+
+def test_combine_bf16_matches_float_combine():
+    T, K, E, H = 7, 4, 6, 32
+    ids = wl.random_ids(T, K, E, seed=4)
+    _, _, inv, _ = oracle.sort(ids, E)
+    ys = wl.random_rows_bf16(T * K, H, seed=6)
+    sh = wl.random_rows_bf16(T, H, seed=7)
+    a = oracle.combine_bf16(ys, inv, sh, T, K)
+    b = oracle.combine(oracle.bf16_array(ys), inv, oracle.bf16_array(sh), T, K)
+    assert np.array_equal(a, b)
+
+
+def test_oracle_matches_stored_golden(tiny):
+    """The stored oracle output of the tiny workload (tests/golden/make_golden.py)."""
+    import os
+    path = os.path.join(os.path.dirname(__file__), "golden", "tiny_oracle.txt")
+    rows = {}
+    for line in open(path):
+        if line.startswith("#"):
+            continue
+        key, *vals = line.split()
+        rows[key] = vals
+    o = oracle.workload(tiny)
+    assert list(map(int, rows["ids"])) == list(o["ids"].ravel())
+    assert list(map(int, rows["offsets"])) == list(o["offsets"])
+    assert list(map(int, rows["sorted_route"])) == list(o["sorted_route"])
+    np.testing.assert_allclose(np.array(rows["w"], float), o["w"].ravel(), rtol=1e-15)
+    for t in range(4):
+        np.testing.assert_allclose(np.array(rows["out%d" % t], float), o["out"][t, :16],
+                                   rtol=1e-13, atol=1e-15)
