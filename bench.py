@@ -1,0 +1,365 @@
+"""Benchmark of the routed MoE FFN hot path on B200.
+
+One step = one pass of the whole path over one batch: moe_route -> moe_sort ->
+moe_expert_ffn -> moe_combine, replayed from a CUDA graph.  The default
+workload is the decode MoE (T=64 tokens, H=2048, I=512, 256 experts, top-8,
+FP8 E4M3 weights with 128x128 block scales, bf16 activations).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload decode|tiny|decode_skew|prefill|prefill_large]
+
+Prints one JSON line (rank 0).  With N > 1 (torchrun), every rank runs an
+independent replica of the workload (the path has no cross-token exchange);
+the time is the max over ranks and the value counts all ranks' tokens.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from mixture_experts_ffn_sort_b200 import workloads as wl  # noqa: E402
+
+METRIC = "MoE FFN tokens/s at 1 B200; % HBM roofline (decode) / % BF16 TC peak (prefill)"
+UNIT = "tokens/s"
+# Bytes of one expert's FP8 weights and fp32 block scales, used for the decode roofline.
+
+
+def expert_bytes(H, I):
+    return 3 * H * I + 3 * (H // 128) * (I // 128) * 4
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm=d["hbm_gbs"], bf16=d["bf16_tflops"], bf16_sus=d["bf16_tflops_sustained"],
+                    src="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
+
+
+def profile_traffic(workload):
+    """DRAM bytes per FFN call from the committed ncu summary, if the kernel
+    sources it was taken on are unchanged (else None)."""
+    path = os.path.join(ROOT, "profiles", "ffn_%s_traffic.md" % workload)
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    m = re.search(r"traffic_bytes_per_call:\s*([0-9.eE+]+)", text)
+    h = re.search(r"sources_sha256:\s*([0-9a-f]+)", text)
+    if not m or not h or h.group(1) != sources_hash():
+        return None
+    return float(m.group(1))
+
+
+def sources_hash():
+    d = os.path.join(ROOT, "mixture_experts_ffn_sort_b200", "csrc")
+    hs = hashlib.sha256()
+    for f in sorted(os.listdir(d)):
+        if f.endswith((".cu", ".cuh", ".h")):
+            hs.update(open(os.path.join(d, f), "rb").read())
+    return hs.hexdigest()[:16]
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons every 100 ms while running."""
+
+    Q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index, self.lines, self.proc = index, [], None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.Q,
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in self.lines:
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 8:
+                continue
+            try:
+                sm.append(float(f[0]))
+                mx.append(float(f[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- reference arm (CPU oracle)
+
+def run_reference(args, shape):
+    import oracle
+    w = wl.make_workload(shape.name)
+    cores = oracle.threads()
+    tk = np.arange(min(shape.T, 64 if shape.T > 512 else shape.T), dtype=np.int32)
+
+    def one():
+        t0 = time.perf_counter()
+        oracle.moe_tokens(w.x, w.logits, shape.K, w.routed, w.shared, w.zero_mask, tokens=tk)
+        return time.perf_counter() - t0
+
+    for _ in range(args.warmup):
+        one()
+    ts = [one() for _ in range(args.steps)]
+    tot = sum(ts)
+    value = len(tk) * len(ts) / tot
+    sample = "%d of the %d tokens per step (brute-force per-token oracle, fp64)" % (len(tk), shape.T)
+    return {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * tot / len(ts), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference", "config": config_of(shape),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def cpu_baseline(shape, budget_s=10.0):
+    """The oracle as it stands, on the host cores, on a bounded sample."""
+    import oracle
+    w = wl.make_workload(shape.name)
+    tk = np.arange(min(shape.T, 64), dtype=np.int32)
+    n, t0 = 0, time.perf_counter()
+    while time.perf_counter() - t0 < budget_s or n == 0:
+        oracle.moe_tokens(w.x, w.logits, shape.K, w.routed, w.shared, w.zero_mask, tokens=tk)
+        n += 1
+    dt = time.perf_counter() - t0
+    return {"value": n * len(tk) / dt, "unit": UNIT, "cores": oracle.threads(), "kind": "oracle",
+            "sample": "%d x %d tokens of the workload, %.1f s, brute-force per-token oracle in fp64"
+                      % (n, len(tk), dt)}
+
+
+def config_of(shape):
+    return {"workload": shape.name, "T": shape.T, "H": shape.H, "I": shape.I, "E": shape.E, "K": shape.K,
+            "I_shared": shape.I_shared, "weights": "fp8 e4m3fn, fp32 scale per 128x128 block",
+            "activations": "bf16", "logit_bias": shape.bias, "zero_route_frac": shape.zero_frac,
+            "seed": shape.seed}
+
+
+# ---------------------------------------------------------------- our arm
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=None)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="decode", choices=wl.SHAPE_ORDER)
+    ap.add_argument("--mode", type=int, default=0, help="moe_expert_ffn mode: 0 AUTO, 1 DECODE, 2 PREFILL")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    shape = wl.SHAPES[args.workload]
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if args.steps is None:
+            args.steps = 3
+        if rank == 0:
+            print(json.dumps(run_reference(args, shape)), flush=True)
+        return
+
+    import torch
+    import torch.distributed as dist
+    import mixture_experts_ffn_sort_b200 as moe
+
+    if args.steps is None:
+        args.steps = {"tiny": 2000, "decode": 5000, "decode_skew": 2000, "prefill": 200,
+                      "prefill_large": 30}[shape.name]
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    w = wl.make_workload(shape.name)
+    T, K, E, H, I = shape.T, shape.K, shape.E, shape.H, shape.I
+    x = torch.from_numpy(w.x.view(np.int16)).view(torch.bfloat16).to(dev)
+    logits = torch.from_numpy(w.logits).to(dev)
+    zmask = torch.from_numpy(w.zero_mask).to(dev) if w.zero_mask is not None else None
+    routed = moe.Experts.from_host(w.routed, dev)
+    shared = moe.Experts.from_host(w.shared, dev) if w.shared is not None else None
+    layer = moe.MoEFFN(routed, T, K, shared, mode=args.mode, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+
+    def step():
+        layer(x, logits, zmask)
+
+    with torch.cuda.stream(stream):
+        for _ in range(max(1, args.warmup)):
+            step()
+    stream.synchronize()
+    if layer.status.item() != 0:
+        raise RuntimeError("status word %d after warm-up" % layer.status.item())
+
+    # Graph of one step; the timed region replays it K times.
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        step()
+    # Instrumented graph: events around each call, for the per-call breakdown.
+    ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(5)]
+    g2 = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g2, stream=stream):
+        ev[0].record()
+        moe.moe_route(logits, K, zmask, layer.topk_ids, layer.topk_w)
+        ev[1].record()
+        moe.moe_sort(layer.topk_ids, E, layer.status, layer.offsets, layer.sorted_route, layer.inv_route,
+                     layer.sort_ws)
+        ev[2].record()
+        moe.moe_expert_ffn(x, K, routed, layer.offsets, layer.sorted_route, layer.topk_w, shared, args.mode,
+                           layer.status, layer.y_sorted, layer.y_shared, layer.ffn_ws)
+        ev[3].record()
+        moe.moe_combine(layer.y_sorted, layer.inv_route, layer.y_shared, T, K, moe.MOE_OUT_BF16, layer.out)
+        ev[4].record()
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            g.replay()
+            g2.replay()
+    stream.synchronize()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        barrier()
+        torch.cuda.synchronize(dev)
+        start.record(stream)
+        with torch.cuda.stream(stream):
+            for _ in range(args.steps):
+                g.replay()
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+    ms = start.elapsed_time(end)
+    t_local = ms / args.steps
+    # Per-call breakdown from the instrumented graph (same stream, after the timed region).
+    parts = {k: [] for k in ("route", "sort", "ffn", "combine")}
+    with torch.cuda.stream(stream):
+        for _ in range(min(args.steps, 200)):
+            g2.replay()
+            stream.synchronize()
+            for i, k in enumerate(parts):
+                parts[k].append(ev[i].elapsed_time(ev[i + 1]))
+    t_max = t_local
+    if world > 1:
+        tt = torch.tensor([t_local], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        t_max = tt.item()
+
+    # End to end through the public API with host buffers: pinned x and logits
+    # copied in, the layer output copied back, every step.
+    xh = torch.from_numpy(w.x.view(np.int16)).view(torch.bfloat16).pin_memory()
+    lh = torch.from_numpy(w.logits).pin_memory()
+    oh = torch.empty((T, H), dtype=torch.bfloat16).pin_memory()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n_e2e = min(args.steps, 500)
+    barrier()
+    torch.cuda.synchronize(dev)
+    with torch.cuda.stream(stream):
+        e0.record()
+        for _ in range(n_e2e):
+            x.copy_(xh, non_blocking=True)
+            logits.copy_(lh, non_blocking=True)
+            step()
+            oh.copy_(layer.out, non_blocking=True)
+        e1.record()
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1) / n_e2e
+    if world > 1:
+        tt = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = tt.item()
+    if layer.status.item() != 0:
+        raise RuntimeError("status word %d after the timed region" % layer.status.item())
+
+    peaks = load_peaks()
+    off = layer.offsets.cpu().numpy()
+    touched = int(np.count_nonzero(np.diff(off)))
+    ffn_ms = statistics.median(parts["ffn"])
+    R_nz = int(np.count_nonzero(layer.topk_w.cpu().numpy()))
+    flops = (R_nz + (T if shape.I_shared else 0)) * 6 * H * I
+    decode_path = (args.mode == 1) or (args.mode == 0 and T * K <= 8192)
+    if decode_path:
+        algo = touched * expert_bytes(H, I) + (expert_bytes(H, shape.I_shared) if shape.I_shared else 0)
+        ach = algo / (ffn_ms * 1e-3) / 1e9
+        traffic = profile_traffic(shape.name)
+        roof = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm"], "unit": "GB/s",
+                "frac": ach / peaks["hbm"], "traffic": traffic,
+                "kernel": "moe_expert_ffn (gate/up + down kernels)", "algorithmic_bytes": algo,
+                "touched_experts": touched, "peak_source": peaks["src"]}
+    else:
+        ach = flops / (ffn_ms * 1e-3) / 1e12
+        pk = peaks["bf16_sus"]
+        roof = {"bound": "tensor", "achieved": ach, "peak": pk, "unit": "TFLOP/s", "frac": ach / pk,
+                "traffic": profile_traffic(shape.name), "kernel": "moe_expert_ffn", "flops": flops,
+                "peak_source": peaks["src"] + " sustained"}
+    n_launch = layer.launches()
+    out = {"metric": METRIC, "value": T * world / (t_max * 1e-3), "unit": UNIT, "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_max, "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+           "config": dict(config_of(shape), parallelism="replicas x%d" % world,
+                          l2="inputs larger than L2 (touched expert weights %.2f GB > 126 MB)"
+                             % (touched * expert_bytes(H, I) / 1e9) if decode_path else
+                             "inputs larger than L2 (expert weights %.2f GB > 126 MB)" % (E * expert_bytes(H, I) / 1e9),
+                          timing="CUDA events around %d CUDA-graph replays of one step" % args.steps),
+           "roofline": roof,
+           "breakdown_ms": {k: statistics.median(v) for k, v in parts.items()},
+           "e2e": {"value": T * world / (e2e_ms * 1e-3), "unit": UNIT,
+                   "h2d_bytes_per_step": x.numel() * 2 + logits.numel() * 4,
+                   "d2h_bytes_per_step": layer.out.numel() * 2},
+           "gpu_launches": n_launch * args.steps,
+           "clocks": clk.summary()}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(shape)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    del g, g2
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,233 @@
+/*
+ * moe_ffn.h -- C ABI of the routed Mixture-of-Experts FFN library for NVIDIA
+ * B200 (sm_100a).
+ *
+ * The four calls run the routed MoE FFN hot path:
+ *
+ *   moe_route      router logits -> top-K expert ids and renormalised weights
+ *   moe_sort       ids -> expert-contiguous route order, per-expert offsets,
+ *                  inverse route map (all on the device, no host sync)
+ *   moe_expert_ffn grouped gate/up GEMM over block-scaled E4M3FN weights
+ *                  decoded to BF16, fused SwiGLU, down GEMM with the routing
+ *                  weight fused in; optional always-on shared expert
+ *   moe_combine    top-K reduce back to token order (+ shared expert)
+ *
+ * Sources (page title, section):
+ *  - dstair/gated-deltanet-nki-trainium, "FP8 MoE decode kernel
+ *    (moe_fused_w8_35b)": the fused chain gate/up GEMM -> SwiGLU -> down GEMM
+ *    -> affinity scale -> expert-sum, official E4M3FN weights with 128x128
+ *    block scales decoded to BF16 tile by tile; "Interface" (hidden, gate_up,
+ *    down, scales, affinities -> [B, H] f32); "Serving contract" (softmax ->
+ *    top-8 -> norm router; the shared expert is added after the routed sum).
+ *  - spark_model/layers/nemotron_moe.rs: module doc ("all expert dispatch is
+ *    device-side ... zero D2H sync"), `new` (top_k bounds checked with an error
+ *    message), `prefill` step 5 (sort by expert, grouped GEMM, unpermute-reduce,
+ *    ids and weights as [N, top_k] 4-byte arrays).
+ *  - ROCm/aiter PR #5988: ctypes C-ABI entry point whose launcher validates the
+ *    tensor contracts; reuse of a sort with an inverse route map; FP32 route
+ *    reduction; zero routing weights and caller-provided output buffers.
+ *  - NKI Library kernel reference, MoE kernels: Router Top-K, Permute Routed
+ *    Tokens, Top-K Reduce, MoE TKG (decode) / MoE CTE (prefill).
+ *
+ * Conventions for every call:
+ *  - All tensor pointers are DEVICE pointers owned by the caller.  The library
+ *    allocates no device memory in any call; scratch is caller-provided through
+ *    the `workspace` arguments, sized by the *_workspace_bytes queries.
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *    default stream), never synchronises the host, and reads no device value
+ *    back.  The first call of a process also does one-time host set-up (kernel
+ *    attributes, driver entry points); make one call before capturing a CUDA
+ *    graph, after which the calls may be captured.
+ *  - Return value: MOE_OK (0) or a negative moe_status.  On error nothing has
+ *    been launched and moe_last_error() holds a message (thread-local, valid
+ *    until the next call on the same thread).  MOE_ERR_CUDA reports a launch
+ *    error, with the CUDA error string in the message.
+ *  - T = 0 (no tokens) is valid: nothing is launched and MOE_OK is returned.
+ *  - Tensor base addresses must be 16-byte aligned (MOE_ERR_MISALIGNED).
+ *  - Layouts are row-major with the last index contiguous.  Route r = t*K + j
+ *    is token t's j-th choice (descending weight).
+ *  - bf16 tensors are passed as uint16_t bit patterns.
+ */
+#ifndef MOE_FFN_H
+#define MOE_FFN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Exported symbols of the shared library (everything else is hidden). */
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+/* A cudaStream_t (the runtime's stream handle type is `struct CUstream_st*`). */
+typedef struct CUstream_st* moe_stream_t;
+
+typedef enum moe_status {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = -1,          /* NULL pointer, negative size, bad enum, K > E */
+    MOE_ERR_UNSUPPORTED_SHAPE = -2,    /* H or I not a multiple of 128, E > MOE_MAX_E, ... */
+    MOE_ERR_MISALIGNED = -3,           /* a tensor base not 16-byte aligned */
+    MOE_ERR_WORKSPACE_TOO_SMALL = -4,  /* workspace_bytes below the query's answer */
+    MOE_ERR_CUDA = -5                  /* the CUDA runtime reported an error */
+} moe_status;
+
+#define MOE_MAX_E 1024      /* experts per call */
+#define MOE_MAX_K 32        /* top-K */
+#define MOE_BLOCK 128       /* FP8 scale block edge: one fp32 scale per 128 x 128 */
+#define MOE_MAX_T (1 << 24) /* tokens per call */
+
+/* Bits OR-ed into the optional device status word (int32) by the kernels. */
+#define MOE_STATUS_BAD_ID 1      /* an expert id outside [0, E) was skipped */
+#define MOE_STATUS_BAD_MAP 2     /* offsets / route map out of range: rows skipped */
+
+/* moe_expert_ffn `mode`. */
+#define MOE_MODE_AUTO 0     /* DECODE when T*K <= MOE_DECODE_MAX_ROUTES, else PREFILL */
+#define MOE_MODE_DECODE 1   /* weight-streaming kernels (memory-bound regime) */
+#define MOE_MODE_PREFILL 2  /* tcgen05 / TMEM grouped GEMM kernels (compute-bound regime) */
+#define MOE_DECODE_MAX_ROUTES 8192
+
+/* moe_combine `out_dtype`. */
+#define MOE_OUT_BF16 0
+#define MOE_OUT_F32 1
+
+/* Thread-local message describing the last error on this thread ("" if none). */
+MOE_API const char* moe_last_error(void);
+
+/* ABI version of this header (incremented on incompatible changes). */
+#define MOE_ABI_VERSION 1
+MOE_API int moe_abi_version(void);
+
+/* ---------------------------------------------------------------------------
+ * moe_route -- softmax top-K routing with renormalisation.
+ *
+ * Defined by the decode kernel page's serving contract (router "softmax ->
+ * top-8 -> norm") and the NKI Router Top-K kernel.  Per token t:
+ *   p = softmax(logits[t, :]);  topk_ids[t, 0..K-1] = the K largest p in
+ *   descending order, equal logits going to the lower expert id;
+ *   topk_w[t, j] = p[topk_ids[t, j]] / sum_j' p[topk_ids[t, j']].
+ * The kernel ranks by the fp32 logit (softmax is strictly increasing, so the
+ * order is the same) and computes the weights in fp32 as
+ * exp(l_j - l_max) / sum_j' exp(l_j' - l_max).
+ *
+ *   logits    [T, E] f32 (read)
+ *   zero_mask [T, K] u8 or NULL (read): a nonzero entry sets topk_w[t, j] = 0
+ *             after the renormalisation, with no second renormalisation (the
+ *             zero-routing-weight case of the aiter prefill PR)
+ *   topk_ids  [T, K] i32 (written)
+ *   topk_w    [T, K] f32 (written)
+ * Limits: 1 <= K <= min(E, MOE_MAX_K), 1 <= E <= MOE_MAX_E, 0 <= T <= MOE_MAX_T.
+ * Logits must be finite; a NaN logit gives unspecified ids for that token.
+ * ------------------------------------------------------------------------- */
+MOE_API int moe_route(const float* logits, int T, int E, int K, const uint8_t* zero_mask,
+              int32_t* topk_ids, float* topk_w, moe_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * moe_sort -- stable sort of the R = T*K routes by expert.
+ *
+ * The "sort tokens by expert" step of the Nemotron prefill path, the NKI
+ * Permute Routed Tokens kernel, and the aiter pipeline's sort with inverse
+ * route map.  A counting sort: per-chunk expert histograms, an expert-major
+ * exclusive scan, and an in-order scatter, so the result is deterministic.
+ *   expert_offsets[e]   = number of valid routes with id < e;
+ *                         expert_offsets[E] = number of valid routes   [E+1] i32
+ *   sorted_route[p]     = route r at sorted position p, routes of one expert in
+ *                         increasing r; -1 for p >= expert_offsets[E]  [R] i32
+ *   inv_route[r]        = sorted position of route r, -1 if skipped    [R] i32
+ * Ids outside [0, E) are skipped (never written out of bounds) and set
+ * MOE_STATUS_BAD_ID in *status (optional device int32, may be NULL; the
+ * library only ORs bits into it, the caller clears it).
+ *   workspace: device scratch of moe_sort_workspace_bytes(T, K, E) bytes, any
+ *   contents; overwritten.
+ * ------------------------------------------------------------------------- */
+MOE_API size_t moe_sort_workspace_bytes(int T, int K, int E);
+MOE_API int moe_sort(const int32_t* topk_ids, int T, int K, int E, int32_t* expert_offsets,
+             int32_t* sorted_route, int32_t* inv_route, void* workspace,
+             size_t workspace_bytes, int32_t* status, moe_stream_t stream);
+
+/* Block-scaled FP8 expert weights, expert-major (the caller owns the memory).
+ * Rows are output features and the reduction index is contiguous:
+ *   w_gate, w_up  [n_experts, inter, H] u8 E4M3FN codes
+ *   w_down        [n_experts, H, inter] u8 E4M3FN codes
+ *   s_gate, s_up  [n_experts, inter/128, H/128] f32 block scales
+ *   s_down        [n_experts, H/128, inter/128] f32 block scales
+ * Weight value W[n, k] = e4m3fn(code[n, k]) * s[n/128, k/128] (the exact
+ * 128x128 block mapping of the decode kernel page's block_pow2 variant).
+ * E4M3FN: bias 7, 3 mantissa bits, subnormals, S.1111.111 = NaN, no inf. */
+typedef struct moe_fp8_experts {
+    const uint8_t* w_gate;
+    const uint8_t* w_up;
+    const uint8_t* w_down;
+    const float* s_gate;
+    const float* s_up;
+    const float* s_down;
+    int n_experts;
+    int inter;
+} moe_fp8_experts;
+
+/* ---------------------------------------------------------------------------
+ * moe_expert_ffn -- grouped expert FFN over the sorted routes.
+ *
+ * For every expert e and sorted position p in [expert_offsets[e],
+ * expert_offsets[e+1]), with route r = sorted_route[p] and token t = r / K:
+ *   h        = silu(Wg_e x[t]) * (Wu_e x[t])          (SwiGLU, `_silu_mul`)
+ *   y_sorted[p, :] = bf16( topk_w[r] * (Wd_e h) )     (affinity in the epilogue)
+ * and, when `shared` is not NULL, for every token t:
+ *   y_shared[t, :] = bf16( Wd_s (silu(Wg_s x[t]) * (Wu_s x[t])) )
+ * This is the decode kernel page's fused chain (gate/up -> SwiGLU -> down ->
+ * affinity scale) over the Nemotron page's sorted grouped-GEMM order; the
+ * shared expert is the "one shared expert" of the aiter PR, weight 1.
+ * Numerics: bf16 x bf16 products accumulated in fp32; weights decoded from
+ * E4M3FN to BF16 (DECODE mode: the exact E4M3 value, its block scale applied to
+ * each 128-wide fp32 partial sum; PREFILL mode: bf16(e4m3 * scale));
+ * h is rounded to bf16 between the two GEMMs.
+ *
+ *   x              [T, H] bf16 (read)
+ *   routed         routed experts; routed->n_experts = E, routed->inter = I
+ *   shared         NULL or one always-on expert (n_experts = 1, inter = I_s)
+ *   expert_offsets [E+1] i32, sorted_route [T*K] i32 (as moe_sort writes them)
+ *   topk_w         [T, K] f32 (read; route r's weight is topk_w[r])
+ *   y_sorted       [T*K, H] bf16 (written for rows p < expert_offsets[E])
+ *   y_shared       [T, H] bf16 (written) when shared != NULL, else ignored
+ *   mode           MOE_MODE_AUTO | MOE_MODE_DECODE | MOE_MODE_PREFILL
+ *   workspace      moe_ffn_workspace_bytes(...) bytes of device scratch
+ *   status         optional device int32: MOE_STATUS_BAD_MAP is OR-ed in when
+ *                  offsets or route ids are out of range (those rows skipped)
+ * Limits: H % 128 == 0, I % 128 == 0, I_s % 128 == 0, 128 <= H <= 8192,
+ *   128 <= I, I_s <= 4096, 1 <= E <= MOE_MAX_E, 1 <= K <= MOE_MAX_K
+ *   (MOE_ERR_UNSUPPORTED_SHAPE otherwise).
+ * Zero-weight routes produce rows equal to +0 or -0 (a zero contribution) as
+ * long as Wd_e h is finite.
+ * ------------------------------------------------------------------------- */
+MOE_API size_t moe_ffn_workspace_bytes(int T, int K, int H, int E, int I, int I_shared, int mode);
+MOE_API int moe_expert_ffn(const uint16_t* x, int T, int H, int K, const moe_fp8_experts* routed,
+                   const moe_fp8_experts* shared, const int32_t* expert_offsets,
+                   const int32_t* sorted_route, const float* topk_w, uint16_t* y_sorted,
+                   uint16_t* y_shared, int mode, void* workspace, size_t workspace_bytes,
+                   int32_t* status, moe_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * moe_combine -- top-K reduce back to token order.
+ *
+ * The Nemotron unpermute-reduce, the aiter FP32 route reduction and the NKI
+ * Top-K Reduce:  out[t, :] = sum_{j=0..K-1} y_sorted[inv_route[t*K + j], :]
+ *                            (+ y_shared[t, :] if y_shared != NULL),
+ * summed in fp32 in slot order j = 0..K-1 (then the shared term), one rounding
+ * at the end.  Routes with inv_route = -1 add nothing.
+ *   y_sorted  [T*K, H] bf16; inv_route [T*K] i32; y_shared [T, H] bf16 or NULL
+ *   out       [T, H], bf16 (out_dtype MOE_OUT_BF16) or f32 (MOE_OUT_F32)
+ * Limits: H % 8 == 0, 1 <= K <= MOE_MAX_K.
+ * ------------------------------------------------------------------------- */
+MOE_API int moe_combine(const uint16_t* y_sorted, const int32_t* inv_route, const uint16_t* y_shared,
+                int T, int K, int H, void* out, int out_dtype, moe_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_FFN_H */

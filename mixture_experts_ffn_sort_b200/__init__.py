@@ -1,0 +1,267 @@
+"""Routed MoE FFN for NVIDIA B200: Python binding of libmoe_ffn_b200.so.
+
+The library (include/moe_ffn.h) exports moe_route, moe_sort, moe_expert_ffn
+and moe_combine.  This module marshals torch tensors into those calls: device
+pointers, sizes and the current CUDA stream.  Every step of the computation
+runs in the library's kernels; torch only allocates device memory.  There is no
+fallback: if the library is missing, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe_ffn_b200.so")
+
+MOE_OK = 0
+MOE_ERR_INVALID_ARG = -1
+MOE_ERR_UNSUPPORTED_SHAPE = -2
+MOE_ERR_MISALIGNED = -3
+MOE_ERR_WORKSPACE_TOO_SMALL = -4
+MOE_ERR_CUDA = -5
+MOE_MODE_AUTO, MOE_MODE_DECODE, MOE_MODE_PREFILL = 0, 1, 2
+MOE_OUT_BF16, MOE_OUT_F32 = 0, 1
+MOE_STATUS_BAD_ID, MOE_STATUS_BAD_MAP, MOE_STATUS_TIMEOUT = 1, 2, 4
+MOE_MAX_E, MOE_MAX_K = 1024, 32
+
+EXPORTED = ("moe_last_error", "moe_abi_version", "moe_route", "moe_sort_workspace_bytes", "moe_sort",
+            "moe_ffn_workspace_bytes", "moe_expert_ffn", "moe_combine")
+
+
+class MoEError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__("MoE call failed (%d): %s" % (code, msg))
+        self.code = code
+
+
+class _Experts(ctypes.Structure):
+    _fields_ = [("w_gate", ctypes.c_void_p), ("w_up", ctypes.c_void_p), ("w_down", ctypes.c_void_p),
+                ("s_gate", ctypes.c_void_p), ("s_up", ctypes.c_void_p), ("s_down", ctypes.c_void_p),
+                ("n_experts", ctypes.c_int), ("inter", ctypes.c_int)]
+
+
+_lock = threading.Lock()
+_L = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load the CUDA library (raises if it has not been built)."""
+    global _L
+    with _lock:
+        if _L is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError("%s is missing: build it with "
+                                   "`python -m mixture_experts_ffn_sort_b200.build`" % LIB_PATH)
+            L = ctypes.CDLL(LIB_PATH)
+            P, I, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+            L.moe_last_error.restype = ctypes.c_char_p
+            L.moe_abi_version.restype = I
+            L.moe_route.argtypes = [P, I, I, I, P, P, P, P]
+            L.moe_route.restype = I
+            L.moe_sort_workspace_bytes.argtypes = [I, I, I]
+            L.moe_sort_workspace_bytes.restype = S
+            L.moe_sort.argtypes = [P, I, I, I, P, P, P, P, S, P, P]
+            L.moe_sort.restype = I
+            L.moe_ffn_workspace_bytes.argtypes = [I, I, I, I, I, I, I]
+            L.moe_ffn_workspace_bytes.restype = S
+            L.moe_expert_ffn.argtypes = [P, I, I, I, P, P, P, P, P, P, P, I, P, S, P, P]
+            L.moe_expert_ffn.restype = I
+            L.moe_combine.argtypes = [P, P, P, I, I, I, P, I, P]
+            L.moe_combine.restype = I
+            _L = L
+    return _L
+
+
+def _check(rc: int):
+    if rc != MOE_OK:
+        raise MoEError(rc, lib().moe_last_error().decode())
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("tensors must be CUDA tensors")
+
+
+@dataclass
+class Experts:
+    """Block-scaled FP8 experts resident on the device (see moe_fp8_experts).
+
+    w_gate, w_up: uint8 [n, I, H]; w_down: uint8 [n, H, I];
+    s_gate, s_up: float32 [n, I/128, H/128]; s_down: float32 [n, H/128, I/128].
+    """
+
+    w_gate: torch.Tensor
+    s_gate: torch.Tensor
+    w_up: torch.Tensor
+    s_up: torch.Tensor
+    w_down: torch.Tensor
+    s_down: torch.Tensor
+
+    @property
+    def n(self) -> int:
+        return self.w_gate.shape[0]
+
+    @property
+    def inter(self) -> int:
+        return self.w_gate.shape[1]
+
+    def struct(self) -> _Experts:
+        return _Experts(self.w_gate.data_ptr(), self.w_up.data_ptr(), self.w_down.data_ptr(),
+                        self.s_gate.data_ptr(), self.s_up.data_ptr(), self.s_down.data_ptr(),
+                        self.n, self.inter)
+
+    @staticmethod
+    def from_host(ex, device="cuda") -> "Experts":
+        """Copy host experts (any object with numpy w_*/s_* arrays) to the device."""
+        def t(a):
+            return torch.from_numpy(a).to(device)
+        return Experts(t(ex.w_gate), t(ex.s_gate), t(ex.w_up), t(ex.s_up), t(ex.w_down), t(ex.s_down))
+
+
+# ---------------------------------------------------------------- the four calls
+
+def moe_route(logits: torch.Tensor, K: int, zero_mask: Optional[torch.Tensor] = None,
+              topk_ids: Optional[torch.Tensor] = None, topk_w: Optional[torch.Tensor] = None,
+              stream=None):
+    """logits [T, E] f32 -> (topk_ids [T, K] i32, topk_w [T, K] f32)."""
+    _need_cuda(logits, zero_mask)
+    T, E = logits.shape
+    if topk_ids is None:
+        topk_ids = torch.empty((T, K), dtype=torch.int32, device=logits.device)
+    if topk_w is None:
+        topk_w = torch.empty((T, K), dtype=torch.float32, device=logits.device)
+    _check(lib().moe_route(_ptr(logits), T, E, K, _ptr(zero_mask), _ptr(topk_ids), _ptr(topk_w),
+                           _stream(stream)))
+    return topk_ids, topk_w
+
+
+def moe_sort_workspace_bytes(T: int, K: int, E: int) -> int:
+    return int(lib().moe_sort_workspace_bytes(T, K, E))
+
+
+def moe_sort(topk_ids: torch.Tensor, E: int, status: Optional[torch.Tensor] = None,
+             expert_offsets=None, sorted_route=None, inv_route=None, workspace=None, stream=None):
+    """topk_ids [T, K] i32 -> (expert_offsets [E+1], sorted_route [T*K], inv_route [T*K])."""
+    _need_cuda(topk_ids, status)
+    T, K = topk_ids.shape
+    dev = topk_ids.device
+    if expert_offsets is None:
+        expert_offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    if sorted_route is None:
+        sorted_route = torch.empty(T * K, dtype=torch.int32, device=dev)
+    if inv_route is None:
+        inv_route = torch.empty(T * K, dtype=torch.int32, device=dev)
+    need = moe_sort_workspace_bytes(T, K, E)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    _check(lib().moe_sort(_ptr(topk_ids), T, K, E, _ptr(expert_offsets), _ptr(sorted_route),
+                          _ptr(inv_route), _ptr(workspace), workspace.numel(), _ptr(status),
+                          _stream(stream)))
+    return expert_offsets, sorted_route, inv_route
+
+
+def moe_ffn_workspace_bytes(T, K, H, E, I, I_shared=0, mode=MOE_MODE_AUTO) -> int:
+    return int(lib().moe_ffn_workspace_bytes(T, K, H, E, I, I_shared, mode))
+
+
+def moe_expert_ffn(x: torch.Tensor, K: int, routed: Experts, expert_offsets: torch.Tensor,
+                   sorted_route: torch.Tensor, topk_w: torch.Tensor, shared: Optional[Experts] = None,
+                   mode: int = MOE_MODE_AUTO, status: Optional[torch.Tensor] = None,
+                   y_sorted=None, y_shared=None, workspace=None, stream=None):
+    """x [T, H] bf16 -> (y_sorted [T*K, H] bf16, y_shared [T, H] bf16 or None)."""
+    _need_cuda(x, expert_offsets, sorted_route, topk_w, status)
+    T, H = x.shape
+    dev = x.device
+    if y_sorted is None:
+        y_sorted = torch.empty((T * K, H), dtype=torch.bfloat16, device=dev)
+    if shared is not None and y_shared is None:
+        y_shared = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    need = moe_ffn_workspace_bytes(T, K, H, routed.n, routed.inter, shared.inter if shared else 0, mode)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    rs = routed.struct()
+    ss = shared.struct() if shared is not None else None
+    _check(lib().moe_expert_ffn(_ptr(x), T, H, K, ctypes.byref(rs),
+                                ctypes.byref(ss) if ss is not None else None,
+                                _ptr(expert_offsets), _ptr(sorted_route), _ptr(topk_w), _ptr(y_sorted),
+                                _ptr(y_shared) if shared is not None else None, mode, _ptr(workspace),
+                                workspace.numel(), _ptr(status), _stream(stream)))
+    return y_sorted, (y_shared if shared is not None else None)
+
+
+def moe_combine(y_sorted: torch.Tensor, inv_route: torch.Tensor, y_shared: Optional[torch.Tensor],
+                T: int, K: int, out_dtype: int = MOE_OUT_BF16, out=None, stream=None):
+    """-> out [T, H] (bf16 or f32)."""
+    _need_cuda(y_sorted, inv_route, y_shared)
+    H = y_sorted.shape[1]
+    if out is None:
+        dt = torch.bfloat16 if out_dtype == MOE_OUT_BF16 else torch.float32
+        out = torch.empty((T, H), dtype=dt, device=y_sorted.device)
+    _check(lib().moe_combine(_ptr(y_sorted), _ptr(inv_route), _ptr(y_shared), T, K, H, _ptr(out),
+                             out_dtype, _stream(stream)))
+    return out
+
+
+# ---------------------------------------------------------------- whole layer
+
+class MoEFFN:
+    """The routed MoE FFN of one layer on fixed shapes: route -> sort -> expert
+    FFN -> combine, with every buffer allocated once (no allocation per call,
+    so a call can be captured in a CUDA graph after the first one)."""
+
+    def __init__(self, routed: Experts, T: int, K: int, shared: Optional[Experts] = None,
+                 mode: int = MOE_MODE_AUTO, out_dtype: int = MOE_OUT_BF16, device="cuda"):
+        self.routed, self.shared, self.T, self.K = routed, shared, T, K
+        self.E, self.I, self.H = routed.n, routed.inter, routed.w_gate.shape[2]
+        self.mode, self.out_dtype = mode, out_dtype
+        d = device
+        R = T * K
+        self.topk_ids = torch.empty((T, K), dtype=torch.int32, device=d)
+        self.topk_w = torch.empty((T, K), dtype=torch.float32, device=d)
+        self.offsets = torch.empty(self.E + 1, dtype=torch.int32, device=d)
+        self.sorted_route = torch.empty(R, dtype=torch.int32, device=d)
+        self.inv_route = torch.empty(R, dtype=torch.int32, device=d)
+        self.sort_ws = torch.empty(max(16, moe_sort_workspace_bytes(T, K, self.E)), dtype=torch.uint8, device=d)
+        self.ffn_ws = torch.empty(max(16, moe_ffn_workspace_bytes(T, K, self.H, self.E, self.I,
+                                                                  shared.inter if shared else 0, mode)),
+                                  dtype=torch.uint8, device=d)
+        self.y_sorted = torch.empty((R, self.H), dtype=torch.bfloat16, device=d)
+        self.y_shared = torch.empty((T, self.H), dtype=torch.bfloat16, device=d) if shared else None
+        dt = torch.bfloat16 if out_dtype == MOE_OUT_BF16 else torch.float32
+        self.out = torch.empty((T, self.H), dtype=dt, device=d)
+        self.status = torch.zeros(1, dtype=torch.int32, device=d)
+
+    # Number of the library's kernel launches one forward makes.
+    def launches(self) -> int:
+        R = self.T * self.K
+        n = 1 + (1 if R <= 16384 else 3) + 2 + (2 if self.shared is not None else 0) + 1
+        return n
+
+    def forward(self, x: torch.Tensor, logits: torch.Tensor, zero_mask: Optional[torch.Tensor] = None,
+                stream=None) -> torch.Tensor:
+        moe_route(logits, self.K, zero_mask, self.topk_ids, self.topk_w, stream=stream)
+        moe_sort(self.topk_ids, self.E, self.status, self.offsets, self.sorted_route, self.inv_route,
+                 self.sort_ws, stream=stream)
+        moe_expert_ffn(x, self.K, self.routed, self.offsets, self.sorted_route, self.topk_w, self.shared,
+                       self.mode, self.status, self.y_sorted, self.y_shared, self.ffn_ws, stream=stream)
+        moe_combine(self.y_sorted, self.inv_route, self.y_shared, self.T, self.K, self.out_dtype, self.out,
+                    stream=stream)
+        return self.out
+
+    __call__ = forward

@@ -1,0 +1,67 @@
+// launch.h -- internal host-side launchers of the library's kernels (C++ only;
+// the public boundary is include/moe_ffn.h).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace moe {
+
+// ---------------------------------------------------------------- route
+cudaError_t launch_route(const float* logits, int T, int E, int K, const uint8_t* zero_mask,
+                         int32_t* ids, float* w, cudaStream_t stream);
+
+// ---------------------------------------------------------------- sort
+// Routes per warp-chunk of the multi-kernel sort, and the largest route count
+// handled by the single-block sort.
+constexpr int kSortChunk = 2048;
+constexpr long kSortSmallMaxRoutes = 16384;
+size_t sort_workspace_bytes(long R, int E);
+cudaError_t launch_sort(const int32_t* ids, long R, int E, int32_t* offsets, int32_t* sorted_route,
+                        int32_t* inv_route, void* ws, int32_t* status, cudaStream_t stream);
+
+// ---------------------------------------------------------------- combine
+cudaError_t launch_combine(const uint16_t* y_sorted, const int32_t* inv_route,
+                           const uint16_t* y_shared, int T, int K, int H, void* out, int out_f32,
+                           cudaStream_t stream);
+
+// ---------------------------------------------------------------- expert FFN (decode)
+// One projection set of experts as the kernels see it.
+struct ExpertsView {
+    const uint8_t* w_gate;
+    const uint8_t* w_up;
+    const uint8_t* w_down;
+    const float* s_gate;
+    const float* s_up;
+    const float* s_down;
+    int n;      // experts
+    int inter;  // I
+};
+
+struct FfnArgs {
+    const uint16_t* x;  // [T, H]
+    int T, H, K;
+    ExpertsView ex;
+    // Rows of this call: either routed (offsets / sorted_route / topk_w) or
+    // the identity group of all T tokens with weight 1 (shared expert).
+    bool identity;
+    const int32_t* offsets;
+    const int32_t* sorted_route;
+    const float* topk_w;
+    uint16_t* h;  // [rows, I] bf16 scratch
+    uint16_t* y;  // [rows, H] bf16 output
+    int32_t* status;
+    int avg_rows;  // host-known rows per expert (sizes the token tile)
+};
+
+cudaError_t launch_ffn_decode(const FfnArgs& a, cudaStream_t stream);
+
+// ---------------------------------------------------------------- TMA descriptors
+// 2-D row-major uint8 matrix [rows, cols] (cols contiguous), box
+// {box_cols, box_rows}, 128-byte swizzle.
+cudaError_t make_tmap_u8_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                            uint32_t box_cols, uint32_t box_rows);
+
+}  // namespace moe

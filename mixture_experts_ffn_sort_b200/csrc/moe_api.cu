@@ -1,0 +1,220 @@
+// moe_api.cu -- the extern "C" boundary (include/moe_ffn.h): argument and
+// tensor-contract validation on the host, workspace carving, kernel launch,
+// and the thread-local error message.  Like the C-ABI entry points of the
+// aiter gfx950 prefill PR, the launcher checks the tensor contracts; like the
+// Nemotron-H layer's constructor, an out-of-range top_k is reported with a
+// message naming the bound.
+#include <stdarg.h>
+#include <stdio.h>
+
+#include <string>
+
+#include "../../include/moe_ffn.h"
+#include "launch.h"
+
+namespace moe {
+bool ffn_decode_supported(int H, int I);
+}
+
+namespace {
+
+thread_local std::string g_err;
+
+int fail(int code, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_err = buf;
+    return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+    return fail(MOE_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorString(e), cudaGetErrorName(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t round256(size_t n) { return (n + 255) & ~size_t(255); }
+
+int check_topk(int T, int E, int K) {
+    if (T < 0 || T > MOE_MAX_T) return fail(MOE_ERR_INVALID_ARG, "T=%d must be in 0..=%d", T, MOE_MAX_T);
+    if (E < 1 || E > MOE_MAX_E)
+        return fail(MOE_ERR_UNSUPPORTED_SHAPE, "num_experts=%d must be in 1..=%d", E, MOE_MAX_E);
+    if (K < 1 || K > E || K > MOE_MAX_K)
+        return fail(MOE_ERR_INVALID_ARG,
+                    "top_k=%d must be in 1..=%d and within the routing kernels' bounds "
+                    "(top_k max %d, num_experts=%d max %d)",
+                    K, E, MOE_MAX_K, E, MOE_MAX_E);
+    return MOE_OK;
+}
+
+int check_experts(const moe_fp8_experts* ex, int H, const char* which) {
+    if (!ex->w_gate || !ex->w_up || !ex->w_down || !ex->s_gate || !ex->s_up || !ex->s_down)
+        return fail(MOE_ERR_INVALID_ARG, "%s experts: NULL weight or scale pointer", which);
+    if (!aligned16(ex->w_gate) || !aligned16(ex->w_up) || !aligned16(ex->w_down) ||
+        !aligned16(ex->s_gate) || !aligned16(ex->s_up) || !aligned16(ex->s_down))
+        return fail(MOE_ERR_MISALIGNED, "%s experts: weight and scale bases must be 16-byte aligned", which);
+    const int I = ex->inter;
+    if (I < 128 || I > 4096 || I % MOE_BLOCK)
+        return fail(MOE_ERR_UNSUPPORTED_SHAPE, "%s experts: inter=%d must be a multiple of 128 in 128..=4096",
+                    which, I);
+    if (!moe::ffn_decode_supported(H, I))
+        return fail(MOE_ERR_UNSUPPORTED_SHAPE, "%s experts: H=%d, inter=%d exceed the shared-memory tiles",
+                    which, H, I);
+    return MOE_OK;
+}
+
+size_t ffn_h_bytes(long R, int I) { return round256(static_cast<size_t>(R) * I * 2); }
+
+}  // namespace
+
+extern "C" {
+
+const char* moe_last_error(void) { return g_err.c_str(); }
+
+int moe_abi_version(void) { return MOE_ABI_VERSION; }
+
+int moe_route(const float* logits, int T, int E, int K, const uint8_t* zero_mask, int32_t* topk_ids,
+              float* topk_w, moe_stream_t stream) {
+    g_err.clear();
+    int rc = check_topk(T, E, K);
+    if (rc) return rc;
+    if (T == 0) return MOE_OK;
+    if (!logits || !topk_ids || !topk_w)
+        return fail(MOE_ERR_INVALID_ARG, "moe_route: logits, topk_ids and topk_w must not be NULL");
+    if (!aligned16(logits) || !aligned16(topk_ids) || !aligned16(topk_w))
+        return fail(MOE_ERR_MISALIGNED, "moe_route: tensor bases must be 16-byte aligned");
+    cudaError_t e = moe::launch_route(logits, T, E, K, zero_mask, topk_ids, topk_w, stream);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_route launch");
+}
+
+size_t moe_sort_workspace_bytes(int T, int K, int E) {
+    if (T < 0 || K < 1 || E < 1) return 0;
+    return moe::sort_workspace_bytes(static_cast<long>(T) * K, E);
+}
+
+int moe_sort(const int32_t* topk_ids, int T, int K, int E, int32_t* expert_offsets,
+             int32_t* sorted_route, int32_t* inv_route, void* workspace, size_t workspace_bytes,
+             int32_t* status, moe_stream_t stream) {
+    g_err.clear();
+    int rc = check_topk(T, E, K);
+    if (rc) return rc;
+    if (!expert_offsets) return fail(MOE_ERR_INVALID_ARG, "moe_sort: expert_offsets must not be NULL");
+    if (T > 0 && (!topk_ids || !sorted_route || !inv_route))
+        return fail(MOE_ERR_INVALID_ARG, "moe_sort: topk_ids, sorted_route and inv_route must not be NULL");
+    if (!aligned16(topk_ids) || !aligned16(expert_offsets) || !aligned16(sorted_route) ||
+        !aligned16(inv_route) || !aligned16(workspace) || (status && (reinterpret_cast<uintptr_t>(status) & 3)))
+        return fail(MOE_ERR_MISALIGNED, "moe_sort: tensor bases must be 16-byte aligned");
+    const long R = static_cast<long>(T) * K;
+    const size_t need = moe::sort_workspace_bytes(R, E);
+    if (workspace_bytes < need || (need && !workspace))
+        return fail(MOE_ERR_WORKSPACE_TOO_SMALL, "moe_sort: workspace of %zu bytes, need %zu",
+                    workspace_bytes, need);
+    if (T == 0) {
+        // No routes: all offsets are 0.
+        cudaError_t e = cudaMemsetAsync(expert_offsets, 0, sizeof(int32_t) * (E + 1), stream);
+        return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_sort memset");
+    }
+    cudaError_t e = moe::launch_sort(topk_ids, R, E, expert_offsets, sorted_route, inv_route, workspace,
+                                     status, stream);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_sort launch");
+}
+
+size_t moe_ffn_workspace_bytes(int T, int K, int H, int E, int I, int I_shared, int mode) {
+    (void)H;
+    (void)E;
+    (void)mode;
+    if (T < 0 || K < 1 || I < 0 || I_shared < 0) return 0;
+    const long R = static_cast<long>(T) * K;
+    return ffn_h_bytes(R, I) + ffn_h_bytes(T, I_shared);
+}
+
+int moe_expert_ffn(const uint16_t* x, int T, int H, int K, const moe_fp8_experts* routed,
+                   const moe_fp8_experts* shared, const int32_t* expert_offsets,
+                   const int32_t* sorted_route, const float* topk_w, uint16_t* y_sorted,
+                   uint16_t* y_shared, int mode, void* workspace, size_t workspace_bytes,
+                   int32_t* status, moe_stream_t stream) {
+    g_err.clear();
+    if (!routed) return fail(MOE_ERR_INVALID_ARG, "moe_expert_ffn: routed must not be NULL");
+    const int E = routed->n_experts, I = routed->inter;
+    int rc = check_topk(T, E, K);
+    if (rc) return rc;
+    if (mode != MOE_MODE_AUTO && mode != MOE_MODE_DECODE && mode != MOE_MODE_PREFILL)
+        return fail(MOE_ERR_INVALID_ARG, "moe_expert_ffn: mode=%d is not AUTO/DECODE/PREFILL", mode);
+    if (H < 128 || H % MOE_BLOCK || H > 8192)
+        return fail(MOE_ERR_UNSUPPORTED_SHAPE, "moe_expert_ffn: H=%d must be a multiple of 128 in 128..=8192", H);
+    if ((rc = check_experts(routed, H, "routed"))) return rc;
+    if (shared) {
+        if (shared->n_experts != 1)
+            return fail(MOE_ERR_INVALID_ARG, "moe_expert_ffn: shared->n_experts=%d must be 1", shared->n_experts);
+        if ((rc = check_experts(shared, H, "shared"))) return rc;
+    }
+    if (T == 0) return MOE_OK;
+    if (!x || !expert_offsets || !sorted_route || !topk_w || !y_sorted || (shared && !y_shared))
+        return fail(MOE_ERR_INVALID_ARG, "moe_expert_ffn: NULL tensor pointer");
+    if (!aligned16(x) || !aligned16(expert_offsets) || !aligned16(sorted_route) || !aligned16(topk_w) ||
+        !aligned16(y_sorted) || (shared && !aligned16(y_shared)) || !aligned16(workspace))
+        return fail(MOE_ERR_MISALIGNED, "moe_expert_ffn: tensor bases must be 16-byte aligned");
+    const long R = static_cast<long>(T) * K;
+    const int Is = shared ? shared->inter : 0;
+    const size_t need = moe_ffn_workspace_bytes(T, K, H, E, I, Is, mode);
+    if (workspace_bytes < need || !workspace)
+        return fail(MOE_ERR_WORKSPACE_TOO_SMALL, "moe_expert_ffn: workspace of %zu bytes, need %zu",
+                    workspace_bytes, need);
+    if (mode == MOE_MODE_PREFILL)
+        return fail(MOE_ERR_UNSUPPORTED_SHAPE, "moe_expert_ffn: PREFILL kernels are not available in this build");
+
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    moe::FfnArgs a{};
+    a.x = x;
+    a.T = T;
+    a.H = H;
+    a.K = K;
+    a.ex = {routed->w_gate, routed->w_up, routed->w_down, routed->s_gate, routed->s_up, routed->s_down, E, I};
+    a.identity = false;
+    a.offsets = expert_offsets;
+    a.sorted_route = sorted_route;
+    a.topk_w = topk_w;
+    a.h = reinterpret_cast<uint16_t*>(ws);
+    a.y = y_sorted;
+    a.status = status;
+    a.avg_rows = static_cast<int>((R + E - 1) / E);
+    cudaError_t e = moe::launch_ffn_decode(a, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "moe_expert_ffn routed launch");
+    if (shared) {
+        moe::FfnArgs s = a;
+        s.ex = {shared->w_gate, shared->w_up, shared->w_down, shared->s_gate, shared->s_up, shared->s_down, 1, Is};
+        s.identity = true;
+        s.offsets = nullptr;
+        s.sorted_route = nullptr;
+        s.topk_w = nullptr;
+        s.h = reinterpret_cast<uint16_t*>(ws + ffn_h_bytes(R, I));
+        s.y = y_shared;
+        s.avg_rows = T;
+        e = moe::launch_ffn_decode(s, stream);
+        if (e != cudaSuccess) return cuda_fail(e, "moe_expert_ffn shared launch");
+    }
+    return MOE_OK;
+}
+
+int moe_combine(const uint16_t* y_sorted, const int32_t* inv_route, const uint16_t* y_shared, int T,
+                int K, int H, void* out, int out_dtype, moe_stream_t stream) {
+    g_err.clear();
+    if (T < 0 || T > MOE_MAX_T) return fail(MOE_ERR_INVALID_ARG, "moe_combine: T=%d out of range", T);
+    if (K < 1 || K > MOE_MAX_K) return fail(MOE_ERR_INVALID_ARG, "moe_combine: K=%d must be in 1..=%d", K, MOE_MAX_K);
+    if (H < 8 || H % 8) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "moe_combine: H=%d must be a positive multiple of 8", H);
+    if (out_dtype != MOE_OUT_BF16 && out_dtype != MOE_OUT_F32)
+        return fail(MOE_ERR_INVALID_ARG, "moe_combine: out_dtype=%d is not BF16/F32", out_dtype);
+    if (T == 0) return MOE_OK;
+    if (!y_sorted || !inv_route || !out)
+        return fail(MOE_ERR_INVALID_ARG, "moe_combine: y_sorted, inv_route and out must not be NULL");
+    if (!aligned16(y_sorted) || !aligned16(inv_route) || !aligned16(y_shared) || !aligned16(out))
+        return fail(MOE_ERR_MISALIGNED, "moe_combine: tensor bases must be 16-byte aligned");
+    cudaError_t e = moe::launch_combine(y_sorted, inv_route, y_shared, T, K, H, out,
+                                        out_dtype == MOE_OUT_F32, stream);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_combine launch");
+}
+
+}  // extern "C"

@@ -1,0 +1,240 @@
+// sort.cu -- stable sort of the routes by expert (moe_sort).
+//
+// The "sort tokens by expert" step of the Nemotron-H sorted prefill path
+// (spark_model/layers/nemotron_moe.rs, `prefill` step 5), the NKI Permute
+// Routed Tokens kernel, and the sort with an inverse route map that the aiter
+// gfx950 prefill PR reuses.  A counting sort in three passes:
+//   1. each warp-chunk of routes builds an expert histogram;
+//   2. an exclusive scan in (expert, chunk) order gives every chunk the first
+//      sorted position of each of its experts, and the per-expert offsets;
+//   3. each warp-chunk walks its routes in order and scatters them, ranking
+//      equal experts within a 32-route step with __match_any_sync.
+// Order within an expert is therefore route order: the result is unique and
+// deterministic.  Small inputs run all three passes in one thread block.
+#include "device_common.cuh"
+#include "launch.h"
+
+namespace moe {
+
+namespace {
+
+__device__ __forceinline__ uint32_t lanemask_lt() {
+    uint32_t m;
+    asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+    return m;
+}
+
+// Scatter one warp-chunk [r_begin, r_end) given the chunk's start positions
+// `cursor[e]` (shared memory, advanced in place).
+__device__ __forceinline__ void scatter_chunk(const int32_t* __restrict__ ids, long r_begin,
+                                              long r_end, int E, int32_t* cursor,
+                                              int32_t* __restrict__ sorted_route,
+                                              int32_t* __restrict__ inv_route) {
+    const int lane = threadIdx.x & 31;
+    const uint32_t lt = lanemask_lt();
+    for (long r0 = r_begin; r0 < r_end; r0 += 32) {
+        const long r = r0 + lane;
+        const bool in = r < r_end;
+        const int e = in ? ids[r] : -1;
+        const bool ok = in && e >= 0 && e < E;
+        const uint32_t peers = __match_any_sync(0xffffffffu, ok ? e : (E + lane));
+        int32_t pos = 0;
+        if (ok) pos = cursor[e] + __popc(peers & lt);
+        __syncwarp();
+        // The highest lane of each group of equal experts advances the cursor.
+        if (ok && (peers >> lane) == 1u) cursor[e] += __popc(peers);
+        __syncwarp();
+        if (ok) {
+            sorted_route[pos] = static_cast<int32_t>(r);
+            inv_route[r] = pos;
+        } else if (in) {
+            inv_route[r] = -1;
+        }
+    }
+}
+
+// Count one warp-chunk into hist[E] (shared memory, zeroed by the caller).
+// Returns true if an id outside [0, E) was seen.
+__device__ __forceinline__ bool count_chunk(const int32_t* __restrict__ ids, long r_begin,
+                                            long r_end, int E, int32_t* hist) {
+    const int lane = threadIdx.x & 31;
+    bool bad = false;
+    for (long r = r_begin + lane; r < r_end; r += 32) {
+        const int e = ids[r];
+        if (e >= 0 && e < E)
+            atomicAdd(&hist[e], 1);
+        else
+            bad = true;
+    }
+    return __any_sync(0xffffffffu, bad);
+}
+
+// Block-wide exclusive scan of one int per thread; returns the prefix and
+// writes the block total to *total.  blockDim.x is a multiple of 32, <= 1024.
+__device__ int block_exclusive_scan(int v, int* scratch /*[32]*/, int* total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int nw = blockDim.x >> 5;
+    int x = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, off);
+        if (lane >= off) x += y;
+    }
+    if (lane == 31) scratch[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+        int s = lane < nw ? scratch[lane] : 0;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, s, off);
+            if (lane >= off) s += y;
+        }
+        scratch[lane] = s;  // inclusive warp totals
+    }
+    __syncthreads();
+    const int warp_prefix = warp ? scratch[warp - 1] : 0;
+    *total = scratch[nw - 1];
+    __syncthreads();
+    return warp_prefix + x - v;
+}
+
+// ---------------------------------------------------------------- small: one block
+
+// smem: hist[NW][E] ints, then 32 ints of scan scratch.
+__global__ void __launch_bounds__(1024) sort_small_kernel(const int32_t* __restrict__ ids, long R,
+                                                          int E, int32_t* __restrict__ offsets,
+                                                          int32_t* __restrict__ sorted_route,
+                                                          int32_t* __restrict__ inv_route,
+                                                          int32_t* status) {
+    extern __shared__ int32_t sm[];
+    const int NW = blockDim.x >> 5;
+    const int warp = threadIdx.x >> 5;
+    int32_t* hist = sm;                      // [NW][E]
+    int32_t* scratch = sm + NW * E;          // [32]
+    for (int i = threadIdx.x; i < NW * E; i += blockDim.x) hist[i] = 0;
+    __syncthreads();
+
+    const long chunk = ((R + NW - 1) / NW + 31) / 32 * 32;
+    const long rb = min(R, warp * chunk), re = min(R, rb + chunk);
+    if (count_chunk(ids, rb, re, E, hist + warp * E) && (threadIdx.x & 31) == 0)
+        report_status(status, MOE_STATUS_BAD_ID);
+    __syncthreads();
+
+    // Exclusive scan over (expert, warp) order; each thread owns a contiguous
+    // run of that order.
+    const int N = NW * E;
+    const int per = (N + blockDim.x - 1) / blockDim.x;
+    const int i0 = min(N, static_cast<int>(threadIdx.x) * per), i1 = min(N, i0 + per);
+    int s = 0;
+    for (int i = i0; i < i1; ++i) s += hist[(i % NW) * E + i / NW];
+    int total;
+    int prefix = block_exclusive_scan(s, scratch, &total);
+    for (int i = i0; i < i1; ++i) {
+        const int idx = (i % NW) * E + i / NW;
+        const int c = hist[idx];
+        if (i % NW == 0) offsets[i / NW] = prefix;
+        hist[idx] = prefix;
+        prefix += c;
+    }
+    if (threadIdx.x == 0) offsets[E] = total;
+    for (long p = total + threadIdx.x; p < R; p += blockDim.x) sorted_route[p] = -1;
+    __syncthreads();
+
+    scatter_chunk(ids, rb, re, E, hist + warp * E, sorted_route, inv_route);
+}
+
+// ---------------------------------------------------------------- large: three kernels
+
+constexpr int kSortWarpsPerBlock = 8;
+
+// counts[e * nchunks + c] = routes of chunk c with expert e.
+__global__ void __launch_bounds__(kSortWarpsPerBlock * 32)
+    sort_count_kernel(const int32_t* __restrict__ ids, long R, int E, int nchunks,
+                      int32_t* __restrict__ counts, int32_t* status) {
+    extern __shared__ int32_t sm[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int c = blockIdx.x * kSortWarpsPerBlock + warp;
+    int32_t* hist = sm + warp * E;
+    for (int e = lane; e < E; e += 32) hist[e] = 0;
+    __syncwarp();
+    if (c >= nchunks) return;
+    const long rb = static_cast<long>(c) * kSortChunk, re = min(R, rb + kSortChunk);
+    if (count_chunk(ids, rb, re, E, hist) && lane == 0) report_status(status, MOE_STATUS_BAD_ID);
+    __syncwarp();
+    for (int e = lane; e < E; e += 32) counts[static_cast<size_t>(e) * nchunks + c] = hist[e];
+}
+
+// In-place exclusive scan of counts[E * nchunks] (expert-major); offsets[e] is
+// the scan value at (e, chunk 0) and offsets[E] the total.
+__global__ void __launch_bounds__(1024)
+    sort_scan_kernel(int32_t* __restrict__ counts, int E, int nchunks, long R,
+                     int32_t* __restrict__ offsets, int32_t* __restrict__ sorted_route) {
+    __shared__ int scratch[32];
+    const int N = E * nchunks;
+    const int per = (N + blockDim.x - 1) / blockDim.x;
+    const int i0 = min(N, static_cast<int>(threadIdx.x) * per), i1 = min(N, i0 + per);
+    int s = 0;
+    for (int i = i0; i < i1; ++i) s += counts[i];
+    int total;
+    int prefix = block_exclusive_scan(s, scratch, &total);
+    for (int i = i0; i < i1; ++i) {
+        const int c = counts[i];
+        if (i % nchunks == 0) offsets[i / nchunks] = prefix;
+        counts[i] = prefix;
+        prefix += c;
+    }
+    if (threadIdx.x == 0) offsets[E] = total;
+    for (long p = total + threadIdx.x; p < R; p += blockDim.x) sorted_route[p] = -1;
+}
+
+__global__ void __launch_bounds__(kSortWarpsPerBlock * 32)
+    sort_scatter_kernel(const int32_t* __restrict__ ids, long R, int E, int nchunks,
+                        const int32_t* __restrict__ base, int32_t* __restrict__ sorted_route,
+                        int32_t* __restrict__ inv_route) {
+    extern __shared__ int32_t sm[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int c = blockIdx.x * kSortWarpsPerBlock + warp;
+    if (c >= nchunks) return;
+    int32_t* cursor = sm + warp * E;
+    for (int e = lane; e < E; e += 32) cursor[e] = base[static_cast<size_t>(e) * nchunks + c];
+    __syncwarp();
+    const long rb = static_cast<long>(c) * kSortChunk, re = min(R, rb + kSortChunk);
+    scatter_chunk(ids, rb, re, E, cursor, sorted_route, inv_route);
+}
+
+int small_sort_warps(int E) {
+    int nw = 32;
+    while (nw > 1 && (static_cast<long>(nw) * E + 32) * 4 > 48 * 1024) nw >>= 1;
+    return nw;
+}
+
+}  // namespace
+
+size_t sort_workspace_bytes(long R, int E) {
+    if (R <= kSortSmallMaxRoutes) return 0;
+    const long nchunks = (R + kSortChunk - 1) / kSortChunk;
+    return static_cast<size_t>(nchunks) * E * sizeof(int32_t);
+}
+
+cudaError_t launch_sort(const int32_t* ids, long R, int E, int32_t* offsets, int32_t* sorted_route,
+                        int32_t* inv_route, void* ws, int32_t* status, cudaStream_t stream) {
+    if (R <= kSortSmallMaxRoutes) {
+        const int nw = small_sort_warps(E);
+        const size_t smem = (static_cast<size_t>(nw) * E + 32) * sizeof(int32_t);
+        sort_small_kernel<<<1, nw * 32, smem, stream>>>(ids, R, E, offsets, sorted_route, inv_route,
+                                                        status);
+        return cudaGetLastError();
+    }
+    const int nchunks = static_cast<int>((R + kSortChunk - 1) / kSortChunk);
+    int32_t* counts = static_cast<int32_t*>(ws);
+    const int blocks = (nchunks + kSortWarpsPerBlock - 1) / kSortWarpsPerBlock;
+    const size_t smem = static_cast<size_t>(kSortWarpsPerBlock) * E * sizeof(int32_t);
+    sort_count_kernel<<<blocks, kSortWarpsPerBlock * 32, smem, stream>>>(ids, R, E, nchunks, counts,
+                                                                         status);
+    sort_scan_kernel<<<1, 1024, 0, stream>>>(counts, E, nchunks, R, offsets, sorted_route);
+    sort_scatter_kernel<<<blocks, kSortWarpsPerBlock * 32, smem, stream>>>(
+        ids, R, E, nchunks, counts, sorted_route, inv_route);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

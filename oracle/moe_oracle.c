@@ -92,11 +92,21 @@ double oracle_bf16_value(uint16_t bits) {
     return (double)f;
 }
 
+/* oracle_e4m3fn_value of every code, filled once before any parallel region. */
+static double g_e4m3[256];
+static int g_e4m3_ready = 0;
+
+static void init_tables(void) {
+    if (g_e4m3_ready) return;
+    for (int c = 0; c < 256; ++c) g_e4m3[c] = oracle_e4m3fn_value((uint8_t)c);
+    g_e4m3_ready = 1;
+}
+
 /* One weight element of a block-scaled FP8 matrix [rows, cols] (cols contiguous):
  * W[n, k] = e4m3fn(q[n, k]) * s[n / 128, k / 128]. */
 static double weight(const uint8_t* q, const float* s, int cols, int n, int k) {
     int ncb = cols / ORACLE_BLOCK;
-    return oracle_e4m3fn_value(q[(size_t)n * cols + k]) *
+    return g_e4m3[q[(size_t)n * cols + k]] *
            (double)s[(size_t)(n / ORACLE_BLOCK) * ncb + (k / ORACLE_BLOCK)];
 }
 
@@ -234,6 +244,7 @@ static void load_row(const uint16_t* x, int H, int t, double* xr) {
 void oracle_ffn_sorted(const uint16_t* x, int T, int H, int K, const oracle_experts* ex,
                        const int32_t* offsets, const int32_t* sorted_route, const double* w,
                        double* y_sorted) {
+    init_tables();
     (void)T;
     int E = ex->n_experts, I = ex->inter;
     for (int e = 0; e < E; ++e) {
@@ -258,6 +269,7 @@ void oracle_ffn_sorted(const uint16_t* x, int T, int H, int K, const oracle_expe
 /* The always-on shared expert (weight 1, every token): y_shared[t] = FFN_s(x[t]). */
 void oracle_ffn_shared(const uint16_t* x, int T, int H, const oracle_experts* sh,
                        double* y_shared) {
+    init_tables();
     const uint8_t *wg, *wu, *wd; const float *sg, *su, *sd;
     expert_ptrs(sh, 0, H, &wg, &sg, &wu, &su, &wd, &sd);
     int I = sh->inter;
@@ -329,6 +341,7 @@ void oracle_moe_tokens(const uint16_t* x, const float* logits, int T, int H, int
                        const uint8_t* zero_mask, const oracle_experts* routed,
                        const oracle_experts* sh, const int32_t* tokens, int n_tokens,
                        double* out) {
+    init_tables();
     (void)T;
     int I = routed->inter;
     int Is = sh ? sh->inter : 0;
@@ -365,6 +378,7 @@ void oracle_moe_tokens(const uint16_t* x, const float* logits, int T, int H, int
 /* One expert FFN on explicit rows (no routing): y[i] = FFN_e(x[rows[i]]). */
 void oracle_expert_rows(const uint16_t* x, int H, const oracle_experts* ex, int e,
                         const int32_t* rows, int n_rows, double* y) {
+    init_tables();
     const uint8_t *wg, *wu, *wd; const float *sg, *su, *sd;
     expert_ptrs(ex, e, H, &wg, &sg, &wu, &su, &wd, &sd);
     int I = ex->inter;

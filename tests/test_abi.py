@@ -1,0 +1,140 @@
+"""The C-ABI library loads and exports every symbol include/*.h declares, and
+its host-side contract checks reject bad arguments before touching the device
+(CPU only: every call here returns from validation, none reaches a kernel)."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+import mixture_experts_ffn_sort_b200 as moe
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from mixture_experts_ffn_sort_b200 import build
+    build.build()
+    return moe.lib()
+
+
+def declared_symbols():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        for m in re.finditer(r"MOE_API\s+[\w\s\*]+?\b(moe_\w+)\s*\(", text):
+            names.add(m.group(1))
+    return names
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = declared_symbols()
+    assert {"moe_route", "moe_sort", "moe_expert_ffn", "moe_combine"} <= names
+    for n in names:
+        assert hasattr(L, n), n
+    assert names == set(moe.EXPORTED)
+
+
+def test_no_other_symbols_exported(L):
+    out = os.popen("nm -D --defined-only %s" % moe.LIB_PATH).read()
+    exported = {l.split()[-1] for l in out.splitlines() if " T " in l}
+    assert exported == set(moe.EXPORTED)
+
+
+def test_abi_version(L):
+    assert L.moe_abi_version() == 1
+
+
+def test_workspace_queries(L):
+    assert L.moe_sort_workspace_bytes(64, 8, 256) == 0            # single-block sort
+    assert L.moe_sort_workspace_bytes(32768, 10, 512) == 160 * 512 * 4
+    assert L.moe_ffn_workspace_bytes(64, 8, 2048, 256, 512, 0, 0) == 512 * 512 * 2
+    assert L.moe_ffn_workspace_bytes(16, 2, 256, 8, 128, 0, 0) == 8192
+    assert L.moe_ffn_workspace_bytes(8192, 10, 4096, 512, 256, 256, 0) == 81920 * 512 + 8192 * 512
+
+
+P = ctypes.c_void_p
+
+
+def _err(L):
+    return L.moe_last_error().decode()
+
+
+@pytest.mark.parametrize("T,E,K,code", [(4, 8, 0, moe.MOE_ERR_INVALID_ARG), (4, 8, 9, moe.MOE_ERR_INVALID_ARG),
+                                        (4, 1025, 2, moe.MOE_ERR_UNSUPPORTED_SHAPE),
+                                        (4, 64, 33, moe.MOE_ERR_INVALID_ARG), (-1, 8, 2, moe.MOE_ERR_INVALID_ARG)])
+def test_route_rejects_bad_sizes(L, T, E, K, code):
+    assert L.moe_route(P(16), T, E, K, None, P(16), P(16), None) == code
+    assert _err(L)
+
+
+def test_route_top_k_message_names_bounds(L):
+    assert L.moe_route(P(16), 4, 8, 9, None, P(16), P(16), None) == moe.MOE_ERR_INVALID_ARG
+    assert "top_k=9 must be in 1..=8" in _err(L)
+
+
+def test_route_zero_tokens_is_a_no_op(L):
+    assert L.moe_route(None, 0, 8, 2, None, None, None, None) == moe.MOE_OK
+    assert _err(L) == ""
+
+
+def test_route_null_and_misaligned(L):
+    assert L.moe_route(None, 4, 8, 2, None, P(16), P(16), None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_route(P(0x1008), 4, 8, 2, None, P(16), P(16), None) == moe.MOE_ERR_MISALIGNED
+
+
+def test_sort_checks(L):
+    assert L.moe_sort(P(16), 4, 2, 8, None, P(16), P(16), None, 0, None, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_sort(P(16), 4, 2, 8, P(20), P(16), P(16), None, 0, None, None) == moe.MOE_ERR_MISALIGNED
+    # Large sorts need the workspace the query reports.
+    assert L.moe_sort(P(16), 4096, 8, 64, P(16), P(16), P(16), P(16), 10, None, None) == \
+        moe.MOE_ERR_WORKSPACE_TOO_SMALL
+    assert "need" in _err(L)
+
+
+def _experts(inter=128, n=4, base=0x10000):
+    return moe._Experts(base, base + 0x100, base + 0x200, base + 0x300, base + 0x400, base + 0x500, n, inter)
+
+
+def test_expert_ffn_checks(L):
+    ex = _experts()
+    ws = L.moe_ffn_workspace_bytes(8, 2, 256, 4, 128, 0, 0)
+    args = lambda **kw: dict(dict(x=P(16), T=8, H=256, K=2, routed=ctypes.byref(ex), shared=None,
+                                  off=P(16), sr=P(16), w=P(16), y=P(16), ys=None, mode=0, ws=P(16),
+                                  wsb=ws, status=None, stream=None), **kw)
+
+    def call(**kw):
+        a = args(**kw)
+        return L.moe_expert_ffn(a["x"], a["T"], a["H"], a["K"], a["routed"], a["shared"], a["off"], a["sr"],
+                                a["w"], a["y"], a["ys"], a["mode"], a["ws"], a["wsb"], a["status"], a["stream"])
+
+    assert call(H=200) == moe.MOE_ERR_UNSUPPORTED_SHAPE
+    assert call(H=16384) == moe.MOE_ERR_UNSUPPORTED_SHAPE
+    assert call(mode=7) == moe.MOE_ERR_INVALID_ARG
+    assert call(K=5) == moe.MOE_ERR_INVALID_ARG
+    assert call(x=P(24)) == moe.MOE_ERR_MISALIGNED
+    assert call(wsb=ws - 1) == moe.MOE_ERR_WORKSPACE_TOO_SMALL
+    assert call(y=None) == moe.MOE_ERR_INVALID_ARG
+    bad_inter = _experts(inter=192)
+    assert call(routed=ctypes.byref(bad_inter)) == moe.MOE_ERR_UNSUPPORTED_SHAPE
+    two = _experts(n=2)
+    assert call(shared=ctypes.byref(two), ys=P(16)) == moe.MOE_ERR_INVALID_ARG   # shared must hold 1 expert
+    assert call(T=0) == moe.MOE_OK
+    assert L.moe_expert_ffn(P(16), 8, 256, 2, None, None, P(16), P(16), P(16), P(16), None, 0, P(16), ws,
+                            None, None) == moe.MOE_ERR_INVALID_ARG
+
+
+def test_combine_checks(L):
+    assert L.moe_combine(P(16), P(16), None, 4, 2, 12, P(16), 0, None) == moe.MOE_ERR_UNSUPPORTED_SHAPE
+    assert L.moe_combine(P(16), P(16), None, 4, 2, 16, P(16), 3, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_combine(P(16), P(16), P(40), 4, 2, 16, P(16), 0, None) == moe.MOE_ERR_MISALIGNED
+    assert L.moe_combine(None, None, None, 0, 2, 16, None, 0, None) == moe.MOE_OK
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(moe, "LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(moe, "_L", None)
+    with pytest.raises(RuntimeError, match="missing"):
+        moe.lib()
