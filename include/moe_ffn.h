@@ -144,6 +144,8 @@ MOE_API int moe_route(const float* logits, int T, int E, int K, const uint8_t* z
  * library only ORs bits into it, the caller clears it).
  *   workspace: device scratch of moe_sort_workspace_bytes(T, K, E) bytes, any
  *   contents; overwritten.
+ * Limits: 1 <= K <= MOE_MAX_K, 1 <= E <= MOE_MAX_E (K > E is allowed: ids
+ * need not be distinct within a token).
  * ------------------------------------------------------------------------- */
 MOE_API size_t moe_sort_workspace_bytes(int T, int K, int E);
 MOE_API int moe_sort(const int32_t* topk_ids, int T, int K, int E, int32_t* expert_offsets,
@@ -200,7 +202,7 @@ typedef struct moe_fp8_experts {
  *                  offsets or route ids are out of range (those rows skipped)
  * Limits: H % 128 == 0, I % 128 == 0, I_s % 128 == 0, 128 <= H <= 8192,
  *   128 <= I, I_s <= 4096, 1 <= E <= MOE_MAX_E, 1 <= K <= MOE_MAX_K
- *   (MOE_ERR_UNSUPPORTED_SHAPE otherwise).
+ *   (MOE_ERR_UNSUPPORTED_SHAPE / MOE_ERR_INVALID_ARG otherwise).
  * Zero-weight routes produce rows equal to +0 or -0 (a zero contribution) as
  * long as Wd_e h is finite.
  * ------------------------------------------------------------------------- */

@@ -5,6 +5,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -121,6 +122,24 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
         : "memory");
 }
 
+// Same load with an L2 cache-policy hint (see l2_evict_first_policy).
+__device__ __forceinline__ void tma_load_2d_hint(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                                 int x, int y, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "l"(policy)
+        : "memory");
+}
+
+// L2 policy for data read exactly once (streamed expert weights): evict first,
+// so activations and outputs keep their L2 residency.
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
 // Byte offset of 16-byte chunk q of row r in a tile written by TMA with
 // CU_TENSOR_MAP_SWIZZLE_128B (128-byte rows, tile base 1024-byte aligned):
 // the chunk index is XOR-ed with the row index modulo 8.
@@ -147,14 +166,38 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint3
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// D += A(16x16, row) * B(16x8, col), f16 inputs, fp32 accumulators.
+__device__ __forceinline__ void mma_f16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                              uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
 // ---------------------------------------------------------------- FP8 decode
+
+// Two E4M3FN codes (low byte -> low half) to two f16 values.  Every finite
+// E4M3FN value (|v| in [2^-9, 448] or 0) is an f16 normal or zero, so the
+// hardware conversion is exact.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t codes) {
+    uint32_t f;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(f) : "h"(codes));
+    return f;
+}
+
+__device__ __forceinline__ void e4m3x4_to_f16(uint32_t w, uint32_t& lo, uint32_t& hi) {
+    lo = e4m3x2_to_f16x2(static_cast<uint16_t>(w & 0xFFFFu));
+    hi = e4m3x2_to_f16x2(static_cast<uint16_t>(w >> 16));
+}
 
 // Two E4M3FN codes (low byte -> low half) to two BF16 values, exactly.
 // Every E4M3FN value is an f16 normal (or zero), so the hardware conversion to
 // f16x2 is exact.  Dropping the 7 low mantissa bits (always zero here) and
 // shifting the exponent into BF16's field gives |v| * 2^-112, a BF16 normal;
-// one BF16 multiply by 2^112 restores v with no rounding.  NaN codes become
-// NaN.
+// one BF16 multiply by 2^112 restores v with no rounding.  (NaN codes are not
+// valid weights; they decode to an unspecified value.)
 __device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint16_t codes) {
     uint32_t f;
     asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(f) : "h"(codes));

@@ -4,28 +4,37 @@
 // The computation of the FP8 W8A16 MoE decode kernel
 // (dstair/gated-deltanet-nki-trainium, "FP8 MoE decode kernel"): gate/up GEMM
 // -> SwiGLU -> down GEMM -> affinity scale, with E4M3FN weights and one fp32
-// scale per 128x128 block decoded to BF16 tile by tile; the row order is the
-// expert-sorted order of the Nemotron-H sorted path, read from device-side
-// offsets (no host sync).
+// scale per 128x128 block decoded tile by tile into 16-bit MMA operands; the
+// row order is the expert-sorted order of the Nemotron-H sorted path, read from
+// device-side offsets (no host sync).
 //
 // Design (B200):
-//  * One CTA owns a slice of ONE expert's weights: 32 intermediate features
-//    (gate and up rows) in the gate/up kernel, 64 output features in the down
-//    kernel.  CTAs whose expert received no route exit at once, so only the
-//    touched experts' weights are read, each exactly once per token group.
-//  * A producer warp streams the slice from HBM with TMA in stages of 128
-//    reduction columns (one scale block), 128-byte swizzled, through a
-//    6-deep shared-memory ring (mbarrier full/empty pairs, bounded waits).
-//  * Eight consumer warps load the FP8 bytes with ldmatrix, decode them to
-//    BF16 in registers (exact), and run mma.sync m16n8k16 against the
-//    expert's token rows staged in shared memory.  The reduction columns are
-//    permuted identically on both operands so that one ldmatrix register (4
-//    codes of one row) feeds one A-fragment pair.  Each 128-wide fp32 partial
-//    sum is multiplied by its block scale.
+//  * One CTA owns a slice of ONE expert's weights: 64 intermediate features
+//    (their gate and up rows) in the gate/up kernel, 128 output features in the
+//    down kernel.  CTAs whose expert received no route exit at once, so only
+//    the touched experts' weights are read, once per token group.
+//  * A producer warp streams the slice from HBM with TMA (evict-first L2
+//    policy) in 16 KB stages of 128 reduction columns (one scale block),
+//    128-byte swizzled, through a 4-deep shared-memory ring (mbarrier
+//    full/empty pairs with bounded waits).
+//  * Eight consumer warps each own 16 MMA rows.  They read the FP8 bytes with
+//    ldmatrix (conflict-free on the swizzled tile) and convert them with the
+//    one-instruction E4M3x2 -> f16x2 conversion, which is exact: the decoded
+//    weight is the E4M3 value itself.  Its 128x128 block scale multiplies each
+//    128-column fp32 partial sum.  mma.sync m16n8k16 (f16 x f16 -> fp32) runs
+//    against the expert's token rows staged in shared memory.  The reduction
+//    columns are permuted identically on both operands so that one ldmatrix
+//    register (4 codes of one row) feeds one A-fragment pair.
+//  * Activations reach the MMA as f16: each bf16 row is multiplied by a power
+//    of two 2^k that puts its largest magnitude in [2^14, 2^15), which makes
+//    the bf16 -> f16 conversion exact (f16 holds 11 significant bits to bf16's
+//    8); the epilogue multiplies by 2^-k in fp32.
 //  * In the gate/up tile the 16 MMA rows are 8 gate + 8 up rows of the same
-//    features, so SwiGLU is thread-local in the epilogue.
-//  * Two warps share each 16-row tile, each taking half of every stage's
-//    columns; their sums meet in shared memory for a coalesced epilogue.
+//    features, so SwiGLU is thread-local in the epilogue; outputs go through a
+//    shared-memory tile to coalesced 16-byte stores.
+//  * The down kernel is a programmatic dependent launch: its producer starts
+//    streaming weights while the gate/up grid drains, and its consumers wait
+//    (griddepcontrol.wait) before reading h.
 #include <algorithm>
 
 #include "device_common.cuh"
@@ -35,14 +44,15 @@ namespace moe {
 
 namespace {
 
-constexpr int kStages = 6;
+constexpr int kStages = 4;
 constexpr int kConsumerWarps = 8;
-constexpr int kThreads = (kConsumerWarps + 1) * 32;
-constexpr int kStageBytes = 8192;  // 64 rows x 128 bytes
-constexpr int kGateUpRows = 32;    // intermediate features per gate/up CTA
-constexpr int kDownRows = 64;      // output features per down CTA
-constexpr int kRedGU = 36;         // padded token stride (floats) of the gate/up reduction tile
-constexpr int kRedDn = 68;         // same for the down tile
+constexpr int kConsumers = kConsumerWarps * 32;
+constexpr int kThreads = kConsumers + 32;
+constexpr int kStageBytes = 16384;  // 128 rows x 128 bytes
+constexpr int kGateUpFeat = 64;     // intermediate features per gate/up CTA (8 per warp)
+constexpr int kDownRows = 128;      // output features per down CTA (16 per warp)
+constexpr int kGuTile = kGateUpFeat + 8;  // bf16 stride of the gate/up output tile
+constexpr int kDnTile = kDownRows + 8;    // bf16 stride of the down output tile
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
     return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
@@ -54,15 +64,15 @@ __device__ __forceinline__ uint2 lds64(uint32_t addr) {
     return v;
 }
 
-__device__ __forceinline__ uint4 ldg_nc_v4(const void* p) {
+__device__ __forceinline__ uint4 ldg_v4(const void* p) {
     uint4 v;
-    asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
+    asm volatile("ld.global.v4.u32 {%0,%1,%2,%3}, [%4];"
                  : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                  : "l"(p));
     return v;
 }
 
-// Row range [p0, p0 + n) of expert e.  Returns false (BAD_MAP) for corrupt offsets.
+// Row range [p0, p0 + n) of expert e.  Returns false for corrupt offsets.
 __device__ __forceinline__ bool expert_rows(const FfnArgs& a, int e, long& p0, long& n) {
     if (a.identity) {
         p0 = 0;
@@ -77,61 +87,163 @@ __device__ __forceinline__ bool expert_rows(const FfnArgs& a, int e, long& p0, l
     return true;
 }
 
-// Token of sorted row p, -1 if the route map entry is out of range.
-__device__ __forceinline__ int row_token(const FfnArgs& a, long p) {
-    if (a.identity) return static_cast<int>(p);
-    const int r = a.sorted_route[p];
-    const long R = static_cast<long>(a.T) * a.K;
-    if (r < 0 || r >= R) return -1;
-    return r / a.K;
-}
-
 // Producer: stream `total` stages (cycling the slice's KB column blocks) into the ring.
 __device__ __forceinline__ void produce(const CUtensorMap* m0, const CUtensorMap* m1, int row,
                                         int KB, long total, uint8_t* ring, uint64_t* full,
-                                        uint64_t* empty, uint32_t bytes_each, volatile int* abort_flag,
-                                        int32_t* status) {
+                                        uint64_t* empty, volatile int* abort_flag, int32_t* status) {
     tma_prefetch_desc(m0);
     if (m1) tma_prefetch_desc(m1);
+    const uint64_t policy = l2_evict_first_policy();
     for (long it = 0; it < total; ++it) {
         const int s = static_cast<int>(it % kStages);
         if (it >= kStages &&
             !mbar_wait_or_abort(&empty[s], static_cast<uint32_t>((it / kStages - 1) & 1), abort_flag, status))
             return;
-        mbar_arrive_expect_tx(&full[s], m1 ? 2 * bytes_each : bytes_each);
+        mbar_arrive_expect_tx(&full[s], kStageBytes);
         const int kb = static_cast<int>(it % KB);
         uint8_t* dst = ring + static_cast<size_t>(s) * kStageBytes;
-        tma_load_2d(dst, m0, &full[s], kb * 128, row);
-        if (m1) tma_load_2d(dst + bytes_each, m1, &full[s], kb * 128, row);
+        if (m1) {
+            tma_load_2d_hint(dst, m0, &full[s], kb * 128, row, policy);
+            tma_load_2d_hint(dst + kStageBytes / 2, m1, &full[s], kb * 128, row, policy);
+        } else {
+            tma_load_2d_hint(dst, m0, &full[s], kb * 128, row, policy);
+        }
     }
 }
 
-// One stage of one warp: 16 rows (two 8-row halves r_lo / r_hi from the
-// ldmatrix register pairs) x 64 columns (chunks j0..j0+3) against NT token tiles.
-template <int NT>
-__device__ __forceinline__ void stage_mma(uint32_t stage_base, uint32_t lm_off0, uint32_t lm_off1,
-                                          uint32_t b_base, int xstride, int b_col_bytes,
-                                          float (&part)[NT][4]) {
-#pragma unroll
-    for (int q = 0; q < 2; ++q) {
-        uint32_t r0, r1, r2, r3;
-        ldmatrix_x4(stage_base + (q ? lm_off1 : lm_off0), r0, r1, r2, r3);
-        uint32_t lo0, hi0, lo1, hi1;
-        e4m3x4_to_bf16(r0, lo0, hi0);
-        e4m3x4_to_bf16(r1, lo1, hi1);
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-            const uint2 b = lds64(b_base + nt * 8 * xstride + b_col_bytes + (2 * q) * 32);
-            mma_bf16_16816(part[nt], lo0, lo1, hi0, hi1, b.x, b.y);
+// Largest |x| bit pattern (sign cleared) among the 8 bf16 of a 16-byte vector.
+__device__ __forceinline__ uint32_t absmax_bf16x8(const uint4& v) {
+    uint32_t m = __vmaxu2(__vmaxu2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu),
+                          __vmaxu2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu));
+    return max(m & 0xFFFFu, m >> 16);
+}
+
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2_scaled(uint32_t w, float up) {
+    const float a = __uint_as_float(w << 16) * up;
+    const float b = __uint_as_float(w & 0xFFFF0000u) * up;
+    __half2 h = __floats2half2_rn(a, b);
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// Stage NG rows of W bf16 values into shared memory (row stride `stride`
+// bytes) as f16 times 2^k, k chosen per row so that its largest magnitude
+// lies in [2^14, 2^15); inv_scale[q] = 2^-k.  row_ptr(q) gives the source row
+// or nullptr for a padding row (zeros).  Warp w handles rows w, w + 8, ...
+template <int NG, class RowPtr>
+__device__ __forceinline__ void stage_rows_f16(RowPtr row_ptr, int W, uint8_t* dst, int stride,
+                                               float* inv_scale) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int vpr = W / 8;
+    for (int q = warp; q < NG; q += kConsumerWarps) {
+        const uint16_t* src = row_ptr(q);
+        uint8_t* d = dst + q * stride;
+        uint32_t amax = 0;
+        for (int v = lane; v < vpr; v += 32) {
+            const uint4 val = src ? ldg_v4(src + v * 8) : make_uint4(0, 0, 0, 0);
+            *reinterpret_cast<uint4*>(d + v * 16) = val;
+            amax = max(amax, absmax_bf16x8(val));
         }
-        e4m3x4_to_bf16(r2, lo0, hi0);
-        e4m3x4_to_bf16(r3, lo1, hi1);
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-            const uint2 b = lds64(b_base + nt * 8 * xstride + b_col_bytes + (2 * q + 1) * 32);
-            mma_bf16_16816(part[nt], lo0, lo1, hi0, hi1, b.x, b.y);
+        amax = __reduce_max_sync(0xffffffffu, amax);
+        // |x|max = 2^e * m with e = (bits >> 7) - 127; k = 14 - e, at most 64.
+        const int k = amax ? min(64, 14 - (static_cast<int>(amax >> 7) - 127)) : 0;
+        const float up = __uint_as_float(static_cast<uint32_t>(k + 127) << 23);
+        if (lane == 0) inv_scale[q] = __uint_as_float(static_cast<uint32_t>(127 - k) << 23);
+        __syncwarp();
+        for (int v = lane; v < vpr; v += 32) {
+            uint4 val = *reinterpret_cast<const uint4*>(d + v * 16);
+            val.x = bf16x2_to_f16x2_scaled(val.x, up);
+            val.y = bf16x2_to_f16x2_scaled(val.y, up);
+            val.z = bf16x2_to_f16x2_scaled(val.z, up);
+            val.w = bf16x2_to_f16x2_scaled(val.w, up);
+            *reinterpret_cast<uint4*>(d + v * 16) = val;
         }
     }
+}
+
+// One 128-column stage of one warp: 16 rows x 128 columns against NT token
+// tiles.  This lane's ldmatrix row is `row` of sub-tile tile0 (chunk_sel bit 1
+// clear) or tile1 (set), in chunk j (bit 0 clear) or j+1 (set) of each chunk
+// pair; b_addr is this lane's B address for chunk 0 of the stage.
+template <int NT>
+__device__ __forceinline__ void stage_mma(uint32_t tile0, uint32_t tile1, uint32_t row,
+                                          uint32_t chunk_sel, uint32_t b_addr, int xstride,
+                                          float (&part)[NT][4]) {
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+        const uint32_t chunk = 2 * p + (chunk_sel & 1);
+        uint32_t r0, r1, r2, r3;
+        ldmatrix_x4((chunk_sel & 2 ? tile1 : tile0) + sw128_offset(row, chunk & 7), r0, r1, r2, r3);
+        uint32_t lo0, hi0, lo1, hi1;
+        e4m3x4_to_f16(r0, lo0, hi0);
+        e4m3x4_to_f16(r1, lo1, hi1);
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            const uint2 b = lds64(b_addr + nt * 8 * xstride + (2 * p) * 32);
+            mma_f16_16816(part[nt], lo0, lo1, hi0, hi1, b.x, b.y);
+        }
+        e4m3x4_to_f16(r2, lo0, hi0);
+        e4m3x4_to_f16(r3, lo1, hi1);
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            const uint2 b = lds64(b_addr + nt * 8 * xstride + (2 * p + 1) * 32);
+            mma_f16_16816(part[nt], lo0, lo1, hi0, hi1, b.x, b.y);
+        }
+    }
+}
+
+template <int NT>
+__device__ __forceinline__ void zero_acc(float (&a)[NT][4]) {
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) a[nt][0] = a[nt][1] = a[nt][2] = a[nt][3] = 0.f;
+}
+
+// Shared-memory carve-up common to both kernels.
+struct Smem {
+    uint8_t* ring;
+    uint8_t* rows;    // staged activation rows (f16)
+    uint16_t* otile;  // output tile (bf16)
+    int* tok;
+    float* wr;
+    float* inv;
+    uint64_t* full;
+    uint64_t* empty;
+    volatile int* abort_flag;
+};
+
+__host__ __device__ constexpr size_t smem_bytes(int NG, int row_stride, int otile_stride) {
+    return 1024 + static_cast<size_t>(kStages) * kStageBytes + static_cast<size_t>(NG) * row_stride +
+           static_cast<size_t>(NG) * otile_stride * 2 + 3 * NG * 4 + 2 * kStages * 8 + 16;
+}
+
+__device__ __forceinline__ Smem carve(uint8_t* raw, int NG, int row_stride, int otile_stride) {
+    Smem s;
+    uint8_t* p = align1024(raw);
+    s.ring = p;
+    p += kStages * kStageBytes;
+    s.rows = p;
+    p += NG * row_stride;
+    s.otile = reinterpret_cast<uint16_t*>(p);
+    p += NG * otile_stride * 2;
+    s.tok = reinterpret_cast<int*>(p);
+    s.wr = reinterpret_cast<float*>(s.tok + NG);
+    s.inv = s.wr + NG;
+    p = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(s.inv + NG) + 7) & ~uintptr_t(7));
+    s.full = reinterpret_cast<uint64_t*>(p);
+    s.empty = s.full + kStages;
+    s.abort_flag = reinterpret_cast<volatile int*>(s.empty + kStages);
+    return s;
+}
+
+__device__ __forceinline__ void init_barriers(const Smem& s) {
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kStages; ++i) {
+            mbar_init(&s.full[i], 1);
+            mbar_init(&s.empty[i], kConsumerWarps);
+        }
+        *s.abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
 }
 
 // ------------------------------------------------------------------ gate/up + SwiGLU
@@ -141,11 +253,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     gateup_decode_kernel(const __grid_constant__ CUtensorMap tm_gate,
                          const __grid_constant__ CUtensorMap tm_up, const FfnArgs a) {
     constexpr int NG = 8 * NT;  // tokens per group
+    if (threadIdx.x == 0) grid_dependency_launch();  // the down kernel may start streaming
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = align1024(smem_raw);
     const int e = blockIdx.y;
     const int H = a.H, I = a.ex.inter;
-    const int i0 = blockIdx.x * kGateUpRows;
+    const int i0 = blockIdx.x * kGateUpFeat;
     long p0, n;
     if (!expert_rows(a, e, p0, n)) {
         if (threadIdx.x == 0) report_status(a.status, MOE_STATUS_BAD_MAP);
@@ -155,44 +267,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int KB = H / 128;
     const int groups = static_cast<int>((n + NG - 1) / NG);
     const int xstride = 2 * H + 32;
-
-    uint8_t* ring = smem;
-    uint8_t* xs = ring + kStages * kStageBytes;
-    float* red = reinterpret_cast<float*>(xs + NG * xstride);  // [2 halves][gate, up][NG][kRedGU]
-    int* tok = reinterpret_cast<int*>(red + 4 * NG * kRedGU);
-    uint64_t* full = reinterpret_cast<uint64_t*>(tok + NG + (NG & 1));
-    uint64_t* empty = full + kStages;
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + kStages);
+    const Smem s = carve(smem_raw, NG, xstride, kGuTile);
+    init_barriers(s);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], kConsumerWarps);
-        }
-        *abort_flag = 0;
-        fence_mbar_init();
-    }
-    __syncthreads();
-
     if (warp == kConsumerWarps) {
         if (lane == 0)
-            produce(&tm_gate, &tm_up, e * I + i0, KB, static_cast<long>(groups) * KB, ring, full,
-                    empty, kStageBytes / 2, abort_flag, a.status);
+            produce(&tm_gate, &tm_up, e * I + i0, KB, static_cast<long>(groups) * KB, s.ring, s.full,
+                    s.empty, s.abort_flag, a.status);
         return;
     }
 
-    const int u = warp & 3, hh = warp >> 2;  // 16-row tile (8 gate + 8 up), column half
     const int g = lane >> 2, c = lane & 3;
     const int mi = lane >> 3, rr = lane & 7;
-    const uint32_t lm_tile = (mi & 1) ? kStageBytes / 2 : 0;  // gate / up sub-tile
-    const uint32_t lm_off0 = lm_tile + sw128_offset(8 * u + rr, 4 * hh + (mi >> 1));
-    const uint32_t lm_off1 = lm_tile + sw128_offset(8 * u + rr, 4 * hh + 2 + (mi >> 1));
-    const uint32_t ring_u32 = smem_u32(ring);
-    const uint32_t b_base = smem_u32(xs) + g * xstride + 4 * c * 2 + 4 * hh * 32;
+    // ldmatrix: matrices 0/2 read gate rows 8w+rr, 1/3 the up rows; 0/1 chunk j, 2/3 chunk j+1.
+    const uint32_t lm_row = 8 * warp + rr;
+    const uint32_t chunk_sel = (mi >> 1) | ((mi & 1) << 1);  // bit 0: chunk j+1, bit 1: up tile
+    const uint32_t ring_u32 = smem_u32(s.ring);
+    const uint32_t b_lane = smem_u32(s.rows) + g * xstride + 8 * c;
     const size_t sblk = (static_cast<size_t>(e) * (I / 128) + i0 / 128) * KB;
     const float* sg = a.ex.s_gate + sblk;
     const float* su = a.ex.s_up + sblk;
+    const long R = static_cast<long>(a.T) * a.K;
 
     long it = 0;
     for (int grp = 0; grp < groups; ++grp) {
@@ -201,34 +297,41 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (threadIdx.x < NG) {
             int t = -1;
             if (static_cast<int>(threadIdx.x) < gn) {
-                t = row_token(a, gp0 + threadIdx.x);
-                if (t < 0) report_status(a.status, MOE_STATUS_BAD_MAP);
+                if (a.identity) {
+                    t = static_cast<int>(gp0 + threadIdx.x);
+                } else {
+                    const int r = a.sorted_route[gp0 + threadIdx.x];
+                    if (r >= 0 && r < R)
+                        t = r / a.K;
+                    else
+                        report_status(a.status, MOE_STATUS_BAD_MAP);
+                }
             }
-            tok[threadIdx.x] = t;
+            s.tok[threadIdx.x] = t;
         }
-        named_barrier_sync(1, kConsumerWarps * 32);
-        const int vpr = H / 8;  // 16-byte vectors per row
-        for (int v = threadIdx.x; v < NG * vpr; v += kConsumerWarps * 32) {
-            const int q = v / vpr, col = v - q * vpr;
-            const int t = tok[q];
-            uint4 val = make_uint4(0, 0, 0, 0);
-            if (t >= 0) val = ldg_nc_v4(a.x + static_cast<size_t>(t) * H + col * 8);
-            *reinterpret_cast<uint4*>(xs + q * xstride + col * 16) = val;
-        }
-        named_barrier_sync(1, kConsumerWarps * 32);
+        named_barrier_sync(1, kConsumers);
+        stage_rows_f16<NG>(
+            [&](int q) -> const uint16_t* {
+                const int t = s.tok[q];
+                return t >= 0 ? a.x + static_cast<size_t>(t) * H : nullptr;
+            },
+            H, s.rows, xstride, s.inv);
+        named_barrier_sync(1, kConsumers);
 
         float acc[NT][4];
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+        zero_acc<NT>(acc);
         for (int kb = 0; kb < KB; ++kb, ++it) {
-            const int s = static_cast<int>(it % kStages);
+            const int st = static_cast<int>(it % kStages);
             float part[NT][4];
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) part[nt][0] = part[nt][1] = part[nt][2] = part[nt][3] = 0.f;
-            if (mbar_wait_or_abort(&full[s], static_cast<uint32_t>((it / kStages) & 1), abort_flag, a.status)) {
-                stage_mma<NT>(ring_u32 + s * kStageBytes, lm_off0, lm_off1, b_base, xstride, kb * 256, part);
+            zero_acc<NT>(part);
+            if (mbar_wait_or_abort(&s.full[st], static_cast<uint32_t>((it / kStages) & 1), s.abort_flag,
+                                   a.status)) {
+                const uint32_t tile = ring_u32 + st * kStageBytes;
+                // chunk_sel bit 1 selects the up sub-tile (second half of the stage).
+                stage_mma<NT>(tile, tile + kStageBytes / 2, lm_row, chunk_sel, b_lane + kb * 256, xstride,
+                              part);
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&empty[s]);
+                if (lane == 0) mbar_arrive(&s.empty[st]);
             }
             const float gs = __ldg(sg + kb), us = __ldg(su + kb);
 #pragma unroll
@@ -239,39 +342,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                 acc[nt][3] = fmaf(part[nt][3], us, acc[nt][3]);
             }
         }
-        // Partial sums of this column half -> shared memory.
-        float* rg = red + (hh * 2 + 0) * NG * kRedGU;
-        float* ru = red + (hh * 2 + 1) * NG * kRedGU;
-        const int il = 8 * u + g;
+        // SwiGLU on the true sums (undo the activation scale first).
+        const int il = 8 * warp + g;
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
             const int t0 = nt * 8 + 2 * c;
-            rg[t0 * kRedGU + il] = acc[nt][0];
-            rg[(t0 + 1) * kRedGU + il] = acc[nt][1];
-            ru[t0 * kRedGU + il] = acc[nt][2];
-            ru[(t0 + 1) * kRedGU + il] = acc[nt][3];
+            const float s0 = s.inv[t0], s1 = s.inv[t0 + 1];
+            const float h0 = silu_f32(acc[nt][0] * s0) * (acc[nt][2] * s0);
+            const float h1 = silu_f32(acc[nt][1] * s1) * (acc[nt][3] * s1);
+            s.otile[t0 * kGuTile + il] = __bfloat16_as_ushort(__float2bfloat16_rn(h0));
+            s.otile[(t0 + 1) * kGuTile + il] = __bfloat16_as_ushort(__float2bfloat16_rn(h1));
         }
-        named_barrier_sync(1, kConsumerWarps * 32);
-        // SwiGLU and a coalesced bf16 store of h[row, i0 .. i0+31].
-        for (int v = threadIdx.x; v < NG * 4; v += kConsumerWarps * 32) {
-            const int q = v >> 2, ch = v & 3;
-            if (q < gn && tok[q] >= 0) {
-                const float* g0 = red + (0 * NG + q) * kRedGU + ch * 8;
-                const float* u0 = red + (1 * NG + q) * kRedGU + ch * 8;
-                const float* g1 = red + (2 * NG + q) * kRedGU + ch * 8;
-                const float* u1 = red + (3 * NG + q) * kRedGU + ch * 8;
-                uint32_t pk[4];
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const float ga = g0[2 * k] + g1[2 * k], gb = g0[2 * k + 1] + g1[2 * k + 1];
-                    const float ua = u0[2 * k] + u1[2 * k], ub = u0[2 * k + 1] + u1[2 * k + 1];
-                    pk[k] = pack_bf16x2(silu_f32(ga) * ua, silu_f32(gb) * ub);
-                }
+        named_barrier_sync(1, kConsumers);
+        for (int v = threadIdx.x; v < NG * (kGateUpFeat / 8); v += kConsumers) {
+            const int q = v / (kGateUpFeat / 8), ch = v % (kGateUpFeat / 8);
+            if (q < gn && s.tok[q] >= 0)
                 *reinterpret_cast<uint4*>(a.h + static_cast<size_t>(gp0 + q) * I + i0 + ch * 8) =
-                    make_uint4(pk[0], pk[1], pk[2], pk[3]);
-            }
+                    *reinterpret_cast<const uint4*>(s.otile + q * kGuTile + ch * 8);
         }
-        named_barrier_sync(1, kConsumerWarps * 32);
+        named_barrier_sync(1, kConsumers);
     }
 }
 
@@ -282,10 +371,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     down_decode_kernel(const __grid_constant__ CUtensorMap tm_down, const FfnArgs a) {
     constexpr int NG = 8 * NT;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = align1024(smem_raw);
     const int e = blockIdx.y;
     const int H = a.H, I = a.ex.inter;
     const int n0 = blockIdx.x * kDownRows;
+    // Offsets come from the sort, which finished before the gate/up grid began.
     long p0, n;
     if (!expert_rows(a, e, p0, n)) {
         if (threadIdx.x == 0) report_status(a.status, MOE_STATUS_BAD_MAP);
@@ -295,43 +384,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int KB = I / 128;
     const int groups = static_cast<int>((n + NG - 1) / NG);
     const int hstride = 2 * I + 32;
-
-    uint8_t* ring = smem;
-    uint8_t* hs = ring + kStages * kStageBytes;
-    float* red = reinterpret_cast<float*>(hs + NG * hstride);  // [2 halves][NG][kRedDn]
-    float* wr = red + 2 * NG * kRedDn;                         // [NG] route weights
-    int* tok = reinterpret_cast<int*>(wr + NG);
-    uint64_t* full = reinterpret_cast<uint64_t*>(tok + NG + (NG & 1));
-    uint64_t* empty = full + kStages;
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + kStages);
+    const Smem s = carve(smem_raw, NG, hstride, kDnTile);
+    init_barriers(s);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], kConsumerWarps);
-        }
-        *abort_flag = 0;
-        fence_mbar_init();
-    }
-    __syncthreads();
-
     if (warp == kConsumerWarps) {
         if (lane == 0)
-            produce(&tm_down, nullptr, e * H + n0, KB, static_cast<long>(groups) * KB, ring, full,
-                    empty, kStageBytes, abort_flag, a.status);
+            produce(&tm_down, nullptr, e * H + n0, KB, static_cast<long>(groups) * KB, s.ring, s.full,
+                    s.empty, s.abort_flag, a.status);
         return;
     }
+    grid_dependency_wait();  // h is written by the gate/up grid
 
-    const int mt = warp & 3, hh = warp >> 2;
     const int g = lane >> 2, c = lane & 3;
     const int mi = lane >> 3, rr = lane & 7;
-    const int lm_row = 16 * mt + ((mi & 1) ? 8 : 0) + rr;
-    const uint32_t lm_off0 = sw128_offset(lm_row, 4 * hh + (mi >> 1));
-    const uint32_t lm_off1 = sw128_offset(lm_row, 4 * hh + 2 + (mi >> 1));
-    const uint32_t ring_u32 = smem_u32(ring);
-    const uint32_t b_base = smem_u32(hs) + g * hstride + 4 * c * 2 + 4 * hh * 32;
+    // ldmatrix: matrices 0/2 rows 16w+rr, 1/3 rows 16w+8+rr; 0/1 chunk j, 2/3 chunk j+1.
+    const uint32_t lm_row = 16 * warp + ((mi & 1) << 3) + rr;
+    const uint32_t chunk_sel = mi >> 1;
+    const uint32_t ring_u32 = smem_u32(s.ring);
+    const uint32_t b_lane = smem_u32(s.rows) + g * hstride + 8 * c;
     const float* sd = a.ex.s_down + (static_cast<size_t>(e) * (H / 128) + n0 / 128) * KB;
+    const long R = static_cast<long>(a.T) * a.K;
 
     long it = 0;
     for (int grp = 0; grp < groups; ++grp) {
@@ -347,7 +420,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     wv = 1.f;
                 } else {
                     const int r = a.sorted_route[p];
-                    if (r >= 0 && r < static_cast<long>(a.T) * a.K) {
+                    if (r >= 0 && r < R) {
                         t = r / a.K;
                         wv = a.topk_w[r];
                     } else {
@@ -355,31 +428,29 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
             }
-            tok[threadIdx.x] = t;
-            wr[threadIdx.x] = wv;
+            s.tok[threadIdx.x] = t;
+            s.wr[threadIdx.x] = wv;
         }
-        // h rows of this group are contiguous: rows gp0 .. gp0 + gn - 1.
-        const int vpr = I / 8;
-        for (int v = threadIdx.x; v < NG * vpr; v += kConsumerWarps * 32) {
-            const int q = v / vpr, col = v - q * vpr;
-            uint4 val = make_uint4(0, 0, 0, 0);
-            if (q < gn) val = *reinterpret_cast<const uint4*>(a.h + static_cast<size_t>(gp0 + q) * I + col * 8);
-            *reinterpret_cast<uint4*>(hs + q * hstride + col * 16) = val;
-        }
-        named_barrier_sync(1, kConsumerWarps * 32);
+        named_barrier_sync(1, kConsumers);
+        stage_rows_f16<NG>(
+            [&](int q) -> const uint16_t* {
+                return (q < gn && s.tok[q] >= 0) ? a.h + static_cast<size_t>(gp0 + q) * I : nullptr;
+            },
+            I, s.rows, hstride, s.inv);
+        named_barrier_sync(1, kConsumers);
 
         float acc[NT][4];
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+        zero_acc<NT>(acc);
         for (int kb = 0; kb < KB; ++kb, ++it) {
-            const int s = static_cast<int>(it % kStages);
+            const int st = static_cast<int>(it % kStages);
             float part[NT][4];
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) part[nt][0] = part[nt][1] = part[nt][2] = part[nt][3] = 0.f;
-            if (mbar_wait_or_abort(&full[s], static_cast<uint32_t>((it / kStages) & 1), abort_flag, a.status)) {
-                stage_mma<NT>(ring_u32 + s * kStageBytes, lm_off0, lm_off1, b_base, hstride, kb * 256, part);
+            zero_acc<NT>(part);
+            if (mbar_wait_or_abort(&s.full[st], static_cast<uint32_t>((it / kStages) & 1), s.abort_flag,
+                                   a.status)) {
+                const uint32_t tile = ring_u32 + st * kStageBytes;
+                stage_mma<NT>(tile, tile, lm_row, chunk_sel, b_lane + kb * 256, hstride, part);
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&empty[s]);
+                if (lane == 0) mbar_arrive(&s.empty[st]);
             }
             const float ds = __ldg(sd + kb);
 #pragma unroll
@@ -387,48 +458,29 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int k = 0; k < 4; ++k) acc[nt][k] = fmaf(part[nt][k], ds, acc[nt][k]);
         }
-        float* rh = red + hh * NG * kRedDn;
-        const int rl = 16 * mt + g;
+        const int rl = 16 * warp + g;
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
             const int t0 = nt * 8 + 2 * c;
-            rh[t0 * kRedDn + rl] = acc[nt][0];
-            rh[(t0 + 1) * kRedDn + rl] = acc[nt][1];
-            rh[t0 * kRedDn + rl + 8] = acc[nt][2];
-            rh[(t0 + 1) * kRedDn + rl + 8] = acc[nt][3];
+            const float f0 = s.inv[t0] * s.wr[t0], f1 = s.inv[t0 + 1] * s.wr[t0 + 1];
+            s.otile[t0 * kDnTile + rl] = __bfloat16_as_ushort(__float2bfloat16_rn(acc[nt][0] * f0));
+            s.otile[(t0 + 1) * kDnTile + rl] = __bfloat16_as_ushort(__float2bfloat16_rn(acc[nt][1] * f1));
+            s.otile[t0 * kDnTile + rl + 8] = __bfloat16_as_ushort(__float2bfloat16_rn(acc[nt][2] * f0));
+            s.otile[(t0 + 1) * kDnTile + rl + 8] = __bfloat16_as_ushort(__float2bfloat16_rn(acc[nt][3] * f1));
         }
-        named_barrier_sync(1, kConsumerWarps * 32);
-        // y[row, n0 .. n0+63] = bf16(w * (sum of both halves)), 16-byte stores.
-        for (int v = threadIdx.x; v < NG * 8; v += kConsumerWarps * 32) {
-            const int q = v >> 3, ch = v & 7;
-            if (q < gn && tok[q] >= 0) {
-                const float* y0 = red + q * kRedDn + ch * 8;
-                const float* y1 = red + (NG + q) * kRedDn + ch * 8;
-                const float wv = wr[q];
-                uint32_t pk[4];
-#pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    pk[k] = pack_bf16x2(wv * (y0[2 * k] + y1[2 * k]), wv * (y0[2 * k + 1] + y1[2 * k + 1]));
+        named_barrier_sync(1, kConsumers);
+        for (int v = threadIdx.x; v < NG * (kDownRows / 8); v += kConsumers) {
+            const int q = v / (kDownRows / 8), ch = v % (kDownRows / 8);
+            if (q < gn && s.tok[q] >= 0)
                 *reinterpret_cast<uint4*>(a.y + static_cast<size_t>(gp0 + q) * H + n0 + ch * 8) =
-                    make_uint4(pk[0], pk[1], pk[2], pk[3]);
-            }
+                    *reinterpret_cast<const uint4*>(s.otile + q * kDnTile + ch * 8);
         }
-        named_barrier_sync(1, kConsumerWarps * 32);
+        named_barrier_sync(1, kConsumers);
     }
 }
 
-size_t gateup_smem(int NT, int H) {
-    const int NG = 8 * NT;
-    return 1024 + kStages * kStageBytes + static_cast<size_t>(NG) * (2 * H + 32) +
-           4 * NG * kRedGU * sizeof(float) + (NG + 2) * sizeof(int) + 2 * kStages * sizeof(uint64_t) + 16;
-}
-
-size_t down_smem(int NT, int I) {
-    const int NG = 8 * NT;
-    return 1024 + kStages * kStageBytes + static_cast<size_t>(NG) * (2 * I + 32) +
-           2 * NG * kRedDn * sizeof(float) + NG * sizeof(float) + (NG + 2) * sizeof(int) +
-           2 * kStages * sizeof(uint64_t) + 16;
-}
+size_t gateup_smem(int NT, int H) { return smem_bytes(8 * NT, 2 * H + 32, kGuTile); }
+size_t down_smem(int NT, int I) { return smem_bytes(8 * NT, 2 * I + 32, kDnTile); }
 
 constexpr size_t kSmemLimit = 227 * 1024;
 
@@ -443,24 +495,35 @@ cudaError_t launch_nt(const FfnArgs& a, const CUtensorMap& tg, const CUtensorMap
                                static_cast<int>(s2));
     if (err != cudaSuccess) return err;
     const int E = a.ex.n;
-    gateup_decode_kernel<NT><<<dim3(a.ex.inter / kGateUpRows, E), kThreads, s1, stream>>>(tg, tu, a);
+    gateup_decode_kernel<NT><<<dim3(a.ex.inter / kGateUpFeat, E), kThreads, s1, stream>>>(tg, tu, a);
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
-    down_decode_kernel<NT><<<dim3(a.H / kDownRows, E), kThreads, s2, stream>>>(td, a);
-    return cudaGetLastError();
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(a.H / kDownRows, E);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = s2;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, down_decode_kernel<NT>, td, a);
 }
 
 }  // namespace
 
 bool ffn_decode_supported(int H, int I) {
-    return gateup_smem(1, H) <= kSmemLimit && down_smem(1, I) <= kSmemLimit;
+    return H % kDownRows == 0 && I % kGateUpFeat == 0 && gateup_smem(1, H) <= kSmemLimit &&
+           down_smem(1, I) <= kSmemLimit;
 }
 
 cudaError_t launch_ffn_decode(const FfnArgs& a, cudaStream_t stream) {
     CUtensorMap tg, tu, td;
     const uint64_t E = static_cast<uint64_t>(a.ex.n), I = a.ex.inter, H = a.H;
-    cudaError_t err = make_tmap_u8_2d(&tg, a.ex.w_gate, E * I, H, 128, kGateUpRows);
-    if (err == cudaSuccess) err = make_tmap_u8_2d(&tu, a.ex.w_up, E * I, H, 128, kGateUpRows);
+    cudaError_t err = make_tmap_u8_2d(&tg, a.ex.w_gate, E * I, H, 128, kGateUpFeat);
+    if (err == cudaSuccess) err = make_tmap_u8_2d(&tu, a.ex.w_up, E * I, H, 128, kGateUpFeat);
     if (err == cudaSuccess) err = make_tmap_u8_2d(&td, a.ex.w_down, E * H, I, 128, kDownRows);
     if (err != cudaSuccess) return err;
     // Token tile: the host only knows the average rows per expert.

@@ -50,6 +50,15 @@ int check_topk(int T, int E, int K) {
     return MOE_OK;
 }
 
+// Sizes of the calls after routing: they need no K <= E (any ids sort).
+int check_sizes(int T, int E, int K) {
+    if (T < 0 || T > MOE_MAX_T) return fail(MOE_ERR_INVALID_ARG, "T=%d must be in 0..=%d", T, MOE_MAX_T);
+    if (E < 1 || E > MOE_MAX_E)
+        return fail(MOE_ERR_UNSUPPORTED_SHAPE, "num_experts=%d must be in 1..=%d", E, MOE_MAX_E);
+    if (K < 1 || K > MOE_MAX_K) return fail(MOE_ERR_INVALID_ARG, "top_k=%d must be in 1..=%d", K, MOE_MAX_K);
+    return MOE_OK;
+}
+
 int check_experts(const moe_fp8_experts* ex, int H, const char* which) {
     if (!ex->w_gate || !ex->w_up || !ex->w_down || !ex->s_gate || !ex->s_up || !ex->s_down)
         return fail(MOE_ERR_INVALID_ARG, "%s experts: NULL weight or scale pointer", which);
@@ -99,7 +108,7 @@ int moe_sort(const int32_t* topk_ids, int T, int K, int E, int32_t* expert_offse
              int32_t* sorted_route, int32_t* inv_route, void* workspace, size_t workspace_bytes,
              int32_t* status, moe_stream_t stream) {
     g_err.clear();
-    int rc = check_topk(T, E, K);
+    int rc = check_sizes(T, E, K);
     if (rc) return rc;
     if (!expert_offsets) return fail(MOE_ERR_INVALID_ARG, "moe_sort: expert_offsets must not be NULL");
     if (T > 0 && (!topk_ids || !sorted_route || !inv_route))
@@ -139,7 +148,7 @@ int moe_expert_ffn(const uint16_t* x, int T, int H, int K, const moe_fp8_experts
     g_err.clear();
     if (!routed) return fail(MOE_ERR_INVALID_ARG, "moe_expert_ffn: routed must not be NULL");
     const int E = routed->n_experts, I = routed->inter;
-    int rc = check_topk(T, E, K);
+    int rc = check_sizes(T, E, K);
     if (rc) return rc;
     if (mode != MOE_MODE_AUTO && mode != MOE_MODE_DECODE && mode != MOE_MODE_PREFILL)
         return fail(MOE_ERR_INVALID_ARG, "moe_expert_ffn: mode=%d is not AUTO/DECODE/PREFILL", mode);

@@ -113,7 +113,7 @@ def test_expert_ffn_checks(L):
     assert call(H=200) == moe.MOE_ERR_UNSUPPORTED_SHAPE
     assert call(H=16384) == moe.MOE_ERR_UNSUPPORTED_SHAPE
     assert call(mode=7) == moe.MOE_ERR_INVALID_ARG
-    assert call(K=5) == moe.MOE_ERR_INVALID_ARG
+    assert call(K=33) == moe.MOE_ERR_INVALID_ARG
     assert call(x=P(24)) == moe.MOE_ERR_MISALIGNED
     assert call(wsb=ws - 1) == moe.MOE_ERR_WORKSPACE_TOO_SMALL
     assert call(y=None) == moe.MOE_ERR_INVALID_ARG
