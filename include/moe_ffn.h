@@ -152,6 +152,37 @@ MOE_API int moe_sort(const int32_t* topk_ids, int T, int K, int E, int32_t* expe
              int32_t* sorted_route, int32_t* inv_route, void* workspace,
              size_t workspace_bytes, int32_t* status, moe_stream_t stream);
 
+/* ---------------------------------------------------------------------------
+ * moe_sort_static_ws -- moe_sort for callers that cannot allocate device memory.
+ *
+ * The source paper has no counterpart of this call; it exists for callers that
+ * may not call cudaMalloc or any allocating routine: plugins whose host
+ * framework owns every device allocation, code that runs while a stream is
+ * being captured into a CUDA graph (where allocation is not allowed), and
+ * processes held to a fixed device-memory budget.  It computes exactly what
+ * moe_sort computes (same arguments, same outputs, bit for bit) but takes no
+ * workspace: the scratch its multi-kernel path needs (one int32 counter per
+ * expert per 2048-route chunk) lives in a statically allocated device array of
+ * MOE_SORT_STATIC_WS_BYTES bytes inside the library, which every GPU that
+ * loads the library holds until the process exits.  The call itself allocates
+ * nothing.
+ *  - Sizes whose scratch would exceed the array (E * ceil(T*K / 2048) * 4 >
+ *    MOE_SORT_STATIC_WS_BYTES) are rejected with MOE_ERR_UNSUPPORTED_SHAPE and a
+ *    message naming both byte counts; use moe_sort with a workspace for them.
+ *  - The first call on a device looks up the array's device address (a host
+ *    set-up step, with that device current).  Make that first call before
+ *    capturing a stream into a CUDA graph.
+ *  - Every call shares the one array and leaves its contents behind.  Nothing
+ *    in it needs to start at zero: each call overwrites every counter it reads.
+ *    Calls that overlap on the GPU (on different streams without ordering, or
+ *    from several host threads) race on the array and give undefined results;
+ *    order them on one stream.
+ * ------------------------------------------------------------------------- */
+#define MOE_SORT_STATIC_WS_BYTES (1u << 20)
+MOE_API int moe_sort_static_ws(const int32_t* topk_ids, int T, int K, int E, int32_t* expert_offsets,
+                               int32_t* sorted_route, int32_t* inv_route, int32_t* status,
+                               moe_stream_t stream);
+
 /* Block-scaled FP8 expert weights, expert-major (the caller owns the memory).
  * Rows are output features and the reduction index is contiguous:
  *   w_gate, w_up  [n_experts, inter, H] u8 E4M3FN codes

@@ -31,7 +31,7 @@ MOE_STATUS_BAD_ID, MOE_STATUS_BAD_MAP, MOE_STATUS_TIMEOUT = 1, 2, 4
 MOE_MAX_E, MOE_MAX_K = 1024, 32
 
 EXPORTED = ("moe_last_error", "moe_abi_version", "moe_route", "moe_sort_workspace_bytes", "moe_sort",
-            "moe_ffn_workspace_bytes", "moe_expert_ffn", "moe_combine")
+            "moe_sort_static_ws", "moe_ffn_workspace_bytes", "moe_expert_ffn", "moe_combine")
 
 
 class MoEError(RuntimeError):
@@ -68,6 +68,8 @@ def lib() -> ctypes.CDLL:
             L.moe_sort_workspace_bytes.restype = S
             L.moe_sort.argtypes = [P, I, I, I, P, P, P, P, S, P, P]
             L.moe_sort.restype = I
+            L.moe_sort_static_ws.argtypes = [P, I, I, I, P, P, P, P, P]
+            L.moe_sort_static_ws.restype = I
             L.moe_ffn_workspace_bytes.argtypes = [I, I, I, I, I, I, I]
             L.moe_ffn_workspace_bytes.restype = S
             L.moe_expert_ffn.argtypes = [P, I, I, I, P, P, P, P, P, P, P, I, P, S, P, P]

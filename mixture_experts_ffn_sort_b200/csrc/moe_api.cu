@@ -79,6 +79,15 @@ size_t ffn_h_bytes(long R, int I) { return round256(static_cast<size_t>(R) * I *
 
 }  // namespace
 
+namespace moe {
+// Records an error message for moe_last_error() from another translation unit.
+int api_error(int code, const char* msg) {
+    g_err = msg;
+    return code;
+}
+void api_clear_error() { g_err.clear(); }
+}  // namespace moe
+
 extern "C" {
 
 const char* moe_last_error(void) { return g_err.c_str(); }

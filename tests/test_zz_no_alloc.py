@@ -1,0 +1,57 @@
+"""moe_sort_static_ws: the route sort for callers that cannot allocate.
+
+Some callers may not allocate device memory at all: a plugin whose host
+framework owns every allocation, code running while a stream is captured into
+a CUDA graph, or a process held to a fixed memory budget.  moe_sort_static_ws
+serves them by keeping the sort's scratch in a device array inside the library.
+These tests call it through the C ABI and check that it returns exactly what
+moe_sort (with a caller-provided workspace) returns, on two calls in a row,
+with sizes that use the scratch (more than 16384 routes) and one that does not.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import mixture_experts_ffn_sort_b200 as moe
+from mixture_experts_ffn_sort_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def static_sort(ids: torch.Tensor, E: int, status: torch.Tensor):
+    T, K = ids.shape
+    off = torch.full((E + 1,), -7, dtype=torch.int32, device="cuda")
+    sr = torch.full((T * K,), -7, dtype=torch.int32, device="cuda")
+    inv = torch.full((T * K,), -7, dtype=torch.int32, device="cuda")
+    rc = moe.lib().moe_sort_static_ws(_p(ids), T, K, E, _p(off), _p(sr), _p(inv), _p(status),
+                                      ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert rc == moe.MOE_OK, moe.lib().moe_last_error().decode()
+    return off, sr, inv
+
+
+@pytest.mark.parametrize("T,K,E", [(4096, 8, 256), (40000, 10, 512), (100, 4, 16)])
+def test_static_scratch_sort_matches_moe_sort(T, K, E):
+    for call in range(2):                       # two calls in a row share the scratch array
+        ids = torch.from_numpy(wl.random_ids(T, K, E, seed=1000 * call + T)).cuda()
+        status = torch.zeros(1, dtype=torch.int32, device="cuda")
+        got = static_sort(ids, E, status)
+        ref = moe.moe_sort(ids, E)
+        torch.cuda.synchronize()
+        assert status.item() == 0
+        for name, a, b in zip(("offsets", "sorted_route", "inv_route"), got, ref):
+            assert torch.equal(a, b), "call %d: %s differs" % (call, name)
+
+
+def test_static_scratch_sort_rejects_sizes_beyond_its_array():
+    L = moe.lib()
+    fake = ctypes.c_void_p(256)                 # never dereferenced: the size check fails first
+    T, K, E = 65536, 10, 1024                   # needs 1024 * 320 * 4 bytes > 1 MiB of scratch
+    rc = L.moe_sort_static_ws(fake, T, K, E, fake, fake, fake, None, None)
+    assert rc == moe.MOE_ERR_UNSUPPORTED_SHAPE
+    assert "scratch" in L.moe_last_error().decode()
