@@ -50,26 +50,32 @@ def load_peaks():
     return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
 
 
-def profile_traffic(workload):
-    """DRAM bytes per FFN call from the committed ncu summary, if the kernel
-    sources it was taken on are unchanged (else None)."""
-    path = os.path.join(ROOT, "profiles", "ffn_%s_traffic.md" % workload)
+def profile_traffic(workload, kind):
+    """DRAM bytes per FFN call from the committed ncu summary of this workload,
+    if the kernel sources it was taken on are unchanged (else None)."""
+    path = os.path.join(ROOT, "profiles", "ffn_%s_%s.md" % (kind, workload))
     if not os.path.exists(path):
         return None
     text = open(path).read()
     m = re.search(r"traffic_bytes_per_call:\s*([0-9.eE+]+)", text)
     h = re.search(r"sources_sha256:\s*([0-9a-f]+)", text)
-    if not m or not h or h.group(1) != sources_hash():
+    if not m or not h or h.group(1) != sources_hash(kind):
         return None
     return float(m.group(1))
 
 
-def sources_hash():
+FFN_SOURCES = {"decode": ("ffn_decode.cu", "device_common.cuh", "launch.h"),
+               "prefill": ("ffn_prefill.cu", "device_common.cuh", "launch.h")}
+
+
+def sources_hash(kind="decode"):
+    """Hash of the sources of the FFN kernels a profile summary was taken on."""
     d = os.path.join(ROOT, "mixture_experts_ffn_sort_b200", "csrc")
     hs = hashlib.sha256()
-    for f in sorted(os.listdir(d)):
-        if f.endswith((".cu", ".cuh", ".h")):
-            hs.update(open(os.path.join(d, f), "rb").read())
+    for f in FFN_SOURCES[kind]:
+        path = os.path.join(d, f)
+        if os.path.exists(path):
+            hs.update(open(path, "rb").read())
     return hs.hexdigest()[:16]
 
 
@@ -325,7 +331,7 @@ def main():
     if decode_path:
         algo = touched * expert_bytes(H, I) + (expert_bytes(H, shape.I_shared) if shape.I_shared else 0)
         ach = algo / (ffn_ms * 1e-3) / 1e9
-        traffic = profile_traffic(shape.name)
+        traffic = profile_traffic(shape.name, "decode")
         roof = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm"], "unit": "GB/s",
                 "frac": ach / peaks["hbm"], "traffic": traffic,
                 "kernel": "moe_expert_ffn (gate/up + down kernels)", "algorithmic_bytes": algo,
@@ -334,7 +340,7 @@ def main():
         ach = flops / (ffn_ms * 1e-3) / 1e12
         pk = peaks["bf16_sus"]
         roof = {"bound": "tensor", "achieved": ach, "peak": pk, "unit": "TFLOP/s", "frac": ach / pk,
-                "traffic": profile_traffic(shape.name), "kernel": "moe_expert_ffn", "flops": flops,
+                "traffic": profile_traffic(shape.name, "prefill"), "kernel": "moe_expert_ffn", "flops": flops,
                 "peak_source": peaks["src"] + " sustained"}
     n_launch = layer.launches()
     out = {"metric": METRIC, "value": T * world / (t_max * 1e-3), "unit": UNIT, "n_gpus": world,
