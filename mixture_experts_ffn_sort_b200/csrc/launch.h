@@ -60,8 +60,12 @@ cudaError_t launch_ffn_decode(const FfnArgs& a, cudaStream_t stream);
 
 // ---------------------------------------------------------------- TMA descriptors
 // 2-D row-major uint8 matrix [rows, cols] (cols contiguous), box
-// {box_cols, box_rows}, 128-byte swizzle.
+// {box_cols, box_rows}, 128-byte (default) or 64-byte swizzle.
 cudaError_t make_tmap_u8_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
-                            uint32_t box_cols, uint32_t box_rows);
+                            uint32_t box_cols, uint32_t box_rows, int swizzle_bytes = 128);
+
+// ---------------------------------------------------------------- expert FFN (prefill, tcgen05)
+cudaError_t launch_ffn_prefill(const FfnArgs& a, cudaStream_t stream);
+bool ffn_prefill_supported(int H, int I);
 
 }  // namespace moe

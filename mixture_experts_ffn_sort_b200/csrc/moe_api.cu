@@ -181,8 +181,9 @@ int moe_expert_ffn(const uint16_t* x, int T, int H, int K, const moe_fp8_experts
     if (workspace_bytes < need || !workspace)
         return fail(MOE_ERR_WORKSPACE_TOO_SMALL, "moe_expert_ffn: workspace of %zu bytes, need %zu",
                     workspace_bytes, need);
-    if (mode == MOE_MODE_PREFILL)
-        return fail(MOE_ERR_UNSUPPORTED_SHAPE, "moe_expert_ffn: PREFILL kernels are not available in this build");
+    const bool prefill = mode == MOE_MODE_PREFILL || (mode == MOE_MODE_AUTO && R > MOE_DECODE_MAX_ROUTES);
+    if (prefill && !moe::ffn_prefill_supported(H, I))
+        return fail(MOE_ERR_UNSUPPORTED_SHAPE, "moe_expert_ffn: H=%d, inter=%d not supported by the PREFILL kernels", H, I);
 
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     moe::FfnArgs a{};
@@ -199,7 +200,7 @@ int moe_expert_ffn(const uint16_t* x, int T, int H, int K, const moe_fp8_experts
     a.y = y_sorted;
     a.status = status;
     a.avg_rows = static_cast<int>((R + E - 1) / E);
-    cudaError_t e = moe::launch_ffn_decode(a, stream);
+    cudaError_t e = prefill ? moe::launch_ffn_prefill(a, stream) : moe::launch_ffn_decode(a, stream);
     if (e != cudaSuccess) return cuda_fail(e, "moe_expert_ffn routed launch");
     if (shared) {
         moe::FfnArgs s = a;
@@ -211,7 +212,7 @@ int moe_expert_ffn(const uint16_t* x, int T, int H, int K, const moe_fp8_experts
         s.h = reinterpret_cast<uint16_t*>(ws + ffn_h_bytes(R, I));
         s.y = y_shared;
         s.avg_rows = T;
-        e = moe::launch_ffn_decode(s, stream);
+        e = prefill ? moe::launch_ffn_prefill(s, stream) : moe::launch_ffn_decode(s, stream);
         if (e != cudaSuccess) return cuda_fail(e, "moe_expert_ffn shared launch");
     }
     return MOE_OK;

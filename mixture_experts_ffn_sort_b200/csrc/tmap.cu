@@ -32,7 +32,7 @@ EncodeTiledFn encode_fn(cudaError_t* err) {
 }  // namespace
 
 cudaError_t make_tmap_u8_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
-                            uint32_t box_cols, uint32_t box_rows) {
+                            uint32_t box_cols, uint32_t box_rows, int swizzle_bytes) {
     cudaError_t err;
     EncodeTiledFn fn = encode_fn(&err);
     if (!fn) return err == cudaSuccess ? cudaErrorNotSupported : err;
@@ -41,7 +41,8 @@ cudaError_t make_tmap_u8_2d(CUtensorMap* map, const void* base, uint64_t rows, u
     const cuuint32_t box[2] = {box_cols, box_rows};
     const cuuint32_t estride[2] = {1, 1};
     CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
-                    estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    swizzle_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
