@@ -193,6 +193,8 @@ def main():
     ap.add_argument("--workload", default="decode", choices=wl.SHAPE_ORDER)
     ap.add_argument("--mode", type=int, default=0, help="moe_expert_ffn mode: 0 AUTO, 1 DECODE, 2 PREFILL")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--eager", action="store_true",
+                    help="launch every call directly instead of replaying CUDA graphs (for profilers)")
     args = ap.parse_args()
     shape = wl.SHAPES[args.workload]
     rank = int(os.environ.get("RANK", "0"))
@@ -239,14 +241,14 @@ def main():
     if layer.status.item() != 0:
         raise RuntimeError("status word %d after warm-up" % layer.status.item())
 
-    # Graph of one step; the timed region replays it K times.
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g, stream=stream):
-        step()
-    # Instrumented graph: events around each call, for the per-call breakdown.
-    ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(5)]
-    g2 = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g2, stream=stream):
+    class Eager:
+        def __init__(self, fn):
+            self.fn = fn
+
+        def replay(self):
+            self.fn()
+
+    def instrumented():
         ev[0].record()
         moe.moe_route(logits, K, zmask, layer.topk_ids, layer.topk_w)
         ev[1].record()
@@ -258,6 +260,19 @@ def main():
         ev[3].record()
         moe.moe_combine(layer.y_sorted, layer.inv_route, layer.y_shared, T, K, moe.MOE_OUT_BF16, layer.out)
         ev[4].record()
+
+    # Graph of one step; the timed region replays it K times.  A second graph
+    # records events around each call, for the per-call breakdown.
+    ev = [torch.cuda.Event(enable_timing=True, external=not args.eager) for _ in range(5)]
+    if args.eager:
+        g, g2 = Eager(step), Eager(instrumented)
+    else:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            step()
+        g2 = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g2, stream=stream):
+            instrumented()
     with torch.cuda.stream(stream):
         for _ in range(3):
             g.replay()
@@ -350,7 +365,8 @@ def main():
                           l2="inputs larger than L2 (touched expert weights %.2f GB > 126 MB)"
                              % (touched * expert_bytes(H, I) / 1e9) if decode_path else
                              "inputs larger than L2 (expert weights %.2f GB > 126 MB)" % (E * expert_bytes(H, I) / 1e9),
-                          timing="CUDA events around %d CUDA-graph replays of one step" % args.steps),
+                          timing="CUDA events around %d %s of one step" % (
+                              args.steps, "eager launches" if args.eager else "CUDA-graph replays")),
            "roofline": roof,
            "breakdown_ms": {k: statistics.median(v) for k, v in parts.items()},
            "e2e": {"value": T * world / (e2e_ms * 1e-3), "unit": UNIT,

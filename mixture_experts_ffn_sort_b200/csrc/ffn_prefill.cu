@@ -11,19 +11,24 @@
 //
 // One persistent kernel per GEMM (gate/up, then down); each CTA owns one SM
 // and walks a list of output tiles built on the device from the expert
-// offsets (no host sync).  A tile is 128 weight rows x up to 256 token rows:
+// offsets (no host sync).  A tile is 128 weight rows x up to 192 token rows:
 //  * swap-AB: the weights are the M=128 operand A, the tokens the N operand B,
 //    so the FP8 decode writes tensor memory, not shared memory;
-//  * loader warps 0-3: the weight tile's FP8 bytes by TMA (64-byte swizzle)
-//    and the token rows by cp.async into the 128-byte-swizzled K-major layout
-//    the MMA reads (token rows are gathered through sorted_route for gate/up,
-//    contiguous rows of h for down);
-//  * transform warps 4-7: each thread owns one TMEM lane (one weight row),
-//    decodes its 64 FP8 codes per stage to bf16(e4m3 * block scale) and
-//    stores them to TMEM with tcgen05.st (A operand, two bf16 per column);
-//  * warp 12: one thread issues tcgen05.mma (kind::f16, A in TMEM, B in
-//    shared memory, fp32 accumulator D in TMEM) and commits to mbarriers;
-//  * epilogue warps 8-11: tcgen05.ld of D; gate/up rows are interleaved
+//  * warp 0: the weight tile's FP8 bytes by TMA (64-byte swizzle), up to 8
+//    stages ahead;
+//  * warps 2-3: the token rows into the 128-byte-swizzled K-major layout the
+//    MMA reads -- x rows gathered through sorted_route by cp.async (each
+//    thread arrives on the stage's mbarrier when its copies land) for
+//    gate/up, contiguous rows of h as one 2-D TMA tile for down -- up to 6
+//    stages ahead;
+//  * transform warps 8-15: each thread owns one TMEM lane (one weight row)
+//    and half of a stage's columns, decodes its FP8 codes to
+//    bf16(e4m3 * block scale) and stores them to TMEM with tcgen05.st (A
+//    operand, two bf16 per column), into a 4-deep A ring;
+//  * warp 1: one thread issues tcgen05.mma (kind::f16, A in TMEM, B in
+//    shared memory, fp32 accumulator D in TMEM, double-buffered so the
+//    epilogue of one tile overlaps the main loop of the next);
+//  * epilogue warps 4-7: tcgen05.ld of D; gate/up rows are interleaved
 //    (row 2j = gate of feature j, row 2j+1 = up of feature j), so a lane pair
 //    holds gate and up of one feature and SwiGLU needs one shuffle; the down
 //    epilogue multiplies by the route weight.  bf16 results go to global.
@@ -37,23 +42,43 @@ namespace moe {
 
 namespace {
 
-constexpr int kS = 4;                       // pipeline stages of 64 reduction columns
-constexpr int kNMax = 256;                  // token rows per tile (MMA N)
-constexpr int kWStage = 128 * 64;           // FP8 weight rows x 64 codes (64-byte swizzle)
+constexpr int kSB = 6;                      // token stages
+constexpr int kNMax = 192;                  // token rows per tile (MMA N)
 constexpr int kBStage = kNMax * 128;        // token rows x 64 bf16 (128-byte swizzle)
-constexpr int kWarpXform = 4, kWarpEpi = 8, kWarpMma = 12;
-constexpr int kThreads = 13 * 32;
-constexpr int kLoaders = 128;
+constexpr int kWRing = 64 * 1024;           // FP8 weight ring (64 reduction columns per stage)
+// Per mode: M-tiles (128 weight rows each) per step, weight stage bytes and
+// depths of the weight ring and of the bf16 A ring in TMEM.
+template <int MODE> struct Cfg;
+// Warp roles (transform and epilogue warps sit on their TMEM lane quarter, warp % 4):
+// warps 2-3 load token rows.
+constexpr int kWarpTma = 0, kWarpMma = 1, kWarpTok = 2, kWarpEpi = 4, kWarpXform = 8;
+constexpr int kTokThreads = 64;
+constexpr int kNumWarps = 16;
+constexpr int kThreads = kNumWarps * 32;
+constexpr int kXformWarps = 8;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kDCol = 0;    // D: columns [0, 256)
-constexpr uint32_t kACol = 256;  // A stages: 32 columns each
-constexpr int kLag = 2;          // cp.async stages kept in flight before a stage is published
+constexpr uint32_t kDRegion = kNMax;        // two accumulator regions of kNMax columns
+constexpr uint32_t kACol = 2 * kNMax;       // A ring: 128 columns
+constexpr int kDownGroup = 16;                  // output blocks sharing a resident token tile (down)
+constexpr int kScales = 1024;                   // staged block scales per item (floats)
 
 enum Mode { kGateUp = 0, kDown = 1 };
 
+// gate/up: a step feeds two M-tiles (gate and up rows of 128 features, two
+// accumulator regions); down: one M-tile per step, regions double-buffered.
+template <> struct Cfg<0> {
+    static constexpr int MT = 2, kWStage = 2 * 128 * 64, kSW = kWRing / kWStage, kSA = 2;
+};
+template <> struct Cfg<1> {
+    static constexpr int MT = 1, kWStage = 128 * 64, kSW = kWRing / kWStage, kSA = 4;
+};
+constexpr int kSWMax = 8, kSAMax = 4;
+
 struct Barriers {
-    uint64_t w_full[kS], w_empty[kS], b_full[kS], a_full[kS], done[kS];
-    uint64_t d_full, d_empty, final_bar;
+    uint64_t w_full[kSWMax], w_empty[kSWMax];
+    uint64_t b_full[kSB], b_done[kSB];
+    uint64_t a_full[kSAMax], a_done[kSAMax];
+    uint64_t d_full[2], d_empty[2], final_bar;
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -62,32 +87,41 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
     return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
+// One work item: a token tile of one expert and a group of consecutive
+// output blocks (128 weight rows each) that share that token tile.
 struct Tile {
     int e;
-    long p0;
-    int n;
-    int fb;
+    long p0;  // first sorted row
+    int n;    // rows in the tile (<= kNMax)
+    int fb0;  // first output block
+    int nfb;  // output blocks in the group
 };
 
-// Tile list: expert e contributes ceil(n_e / 256) token tiles x FB feature blocks,
-// pre[] holds the exclusive prefix over experts.  Returns the total.
-__device__ int build_tiles(const FfnArgs& a, int FB, int* pre) {
+// Number of items of expert e with n_e rows.
+__device__ __forceinline__ int items_of(long n_e, int groups) {
+    return static_cast<int>((n_e + kNMax - 1) / kNMax) * groups;
+}
+
+__device__ __forceinline__ long expert_len(const FfnArgs& a, int e, long R, bool* bad) {
+    if (a.identity) return a.T;
+    const long b = a.offsets[e], f = a.offsets[e + 1];
+    if (b < 0 || f < b || f > R) {
+        *bad = true;
+        return 0;
+    }
+    return f - b;
+}
+
+// Item list: pre[] holds the exclusive prefix of items over experts.  Returns the total.
+__device__ int build_tiles(const FfnArgs& a, int groups, int* pre) {
     const int E = a.identity ? 1 : a.ex.n;
     const long R = static_cast<long>(a.T) * a.K;
     const int per = (E + blockDim.x - 1) / blockDim.x;
     const int e0 = min(E, static_cast<int>(threadIdx.x) * per), e1 = min(E, e0 + per);
     int local = 0;
-    for (int e = e0; e < e1; ++e) {
-        long n;
-        if (a.identity) {
-            n = a.T;
-        } else {
-            const long b = a.offsets[e], f = a.offsets[e + 1];
-            n = (b < 0 || f < b || f > R) ? 0 : f - b;
-            if (n == 0 && (b < 0 || f < b || f > R)) report_status(a.status, MOE_STATUS_BAD_MAP);
-        }
-        local += static_cast<int>((n + kNMax - 1) / kNMax) * FB;
-    }
+    bool bad = false;
+    for (int e = e0; e < e1; ++e) local += items_of(expert_len(a, e, R, &bad), groups);
+    if (bad) report_status(a.status, MOE_STATUS_BAD_MAP);
     // Block exclusive scan of `local`.
     __shared__ int warp_sums[32];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
@@ -112,14 +146,7 @@ __device__ int build_tiles(const FfnArgs& a, int FB, int* pre) {
     int run = (warp ? warp_sums[warp - 1] : 0) + x - local;
     for (int e = e0; e < e1; ++e) {
         pre[e] = run;
-        long n;
-        if (a.identity) {
-            n = a.T;
-        } else {
-            const long b = a.offsets[e], f = a.offsets[e + 1];
-            n = (b < 0 || f < b || f > R) ? 0 : f - b;
-        }
-        run += static_cast<int>((n + kNMax - 1) / kNMax) * FB;
+        run += items_of(expert_len(a, e, R, &bad), groups);
     }
     const int total = warp_sums[nw - 1];
     if (threadIdx.x == 0) pre[E] = total;
@@ -127,7 +154,7 @@ __device__ int build_tiles(const FfnArgs& a, int FB, int* pre) {
     return total;
 }
 
-__device__ __forceinline__ Tile tile_of(const FfnArgs& a, const int* pre, int FB, int item) {
+__device__ __forceinline__ Tile tile_of(const FfnArgs& a, const int* pre, int FB, int GFB, int item) {
     const int E = a.identity ? 1 : a.ex.n;
     int lo = 0, hi = E - 1;  // last e with pre[e] <= item
     while (lo < hi) {
@@ -137,15 +164,18 @@ __device__ __forceinline__ Tile tile_of(const FfnArgs& a, const int* pre, int FB
         else
             hi = mid - 1;
     }
+    const int groups = (FB + GFB - 1) / GFB;
     Tile t;
     t.e = lo;
     const int local = item - pre[lo];
-    const int tt = local / FB;
-    t.fb = local - tt * FB;
+    const int tt = local / groups;
+    const int fg = local - tt * groups;
     const long base = a.identity ? 0 : a.offsets[lo];
     const long n_e = a.identity ? a.T : a.offsets[lo + 1] - base;
     t.p0 = base + static_cast<long>(tt) * kNMax;
     t.n = static_cast<int>(min(static_cast<long>(kNMax), n_e - static_cast<long>(tt) * kNMax));
+    t.fb0 = fg * GFB;
+    t.nfb = min(GFB, FB - t.fb0);
     return t;
 }
 
@@ -163,34 +193,49 @@ __device__ __forceinline__ uint32_t decode_scaled(uint16_t codes, float s) {
 template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tm_w0, const __grid_constant__ CUtensorMap tm_w1,
-                   const FfnArgs a) {
+                   const __grid_constant__ CUtensorMap tm_act, const FfnArgs a) {
+    using C = Cfg<MODE>;
+    constexpr int MT = C::MT, kSW = C::kSW, kSA = C::kSA, kWStage = C::kWStage;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = align1024(smem_raw);
-    uint8_t* w_ring = sm;                          // kS x 8 KB
-    uint8_t* b_ring = w_ring + kS * kWStage;       // kS x 32 KB
-    Barriers* B = reinterpret_cast<Barriers*>(b_ring + kS * kBStage);
-    int* row_tok = reinterpret_cast<int*>(B + 1);  // [kNMax] token row offsets of the loaders' tile
-    int* pre = row_tok + kNMax;                    // [E + 1]
+    uint8_t* w_ring = sm;                          // kSW x kWStage (64 KB)
+    uint8_t* b_ring = w_ring + kWRing;             // kSB x 24 KB
+    Barriers* B = reinterpret_cast<Barriers*>(b_ring + kSB * kBStage);
+    int* row_tok = reinterpret_cast<int*>(B + 1);  // [kNMax] activation row of each tile row
+    float* col_w = reinterpret_cast<float*>(row_tok + kNMax);  // [kNMax] route weight of each column (down)
+    float* sc_sm = col_w + kNMax;                              // [kScales] block scales of the item
+    int* pre = reinterpret_cast<int*>(sc_sm + kScales);        // [E + 1]
 
     const int H = a.H, I = a.ex.inter;
     const int Kred = MODE == kGateUp ? H : I;       // reduction length
-    const int KB = Kred / 64;                       // stages per tile
-    const int FB = MODE == kGateUp ? I / 64 : H / 128;
-    const int rowstride = MODE == kGateUp ? H : I;  // elements between activation rows
-    const uint16_t* act = MODE == kGateUp ? a.x : a.h;
+    const int KB = Kred / 64;                       // stages per output block
+    const int KB128 = Kred / 128;                   // scale blocks along the reduction
+    // Output blocks: gate/up -> 128 features (gate + up rows); down -> 128 features.
+    const int FB = MODE == kGateUp ? I / 128 : H / 128;
+    // The down GEMM keeps its token tile resident across a group of output
+    // blocks when the whole reduction fits in the token ring.
+    const bool resident = MODE == kDown && KB <= kSB;
+    const int GFB = resident ? kDownGroup : 1;
     const long R = static_cast<long>(a.T) * a.K;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kS; ++s) {
+        for (int s = 0; s < kSW; ++s) {
             mbar_init(&B->w_full[s], 1);
-            mbar_init(&B->w_empty[s], 4);
-            mbar_init(&B->b_full[s], kLoaders);
-            mbar_init(&B->a_full[s], 4);
-            mbar_init(&B->done[s], 1);
+            mbar_init(&B->w_empty[s], kXformWarps);
         }
-        mbar_init(&B->d_full, 1);
-        mbar_init(&B->d_empty, 4);
+        for (int s = 0; s < kSB; ++s) {
+            mbar_init(&B->b_full[s], MODE == kGateUp ? kTokThreads : 1);
+            mbar_init(&B->b_done[s], 1);
+        }
+        for (int s = 0; s < kSA; ++s) {
+            mbar_init(&B->a_full[s], kXformWarps);
+            mbar_init(&B->a_done[s], 1);
+        }
+        for (int d = 0; d < 2; ++d) {
+            mbar_init(&B->d_full[d], 1);
+            mbar_init(&B->d_empty[d], 4);
+        }
         mbar_init(&B->final_bar, 1);
         B->abort_flag = 0;
         fence_mbar_init();
@@ -199,209 +244,280 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_alloc(&B->tmem_base, kTmemCols);
         tc_fence_before();
     }
-    const int total = build_tiles(a, FB, pre);  // contains __syncthreads
+    const int total = build_tiles(a, (FB + GFB - 1) / GFB, pre);  // contains __syncthreads
     tc_fence_after();
     const uint32_t tmem = B->tmem_base;
     if (MODE == kGateUp && threadIdx.x == 0) grid_dependency_launch();
 
-    if (warp < 4) {
-        // ------------------------------------------------ loaders
-        const int lt = threadIdx.x;
-        if (MODE == kDown) grid_dependency_wait();  // h comes from the gate/up grid
-        if (lt == 0) {
+    if (warp == kWarpTma) {
+        // ------------------------------------------------ FP8 weight tiles (TMA, evict-first)
+        if (lane == 0) {
             tma_prefetch_desc(&tm_w0);
             if (MODE == kGateUp) tma_prefetch_desc(&tm_w1);
+            const uint64_t policy = l2_evict_first_policy();
+            long g = 0;
+            for (int item = blockIdx.x; item < total; item += gridDim.x) {
+                const Tile t = tile_of(a, pre, FB, GFB, item);
+                for (int f = 0; f < t.nfb; ++f) {
+                    const int fb = t.fb0 + f;
+                    for (int kb = 0; kb < KB; ++kb, ++g) {
+                        const int s = static_cast<int>(g % kSW);
+                        if (g >= kSW) wait_bar(&B->w_empty[s], static_cast<uint32_t>((g / kSW - 1) & 1), B, a.status);
+                        uint8_t* dst = w_ring + s * kWStage;
+                        mbar_arrive_expect_tx(&B->w_full[s], kWStage);
+                        if (MODE == kGateUp) {
+                            const int row = t.e * I + fb * 128;  // 128 gate rows, 128 up rows
+                            tma_load_2d_hint(dst, &tm_w0, &B->w_full[s], kb * 64, row, policy);
+                            tma_load_2d_hint(dst + kWStage / 2, &tm_w1, &B->w_full[s], kb * 64, row, policy);
+                        } else {
+                            tma_load_2d_hint(dst, &tm_w0, &B->w_full[s], kb * 64, t.e * H + fb * 128, policy);
+                        }
+                    }
+                }
+            }
         }
+    } else if (warp == kWarpTok || warp == kWarpTok + 1) {
+        // ------------------------------------------------ token rows
+        // gate/up: rows of x gathered through sorted_route by cp.async (16 bytes
+        // per copy, 64 threads), each thread arriving on the stage barrier when
+        // its copies land; down: contiguous rows of h as one 2-D TMA tile.
+        // Padding rows of the last MMA column group are left stale: column j of
+        // D depends on token row j only, and the epilogue drops those columns.
+        const int lt = threadIdx.x - kWarpTok * 32;  // 0..63
+        if (MODE == kDown) grid_dependency_wait();  // h comes from the gate/up grid
+        if (MODE == kDown && lt == 0) tma_prefetch_desc(&tm_act);
         long g = 0;
-        long published = 0;  // stages whose b_full has been signalled
         for (int item = blockIdx.x; item < total; item += gridDim.x) {
-            const Tile t = tile_of(a, pre, FB, item);
-            const int N = (t.n + 15) & ~15;
-            named_barrier_sync(2, kLoaders);
-            for (int r = lt; r < kNMax; r += kLoaders) {
-                int off = -1;
-                if (r < t.n) {
+            const Tile t = tile_of(a, pre, FB, GFB, item);
+            if (MODE == kGateUp) {
+                named_barrier_sync(2, kTokThreads);
+                bool bad = false;
+                for (int r = lt; r < t.n; r += kTokThreads) {
+                    int tok = 0;
                     const long p = t.p0 + r;
-                    if (MODE == kDown || a.identity) {
-                        off = static_cast<int>(p);
+                    if (a.identity) {
+                        tok = static_cast<int>(p);
                     } else {
                         const int rt = a.sorted_route[p];
-                        off = (rt >= 0 && rt < R) ? rt / a.K : -1;
+                        if (rt >= 0 && rt < R)
+                            tok = rt / a.K;
+                        else
+                            bad = true;
                     }
+                    row_tok[r] = tok;
                 }
-                row_tok[r] = off;
+                if (bad) report_status(a.status, MOE_STATUS_BAD_MAP);
+                named_barrier_sync(2, kTokThreads);
             }
-            named_barrier_sync(2, kLoaders);
             for (int kb = 0; kb < KB; ++kb, ++g) {
-                const int s = static_cast<int>(g % kS);
-                if (g >= kS) wait_bar(&B->done[s], static_cast<uint32_t>((g / kS - 1) & 1), B, a.status);
-                if (lt == 0) {
-                    if (g >= kS) wait_bar(&B->w_empty[s], static_cast<uint32_t>((g / kS - 1) & 1), B, a.status);
-                    uint8_t* dst = w_ring + s * kWStage;
-                    mbar_arrive_expect_tx(&B->w_full[s], kWStage);
-                    if (MODE == kGateUp) {
-                        const int row = t.e * I + t.fb * 64;  // 64 gate rows, 64 up rows
-                        tma_load_2d(dst, &tm_w0, &B->w_full[s], kb * 64, row);
-                        tma_load_2d(dst + kWStage / 2, &tm_w1, &B->w_full[s], kb * 64, row);
-                    } else {
-                        tma_load_2d(dst, &tm_w0, &B->w_full[s], kb * 64, t.e * H + t.fb * 128);
+                const int s = static_cast<int>(g % kSB);
+                if (g >= kSB) wait_bar(&B->b_done[s], static_cast<uint32_t>((g / kSB - 1) & 1), B, a.status);
+                uint8_t* dst = b_ring + s * kBStage;
+                if (MODE == kGateUp) {
+                    const uint32_t bdst = smem_u32(dst);
+                    for (int ci = lt; ci < t.n * 8; ci += kTokThreads) {
+                        const int r = ci >> 3, ch = ci & 7;
+                        const uint16_t* src = a.x + static_cast<size_t>(row_tok[r]) * H + kb * 64 + ch * 8;
+                        cp_async16(bdst + r * 128 + ((ch ^ (r & 7)) << 4), src, 16u);
                     }
-                }
-                const uint32_t bdst = smem_u32(b_ring + s * kBStage);
-                for (int ci = lt; ci < N * 8; ci += kLoaders) {
-                    const int r = ci >> 3, ch = ci & 7;
-                    const int off = row_tok[r];
-                    const uint16_t* src = off >= 0 ? act + static_cast<size_t>(off) * rowstride + kb * 64 + ch * 8 : act;
-                    cp_async16(bdst + r * 128 + ((ch ^ (r & 7)) << 4), src, off >= 0 ? 16u : 0u);
-                }
-                cp_async_commit();
-                if (g - published >= kLag) {
-                    cp_async_wait<kLag>();
-                    fence_proxy_async_smem();
-                    mbar_arrive(&B->b_full[published % kS]);
-                    ++published;
+                    cp_async_arrive_noinc(&B->b_full[s]);
+                } else if (lt == 0) {
+                    mbar_arrive_expect_tx(&B->b_full[s], kBStage);
+                    tma_load_2d(dst, &tm_act, &B->b_full[s], kb * 64, static_cast<int>(t.p0));
                 }
             }
         }
-        cp_async_wait<0>();
-        fence_proxy_async_smem();
-        while (published < g) {
-            mbar_arrive(&B->b_full[published % kS]);
-            ++published;
-        }
-    } else if (warp < kWarpEpi) {
+        if (MODE == kGateUp) cp_async_wait<0>();
+    } else if (warp >= kWarpXform) {
         // ------------------------------------------------ transform: FP8 -> bf16 -> TMEM (A)
-        const int q = warp - kWarpXform;
-        const int row = 32 * q + lane;  // TMEM lane = weight row of the tile
+        // gate/up: warp (q, mt) owns lane quarter q of M-tile mt and all 64 codes
+        // of a stage; down: warp (q, hf) owns lane quarter q and half of the codes.
+        const int q = warp & 3, hi = (warp - kWarpXform) >> 2;
+        const int xt = threadIdx.x - kWarpXform * 32;           // 0..255
+        const int row = 32 * q + lane;  // TMEM lane = weight row of the M-tile
+        constexpr int NW = MODE == kGateUp ? 32 : 16;           // words (bf16 pairs) per thread per stage
         long g = 0;
         for (int item = blockIdx.x; item < total; item += gridDim.x) {
-            const Tile t = tile_of(a, pre, FB, item);
-            int srow, sub;
-            const float* sp;
+            const Tile t = tile_of(a, pre, FB, GFB, item);
+            // Block scales of the item, staged once: gate/up -> [gate, up][KB128],
+            // down -> [output block][KB128].
+            named_barrier_sync(3, kXformWarps * 32);
             if (MODE == kGateUp) {
-                const int j = row >> 1, feat = t.fb * 64 + j;
-                sub = (row & 1) ? kWStage / 2 : 0;
-                srow = j;
-                sp = ((row & 1) ? a.ex.s_up : a.ex.s_gate) +
-                     (static_cast<size_t>(t.e) * (I / 128) + feat / 128) * (H / 128);
+                const size_t off = (static_cast<size_t>(t.e) * (I / 128) + t.fb0) * KB128;
+                for (int i = xt; i < 2 * KB128; i += kXformWarps * 32)
+                    sc_sm[i] = __ldg((i < KB128 ? a.ex.s_gate : a.ex.s_up) + off + (i % KB128));
             } else {
-                const int feat = t.fb * 128 + row;
-                sub = 0;
-                srow = row;
-                sp = a.ex.s_down + (static_cast<size_t>(t.e) * (H / 128) + feat / 128) * (I / 128);
-            }
-            for (int kb = 0; kb < KB; ++kb, ++g) {
-                const int s = static_cast<int>(g % kS);
-                const bool ok1 = wait_bar(&B->w_full[s], static_cast<uint32_t>((g / kS) & 1), B, a.status);
-                bool ok2 = true;
-                if (g >= kS) ok2 = wait_bar(&B->done[s], static_cast<uint32_t>((g / kS - 1) & 1), B, a.status);
-                uint32_t v[32];
-                if (ok1 && ok2) {
-                    const float sc = __ldg(sp + (kb >> 1));
-                    const uint8_t* base = w_ring + s * kWStage + sub + srow * 64;
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        const uint4 w = *reinterpret_cast<const uint4*>(base + ((c ^ ((srow >> 1) & 3)) << 4));
-                        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-                        for (int k = 0; k < 4; ++k) {
-                            v[c * 8 + 2 * k] = decode_scaled(static_cast<uint16_t>(ws[k] & 0xFFFFu), sc);
-                            v[c * 8 + 2 * k + 1] = decode_scaled(static_cast<uint16_t>(ws[k] >> 16), sc);
-                        }
-                    }
-                } else {
-#pragma unroll
-                    for (int k = 0; k < 32; ++k) v[k] = 0;
+                for (int i = xt; i < t.nfb * KB128; i += kXformWarps * 32) {
+                    const int f = i / KB128, k = i - f * KB128;
+                    sc_sm[i] = __ldg(a.ex.s_down +
+                                     (static_cast<size_t>(t.e) * (H / 128) + (t.fb0 + f)) * KB128 + k);
                 }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&B->w_empty[s]);
-                tmem_st32(tmem + (static_cast<uint32_t>(32 * q) << 16) + kACol + s * 32, v);
-                tmem_st_wait();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&B->a_full[s]);
+            }
+            named_barrier_sync(3, kXformWarps * 32);
+            // Source row in the weight stage: gate/up rows interleave as
+            // (gate j, up j) pairs, j = feature within the M-tile.
+            const int srow = MODE == kGateUp ? hi * 64 + (row >> 1) : row;
+            const int sub = (MODE == kGateUp && (row & 1)) ? kWStage / 2 : 0;
+            const int c0 = MODE == kGateUp ? 0 : 2 * hi;  // first 16-byte chunk of this thread
+            for (int f = 0; f < t.nfb; ++f) {
+                const float* scr = sc_sm + (MODE == kGateUp ? (row & 1) * KB128 : f * KB128);
+                for (int kb = 0; kb < KB; ++kb, ++g) {
+                    const int sw = static_cast<int>(g % kSW), sa = static_cast<int>(g % kSA);
+                    const bool ok1 = wait_bar(&B->w_full[sw], static_cast<uint32_t>((g / kSW) & 1), B, a.status);
+                    bool ok2 = true;
+                    if (g >= kSA)
+                        ok2 = wait_bar(&B->a_done[sa], static_cast<uint32_t>((g / kSA - 1) & 1), B, a.status);
+                    uint32_t v[NW];
+                    if (ok1 && ok2) {
+                        const float sc = scr[kb >> 1];
+                        const uint8_t* base = w_ring + sw * kWStage + sub + srow * 64;
+#pragma unroll
+                        for (int c = 0; c < NW / 8; ++c) {
+                            const int chunk = c0 + c;
+                            const uint4 w =
+                                *reinterpret_cast<const uint4*>(base + ((chunk ^ ((srow >> 1) & 3)) << 4));
+                            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                            for (int k = 0; k < 4; ++k) {
+                                v[c * 8 + 2 * k] = decode_scaled(static_cast<uint16_t>(ws[k] & 0xFFFFu), sc);
+                                v[c * 8 + 2 * k + 1] = decode_scaled(static_cast<uint16_t>(ws[k] >> 16), sc);
+                            }
+                        }
+                    } else {
+#pragma unroll
+                        for (int k = 0; k < NW; ++k) v[k] = 0;
+                    }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&B->w_empty[sw]);
+                    const uint32_t acol = kACol + sa * (MT * 32) + (MODE == kGateUp ? hi * 32 : hi * 16);
+                    if constexpr (MODE == kGateUp)
+                        tmem_st32(tmem + (static_cast<uint32_t>(32 * q) << 16) + acol, v);
+                    else
+                        tmem_st16(tmem + (static_cast<uint32_t>(32 * q) << 16) + acol, v);
+                    tmem_st_wait();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&B->a_full[sa]);
+                }
             }
         }
-    } else if (warp < kWarpMma) {
+    } else if (warp >= kWarpEpi) {
         // ------------------------------------------------ epilogue
-        const int q = warp - kWarpEpi;
+        const int q = warp & 3;
+        int uses[2] = {0, 0};
         int tc = 0;
-        for (int item = blockIdx.x; item < total; item += gridDim.x, ++tc) {
-            const Tile t = tile_of(a, pre, FB, item);
-            const bool ok = wait_bar(&B->d_full, static_cast<uint32_t>(tc & 1), B, a.status);
-            tc_fence_after();
-            for (int c0 = 0; c0 < t.n; c0 += 32) {
-                uint32_t v[32];
-                tmem_ld32(tmem + (static_cast<uint32_t>(32 * q) << 16) + kDCol + c0, v);
-                tmem_ld_wait();
-                if (!ok) continue;
-                if (MODE == kGateUp) {
-                    // Lane 2j: gate of feature j; lane 2j+1: up of feature j.  Even lanes
-                    // write column c, odd lanes column c+1.
-                    const int feat = t.fb * 64 + 16 * q + (lane >> 1);
-                    const bool odd = lane & 1;
-#pragma unroll
-                    for (int c = 0; c < 32; c += 2) {
-                        const float x0 = __uint_as_float(v[c]), x1 = __uint_as_float(v[c + 1]);
-                        const float y0 = __shfl_xor_sync(0xffffffffu, x0, 1);
-                        const float y1 = __shfl_xor_sync(0xffffffffu, x1, 1);
-                        const float gte = odd ? y1 : x0, up = odd ? x1 : y0;
-                        const int col = c0 + c + (odd ? 1 : 0);
-                        if (col < t.n)
-                            a.h[static_cast<size_t>(t.p0 + col) * I + feat] =
-                                __bfloat16_as_ushort(__float2bfloat16_rn(silu_f32(gte) * up));
+        const int et = threadIdx.x - kWarpEpi * 32;  // 0..127
+        for (int item = blockIdx.x; item < total; item += gridDim.x) {
+            const Tile t = tile_of(a, pre, FB, GFB, item);
+            if (MODE == kDown) {
+                // Route weight of every column of the item, staged once.
+                named_barrier_sync(4, 128);
+                for (int c = et; c < t.n; c += 128) {
+                    float wv = 1.f;
+                    if (!a.identity) {
+                        const int rt = a.sorted_route[t.p0 + c];
+                        wv = (rt >= 0 && rt < R) ? a.topk_w[rt] : 0.f;
                     }
-                } else {
-                    const int feat = t.fb * 128 + 32 * q + lane;
-                    float wl = 0.f;
-                    if (c0 + lane < t.n) {
-                        const long p = t.p0 + c0 + lane;
-                        if (a.identity) {
-                            wl = 1.f;
+                    col_w[c] = wv;
+                }
+                named_barrier_sync(4, 128);
+            }
+            for (int f = 0; f < t.nfb; ++f, ++tc) {
+                for (int mt = 0; mt < MT; ++mt) {
+                    const int r = MODE == kGateUp ? mt : (tc & 1);  // accumulator region
+                    const bool ok = wait_bar(&B->d_full[r], static_cast<uint32_t>(uses[r] & 1), B, a.status);
+                    ++uses[r];
+                    tc_fence_after();
+                    const uint32_t dcol = r * kDRegion;
+                    for (int c0 = 0; c0 < t.n; c0 += 32) {
+                        uint32_t v[32];
+                        tmem_ld32(tmem + (static_cast<uint32_t>(32 * q) << 16) + dcol + c0, v);
+                        tmem_ld_wait();
+                        if (!ok) continue;
+                        if (MODE == kGateUp) {
+                            // Lane 2j: gate of feature j; lane 2j+1: up of feature j.
+                            // Even lanes write column c, odd lanes column c+1.
+                            const int feat = t.fb0 * 128 + mt * 64 + 16 * q + (lane >> 1);
+                            const bool odd = lane & 1;
+#pragma unroll
+                            for (int c = 0; c < 32; c += 2) {
+                                const float x0 = __uint_as_float(v[c]), x1 = __uint_as_float(v[c + 1]);
+                                const float y0 = __shfl_xor_sync(0xffffffffu, x0, 1);
+                                const float y1 = __shfl_xor_sync(0xffffffffu, x1, 1);
+                                const float gte = odd ? y1 : x0, up = odd ? x1 : y0;
+                                const int col = c0 + c + (odd ? 1 : 0);
+                                if (col < t.n)
+                                    a.h[static_cast<size_t>(t.p0 + col) * I + feat] =
+                                        __bfloat16_as_ushort(__float2bfloat16_rn(silu_f32(gte) * up));
+                            }
                         } else {
-                            const int rt = a.sorted_route[p];
-                            wl = (rt >= 0 && rt < R) ? a.topk_w[rt] : 0.f;
+                            const int feat = (t.fb0 + f) * 128 + 32 * q + lane;
+#pragma unroll
+                            for (int c = 0; c < 32; ++c) {
+                                const float wv = col_w[c0 + c];
+                                if (c0 + c < t.n)
+                                    a.y[static_cast<size_t>(t.p0 + c0 + c) * H + feat] =
+                                        __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[c]) * wv));
+                            }
                         }
                     }
-#pragma unroll
-                    for (int c = 0; c < 32; ++c) {
-                        const float wv = __shfl_sync(0xffffffffu, wl, c);
-                        if (c0 + c < t.n)
-                            a.y[static_cast<size_t>(t.p0 + c0 + c) * H + feat] =
-                                __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[c]) * wv));
-                    }
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&B->d_empty[r]);
                 }
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&B->d_empty);
         }
-    } else {
+    } else if (warp == kWarpMma) {
         // ------------------------------------------------ MMA issuer
         if (lane == 0) {
-            long g = 0;
+            long ga = 0, gb = 0;
+            int uses[2] = {0, 0};
             int tc = 0;
-            for (int item = blockIdx.x; item < total; item += gridDim.x, ++tc) {
-                const Tile t = tile_of(a, pre, FB, item);
+            for (int item = blockIdx.x; item < total; item += gridDim.x) {
+                const Tile t = tile_of(a, pre, FB, GFB, item);
                 const int N = (t.n + 15) & ~15;
                 const uint32_t idesc = umma_idesc_bf16(128, N);
-                if (tc >= 1) wait_bar(&B->d_empty, static_cast<uint32_t>((tc - 1) & 1), B, a.status);
-                tc_fence_after();
-                for (int kb = 0; kb < KB; ++kb, ++g) {
-                    const int s = static_cast<int>(g % kS);
-                    const uint32_t ph = static_cast<uint32_t>((g / kS) & 1);
-                    const bool ok = wait_bar(&B->a_full[s], ph, B, a.status) & wait_bar(&B->b_full[s], ph, B, a.status);
-                    tc_fence_after();
-                    if (ok) {
-                        const uint32_t bbase = smem_u32(b_ring + s * kBStage);
-#pragma unroll
-                        for (int k = 0; k < 4; ++k)
-                            umma_ts_f16(tmem + kDCol, tmem + kACol + s * 32 + k * 8, umma_desc_sw128(bbase + k * 32),
-                                        idesc, (kb > 0 || k > 0) ? 1u : 0u);
+                for (int f = 0; f < t.nfb; ++f, ++tc) {
+                    // Accumulator regions of this output block: both (gate/up) or one (down).
+                    const int r0 = MODE == kGateUp ? 0 : (tc & 1);
+                    for (int mt = 0; mt < MT; ++mt) {
+                        const int r = r0 + mt;
+                        if (uses[r] >= 1)
+                            wait_bar(&B->d_empty[r], static_cast<uint32_t>((uses[r] - 1) & 1), B, a.status);
+                        ++uses[r];
                     }
-                    umma_commit(&B->done[s]);
+                    tc_fence_after();
+                    const bool last = f == t.nfb - 1;
+                    for (int kb = 0; kb < KB; ++kb, ++ga) {
+                        const long g_b = resident ? gb + kb : gb;  // token stage of this step
+                        const int sa = static_cast<int>(ga % kSA), sb = static_cast<int>(g_b % kSB);
+                        const bool ok =
+                            wait_bar(&B->a_full[sa], static_cast<uint32_t>((ga / kSA) & 1), B, a.status) &
+                            wait_bar(&B->b_full[sb], static_cast<uint32_t>((g_b / kSB) & 1), B, a.status);
+                        tc_fence_after();
+                        // Token rows written by cp.async (generic proxy) are read by the MMA
+                        // (async proxy).
+                        if (MODE == kGateUp) fence_proxy_async_smem();
+                        if (ok) {
+                            const uint32_t bbase = smem_u32(b_ring + sb * kBStage);
+#pragma unroll
+                            for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                                for (int k = 0; k < 4; ++k)
+                                    umma_ts_f16(tmem + (r0 + mt) * kDRegion, tmem + kACol + sa * (MT * 32) + mt * 32 + k * 8,
+                                                umma_desc_sw128(bbase + k * 32), idesc, (kb > 0 || k > 0) ? 1u : 0u);
+                        }
+                        umma_commit(&B->a_done[sa]);
+                        if (!resident) {
+                            umma_commit(&B->b_done[sb]);
+                            ++gb;
+                        } else if (last) {
+                            umma_commit(&B->b_done[sb]);
+                        }
+                    }
+                    for (int mt = 0; mt < MT; ++mt) umma_commit(&B->d_full[r0 + mt]);
                 }
-                umma_commit(&B->d_full);
+                if (resident) gb += KB;
             }
             // Every MMA has completed once this barrier flips.
             umma_commit(&B->final_bar);
@@ -417,7 +533,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 size_t prefill_smem(int E) {
-    return 1024 + kS * (kWStage + kBStage) + sizeof(Barriers) + kNMax * 4 + (E + 1) * 4 + 64;
+    return 1024 + kWRing + kSB * kBStage + sizeof(Barriers) + 2 * kNMax * 4 + kScales * 4 + (E + 1) * 4 + 64;
 }
 
 int num_sms() {
@@ -433,14 +549,17 @@ int num_sms() {
 
 }  // namespace
 
-bool ffn_prefill_supported(int H, int I) { return H % 128 == 0 && I % 64 == 0 && prefill_smem(MOE_MAX_E) <= 227 * 1024; }
+bool ffn_prefill_supported(int H, int I) { return H % 128 == 0 && I % 128 == 0 && prefill_smem(MOE_MAX_E) <= 227 * 1024; }
 
 cudaError_t launch_ffn_prefill(const FfnArgs& a, cudaStream_t stream) {
     const uint64_t E = static_cast<uint64_t>(a.ex.n), I = a.ex.inter, H = a.H;
-    CUtensorMap tg, tu, td;
-    cudaError_t err = make_tmap_u8_2d(&tg, a.ex.w_gate, E * I, H, 64, 64, 64);
-    if (err == cudaSuccess) err = make_tmap_u8_2d(&tu, a.ex.w_up, E * I, H, 64, 64, 64);
+    const uint64_t rows = a.identity ? static_cast<uint64_t>(a.T) : static_cast<uint64_t>(a.T) * a.K;
+    CUtensorMap tg, tu, td, tx, th;
+    cudaError_t err = make_tmap_u8_2d(&tg, a.ex.w_gate, E * I, H, 64, 128, 64);
+    if (err == cudaSuccess) err = make_tmap_u8_2d(&tu, a.ex.w_up, E * I, H, 64, 128, 64);
     if (err == cudaSuccess) err = make_tmap_u8_2d(&td, a.ex.w_down, E * H, I, 64, 128, 64);
+    if (err == cudaSuccess) err = make_tmap_bf16_2d(&tx, a.x, static_cast<uint64_t>(a.T), H, 64, 1);
+    if (err == cudaSuccess) err = make_tmap_bf16_2d(&th, a.h, rows, I, 64, kNMax);
     if (err != cudaSuccess) return err;
     const size_t smem = prefill_smem(a.identity ? 1 : a.ex.n);
     err = cudaFuncSetAttribute(prefill_kernel<kGateUp>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
@@ -448,7 +567,7 @@ cudaError_t launch_ffn_prefill(const FfnArgs& a, cudaStream_t stream) {
         err = cudaFuncSetAttribute(prefill_kernel<kDown>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (err != cudaSuccess) return err;
     const int grid = num_sms();
-    prefill_kernel<kGateUp><<<grid, kThreads, smem, stream>>>(tg, tu, a);
+    prefill_kernel<kGateUp><<<grid, kThreads, smem, stream>>>(tg, tu, tx, a);
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
     cudaLaunchConfig_t cfg = {};
@@ -461,7 +580,7 @@ cudaError_t launch_ffn_prefill(const FfnArgs& a, cudaStream_t stream) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, prefill_kernel<kDown>, td, td, a);
+    return cudaLaunchKernelEx(&cfg, prefill_kernel<kDown>, td, td, th, a);
 }
 
 }  // namespace moe

@@ -63,6 +63,9 @@ cudaError_t launch_ffn_decode(const FfnArgs& a, cudaStream_t stream);
 // {box_cols, box_rows}, 128-byte (default) or 64-byte swizzle.
 cudaError_t make_tmap_u8_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
                             uint32_t box_cols, uint32_t box_rows, int swizzle_bytes = 128);
+// 2-D row-major bf16 matrix [rows, cols], box {box_cols, box_rows}, 128-byte swizzle.
+cudaError_t make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                              uint32_t box_cols, uint32_t box_rows);
 
 // ---------------------------------------------------------------- expert FFN (prefill, tcgen05)
 cudaError_t launch_ffn_prefill(const FfnArgs& a, cudaStream_t stream);
