@@ -14,8 +14,8 @@
 // offsets (no host sync).  A tile is 128 weight rows x up to 192 token rows:
 //  * swap-AB: the weights are the M=128 operand A, the tokens the N operand B,
 //    so the FP8 decode writes tensor memory, not shared memory;
-//  * warp 0: the weight tile's FP8 bytes by TMA (64-byte swizzle), up to 8
-//    stages ahead;
+//  * warp 0: the weight tile's FP8 bytes by TMA in stages of 128 reduction
+//    columns (128-byte rows, 128-byte swizzle), 64 KB ahead;
 //  * warps 2-3: the token rows into the 128-byte-swizzled K-major layout the
 //    MMA reads -- x rows gathered through sorted_route by cp.async (each
 //    thread arrives on the stage's mbarrier when its copies land) for
@@ -31,7 +31,8 @@
 //  * epilogue warps 4-7: tcgen05.ld of D; gate/up rows are interleaved
 //    (row 2j = gate of feature j, row 2j+1 = up of feature j), so a lane pair
 //    holds gate and up of one feature and SwiGLU needs one shuffle; the down
-//    epilogue multiplies by the route weight.  bf16 results go to global.
+//    epilogue multiplies by the route weight.  bf16 results are staged in
+//    shared memory and leave as 16-byte row-contiguous stores.
 // Every mbarrier wait is bounded; an expired wait sets a CTA-wide abort flag
 // and every role runs to the end without waiting, so the CTA always reaches
 // the TMEM de-allocation.
@@ -42,10 +43,11 @@ namespace moe {
 
 namespace {
 
-constexpr int kSB = 6;                      // token stages
+constexpr int kSB = 4;                      // token stages
 constexpr int kNMax = 192;                  // token rows per tile (MMA N)
 constexpr int kBStage = kNMax * 128;        // token rows x 64 bf16 (128-byte swizzle)
-constexpr int kWRing = 64 * 1024;           // FP8 weight ring (64 reduction columns per stage)
+constexpr int kWRing = 64 * 1024;           // FP8 weight ring (128 reduction columns per TMA stage)
+constexpr int kORow = 288;                  // bytes per row of the bf16 output staging tile (256 + pad)
 // Per mode: M-tiles (128 weight rows each) per step, weight stage bytes and
 // depths of the weight ring and of the bf16 A ring in TMEM.
 template <int MODE> struct Cfg;
@@ -60,17 +62,19 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kDRegion = kNMax;        // two accumulator regions of kNMax columns
 constexpr uint32_t kACol = 2 * kNMax;       // A ring: 128 columns
 constexpr int kDownGroup = 16;                  // output blocks sharing a resident token tile (down)
-constexpr int kScales = 1024;                   // staged block scales per item (floats)
+constexpr int kScales = 512;                    // staged block scales per item (floats)
 
 enum Mode { kGateUp = 0, kDown = 1 };
 
 // gate/up: a step feeds two M-tiles (gate and up rows of 128 features, two
 // accumulator regions); down: one M-tile per step, regions double-buffered.
+// A weight stage holds 128 reduction columns (128-byte rows) and feeds two
+// 64-column MMA steps.
 template <> struct Cfg<0> {
-    static constexpr int MT = 2, kWStage = 2 * 128 * 64, kSW = kWRing / kWStage, kSA = 2;
+    static constexpr int MT = 2, kWStage = 2 * 128 * 128, kSW = kWRing / kWStage, kSA = 2;
 };
 template <> struct Cfg<1> {
-    static constexpr int MT = 1, kWStage = 128 * 64, kSW = kWRing / kWStage, kSA = 4;
+    static constexpr int MT = 1, kWStage = 128 * 128, kSW = kWRing / kWStage, kSA = 4;
 };
 constexpr int kSWMax = 8, kSAMax = 4;
 
@@ -198,19 +202,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr int MT = C::MT, kSW = C::kSW, kSA = C::kSA, kWStage = C::kWStage;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = align1024(smem_raw);
-    uint8_t* w_ring = sm;                          // kSW x kWStage (64 KB)
-    uint8_t* b_ring = w_ring + kWRing;             // kSB x 24 KB
-    Barriers* B = reinterpret_cast<Barriers*>(b_ring + kSB * kBStage);
-    int* row_tok = reinterpret_cast<int*>(B + 1);  // [kNMax] activation row of each tile row
+    uint8_t* w_ring = sm;                              // kSW x kWStage (64 KB)
+    uint8_t* b_ring = w_ring + kWRing;                 // kSB x 24 KB
+    uint8_t* otile = b_ring + kSB * kBStage;           // [kNMax][kORow] bf16 output staging
+    Barriers* B = reinterpret_cast<Barriers*>(otile + kNMax * kORow);
+    int* row_tok = reinterpret_cast<int*>(B + 1);      // [kNMax] activation row of each tile row
     float* col_w = reinterpret_cast<float*>(row_tok + kNMax);  // [kNMax] route weight of each column (down)
     float* sc_sm = col_w + kNMax;                              // [kScales] block scales of the item
     int* pre = reinterpret_cast<int*>(sc_sm + kScales);        // [E + 1]
 
     const int H = a.H, I = a.ex.inter;
     const int Kred = MODE == kGateUp ? H : I;       // reduction length
-    const int KB = Kred / 64;                       // stages per output block
-    const int KB128 = Kred / 128;                   // scale blocks along the reduction
-    // Output blocks: gate/up -> 128 features (gate + up rows); down -> 128 features.
+    const int KB = Kred / 64;                       // MMA steps (64 columns) per output block
+    const int KB128 = Kred / 128;                   // scale blocks = weight TMA stages per output block
+    // Output blocks: 128 features (gate/up: their gate and up rows).
     const int FB = MODE == kGateUp ? I / 128 : H / 128;
     // The down GEMM keeps its token tile resident across a group of output
     // blocks when the whole reduction fits in the token ring.
@@ -255,22 +260,22 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_prefetch_desc(&tm_w0);
             if (MODE == kGateUp) tma_prefetch_desc(&tm_w1);
             const uint64_t policy = l2_evict_first_policy();
-            long g = 0;
+            long g = 0;  // weight stages (128 columns)
             for (int item = blockIdx.x; item < total; item += gridDim.x) {
                 const Tile t = tile_of(a, pre, FB, GFB, item);
                 for (int f = 0; f < t.nfb; ++f) {
                     const int fb = t.fb0 + f;
-                    for (int kb = 0; kb < KB; ++kb, ++g) {
+                    for (int kw = 0; kw < KB128; ++kw, ++g) {
                         const int s = static_cast<int>(g % kSW);
                         if (g >= kSW) wait_bar(&B->w_empty[s], static_cast<uint32_t>((g / kSW - 1) & 1), B, a.status);
                         uint8_t* dst = w_ring + s * kWStage;
                         mbar_arrive_expect_tx(&B->w_full[s], kWStage);
                         if (MODE == kGateUp) {
                             const int row = t.e * I + fb * 128;  // 128 gate rows, 128 up rows
-                            tma_load_2d_hint(dst, &tm_w0, &B->w_full[s], kb * 64, row, policy);
-                            tma_load_2d_hint(dst + kWStage / 2, &tm_w1, &B->w_full[s], kb * 64, row, policy);
+                            tma_load_2d_hint(dst, &tm_w0, &B->w_full[s], kw * 128, row, policy);
+                            tma_load_2d_hint(dst + kWStage / 2, &tm_w1, &B->w_full[s], kw * 128, row, policy);
                         } else {
-                            tma_load_2d_hint(dst, &tm_w0, &B->w_full[s], kb * 64, t.e * H + fb * 128, policy);
+                            tma_load_2d_hint(dst, &tm_w0, &B->w_full[s], kw * 128, t.e * H + fb * 128, policy);
                         }
                     }
                 }
@@ -331,12 +336,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp >= kWarpXform) {
         // ------------------------------------------------ transform: FP8 -> bf16 -> TMEM (A)
         // gate/up: warp (q, mt) owns lane quarter q of M-tile mt and all 64 codes
-        // of a stage; down: warp (q, hf) owns lane quarter q and half of the codes.
+        // of a step; down: warp (q, hf) owns lane quarter q and half of the codes.
         const int q = warp & 3, hi = (warp - kWarpXform) >> 2;
         const int xt = threadIdx.x - kWarpXform * 32;           // 0..255
         const int row = 32 * q + lane;  // TMEM lane = weight row of the M-tile
-        constexpr int NW = MODE == kGateUp ? 32 : 16;           // words (bf16 pairs) per thread per stage
-        long g = 0;
+        constexpr int NW = MODE == kGateUp ? 32 : 16;           // words (bf16 pairs) per thread per step
+        long g = 0;                                             // MMA steps (64 columns)
         for (int item = blockIdx.x; item < total; item += gridDim.x) {
             const Tile t = tile_of(a, pre, FB, GFB, item);
             // Block scales of the item, staged once: gate/up -> [gate, up][KB128],
@@ -358,24 +363,24 @@ __global__ void __launch_bounds__(kThreads, 1)
             // (gate j, up j) pairs, j = feature within the M-tile.
             const int srow = MODE == kGateUp ? hi * 64 + (row >> 1) : row;
             const int sub = (MODE == kGateUp && (row & 1)) ? kWStage / 2 : 0;
-            const int c0 = MODE == kGateUp ? 0 : 2 * hi;  // first 16-byte chunk of this thread
+            const int c0 = MODE == kGateUp ? 0 : 2 * hi;  // first 16-byte chunk of this thread in a step
             for (int f = 0; f < t.nfb; ++f) {
                 const float* scr = sc_sm + (MODE == kGateUp ? (row & 1) * KB128 : f * KB128);
                 for (int kb = 0; kb < KB; ++kb, ++g) {
-                    const int sw = static_cast<int>(g % kSW), sa = static_cast<int>(g % kSA);
-                    const bool ok1 = wait_bar(&B->w_full[sw], static_cast<uint32_t>((g / kSW) & 1), B, a.status);
+                    const long gw = g >> 1;  // weight stage holding this step
+                    const int sw = static_cast<int>(gw % kSW), sa = static_cast<int>(g % kSA);
+                    const bool ok1 = wait_bar(&B->w_full[sw], static_cast<uint32_t>((gw / kSW) & 1), B, a.status);
                     bool ok2 = true;
                     if (g >= kSA)
                         ok2 = wait_bar(&B->a_done[sa], static_cast<uint32_t>((g / kSA - 1) & 1), B, a.status);
                     uint32_t v[NW];
                     if (ok1 && ok2) {
                         const float sc = scr[kb >> 1];
-                        const uint8_t* base = w_ring + sw * kWStage + sub + srow * 64;
+                        const uint8_t* base = w_ring + sw * kWStage + sub + srow * 128;
 #pragma unroll
                         for (int c = 0; c < NW / 8; ++c) {
-                            const int chunk = c0 + c;
-                            const uint4 w =
-                                *reinterpret_cast<const uint4*>(base + ((chunk ^ ((srow >> 1) & 3)) << 4));
+                            const int chunk = (g & 1) * 4 + c0 + c;
+                            const uint4 w = *reinterpret_cast<const uint4*>(base + ((chunk ^ (srow & 7)) << 4));
                             const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
                             for (int k = 0; k < 4; ++k) {
@@ -388,7 +393,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int k = 0; k < NW; ++k) v[k] = 0;
                     }
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&B->w_empty[sw]);
+                    if ((g & 1) && lane == 0) mbar_arrive(&B->w_empty[sw]);
                     const uint32_t acol = kACol + sa * (MT * 32) + (MODE == kGateUp ? hi * 32 : hi * 16);
                     if constexpr (MODE == kGateUp)
                         tmem_st32(tmem + (static_cast<uint32_t>(32 * q) << 16) + acol, v);
@@ -403,10 +408,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp >= kWarpEpi) {
         // ------------------------------------------------ epilogue
+        // bf16 results go through the staging tile (row = token column, 128
+        // features) and leave as 16-byte row-contiguous stores.
         const int q = warp & 3;
+        const int et = threadIdx.x - kWarpEpi * 32;  // 0..127
         int uses[2] = {0, 0};
         int tc = 0;
-        const int et = threadIdx.x - kWarpEpi * 32;  // 0..127
         for (int item = blockIdx.x; item < total; item += gridDim.x) {
             const Tile t = tile_of(a, pre, FB, GFB, item);
             if (MODE == kDown) {
@@ -428,43 +435,53 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const bool ok = wait_bar(&B->d_full[r], static_cast<uint32_t>(uses[r] & 1), B, a.status);
                     ++uses[r];
                     tc_fence_after();
-                    const uint32_t dcol = r * kDRegion;
-                    for (int c0 = 0; c0 < t.n; c0 += 32) {
-                        uint32_t v[32];
-                        tmem_ld32(tmem + (static_cast<uint32_t>(32 * q) << 16) + dcol + c0, v);
+                    const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * q) << 16) + r * kDRegion;
+                    for (int c0 = 0; c0 < t.n; c0 += 64) {
+                        uint32_t v[64];
+                        tmem_ld32(taddr + c0, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+                        tmem_ld32(taddr + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
                         tmem_ld_wait();
                         if (!ok) continue;
                         if (MODE == kGateUp) {
-                            // Lane 2j: gate of feature j; lane 2j+1: up of feature j.
-                            // Even lanes write column c, odd lanes column c+1.
-                            const int feat = t.fb0 * 128 + mt * 64 + 16 * q + (lane >> 1);
+                            // Lane 2j: gate of feature j; lane 2j+1: up of feature j.  Even
+                            // lanes produce column c, odd lanes column c+1.
+                            const int feat = mt * 64 + 16 * q + (lane >> 1);  // within the 128-feature block
                             const bool odd = lane & 1;
 #pragma unroll
-                            for (int c = 0; c < 32; c += 2) {
+                            for (int c = 0; c < 64; c += 2) {
                                 const float x0 = __uint_as_float(v[c]), x1 = __uint_as_float(v[c + 1]);
                                 const float y0 = __shfl_xor_sync(0xffffffffu, x0, 1);
                                 const float y1 = __shfl_xor_sync(0xffffffffu, x1, 1);
                                 const float gte = odd ? y1 : x0, up = odd ? x1 : y0;
                                 const int col = c0 + c + (odd ? 1 : 0);
-                                if (col < t.n)
-                                    a.h[static_cast<size_t>(t.p0 + col) * I + feat] =
-                                        __bfloat16_as_ushort(__float2bfloat16_rn(silu_f32(gte) * up));
+                                const float hv = __fdividef(gte, 1.0f + __expf(-gte)) * up;
+                                *reinterpret_cast<uint16_t*>(otile + col * kORow + feat * 2) =
+                                    __bfloat16_as_ushort(__float2bfloat16_rn(hv));
                             }
                         } else {
-                            const int feat = (t.fb0 + f) * 128 + 32 * q + lane;
+                            const int feat = 32 * q + lane;
 #pragma unroll
-                            for (int c = 0; c < 32; ++c) {
-                                const float wv = col_w[c0 + c];
-                                if (c0 + c < t.n)
-                                    a.y[static_cast<size_t>(t.p0 + c0 + c) * H + feat] =
-                                        __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[c]) * wv));
-                            }
+                            for (int c = 0; c < 64; ++c)
+                                *reinterpret_cast<uint16_t*>(otile + (c0 + c) * kORow + feat * 2) =
+                                    __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[c]) * col_w[c0 + c]));
                         }
                     }
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&B->d_empty[r]);
                 }
+                // Staging tile -> global, 16 bytes per thread, rows of 256 bytes.
+                named_barrier_sync(4, 128);
+                const int fb = t.fb0 + f;
+                uint16_t* dst = MODE == kGateUp ? a.h + static_cast<size_t>(t.p0) * I + fb * 128
+                                                : a.y + static_cast<size_t>(t.p0) * H + fb * 128;
+                const int stride = MODE == kGateUp ? I : H;
+                for (int i = et; i < t.n * 16; i += 128) {
+                    const int rr = i >> 4, ch = i & 15;
+                    *reinterpret_cast<uint4*>(dst + static_cast<size_t>(rr) * stride + ch * 8) =
+                        *reinterpret_cast<const uint4*>(otile + rr * kORow + ch * 16);
+                }
+                named_barrier_sync(4, 128);
             }
         }
     } else if (warp == kWarpMma) {
@@ -504,7 +521,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                             for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
                                 for (int k = 0; k < 4; ++k)
-                                    umma_ts_f16(tmem + (r0 + mt) * kDRegion, tmem + kACol + sa * (MT * 32) + mt * 32 + k * 8,
+                                    umma_ts_f16(tmem + (r0 + mt) * kDRegion,
+                                                tmem + kACol + sa * (MT * 32) + mt * 32 + k * 8,
                                                 umma_desc_sw128(bbase + k * 32), idesc, (kb > 0 || k > 0) ? 1u : 0u);
                         }
                         umma_commit(&B->a_done[sa]);
@@ -533,7 +551,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 size_t prefill_smem(int E) {
-    return 1024 + kWRing + kSB * kBStage + sizeof(Barriers) + 2 * kNMax * 4 + kScales * 4 + (E + 1) * 4 + 64;
+    return 1024 + kWRing + kSB * kBStage + kNMax * kORow + sizeof(Barriers) + 2 * kNMax * 4 + kScales * 4 +
+           (E + 1) * 4 + 64;
 }
 
 int num_sms() {
@@ -555,9 +574,9 @@ cudaError_t launch_ffn_prefill(const FfnArgs& a, cudaStream_t stream) {
     const uint64_t E = static_cast<uint64_t>(a.ex.n), I = a.ex.inter, H = a.H;
     const uint64_t rows = a.identity ? static_cast<uint64_t>(a.T) : static_cast<uint64_t>(a.T) * a.K;
     CUtensorMap tg, tu, td, tx, th;
-    cudaError_t err = make_tmap_u8_2d(&tg, a.ex.w_gate, E * I, H, 64, 128, 64);
-    if (err == cudaSuccess) err = make_tmap_u8_2d(&tu, a.ex.w_up, E * I, H, 64, 128, 64);
-    if (err == cudaSuccess) err = make_tmap_u8_2d(&td, a.ex.w_down, E * H, I, 64, 128, 64);
+    cudaError_t err = make_tmap_u8_2d(&tg, a.ex.w_gate, E * I, H, 128, 128);
+    if (err == cudaSuccess) err = make_tmap_u8_2d(&tu, a.ex.w_up, E * I, H, 128, 128);
+    if (err == cudaSuccess) err = make_tmap_u8_2d(&td, a.ex.w_down, E * H, I, 128, 128);
     if (err == cudaSuccess) err = make_tmap_bf16_2d(&tx, a.x, static_cast<uint64_t>(a.T), H, 64, 1);
     if (err == cudaSuccess) err = make_tmap_bf16_2d(&th, a.h, rows, I, 64, kNMax);
     if (err != cudaSuccess) return err;
