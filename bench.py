@@ -175,6 +175,30 @@ def cpu_baseline(shape, budget_s=10.0):
                       % (n, len(tk), dt)}
 
 
+# ---------------------------------------------------------------- replicas
+
+def dist_env():
+    """(rank, world size, local rank) from the torchrun environment (1 process: 0, 1, 0)."""
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def max_over_ranks(v, device="cpu"):
+    """Largest v over all ranks of the process group (v itself without one)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(v)
+    t = torch.tensor([float(v)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.item()
+
+
+def job_tokens_per_s(T, world, ms_per_step):
+    """Whole-job throughput: every replica processes T tokens per step."""
+    return T * world / (ms_per_step * 1e-3)
+
+
 def config_of(shape):
     return {"workload": shape.name, "T": shape.T, "H": shape.H, "I": shape.I, "E": shape.E, "K": shape.K,
             "I_shared": shape.I_shared, "weights": "fp8 e4m3fn, fp32 scale per 128x128 block",
@@ -197,9 +221,7 @@ def main():
                     help="launch every call directly instead of replaying CUDA graphs (for profilers)")
     args = ap.parse_args()
     shape = wl.SHAPES[args.workload]
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    rank, world, local = dist_env()
 
     if args.impl == "reference":
         if args.steps is None:
@@ -304,11 +326,7 @@ def main():
             stream.synchronize()
             for i, k in enumerate(parts):
                 parts[k].append(ev[i].elapsed_time(ev[i + 1]))
-    t_max = t_local
-    if world > 1:
-        tt = torch.tensor([t_local], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        t_max = tt.item()
+    t_max = max_over_ranks(t_local, dev)
 
     # End to end through the public API with host buffers: pinned x and logits
     # copied in, the layer output copied back, every step.
@@ -328,11 +346,7 @@ def main():
             oh.copy_(layer.out, non_blocking=True)
         e1.record()
     torch.cuda.synchronize(dev)
-    e2e_ms = e0.elapsed_time(e1) / n_e2e
-    if world > 1:
-        tt = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = tt.item()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / n_e2e, dev)
     if layer.status.item() != 0:
         raise RuntimeError("status word %d after the timed region" % layer.status.item())
 
@@ -342,7 +356,7 @@ def main():
     ffn_ms = statistics.median(parts["ffn"])
     R_nz = int(np.count_nonzero(layer.topk_w.cpu().numpy()))
     flops = (R_nz + (T if shape.I_shared else 0)) * 6 * H * I
-    decode_path = (args.mode == 1) or (args.mode == 0 and T * K <= 8192)
+    decode_path = moe.moe_ffn_resolve_mode(T, K, E, args.mode) == moe.MOE_MODE_DECODE
     if decode_path:
         algo = touched * expert_bytes(H, I) + (expert_bytes(H, shape.I_shared) if shape.I_shared else 0)
         ach = algo / (ffn_ms * 1e-3) / 1e9
@@ -358,7 +372,7 @@ def main():
                 "traffic": profile_traffic(shape.name, "prefill"), "kernel": "moe_expert_ffn", "flops": flops,
                 "peak_source": peaks["src"] + " sustained"}
     n_launch = layer.launches()
-    out = {"metric": METRIC, "value": T * world / (t_max * 1e-3), "unit": UNIT, "n_gpus": world,
+    out = {"metric": METRIC, "value": job_tokens_per_s(T, world, t_max), "unit": UNIT, "n_gpus": world,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_max, "higher_is_better": True,
            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
            "config": dict(config_of(shape), parallelism="replicas x%d" % world,
@@ -369,7 +383,7 @@ def main():
                               args.steps, "eager launches" if args.eager else "CUDA-graph replays")),
            "roofline": roof,
            "breakdown_ms": {k: statistics.median(v) for k, v in parts.items()},
-           "e2e": {"value": T * world / (e2e_ms * 1e-3), "unit": UNIT,
+           "e2e": {"value": job_tokens_per_s(T, world, e2e_ms), "unit": UNIT,
                    "h2d_bytes_per_step": x.numel() * 2 + logits.numel() * 4,
                    "d2h_bytes_per_step": layer.out.numel() * 2},
            "gpu_launches": n_launch * args.steps,

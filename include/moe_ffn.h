@@ -87,10 +87,11 @@ typedef enum moe_status {
 #define MOE_STATUS_BAD_MAP 2     /* offsets / route map out of range: rows skipped */
 
 /* moe_expert_ffn `mode`. */
-#define MOE_MODE_AUTO 0     /* DECODE when T*K <= MOE_DECODE_MAX_ROUTES, else PREFILL */
+#define MOE_MODE_AUTO 0     /* see moe_ffn_resolve_mode */
 #define MOE_MODE_DECODE 1   /* weight-streaming kernels (memory-bound regime) */
 #define MOE_MODE_PREFILL 2  /* tcgen05 / TMEM grouped GEMM kernels (compute-bound regime) */
 #define MOE_DECODE_MAX_ROUTES 8192
+#define MOE_DECODE_MAX_ROWS_PER_EXPERT 8
 
 /* moe_combine `out_dtype`. */
 #define MOE_OUT_BF16 0
@@ -204,6 +205,24 @@ typedef struct moe_fp8_experts {
 } moe_fp8_experts;
 
 /* ---------------------------------------------------------------------------
+ * moe_ffn_resolve_mode -- the FFN form moe_expert_ffn runs for a given mode.
+ *
+ * No counterpart on the pages (they pick a kernel per serving phase: the NKI
+ * library's MoE TKG for decode and MoE CTE for prefill).  Host-only, launches
+ * nothing.  DECODE and PREFILL resolve to themselves; AUTO resolves from
+ * host-known sizes alone (never from the device-side expert counts) to
+ *   MOE_MODE_DECODE   when T*K <= MOE_DECODE_MAX_ROUTES and
+ *                     T*K <= MOE_DECODE_MAX_ROWS_PER_EXPERT * E
+ *                     (few rows per expert: streaming the touched weights
+ *                     bounds the time),
+ *   MOE_MODE_PREFILL  otherwise (enough rows per expert for the tensor-core
+ *                     grouped GEMM to win).
+ * Returns the resolved mode, or MOE_ERR_INVALID_ARG for an unknown mode or
+ * T < 0, K < 1, E < 1.
+ * ------------------------------------------------------------------------- */
+MOE_API int moe_ffn_resolve_mode(int T, int K, int E, int mode);
+
+/* ---------------------------------------------------------------------------
  * moe_expert_ffn -- grouped expert FFN over the sorted routes.
  *
  * For every expert e and sorted position p in [expert_offsets[e],
@@ -228,6 +247,7 @@ typedef struct moe_fp8_experts {
  *   y_sorted       [T*K, H] bf16 (written for rows p < expert_offsets[E])
  *   y_shared       [T, H] bf16 (written) when shared != NULL, else ignored
  *   mode           MOE_MODE_AUTO | MOE_MODE_DECODE | MOE_MODE_PREFILL
+ *                  (AUTO as moe_ffn_resolve_mode resolves it)
  *   workspace      moe_ffn_workspace_bytes(...) bytes of device scratch
  *   status         optional device int32: MOE_STATUS_BAD_MAP is OR-ed in when
  *                  offsets or route ids are out of range (those rows skipped)

@@ -31,7 +31,7 @@ MOE_STATUS_BAD_ID, MOE_STATUS_BAD_MAP, MOE_STATUS_TIMEOUT = 1, 2, 4
 MOE_MAX_E, MOE_MAX_K = 1024, 32
 
 EXPORTED = ("moe_last_error", "moe_abi_version", "moe_route", "moe_sort_workspace_bytes", "moe_sort",
-            "moe_sort_static_ws", "moe_ffn_workspace_bytes", "moe_expert_ffn", "moe_combine")
+            "moe_sort_static_ws", "moe_ffn_resolve_mode", "moe_ffn_workspace_bytes", "moe_expert_ffn", "moe_combine")
 
 
 class MoEError(RuntimeError):
@@ -70,6 +70,8 @@ def lib() -> ctypes.CDLL:
             L.moe_sort.restype = I
             L.moe_sort_static_ws.argtypes = [P, I, I, I, P, P, P, P, P]
             L.moe_sort_static_ws.restype = I
+            L.moe_ffn_resolve_mode.argtypes = [I, I, I, I]
+            L.moe_ffn_resolve_mode.restype = I
             L.moe_ffn_workspace_bytes.argtypes = [I, I, I, I, I, I, I]
             L.moe_ffn_workspace_bytes.restype = S
             L.moe_expert_ffn.argtypes = [P, I, I, I, P, P, P, P, P, P, P, I, P, S, P, P]
@@ -176,6 +178,13 @@ def moe_sort(topk_ids: torch.Tensor, E: int, status: Optional[torch.Tensor] = No
                           _ptr(inv_route), _ptr(workspace), workspace.numel(), _ptr(status),
                           _stream(stream)))
     return expert_offsets, sorted_route, inv_route
+
+
+def moe_ffn_resolve_mode(T: int, K: int, E: int, mode: int = MOE_MODE_AUTO) -> int:
+    """The FFN form (MOE_MODE_DECODE or MOE_MODE_PREFILL) moe_expert_ffn runs for `mode`."""
+    rc = int(lib().moe_ffn_resolve_mode(T, K, E, mode))
+    _check(min(rc, 0))
+    return rc
 
 
 def moe_ffn_workspace_bytes(T, K, H, E, I, I_shared=0, mode=MOE_MODE_AUTO) -> int:

@@ -140,6 +140,19 @@ int moe_sort(const int32_t* topk_ids, int T, int K, int E, int32_t* expert_offse
     return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_sort launch");
 }
 
+int moe_ffn_resolve_mode(int T, int K, int E, int mode) {
+    g_err.clear();
+    if (T < 0 || K < 1 || E < 1)
+        return fail(MOE_ERR_INVALID_ARG, "moe_ffn_resolve_mode: T=%d, K=%d, E=%d out of range", T, K, E);
+    if (mode == MOE_MODE_DECODE || mode == MOE_MODE_PREFILL) return mode;
+    if (mode != MOE_MODE_AUTO)
+        return fail(MOE_ERR_INVALID_ARG, "moe_ffn_resolve_mode: mode=%d is not AUTO/DECODE/PREFILL", mode);
+    const long R = static_cast<long>(T) * K;
+    return R <= MOE_DECODE_MAX_ROUTES && R <= static_cast<long>(MOE_DECODE_MAX_ROWS_PER_EXPERT) * E
+               ? MOE_MODE_DECODE
+               : MOE_MODE_PREFILL;
+}
+
 size_t moe_ffn_workspace_bytes(int T, int K, int H, int E, int I, int I_shared, int mode) {
     (void)H;
     (void)E;
@@ -181,7 +194,7 @@ int moe_expert_ffn(const uint16_t* x, int T, int H, int K, const moe_fp8_experts
     if (workspace_bytes < need || !workspace)
         return fail(MOE_ERR_WORKSPACE_TOO_SMALL, "moe_expert_ffn: workspace of %zu bytes, need %zu",
                     workspace_bytes, need);
-    const bool prefill = mode == MOE_MODE_PREFILL || (mode == MOE_MODE_AUTO && R > MOE_DECODE_MAX_ROUTES);
+    const bool prefill = moe_ffn_resolve_mode(T, K, E, mode) == MOE_MODE_PREFILL;
     if (prefill && !moe::ffn_prefill_supported(H, I))
         return fail(MOE_ERR_UNSUPPORTED_SHAPE, "moe_expert_ffn: H=%d, inter=%d not supported by the PREFILL kernels", H, I);
 

@@ -55,6 +55,29 @@ def test_workspace_queries(L):
     assert L.moe_ffn_workspace_bytes(8192, 10, 4096, 512, 256, 256, 0) == 81920 * 512 + 8192 * 512
 
 
+def test_ffn_resolve_mode(L):
+    D, PF = moe.MOE_MODE_DECODE, moe.MOE_MODE_PREFILL
+    # Explicit modes resolve to themselves at any size.
+    assert L.moe_ffn_resolve_mode(32768, 10, 512, D) == D
+    assert L.moe_ffn_resolve_mode(1, 1, 8, PF) == PF
+    # AUTO: decode while routes per expert stay at most 8 and routes at most 8192.
+    assert L.moe_ffn_resolve_mode(16, 2, 8, 0) == D          # 4 routes per expert
+    assert L.moe_ffn_resolve_mode(64, 8, 256, 0) == D        # 2
+    assert L.moe_ffn_resolve_mode(256, 8, 256, 0) == D       # 8: the limit
+    assert L.moe_ffn_resolve_mode(257, 8, 256, 0) == PF
+    assert L.moe_ffn_resolve_mode(512, 8, 256, 0) == PF      # 16
+    assert L.moe_ffn_resolve_mode(1024, 8, 1024, 0) == D     # 8192 routes
+    assert L.moe_ffn_resolve_mode(1025, 8, 1024, 0) == PF    # 8200 routes
+    assert L.moe_ffn_resolve_mode(8192, 10, 512, 0) == PF
+    assert L.moe_ffn_resolve_mode(0, 8, 256, 0) == D
+    assert moe.moe_ffn_resolve_mode(512, 8, 256) == PF
+    for args in ((4, 2, 8, 3), (-1, 2, 8, 0), (4, 0, 8, 0), (4, 2, 0, 0)):
+        assert L.moe_ffn_resolve_mode(*args) == moe.MOE_ERR_INVALID_ARG
+        assert "moe_ffn_resolve_mode" in L.moe_last_error().decode()
+    with pytest.raises(moe.MoEError):
+        moe.moe_ffn_resolve_mode(4, 2, 8, 7)
+
+
 P = ctypes.c_void_p
 
 
