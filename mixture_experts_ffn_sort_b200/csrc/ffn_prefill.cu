@@ -19,7 +19,7 @@
 //  * warps 2-3: the token rows into the 128-byte-swizzled K-major layout the
 //    MMA reads -- x rows gathered through sorted_route by cp.async (each
 //    thread arrives on the stage's mbarrier when its copies land) for
-//    gate/up, contiguous rows of h as one 2-D TMA tile for down -- up to 6
+//    gate/up, contiguous rows of h as one 2-D TMA tile for down -- up to 4
 //    stages ahead;
 //  * transform warps 8-15: each thread owns one TMEM lane (one weight row)
 //    and half of a stage's columns, decodes its FP8 codes to
