@@ -341,6 +341,53 @@ __device__ __forceinline__ void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
+// ---------------------------------------------------------------- TMEM -> registers -> shared (transposed)
+
+// tcgen05.ld 16x256b, 4 repetitions: 16 TMEM lanes x 32 columns starting at
+// `taddr` (lane field = first of the 16 lanes).  Thread t receives, for column
+// group g = 0..3 (8 columns each): r[4g+0], r[4g+1] = lane t/4, columns
+// 8g + 2(t%4) and 8g + 2(t%4) + 1; r[4g+2], r[4g+3] = lane t/4 + 8, same
+// columns -- the accumulator fragment of mma m16n8.
+__device__ __forceinline__ void tmem_ld16x256b_x4(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x256b.x4.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+        "%14, %15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
+
+// Four 8x8 b16 matrices stored transposed: register i of thread t holds
+// elements (row t/4, columns 2(t%4), 2(t%4)+1) of matrix i; they are written
+// to rows 2(t%4), 2(t%4)+1, column t/4 of the stored matrix, whose row j sits
+// at the address given by thread 8i + j.
+__device__ __forceinline__ void stmatrix_x4_trans(uint32_t addr, uint32_t r0, uint32_t r1, uint32_t r2, uint32_t r3) {
+    asm volatile("stmatrix.sync.aligned.x4.trans.m8n8.shared.b16 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(r0),
+                 "r"(r1), "r"(r2), "r"(r3));
+}
+
+// ---------------------------------------------------------------- bulk stores (shared -> global)
+
+// Asynchronous copy of `bytes` (a multiple of 16, both addresses 16-byte
+// aligned) from shared to global memory, tracked by this thread's bulk group.
+// Generic-proxy writes to the source must be fenced (fence_proxy_async_smem)
+// before the copy is issued.
+__device__ __forceinline__ void bulk_store_s2g(void* dst, uint32_t src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(src), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until every committed bulk copy of this thread has finished reading its source.
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// Wait until every committed bulk copy of this thread has completed.
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// 16-bit shared store with no compiler memory clobber: lets the compiler keep
+// unrelated shared loads ahead of it (callers order it with barriers).
+__device__ __forceinline__ void st_shared_u16(uint32_t addr, uint16_t v) {
+    asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"(v));
+}
+
 // ---------------------------------------------------------------- misc
 
 __device__ __forceinline__ float silu_f32(float z) { return z / (1.0f + __expf(-z)); }

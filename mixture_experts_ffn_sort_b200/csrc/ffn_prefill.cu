@@ -18,9 +18,10 @@
 //    columns (128-byte rows, 128-byte swizzle), 64 KB ahead;
 //  * warps 2-3: the token rows into the 128-byte-swizzled K-major layout the
 //    MMA reads -- x rows gathered through sorted_route by cp.async (each
-//    thread arrives on the stage's mbarrier when its copies land) for
-//    gate/up, contiguous rows of h as one 2-D TMA tile for down -- up to 4
-//    stages ahead;
+//    thread keeps its rows' token indices in registers for the whole tile and
+//    arrives on the stage's mbarrier when its copies land) for gate/up,
+//    contiguous rows of h as one 2-D TMA tile for down -- up to 4 stages
+//    ahead;
 //  * transform warps 8-15: each thread owns one TMEM lane (one weight row)
 //    and half of a stage's columns, decodes its FP8 codes to
 //    bf16(e4m3 * block scale) and stores them to TMEM with tcgen05.st (A
@@ -28,11 +29,12 @@
 //  * warp 1: one thread issues tcgen05.mma (kind::f16, A in TMEM, B in
 //    shared memory, fp32 accumulator D in TMEM, double-buffered so the
 //    epilogue of one tile overlaps the main loop of the next);
-//  * epilogue warps 4-7: tcgen05.ld of D; gate/up rows are interleaved
-//    (row 2j = gate of feature j, row 2j+1 = up of feature j), so a lane pair
-//    holds gate and up of one feature and SwiGLU needs one shuffle; the down
+//  * epilogue warps 4-7: tcgen05.ld of D; in each 32-lane quarter of a
+//    gate/up M-tile, lanes 0-15 hold the gate rows and lanes 16-31 the up
+//    rows of the same 16 features, so SwiGLU needs one shuffle; the down
 //    epilogue multiplies by the route weight.  bf16 results are staged in
-//    shared memory and leave as 16-byte row-contiguous stores.
+//    shared memory (one row per token) and leave as one 256-byte bulk async
+//    copy per token row.
 // Every mbarrier wait is bounded; an expired wait sets a CTA-wide abort flag
 // and every role runs to the end without waiting, so the CTA always reaches
 // the TMEM de-allocation.
@@ -47,7 +49,7 @@ constexpr int kSB = 4;                      // token stages
 constexpr int kNMax = 192;                  // token rows per tile (MMA N)
 constexpr int kBStage = kNMax * 128;        // token rows x 64 bf16 (128-byte swizzle)
 constexpr int kWRing = 64 * 1024;           // FP8 weight ring (128 reduction columns per TMA stage)
-constexpr int kORow = 288;                  // bytes per row of the bf16 output staging tile (256 + pad)
+constexpr int kORow = 272;                  // bytes per row of the bf16 output staging tile (256 + pad)
 // Per mode: M-tiles (128 weight rows each) per step, weight stage bytes and
 // depths of the weight ring and of the bf16 A ring in TMEM.
 template <int MODE> struct Cfg;
@@ -230,7 +232,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&B->w_empty[s], kXformWarps);
         }
         for (int s = 0; s < kSB; ++s) {
-            mbar_init(&B->b_full[s], MODE == kGateUp ? kTokThreads : 1);
+            mbar_init(&B->b_full[s], 1);
             mbar_init(&B->b_done[s], 1);
         }
         for (int s = 0; s < kSA; ++s) {
@@ -289,8 +291,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         // Padding rows of the last MMA column group are left stale: column j of
         // D depends on token row j only, and the epilogue drops those columns.
         const int lt = threadIdx.x - kWarpTok * 32;  // 0..63
+        // gate/up: thread lt gathers rows 4lt .. 4lt+3 of the tile (one
+        // tile::gather4 per stage); rows past the tile's end repeat a valid
+        // token and land in padding rows the epilogue drops.
+        uint32_t tok[4] = {0, 0, 0, 0};
+        int ngroups = 0;
         if (MODE == kDown) grid_dependency_wait();  // h comes from the gate/up grid
-        if (MODE == kDown && lt == 0) tma_prefetch_desc(&tm_act);
+        if (lt == 0) tma_prefetch_desc(&tm_act);
         long g = 0;
         for (int item = blockIdx.x; item < total; item += gridDim.x) {
             const Tile t = tile_of(a, pre, FB, GFB, item);
@@ -298,41 +305,43 @@ __global__ void __launch_bounds__(kThreads, 1)
                 named_barrier_sync(2, kTokThreads);
                 bool bad = false;
                 for (int r = lt; r < t.n; r += kTokThreads) {
-                    int tok = 0;
+                    int tk = 0;
                     const long p = t.p0 + r;
                     if (a.identity) {
-                        tok = static_cast<int>(p);
+                        tk = static_cast<int>(p);
                     } else {
                         const int rt = a.sorted_route[p];
                         if (rt >= 0 && rt < R)
-                            tok = rt / a.K;
+                            tk = rt / a.K;
                         else
                             bad = true;
                     }
-                    row_tok[r] = tok;
+                    row_tok[r] = tk;
                 }
                 if (bad) report_status(a.status, MOE_STATUS_BAD_MAP);
                 named_barrier_sync(2, kTokThreads);
+                ngroups = (t.n + 3) >> 2;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int r = 4 * lt + i;
+                    tok[i] = static_cast<uint32_t>(row_tok[r < t.n ? r : 0]);
+                }
             }
             for (int kb = 0; kb < KB; ++kb, ++g) {
                 const int s = static_cast<int>(g % kSB);
                 if (g >= kSB) wait_bar(&B->b_done[s], static_cast<uint32_t>((g / kSB - 1) & 1), B, a.status);
                 uint8_t* dst = b_ring + s * kBStage;
                 if (MODE == kGateUp) {
-                    const uint32_t bdst = smem_u32(dst);
-                    for (int ci = lt; ci < t.n * 8; ci += kTokThreads) {
-                        const int r = ci >> 3, ch = ci & 7;
-                        const uint16_t* src = a.x + static_cast<size_t>(row_tok[r]) * H + kb * 64 + ch * 8;
-                        cp_async16(bdst + r * 128 + ((ch ^ (r & 7)) << 4), src, 16u);
-                    }
-                    cp_async_arrive_noinc(&B->b_full[s]);
+                    if (lt == 0) mbar_arrive_expect_tx(&B->b_full[s], static_cast<uint32_t>(ngroups) * 512u);
+                    if (lt < ngroups)
+                        tma_gather4(dst + lt * 512, &tm_act, &B->b_full[s], kb * 64, static_cast<int>(tok[0]),
+                                    static_cast<int>(tok[1]), static_cast<int>(tok[2]), static_cast<int>(tok[3]));
                 } else if (lt == 0) {
                     mbar_arrive_expect_tx(&B->b_full[s], kBStage);
                     tma_load_2d(dst, &tm_act, &B->b_full[s], kb * 64, static_cast<int>(t.p0));
                 }
             }
         }
-        if (MODE == kGateUp) cp_async_wait<0>();
     } else if (warp >= kWarpXform) {
         // ------------------------------------------------ transform: FP8 -> bf16 -> TMEM (A)
         // gate/up: warp (q, mt) owns lane quarter q of M-tile mt and all 64 codes
@@ -359,13 +368,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             named_barrier_sync(3, kXformWarps * 32);
-            // Source row in the weight stage: gate/up rows interleave as
-            // (gate j, up j) pairs, j = feature within the M-tile.
-            const int srow = MODE == kGateUp ? hi * 64 + (row >> 1) : row;
-            const int sub = (MODE == kGateUp && (row & 1)) ? kWStage / 2 : 0;
+            // Source row in the weight stage.  gate/up: in the lane quarter of
+            // warp q, lanes 0-15 hold the gate rows and lanes 16-31 the up rows
+            // of features 16q .. 16q+15 of the M-tile (so the eight lanes of a
+            // shared-memory phase read eight different rows).
+            const bool up_row = MODE == kGateUp && (lane & 16);
+            const int srow = MODE == kGateUp ? hi * 64 + 16 * q + (lane & 15) : row;
+            const int sub = up_row ? kWStage / 2 : 0;
             const int c0 = MODE == kGateUp ? 0 : 2 * hi;  // first 16-byte chunk of this thread in a step
             for (int f = 0; f < t.nfb; ++f) {
-                const float* scr = sc_sm + (MODE == kGateUp ? (row & 1) * KB128 : f * KB128);
+                const float* scr = sc_sm + (MODE == kGateUp ? (up_row ? KB128 : 0) : f * KB128);
                 for (int kb = 0; kb < KB; ++kb, ++g) {
                     const long gw = g >> 1;  // weight stage holding this step
                     const int sw = static_cast<int>(gw % kSW), sa = static_cast<int>(g % kSA);
@@ -412,6 +424,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // features) and leave as 16-byte row-contiguous stores.
         const int q = warp & 3;
         const int et = threadIdx.x - kWarpEpi * 32;  // 0..127
+        const uint32_t otile_u32 = smem_u32(otile);
         int uses[2] = {0, 0};
         int tc = 0;
         for (int item = blockIdx.x; item < total; item += gridDim.x) {
@@ -435,55 +448,84 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const bool ok = wait_bar(&B->d_full[r], static_cast<uint32_t>(uses[r] & 1), B, a.status);
                     ++uses[r];
                     tc_fence_after();
-                    const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * q) << 16) + r * kDRegion;
-                    for (int c0 = 0; c0 < t.n; c0 += 64) {
-                        uint32_t v[64];
-                        tmem_ld32(taddr + c0, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-                        tmem_ld32(taddr + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
-                        tmem_ld_wait();
-                        if (!ok) continue;
+                    if (mt == 0) {
+                        // The staging tile is free once the previous block's row
+                        // copies have read it.
+                        bulk_wait_read0();
+                        named_barrier_sync(4, 128);
+                    }
+                    const uint32_t tl = tmem + (static_cast<uint32_t>(32 * q) << 16) + r * kDRegion;
+                    for (int c0 = 0; c0 < t.n; c0 += 32) {
                         if (MODE == kGateUp) {
-                            // Lane 2j: gate of feature j; lane 2j+1: up of feature j.  Even
-                            // lanes produce column c, odd lanes column c+1.
-                            const int feat = mt * 64 + 16 * q + (lane >> 1);  // within the 128-feature block
-                            const bool odd = lane & 1;
+                            // Lanes 32q+0..15 hold the gate rows, 32q+16..31 the up rows of
+                            // features 16q..16q+15 of the M-tile: thread t gets gate and up
+                            // of the same (feature, token) pairs.
+                            uint32_t gv[16], uv[16];
+                            tmem_ld16x256b_x4(tl + c0, gv);
+                            tmem_ld16x256b_x4(tl + (16u << 16) + c0, uv);
+                            tmem_ld_wait();
+                            if (!ok) continue;
+                            uint32_t pk[8];
 #pragma unroll
-                            for (int c = 0; c < 64; c += 2) {
-                                const float x0 = __uint_as_float(v[c]), x1 = __uint_as_float(v[c + 1]);
-                                const float y0 = __shfl_xor_sync(0xffffffffu, x0, 1);
-                                const float y1 = __shfl_xor_sync(0xffffffffu, x1, 1);
-                                const float gte = odd ? y1 : x0, up = odd ? x1 : y0;
-                                const int col = c0 + c + (odd ? 1 : 0);
-                                const float hv = __fdividef(gte, 1.0f + __expf(-gte)) * up;
-                                *reinterpret_cast<uint16_t*>(otile + col * kORow + feat * 2) =
-                                    __bfloat16_as_ushort(__float2bfloat16_rn(hv));
+                            for (int k = 0; k < 8; ++k) {
+                                float hv[2];
+#pragma unroll
+                                for (int j = 0; j < 2; ++j) {
+                                    const float z = __uint_as_float(gv[2 * k + j]);
+                                    hv[j] = __fdividef(z, 1.0f + __expf(-z)) * __uint_as_float(uv[2 * k + j]);
+                                }
+                                pk[k] = pack_bf16x2(hv[0], hv[1]);
                             }
+                            const uint32_t o = otile_u32 + (c0 + 8 * (lane >> 4) + (lane & 7)) * kORow +
+                                               (mt * 64 + 16 * q + 8 * ((lane >> 3) & 1)) * 2;
+                            stmatrix_x4_trans(o, pk[0], pk[1], pk[2], pk[3]);
+                            stmatrix_x4_trans(o + 16 * kORow, pk[4], pk[5], pk[6], pk[7]);
                         } else {
-                            const int feat = 32 * q + lane;
+                            uint32_t dv[2][16];
+                            tmem_ld16x256b_x4(tl + c0, dv[0]);
+                            tmem_ld16x256b_x4(tl + (16u << 16) + c0, dv[1]);
+                            tmem_ld_wait();
+                            if (!ok) continue;
+                            // Route weights of this thread's tokens c0 + 8g + 2(t%4) + {0, 1}.
+                            float2 wv[4];
 #pragma unroll
-                            for (int c = 0; c < 64; ++c)
-                                *reinterpret_cast<uint16_t*>(otile + (c0 + c) * kORow + feat * 2) =
-                                    __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[c]) * col_w[c0 + c]));
+                            for (int gq = 0; gq < 4; ++gq)
+                                wv[gq] = *reinterpret_cast<const float2*>(col_w + c0 + 8 * gq + 2 * (lane & 3));
+#pragma unroll
+                            for (int hf = 0; hf < 2; ++hf) {
+                                uint32_t pk[8];
+#pragma unroll
+                                for (int gq = 0; gq < 4; ++gq) {
+                                    const uint32_t* d = dv[hf] + 4 * gq;
+                                    pk[2 * gq] = pack_bf16x2(__uint_as_float(d[0]) * wv[gq].x,
+                                                             __uint_as_float(d[1]) * wv[gq].y);
+                                    pk[2 * gq + 1] = pack_bf16x2(__uint_as_float(d[2]) * wv[gq].x,
+                                                                 __uint_as_float(d[3]) * wv[gq].y);
+                                }
+                                const uint32_t o = otile_u32 + (c0 + 8 * (lane >> 4) + (lane & 7)) * kORow +
+                                                   (32 * q + 16 * hf + 8 * ((lane >> 3) & 1)) * 2;
+                                stmatrix_x4_trans(o, pk[0], pk[1], pk[2], pk[3]);
+                                stmatrix_x4_trans(o + 16 * kORow, pk[4], pk[5], pk[6], pk[7]);
+                            }
                         }
                     }
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&B->d_empty[r]);
                 }
-                // Staging tile -> global, 16 bytes per thread, rows of 256 bytes.
+                // Staging tile -> global: one 256-byte bulk copy per token row.
+                fence_proxy_async_smem();
                 named_barrier_sync(4, 128);
                 const int fb = t.fb0 + f;
                 uint16_t* dst = MODE == kGateUp ? a.h + static_cast<size_t>(t.p0) * I + fb * 128
                                                 : a.y + static_cast<size_t>(t.p0) * H + fb * 128;
-                const int stride = MODE == kGateUp ? I : H;
-                for (int i = et; i < t.n * 16; i += 128) {
-                    const int rr = i >> 4, ch = i & 15;
-                    *reinterpret_cast<uint4*>(dst + static_cast<size_t>(rr) * stride + ch * 8) =
-                        *reinterpret_cast<const uint4*>(otile + rr * kORow + ch * 16);
-                }
-                named_barrier_sync(4, 128);
+                const size_t stride = MODE == kGateUp ? I : H;
+                for (int rr = et; rr < t.n; rr += 128)
+                    bulk_store_s2g(dst + rr * stride, otile_u32 + rr * kORow, 256);
+                bulk_commit();
             }
         }
+        bulk_wait0();
     } else if (warp == kWarpMma) {
         // ------------------------------------------------ MMA issuer
         if (lane == 0) {
@@ -512,9 +554,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                             wait_bar(&B->a_full[sa], static_cast<uint32_t>((ga / kSA) & 1), B, a.status) &
                             wait_bar(&B->b_full[sb], static_cast<uint32_t>((g_b / kSB) & 1), B, a.status);
                         tc_fence_after();
-                        // Token rows written by cp.async (generic proxy) are read by the MMA
-                        // (async proxy).
-                        if (MODE == kGateUp) fence_proxy_async_smem();
                         if (ok) {
                             const uint32_t bbase = smem_u32(b_ring + sb * kBStage);
 #pragma unroll
