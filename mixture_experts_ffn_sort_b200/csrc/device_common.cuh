@@ -368,6 +368,16 @@ __device__ __forceinline__ void stmatrix_x4_trans(uint32_t addr, uint32_t r0, ui
 
 // ---------------------------------------------------------------- bulk stores (shared -> global)
 
+// 2-D tiled store of a shared-memory tile to global memory through the tensor
+// map, tracked by this thread's bulk group (the tile's coordinates must not be
+// negative).  Generic-proxy writes to the tile must be fenced first.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int x, int y) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(src), "r"(x), "r"(y)
+                 : "memory");
+}
+
 // Asynchronous copy of `bytes` (a multiple of 16, both addresses 16-byte
 // aligned) from shared to global memory, tracked by this thread's bulk group.
 // Generic-proxy writes to the source must be fenced (fence_proxy_async_smem)

@@ -49,7 +49,8 @@ constexpr int kSB = 4;                      // token stages
 constexpr int kNMax = 192;                  // token rows per tile (MMA N)
 constexpr int kBStage = kNMax * 128;        // token rows x 64 bf16 (128-byte swizzle)
 constexpr int kWRing = 64 * 1024;           // FP8 weight ring (128 reduction columns per TMA stage)
-constexpr int kORow = 272;                  // bytes per row of the bf16 output staging tile (256 + pad)
+constexpr int kOHalf = kNMax * 128;         // staging tile: two halves of 64 features (128-byte swizzled rows)
+constexpr int kOStoreRows = 32;             // rows per TMA store of the staging tile
 // Per mode: M-tiles (128 weight rows each) per step, weight stage bytes and
 // depths of the weight ring and of the bf16 A ring in TMEM.
 template <int MODE> struct Cfg;
@@ -199,15 +200,16 @@ __device__ __forceinline__ uint32_t decode_scaled(uint16_t codes, float s) {
 template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tm_w0, const __grid_constant__ CUtensorMap tm_w1,
-                   const __grid_constant__ CUtensorMap tm_act, const FfnArgs a) {
+                   const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ CUtensorMap tm_out,
+                   const FfnArgs a) {
     using C = Cfg<MODE>;
     constexpr int MT = C::MT, kSW = C::kSW, kSA = C::kSA, kWStage = C::kWStage;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = align1024(smem_raw);
     uint8_t* w_ring = sm;                              // kSW x kWStage (64 KB)
     uint8_t* b_ring = w_ring + kWRing;                 // kSB x 24 KB
-    uint8_t* otile = b_ring + kSB * kBStage;           // [kNMax][kORow] bf16 output staging
-    Barriers* B = reinterpret_cast<Barriers*>(otile + kNMax * kORow);
+    uint8_t* otile = b_ring + kSB * kBStage;           // 2 x [kNMax][128 B] bf16 output staging
+    Barriers* B = reinterpret_cast<Barriers*>(otile + 2 * kOHalf);
     int* row_tok = reinterpret_cast<int*>(B + 1);      // [kNMax] activation row of each tile row
     float* col_w = reinterpret_cast<float*>(row_tok + kNMax);  // [kNMax] route weight of each column (down)
     float* sc_sm = col_w + kNMax;                              // [kScales] block scales of the item
@@ -232,7 +234,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&B->w_empty[s], kXformWarps);
         }
         for (int s = 0; s < kSB; ++s) {
-            mbar_init(&B->b_full[s], 1);
+            mbar_init(&B->b_full[s], MODE == kGateUp ? kTokThreads : 1);
             mbar_init(&B->b_done[s], 1);
         }
         for (int s = 0; s < kSA; ++s) {
@@ -291,13 +293,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         // Padding rows of the last MMA column group are left stale: column j of
         // D depends on token row j only, and the epilogue drops those columns.
         const int lt = threadIdx.x - kWarpTok * 32;  // 0..63
-        // gate/up: thread lt gathers rows 4lt .. 4lt+3 of the tile (one
-        // tile::gather4 per stage); rows past the tile's end repeat a valid
-        // token and land in padding rows the epilogue drops.
-        uint32_t tok[4] = {0, 0, 0, 0};
-        int ngroups = 0;
+        // gate/up: thread lt copies 16-byte chunk ch of rows r0 + 8k, keeping
+        // those rows' token indices in registers for the whole tile; the
+        // 128-byte swizzle of those rows is the same for every k.
+        const int r0 = lt >> 3, ch = lt & 7;
+        const uint32_t cch = static_cast<uint32_t>((ch ^ (r0 & 7)) << 4);
+        constexpr int kRowsPerThread = kNMax / 8;
+        uint32_t tok[kRowsPerThread];
         if (MODE == kDown) grid_dependency_wait();  // h comes from the gate/up grid
-        if (lt == 0) tma_prefetch_desc(&tm_act);
+        if (MODE == kDown && lt == 0) tma_prefetch_desc(&tm_act);
         long g = 0;
         for (int item = blockIdx.x; item < total; item += gridDim.x) {
             const Tile t = tile_of(a, pre, FB, GFB, item);
@@ -320,28 +324,28 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 if (bad) report_status(a.status, MOE_STATUS_BAD_MAP);
                 named_barrier_sync(2, kTokThreads);
-                ngroups = (t.n + 3) >> 2;
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int r = 4 * lt + i;
-                    tok[i] = static_cast<uint32_t>(row_tok[r < t.n ? r : 0]);
-                }
+                for (int k = 0; k < kRowsPerThread; ++k) tok[k] = r0 + 8 * k < t.n ? row_tok[r0 + 8 * k] : 0u;
             }
             for (int kb = 0; kb < KB; ++kb, ++g) {
                 const int s = static_cast<int>(g % kSB);
                 if (g >= kSB) wait_bar(&B->b_done[s], static_cast<uint32_t>((g / kSB - 1) & 1), B, a.status);
                 uint8_t* dst = b_ring + s * kBStage;
                 if (MODE == kGateUp) {
-                    if (lt == 0) mbar_arrive_expect_tx(&B->b_full[s], static_cast<uint32_t>(ngroups) * 512u);
-                    if (lt < ngroups)
-                        tma_gather4(dst + lt * 512, &tm_act, &B->b_full[s], kb * 64, static_cast<int>(tok[0]),
-                                    static_cast<int>(tok[1]), static_cast<int>(tok[2]), static_cast<int>(tok[3]));
+                    const uint32_t bdst = smem_u32(dst) + r0 * 128 + cch;
+                    const uint16_t* xs = a.x + kb * 64 + ch * 8;
+#pragma unroll
+                    for (int k = 0; k < kRowsPerThread; ++k)
+                        if (r0 + 8 * k < t.n)
+                            cp_async16(bdst + k * 1024, xs + static_cast<size_t>(tok[k]) * H, 16u);
+                    cp_async_arrive_noinc(&B->b_full[s]);
                 } else if (lt == 0) {
                     mbar_arrive_expect_tx(&B->b_full[s], kBStage);
                     tma_load_2d(dst, &tm_act, &B->b_full[s], kb * 64, static_cast<int>(t.p0));
                 }
             }
         }
+        if (MODE == kGateUp) cp_async_wait<0>();
     } else if (warp >= kWarpXform) {
         // ------------------------------------------------ transform: FP8 -> bf16 -> TMEM (A)
         // gate/up: warp (q, mt) owns lane quarter q of M-tile mt and all 64 codes
@@ -476,10 +480,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 }
                                 pk[k] = pack_bf16x2(hv[0], hv[1]);
                             }
-                            const uint32_t o = otile_u32 + (c0 + 8 * (lane >> 4) + (lane & 7)) * kORow +
-                                               (mt * 64 + 16 * q + 8 * ((lane >> 3) & 1)) * 2;
-                            stmatrix_x4_trans(o, pk[0], pk[1], pk[2], pk[3]);
-                            stmatrix_x4_trans(o + 16 * kORow, pk[4], pk[5], pk[6], pk[7]);
+                            // Features mt*64 + 16q + 8(i&1) + 0..7 of matrix i: half mt, 16-byte
+                            // chunk 2q + (i&1) of the token's 128-byte row.
+                            const int row = c0 + 8 * (lane >> 4) + (lane & 7);
+                            const uint32_t o = otile_u32 + mt * kOHalf + row * 128;
+                            const uint32_t fc = 2 * q + ((lane >> 3) & 1);
+                            stmatrix_x4_trans(o + ((fc ^ (row & 7)) << 4), pk[0], pk[1], pk[2], pk[3]);
+                            stmatrix_x4_trans(o + 16 * 128 + ((fc ^ (row & 7)) << 4), pk[4], pk[5], pk[6], pk[7]);
                         } else {
                             uint32_t dv[2][16];
                             tmem_ld16x256b_x4(tl + c0, dv[0]);
@@ -502,10 +509,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                                     pk[2 * gq + 1] = pack_bf16x2(__uint_as_float(d[2]) * wv[gq].x,
                                                                  __uint_as_float(d[3]) * wv[gq].y);
                                 }
-                                const uint32_t o = otile_u32 + (c0 + 8 * (lane >> 4) + (lane & 7)) * kORow +
-                                                   (32 * q + 16 * hf + 8 * ((lane >> 3) & 1)) * 2;
-                                stmatrix_x4_trans(o, pk[0], pk[1], pk[2], pk[3]);
-                                stmatrix_x4_trans(o + 16 * kORow, pk[4], pk[5], pk[6], pk[7]);
+                                // Features 32q + 16hf + 8(i&1) + 0..7: half q/2, chunk
+                                // 4(q&1) + 2hf + (i&1).
+                                const int row = c0 + 8 * (lane >> 4) + (lane & 7);
+                                const uint32_t o = otile_u32 + (q >> 1) * kOHalf + row * 128;
+                                const uint32_t fc = 4 * (q & 1) + 2 * hf + ((lane >> 3) & 1);
+                                stmatrix_x4_trans(o + ((fc ^ (row & 7)) << 4), pk[0], pk[1], pk[2], pk[3]);
+                                stmatrix_x4_trans(o + 16 * 128 + ((fc ^ (row & 7)) << 4), pk[4], pk[5], pk[6],
+                                                  pk[7]);
                             }
                         }
                     }
@@ -513,16 +524,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&B->d_empty[r]);
                 }
-                // Staging tile -> global: one 256-byte bulk copy per token row.
+                // Staging tile -> global: TMA tensor stores of 32 rows x 64 features,
+                // and 16-byte thread stores for the rows past the last full group.
                 fence_proxy_async_smem();
                 named_barrier_sync(4, 128);
                 const int fb = t.fb0 + f;
+                const int n32 = t.n / kOStoreRows;
+                if (et < 2 * n32) {
+                    const int hh = et & 1, k = et >> 1;
+                    tma_store_2d(&tm_out, otile_u32 + hh * kOHalf + k * kOStoreRows * 128, fb * 128 + hh * 64,
+                                 static_cast<int>(t.p0) + k * kOStoreRows);
+                }
+                bulk_commit();
                 uint16_t* dst = MODE == kGateUp ? a.h + static_cast<size_t>(t.p0) * I + fb * 128
                                                 : a.y + static_cast<size_t>(t.p0) * H + fb * 128;
                 const size_t stride = MODE == kGateUp ? I : H;
-                for (int rr = et; rr < t.n; rr += 128)
-                    bulk_store_s2g(dst + rr * stride, otile_u32 + rr * kORow, 256);
-                bulk_commit();
+                for (int i = n32 * kOStoreRows * 16 + et; i < t.n * 16; i += 128) {
+                    const int rr = i >> 4, hh = (i >> 3) & 1, c8 = i & 7;
+                    *reinterpret_cast<uint4*>(dst + rr * stride + hh * 64 + c8 * 8) =
+                        *reinterpret_cast<const uint4*>(otile + hh * kOHalf + rr * 128 + ((c8 ^ (rr & 7)) << 4));
+                }
             }
         }
         bulk_wait0();
@@ -554,6 +575,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                             wait_bar(&B->a_full[sa], static_cast<uint32_t>((ga / kSA) & 1), B, a.status) &
                             wait_bar(&B->b_full[sb], static_cast<uint32_t>((g_b / kSB) & 1), B, a.status);
                         tc_fence_after();
+                        // Token rows written by cp.async (generic proxy) are read by the MMA
+                        // (async proxy).
+                        if (MODE == kGateUp) fence_proxy_async_smem();
                         if (ok) {
                             const uint32_t bbase = smem_u32(b_ring + sb * kBStage);
 #pragma unroll
@@ -590,7 +614,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 size_t prefill_smem(int E) {
-    return 1024 + kWRing + kSB * kBStage + kNMax * kORow + sizeof(Barriers) + 2 * kNMax * 4 + kScales * 4 +
+    return 1024 + kWRing + kSB * kBStage + 2 * kOHalf + sizeof(Barriers) + 2 * kNMax * 4 + kScales * 4 +
            (E + 1) * 4 + 64;
 }
 
@@ -618,6 +642,9 @@ cudaError_t launch_ffn_prefill(const FfnArgs& a, cudaStream_t stream) {
     if (err == cudaSuccess) err = make_tmap_u8_2d(&td, a.ex.w_down, E * H, I, 128, 128);
     if (err == cudaSuccess) err = make_tmap_bf16_2d(&tx, a.x, static_cast<uint64_t>(a.T), H, 64, 1);
     if (err == cudaSuccess) err = make_tmap_bf16_2d(&th, a.h, rows, I, 64, kNMax);
+    CUtensorMap to_h, to_y;  // staging-tile stores: 32 rows x 64 features
+    if (err == cudaSuccess) err = make_tmap_bf16_2d(&to_h, a.h, rows, I, 64, kOStoreRows);
+    if (err == cudaSuccess) err = make_tmap_bf16_2d(&to_y, a.y, rows, H, 64, kOStoreRows);
     if (err != cudaSuccess) return err;
     const size_t smem = prefill_smem(a.identity ? 1 : a.ex.n);
     err = cudaFuncSetAttribute(prefill_kernel<kGateUp>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
@@ -625,7 +652,7 @@ cudaError_t launch_ffn_prefill(const FfnArgs& a, cudaStream_t stream) {
         err = cudaFuncSetAttribute(prefill_kernel<kDown>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (err != cudaSuccess) return err;
     const int grid = num_sms();
-    prefill_kernel<kGateUp><<<grid, kThreads, smem, stream>>>(tg, tu, tx, a);
+    prefill_kernel<kGateUp><<<grid, kThreads, smem, stream>>>(tg, tu, tx, to_h, a);
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
     cudaLaunchConfig_t cfg = {};
@@ -638,7 +665,7 @@ cudaError_t launch_ffn_prefill(const FfnArgs& a, cudaStream_t stream) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, prefill_kernel<kDown>, td, td, th, a);
+    return cudaLaunchKernelEx(&cfg, prefill_kernel<kDown>, td, td, th, to_y, a);
 }
 
 }  // namespace moe
