@@ -38,6 +38,8 @@
 // Every mbarrier wait is bounded; an expired wait sets a CTA-wide abort flag
 // and every role runs to the end without waiting, so the CTA always reaches
 // the TMEM de-allocation.
+#include <cstring>
+
 #include "device_common.cuh"
 #include "launch.h"
 
@@ -94,23 +96,59 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
     return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
+// Tensor maps of one launch, indexed by part: [0] the routed experts, [1] the
+// shared expert.
+struct PrefillMaps {
+    CUtensorMap w0[2];   // gate (gate/up launch) or down (down launch) weights
+    CUtensorMap w1[2];   // up weights (gate/up launch)
+    CUtensorMap act[2];  // rows of h (down launch)
+    CUtensorMap out[2];  // staging-tile stores: h (gate/up) or y (down)
+};
+
+// Shape of one part (routed or shared) in one launch.
+struct PartCfg {
+    int I;         // intermediate size
+    int KB;        // MMA steps (64 columns) per output block
+    int KB128;     // scale blocks = weight TMA stages per output block
+    int FB;        // output blocks of 128 features (gate/up: their gate and up rows)
+    int GFB;       // output blocks per item
+    bool resident; // down: the token tile stays in the ring across the item
+};
+
+template <int MODE>
+__device__ __forceinline__ PartCfg part_cfg(const FfnArgs& a, int pt) {
+    PartCfg c;
+    c.I = pt ? a.sh.inter : a.ex.inter;
+    const int Kred = MODE == kGateUp ? a.H : c.I;
+    c.KB = Kred / 64;
+    c.KB128 = Kred / 128;
+    c.FB = MODE == kGateUp ? c.I / 128 : a.H / 128;
+    // The down GEMM keeps its token tile resident across a group of output
+    // blocks when the whole reduction fits in the token ring.
+    c.resident = MODE == kDown && c.KB <= kSB;
+    c.GFB = c.resident ? kDownGroup : 1;
+    return c;
+}
+
 // One work item: a token tile of one expert and a group of consecutive
 // output blocks (128 weight rows each) that share that token tile.
 struct Tile {
-    int e;
-    long p0;  // first sorted row
+    int e;    // expert within its part
+    int pt;   // part: 0 routed, 1 shared
+    long p0;  // first row (sorted position, or token for the shared expert)
     int n;    // rows in the tile (<= kNMax)
     int fb0;  // first output block
     int nfb;  // output blocks in the group
 };
 
-// Number of items of expert e with n_e rows.
+// Number of items of an expert with n_e rows.
 __device__ __forceinline__ int items_of(long n_e, int groups) {
     return static_cast<int>((n_e + kNMax - 1) / kNMax) * groups;
 }
 
+// Rows of expert e of the combined list (e == E: the shared expert).
 __device__ __forceinline__ long expert_len(const FfnArgs& a, int e, long R, bool* bad) {
-    if (a.identity) return a.T;
+    if (e >= a.ex.n) return a.T;
     const long b = a.offsets[e], f = a.offsets[e + 1];
     if (b < 0 || f < b || f > R) {
         *bad = true;
@@ -119,15 +157,18 @@ __device__ __forceinline__ long expert_len(const FfnArgs& a, int e, long R, bool
     return f - b;
 }
 
-// Item list: pre[] holds the exclusive prefix of items over experts.  Returns the total.
-__device__ int build_tiles(const FfnArgs& a, int groups, int* pre) {
-    const int E = a.identity ? 1 : a.ex.n;
+__device__ __forceinline__ int num_experts(const FfnArgs& a) { return a.ex.n + (a.sh.n ? 1 : 0); }
+
+// Item list over the routed experts then the shared one: pre[] holds the
+// exclusive prefix of items over experts.  Returns the total.
+__device__ int build_tiles(const FfnArgs& a, int groups_r, int groups_s, int* pre) {
+    const int E = num_experts(a);
     const long R = static_cast<long>(a.T) * a.K;
     const int per = (E + blockDim.x - 1) / blockDim.x;
     const int e0 = min(E, static_cast<int>(threadIdx.x) * per), e1 = min(E, e0 + per);
     int local = 0;
     bool bad = false;
-    for (int e = e0; e < e1; ++e) local += items_of(expert_len(a, e, R, &bad), groups);
+    for (int e = e0; e < e1; ++e) local += items_of(expert_len(a, e, R, &bad), e < a.ex.n ? groups_r : groups_s);
     if (bad) report_status(a.status, MOE_STATUS_BAD_MAP);
     // Block exclusive scan of `local`.
     __shared__ int warp_sums[32];
@@ -153,7 +194,7 @@ __device__ int build_tiles(const FfnArgs& a, int groups, int* pre) {
     int run = (warp ? warp_sums[warp - 1] : 0) + x - local;
     for (int e = e0; e < e1; ++e) {
         pre[e] = run;
-        run += items_of(expert_len(a, e, R, &bad), groups);
+        run += items_of(expert_len(a, e, R, &bad), e < a.ex.n ? groups_r : groups_s);
     }
     const int total = warp_sums[nw - 1];
     if (threadIdx.x == 0) pre[E] = total;
@@ -161,9 +202,9 @@ __device__ int build_tiles(const FfnArgs& a, int groups, int* pre) {
     return total;
 }
 
-__device__ __forceinline__ Tile tile_of(const FfnArgs& a, const int* pre, int FB, int GFB, int item) {
-    const int E = a.identity ? 1 : a.ex.n;
-    int lo = 0, hi = E - 1;  // last e with pre[e] <= item
+template <int MODE>
+__device__ __forceinline__ Tile tile_of(const FfnArgs& a, const int* pre, int item) {
+    int lo = 0, hi = num_experts(a) - 1;  // last e with pre[e] <= item
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
         if (pre[mid] <= item)
@@ -171,18 +212,20 @@ __device__ __forceinline__ Tile tile_of(const FfnArgs& a, const int* pre, int FB
         else
             hi = mid - 1;
     }
-    const int groups = (FB + GFB - 1) / GFB;
     Tile t;
-    t.e = lo;
+    t.pt = lo >= a.ex.n ? 1 : 0;
+    t.e = t.pt ? 0 : lo;
+    const PartCfg c = part_cfg<MODE>(a, t.pt);
+    const int groups = (c.FB + c.GFB - 1) / c.GFB;
     const int local = item - pre[lo];
     const int tt = local / groups;
     const int fg = local - tt * groups;
-    const long base = a.identity ? 0 : a.offsets[lo];
-    const long n_e = a.identity ? a.T : a.offsets[lo + 1] - base;
+    const long base = t.pt ? 0 : a.offsets[lo];
+    const long n_e = t.pt ? a.T : a.offsets[lo + 1] - base;
     t.p0 = base + static_cast<long>(tt) * kNMax;
     t.n = static_cast<int>(min(static_cast<long>(kNMax), n_e - static_cast<long>(tt) * kNMax));
-    t.fb0 = fg * GFB;
-    t.nfb = min(GFB, FB - t.fb0);
+    t.fb0 = fg * c.GFB;
+    t.nfb = min(c.GFB, c.FB - t.fb0);
     return t;
 }
 
@@ -199,9 +242,7 @@ __device__ __forceinline__ uint32_t decode_scaled(uint16_t codes, float s) {
 
 template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
-    prefill_kernel(const __grid_constant__ CUtensorMap tm_w0, const __grid_constant__ CUtensorMap tm_w1,
-                   const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ CUtensorMap tm_out,
-                   const FfnArgs a) {
+    prefill_kernel(const __grid_constant__ PrefillMaps M, const FfnArgs a) {
     using C = Cfg<MODE>;
     constexpr int MT = C::MT, kSW = C::kSW, kSA = C::kSA, kWStage = C::kWStage;
     extern __shared__ uint8_t smem_raw[];
@@ -213,18 +254,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     int* row_tok = reinterpret_cast<int*>(B + 1);      // [kNMax] activation row of each tile row
     float* col_w = reinterpret_cast<float*>(row_tok + kNMax);  // [kNMax] route weight of each column (down)
     float* sc_sm = col_w + kNMax;                              // [kScales] block scales of the item
-    int* pre = reinterpret_cast<int*>(sc_sm + kScales);        // [E + 1]
+    int* pre = reinterpret_cast<int*>(sc_sm + kScales);        // [E + 2]
 
-    const int H = a.H, I = a.ex.inter;
-    const int Kred = MODE == kGateUp ? H : I;       // reduction length
-    const int KB = Kred / 64;                       // MMA steps (64 columns) per output block
-    const int KB128 = Kred / 128;                   // scale blocks = weight TMA stages per output block
-    // Output blocks: 128 features (gate/up: their gate and up rows).
-    const int FB = MODE == kGateUp ? I / 128 : H / 128;
-    // The down GEMM keeps its token tile resident across a group of output
-    // blocks when the whole reduction fits in the token ring.
-    const bool resident = MODE == kDown && KB <= kSB;
-    const int GFB = resident ? kDownGroup : 1;
+    const int H = a.H;
+    const bool has_sh = a.sh.n != 0;
     const long R = static_cast<long>(a.T) * a.K;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -253,7 +286,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_alloc(&B->tmem_base, kTmemCols);
         tc_fence_before();
     }
-    const int total = build_tiles(a, (FB + GFB - 1) / GFB, pre);  // contains __syncthreads
+    int total;
+    {
+        const PartCfg cr = part_cfg<MODE>(a, 0), cs = part_cfg<MODE>(a, 1);
+        total = build_tiles(a, (cr.FB + cr.GFB - 1) / cr.GFB, has_sh ? (cs.FB + cs.GFB - 1) / cs.GFB : 1,
+                            pre);  // contains __syncthreads
+    }
     tc_fence_after();
     const uint32_t tmem = B->tmem_base;
     if (MODE == kGateUp && threadIdx.x == 0) grid_dependency_launch();
@@ -261,25 +299,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == kWarpTma) {
         // ------------------------------------------------ FP8 weight tiles (TMA, evict-first)
         if (lane == 0) {
-            tma_prefetch_desc(&tm_w0);
-            if (MODE == kGateUp) tma_prefetch_desc(&tm_w1);
+            for (int pt = 0; pt < (has_sh ? 2 : 1); ++pt) {
+                tma_prefetch_desc(&M.w0[pt]);
+                if (MODE == kGateUp) tma_prefetch_desc(&M.w1[pt]);
+            }
             const uint64_t policy = l2_evict_first_policy();
             long g = 0;  // weight stages (128 columns)
             for (int item = blockIdx.x; item < total; item += gridDim.x) {
-                const Tile t = tile_of(a, pre, FB, GFB, item);
+                const Tile t = tile_of<MODE>(a, pre, item);
+                const PartCfg pc = part_cfg<MODE>(a, t.pt);
                 for (int f = 0; f < t.nfb; ++f) {
                     const int fb = t.fb0 + f;
-                    for (int kw = 0; kw < KB128; ++kw, ++g) {
+                    for (int kw = 0; kw < pc.KB128; ++kw, ++g) {
                         const int s = static_cast<int>(g % kSW);
                         if (g >= kSW) wait_bar(&B->w_empty[s], static_cast<uint32_t>((g / kSW - 1) & 1), B, a.status);
                         uint8_t* dst = w_ring + s * kWStage;
                         mbar_arrive_expect_tx(&B->w_full[s], kWStage);
                         if (MODE == kGateUp) {
-                            const int row = t.e * I + fb * 128;  // 128 gate rows, 128 up rows
-                            tma_load_2d_hint(dst, &tm_w0, &B->w_full[s], kw * 128, row, policy);
-                            tma_load_2d_hint(dst + kWStage / 2, &tm_w1, &B->w_full[s], kw * 128, row, policy);
+                            const int row = t.e * pc.I + fb * 128;  // 128 gate rows, 128 up rows
+                            tma_load_2d_hint(dst, &M.w0[t.pt], &B->w_full[s], kw * 128, row, policy);
+                            tma_load_2d_hint(dst + kWStage / 2, &M.w1[t.pt], &B->w_full[s], kw * 128, row, policy);
                         } else {
-                            tma_load_2d_hint(dst, &tm_w0, &B->w_full[s], kw * 128, t.e * H + fb * 128, policy);
+                            tma_load_2d_hint(dst, &M.w0[t.pt], &B->w_full[s], kw * 128, t.e * H + fb * 128, policy);
                         }
                     }
                 }
@@ -301,17 +342,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         constexpr int kRowsPerThread = kNMax / 8;
         uint32_t tok[kRowsPerThread];
         if (MODE == kDown) grid_dependency_wait();  // h comes from the gate/up grid
-        if (MODE == kDown && lt == 0) tma_prefetch_desc(&tm_act);
+        if (MODE == kDown && lt == 0)
+            for (int pt = 0; pt < (has_sh ? 2 : 1); ++pt) tma_prefetch_desc(&M.act[pt]);
         long g = 0;
         for (int item = blockIdx.x; item < total; item += gridDim.x) {
-            const Tile t = tile_of(a, pre, FB, GFB, item);
+            const Tile t = tile_of<MODE>(a, pre, item);
+            const PartCfg pc = part_cfg<MODE>(a, t.pt);
             if (MODE == kGateUp) {
                 named_barrier_sync(2, kTokThreads);
                 bool bad = false;
                 for (int r = lt; r < t.n; r += kTokThreads) {
                     int tk = 0;
                     const long p = t.p0 + r;
-                    if (a.identity) {
+                    if (t.pt) {
                         tk = static_cast<int>(p);
                     } else {
                         const int rt = a.sorted_route[p];
@@ -327,7 +370,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int k = 0; k < kRowsPerThread; ++k) tok[k] = r0 + 8 * k < t.n ? row_tok[r0 + 8 * k] : 0u;
             }
-            for (int kb = 0; kb < KB; ++kb, ++g) {
+            for (int kb = 0; kb < pc.KB; ++kb, ++g) {
                 const int s = static_cast<int>(g % kSB);
                 if (g >= kSB) wait_bar(&B->b_done[s], static_cast<uint32_t>((g / kSB - 1) & 1), B, a.status);
                 uint8_t* dst = b_ring + s * kBStage;
@@ -341,7 +384,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     cp_async_arrive_noinc(&B->b_full[s]);
                 } else if (lt == 0) {
                     mbar_arrive_expect_tx(&B->b_full[s], kBStage);
-                    tma_load_2d(dst, &tm_act, &B->b_full[s], kb * 64, static_cast<int>(t.p0));
+                    tma_load_2d(dst, &M.act[t.pt], &B->b_full[s], kb * 64, static_cast<int>(t.p0));
                 }
             }
         }
@@ -356,19 +399,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         constexpr int NW = MODE == kGateUp ? 32 : 16;           // words (bf16 pairs) per thread per step
         long g = 0;                                             // MMA steps (64 columns)
         for (int item = blockIdx.x; item < total; item += gridDim.x) {
-            const Tile t = tile_of(a, pre, FB, GFB, item);
+            const Tile t = tile_of<MODE>(a, pre, item);
+            const PartCfg pc = part_cfg<MODE>(a, t.pt);
+            const ExpertsView& ev = t.pt ? a.sh : a.ex;
+            const int KB = pc.KB, KB128 = pc.KB128;
             // Block scales of the item, staged once: gate/up -> [gate, up][KB128],
             // down -> [output block][KB128].
             named_barrier_sync(3, kXformWarps * 32);
             if (MODE == kGateUp) {
-                const size_t off = (static_cast<size_t>(t.e) * (I / 128) + t.fb0) * KB128;
+                const size_t off = (static_cast<size_t>(t.e) * (pc.I / 128) + t.fb0) * KB128;
                 for (int i = xt; i < 2 * KB128; i += kXformWarps * 32)
-                    sc_sm[i] = __ldg((i < KB128 ? a.ex.s_gate : a.ex.s_up) + off + (i % KB128));
+                    sc_sm[i] = __ldg((i < KB128 ? ev.s_gate : ev.s_up) + off + (i % KB128));
             } else {
                 for (int i = xt; i < t.nfb * KB128; i += kXformWarps * 32) {
                     const int f = i / KB128, k = i - f * KB128;
-                    sc_sm[i] = __ldg(a.ex.s_down +
-                                     (static_cast<size_t>(t.e) * (H / 128) + (t.fb0 + f)) * KB128 + k);
+                    sc_sm[i] = __ldg(ev.s_down + (static_cast<size_t>(t.e) * (H / 128) + (t.fb0 + f)) * KB128 + k);
                 }
             }
             named_barrier_sync(3, kXformWarps * 32);
@@ -432,13 +477,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         int uses[2] = {0, 0};
         int tc = 0;
         for (int item = blockIdx.x; item < total; item += gridDim.x) {
-            const Tile t = tile_of(a, pre, FB, GFB, item);
+            const Tile t = tile_of<MODE>(a, pre, item);
+            const PartCfg pc = part_cfg<MODE>(a, t.pt);
             if (MODE == kDown) {
-                // Route weight of every column of the item, staged once.
+                // Route weight of every column of the item, staged once (1 for
+                // the shared expert).
                 named_barrier_sync(4, 128);
                 for (int c = et; c < t.n; c += 128) {
                     float wv = 1.f;
-                    if (!a.identity) {
+                    if (!t.pt) {
                         const int rt = a.sorted_route[t.p0 + c];
                         wv = (rt >= 0 && rt < R) ? a.topk_w[rt] : 0.f;
                     }
@@ -532,13 +579,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int n32 = t.n / kOStoreRows;
                 if (et < 2 * n32) {
                     const int hh = et & 1, k = et >> 1;
-                    tma_store_2d(&tm_out, otile_u32 + hh * kOHalf + k * kOStoreRows * 128, fb * 128 + hh * 64,
-                                 static_cast<int>(t.p0) + k * kOStoreRows);
+                    tma_store_2d(&M.out[t.pt], otile_u32 + hh * kOHalf + k * kOStoreRows * 128,
+                                 fb * 128 + hh * 64, static_cast<int>(t.p0) + k * kOStoreRows);
                 }
                 bulk_commit();
-                uint16_t* dst = MODE == kGateUp ? a.h + static_cast<size_t>(t.p0) * I + fb * 128
-                                                : a.y + static_cast<size_t>(t.p0) * H + fb * 128;
-                const size_t stride = MODE == kGateUp ? I : H;
+                const size_t stride = MODE == kGateUp ? pc.I : H;
+                uint16_t* base = MODE == kGateUp ? (t.pt ? a.h_sh : a.h) : (t.pt ? a.y_sh : a.y);
+                uint16_t* dst = base + static_cast<size_t>(t.p0) * stride + fb * 128;
                 for (int i = n32 * kOStoreRows * 16 + et; i < t.n * 16; i += 128) {
                     const int rr = i >> 4, hh = (i >> 3) & 1, c8 = i & 7;
                     *reinterpret_cast<uint4*>(dst + rr * stride + hh * 64 + c8 * 8) =
@@ -554,7 +601,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             int uses[2] = {0, 0};
             int tc = 0;
             for (int item = blockIdx.x; item < total; item += gridDim.x) {
-                const Tile t = tile_of(a, pre, FB, GFB, item);
+                const Tile t = tile_of<MODE>(a, pre, item);
+                const PartCfg pc = part_cfg<MODE>(a, t.pt);
+                const int KB = pc.KB;
+                const bool resident = pc.resident;
                 const int N = (t.n + 15) & ~15;
                 const uint32_t idesc = umma_idesc_bf16(128, N);
                 for (int f = 0; f < t.nfb; ++f, ++tc) {
@@ -615,7 +665,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 size_t prefill_smem(int E) {
     return 1024 + kWRing + kSB * kBStage + 2 * kOHalf + sizeof(Barriers) + 2 * kNMax * 4 + kScales * 4 +
-           (E + 1) * 4 + 64;
+           (E + 2) * 4 + 64;
 }
 
 int num_sms() {
@@ -634,25 +684,35 @@ int num_sms() {
 bool ffn_prefill_supported(int H, int I) { return H % 128 == 0 && I % 128 == 0 && prefill_smem(MOE_MAX_E) <= 227 * 1024; }
 
 cudaError_t launch_ffn_prefill(const FfnArgs& a, cudaStream_t stream) {
+    if (a.identity) return cudaErrorInvalidValue;
     const uint64_t E = static_cast<uint64_t>(a.ex.n), I = a.ex.inter, H = a.H;
-    const uint64_t rows = a.identity ? static_cast<uint64_t>(a.T) : static_cast<uint64_t>(a.T) * a.K;
-    CUtensorMap tg, tu, td, tx, th;
-    cudaError_t err = make_tmap_u8_2d(&tg, a.ex.w_gate, E * I, H, 128, 128);
-    if (err == cudaSuccess) err = make_tmap_u8_2d(&tu, a.ex.w_up, E * I, H, 128, 128);
-    if (err == cudaSuccess) err = make_tmap_u8_2d(&td, a.ex.w_down, E * H, I, 128, 128);
-    if (err == cudaSuccess) err = make_tmap_bf16_2d(&tx, a.x, static_cast<uint64_t>(a.T), H, 64, 1);
-    if (err == cudaSuccess) err = make_tmap_bf16_2d(&th, a.h, rows, I, 64, kNMax);
-    CUtensorMap to_h, to_y;  // staging-tile stores: 32 rows x 64 features
-    if (err == cudaSuccess) err = make_tmap_bf16_2d(&to_h, a.h, rows, I, 64, kOStoreRows);
-    if (err == cudaSuccess) err = make_tmap_bf16_2d(&to_y, a.y, rows, H, 64, kOStoreRows);
+    const uint64_t R = static_cast<uint64_t>(a.T) * a.K, T = static_cast<uint64_t>(a.T);
+    PrefillMaps mg, md;  // gate/up and down launches
+    memset(&mg, 0, sizeof(mg));
+    memset(&md, 0, sizeof(md));
+    cudaError_t err = make_tmap_u8_2d(&mg.w0[0], a.ex.w_gate, E * I, H, 128, 128);
+    if (err == cudaSuccess) err = make_tmap_u8_2d(&mg.w1[0], a.ex.w_up, E * I, H, 128, 128);
+    if (err == cudaSuccess) err = make_tmap_bf16_2d(&mg.out[0], a.h, R, I, 64, kOStoreRows);
+    if (err == cudaSuccess) err = make_tmap_u8_2d(&md.w0[0], a.ex.w_down, E * H, I, 128, 128);
+    if (err == cudaSuccess) err = make_tmap_bf16_2d(&md.act[0], a.h, R, I, 64, kNMax);
+    if (err == cudaSuccess) err = make_tmap_bf16_2d(&md.out[0], a.y, R, H, 64, kOStoreRows);
+    if (a.sh.n) {
+        const uint64_t Is = a.sh.inter;
+        if (err == cudaSuccess) err = make_tmap_u8_2d(&mg.w0[1], a.sh.w_gate, Is, H, 128, 128);
+        if (err == cudaSuccess) err = make_tmap_u8_2d(&mg.w1[1], a.sh.w_up, Is, H, 128, 128);
+        if (err == cudaSuccess) err = make_tmap_bf16_2d(&mg.out[1], a.h_sh, T, Is, 64, kOStoreRows);
+        if (err == cudaSuccess) err = make_tmap_u8_2d(&md.w0[1], a.sh.w_down, H, Is, 128, 128);
+        if (err == cudaSuccess) err = make_tmap_bf16_2d(&md.act[1], a.h_sh, T, Is, 64, kNMax);
+        if (err == cudaSuccess) err = make_tmap_bf16_2d(&md.out[1], a.y_sh, T, H, 64, kOStoreRows);
+    }
     if (err != cudaSuccess) return err;
-    const size_t smem = prefill_smem(a.identity ? 1 : a.ex.n);
+    const size_t smem = prefill_smem(a.ex.n);
     err = cudaFuncSetAttribute(prefill_kernel<kGateUp>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (err == cudaSuccess)
         err = cudaFuncSetAttribute(prefill_kernel<kDown>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (err != cudaSuccess) return err;
     const int grid = num_sms();
-    prefill_kernel<kGateUp><<<grid, kThreads, smem, stream>>>(tg, tu, tx, to_h, a);
+    prefill_kernel<kGateUp><<<grid, kThreads, smem, stream>>>(mg, a);
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
     cudaLaunchConfig_t cfg = {};
@@ -665,7 +725,7 @@ cudaError_t launch_ffn_prefill(const FfnArgs& a, cudaStream_t stream) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, prefill_kernel<kDown>, td, td, th, to_y, a);
+    return cudaLaunchKernelEx(&cfg, prefill_kernel<kDown>, md, a);
 }
 
 }  // namespace moe

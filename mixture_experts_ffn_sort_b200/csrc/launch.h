@@ -54,6 +54,11 @@ struct FfnArgs {
     uint16_t* y;  // [rows, H] bf16 output
     int32_t* status;
     int avg_rows;  // host-known rows per expert (sizes the token tile)
+    // Prefill form only: an always-on expert run in the same launches as the
+    // routed rows (its rows are the T tokens in order, route weight 1).
+    ExpertsView sh;  // sh.n == 0: none
+    uint16_t* h_sh;  // [T, sh.inter] bf16 scratch
+    uint16_t* y_sh;  // [T, H] bf16 output
 };
 
 cudaError_t launch_ffn_decode(const FfnArgs& a, cudaStream_t stream);
@@ -68,6 +73,7 @@ cudaError_t make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows,
                               uint32_t box_cols, uint32_t box_rows);
 
 // ---------------------------------------------------------------- expert FFN (prefill, tcgen05)
+// Routed rows (a.identity must be false) plus the optional shared expert a.sh.
 cudaError_t launch_ffn_prefill(const FfnArgs& a, cudaStream_t stream);
 bool ffn_prefill_supported(int H, int I);
 

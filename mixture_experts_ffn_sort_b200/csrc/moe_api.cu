@@ -213,7 +213,17 @@ int moe_expert_ffn(const uint16_t* x, int T, int H, int K, const moe_fp8_experts
     a.y = y_sorted;
     a.status = status;
     a.avg_rows = static_cast<int>((R + E - 1) / E);
-    cudaError_t e = prefill ? moe::launch_ffn_prefill(a, stream) : moe::launch_ffn_decode(a, stream);
+    if (prefill) {
+        // The shared expert runs in the same two launches as the routed rows.
+        if (shared) {
+            a.sh = {shared->w_gate, shared->w_up, shared->w_down, shared->s_gate, shared->s_up, shared->s_down, 1, Is};
+            a.h_sh = reinterpret_cast<uint16_t*>(ws + ffn_h_bytes(R, I));
+            a.y_sh = y_shared;
+        }
+        const cudaError_t e = moe::launch_ffn_prefill(a, stream);
+        return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_expert_ffn launch");
+    }
+    cudaError_t e = moe::launch_ffn_decode(a, stream);
     if (e != cudaSuccess) return cuda_fail(e, "moe_expert_ffn routed launch");
     if (shared) {
         moe::FfnArgs s = a;
@@ -225,7 +235,7 @@ int moe_expert_ffn(const uint16_t* x, int T, int H, int K, const moe_fp8_experts
         s.h = reinterpret_cast<uint16_t*>(ws + ffn_h_bytes(R, I));
         s.y = y_shared;
         s.avg_rows = T;
-        e = prefill ? moe::launch_ffn_prefill(s, stream) : moe::launch_ffn_decode(s, stream);
+        e = moe::launch_ffn_decode(s, stream);
         if (e != cudaSuccess) return cuda_fail(e, "moe_expert_ffn shared launch");
     }
     return MOE_OK;
