@@ -596,64 +596,69 @@ __global__ void __launch_bounds__(kThreads, 1)
         bulk_wait0();
     } else if (warp == kWarpMma) {
         // ------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            long ga = 0, gb = 0;
-            int uses[2] = {0, 0};
-            int tc = 0;
-            for (int item = blockIdx.x; item < total; item += gridDim.x) {
-                const Tile t = tile_of<MODE>(a, pre, item);
-                const PartCfg pc = part_cfg<MODE>(a, t.pt);
-                const int KB = pc.KB;
-                const bool resident = pc.resident;
-                const int N = (t.n + 15) & ~15;
-                const uint32_t idesc = umma_idesc_bf16(128, N);
-                for (int f = 0; f < t.nfb; ++f, ++tc) {
-                    // Accumulator regions of this output block: both (gate/up) or one (down).
-                    const int r0 = MODE == kGateUp ? 0 : (tc & 1);
-                    for (int mt = 0; mt < MT; ++mt) {
-                        const int r = r0 + mt;
-                        if (uses[r] >= 1)
-                            wait_bar(&B->d_empty[r], static_cast<uint32_t>((uses[r] - 1) & 1), B, a.status);
-                        ++uses[r];
-                    }
-                    tc_fence_after();
-                    const bool last = f == t.nfb - 1;
-                    for (int kb = 0; kb < KB; ++kb, ++ga) {
-                        const long g_b = resident ? gb + kb : gb;  // token stage of this step
-                        const int sa = static_cast<int>(ga % kSA), sb = static_cast<int>(g_b % kSB);
-                        const bool ok =
-                            wait_bar(&B->a_full[sa], static_cast<uint32_t>((ga / kSA) & 1), B, a.status) &
-                            wait_bar(&B->b_full[sb], static_cast<uint32_t>((g_b / kSB) & 1), B, a.status);
-                        tc_fence_after();
-                        // Token rows written by cp.async (generic proxy) are read by the MMA
-                        // (async proxy).
-                        if (MODE == kGateUp) fence_proxy_async_smem();
-                        if (ok) {
-                            const uint32_t bbase = smem_u32(b_ring + sb * kBStage);
-#pragma unroll
-                            for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-                                for (int k = 0; k < 4; ++k)
-                                    umma_ts_f16(tmem + (r0 + mt) * kDRegion,
-                                                tmem + kACol + sa * (MT * 32) + mt * 32 + k * 8,
-                                                umma_desc_sw128(bbase + k * 32), idesc, (kb > 0 || k > 0) ? 1u : 0u);
-                        }
-                        umma_commit(&B->a_done[sa]);
-                        if (!resident) {
-                            umma_commit(&B->b_done[sb]);
-                            ++gb;
-                        } else if (last) {
-                            umma_commit(&B->b_done[sb]);
-                        }
-                    }
-                    for (int mt = 0; mt < MT; ++mt) umma_commit(&B->d_full[r0 + mt]);
+        // The whole warp runs the loop with warp-uniform operands; one elected
+        // lane issues each tcgen05 instruction.  Operands are bases computed
+        // once plus per-slot offsets.
+        const uint64_t bdesc0 = umma_desc_sw128(smem_u32(b_ring));
+        const uint32_t a_base = tmem + kACol;
+        long ga = 0, gb = 0;
+        int uses[2] = {0, 0};
+        int tc = 0;
+        for (int item = blockIdx.x; item < total; item += gridDim.x) {
+            const Tile t = tile_of<MODE>(a, pre, item);
+            const PartCfg pc = part_cfg<MODE>(a, t.pt);
+            const int KB = pc.KB;
+            const bool resident = pc.resident;
+            const int N = (t.n + 15) & ~15;
+            const uint32_t idesc = umma_idesc_bf16(128, N);
+            for (int f = 0; f < t.nfb; ++f, ++tc) {
+                // Accumulator regions of this output block: both (gate/up) or one (down).
+                const int r0 = MODE == kGateUp ? 0 : (tc & 1);
+                for (int mt = 0; mt < MT; ++mt) {
+                    const int r = r0 + mt;
+                    if (uses[r] >= 1)
+                        wait_bar(&B->d_empty[r], static_cast<uint32_t>((uses[r] - 1) & 1), B, a.status);
+                    ++uses[r];
                 }
-                if (resident) gb += KB;
+                tc_fence_after();
+                const bool last = f == t.nfb - 1;
+                const uint32_t d_base = tmem + r0 * kDRegion;
+                for (int kb = 0; kb < KB; ++kb, ++ga) {
+                    const long g_b = resident ? gb + kb : gb;  // token stage of this step
+                    const int sa = static_cast<int>(ga % kSA), sb = static_cast<int>(g_b % kSB);
+                    const bool ok =
+                        wait_bar(&B->a_full[sa], static_cast<uint32_t>((ga / kSA) & 1), B, a.status) &
+                        wait_bar(&B->b_full[sb], static_cast<uint32_t>((g_b / kSB) & 1), B, a.status);
+                    tc_fence_after();
+                    // Token rows written by cp.async (generic proxy) are read by the MMA
+                    // (async proxy).
+                    if (MODE == kGateUp) fence_proxy_async_smem();
+                    if (ok) {
+                        const uint64_t bdesc = bdesc0 + static_cast<uint64_t>((sb * kBStage) >> 4);
+                        const uint32_t a_slot = a_base + sa * (MT * 32);
+#pragma unroll
+                        for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                            for (int k = 0; k < 4; ++k)
+                                umma_ts_f16_elect(d_base + mt * kDRegion, a_slot + mt * 32 + k * 8,
+                                                  bdesc + static_cast<uint64_t>(k * 2), idesc,
+                                                  (kb > 0 || k > 0) ? 1u : 0u);
+                    }
+                    umma_commit_elect(&B->a_done[sa]);
+                    if (!resident) {
+                        umma_commit_elect(&B->b_done[sb]);
+                        ++gb;
+                    } else if (last) {
+                        umma_commit_elect(&B->b_done[sb]);
+                    }
+                }
+                for (int mt = 0; mt < MT; ++mt) umma_commit_elect(&B->d_full[r0 + mt]);
             }
-            // Every MMA has completed once this barrier flips.
-            umma_commit(&B->final_bar);
-            mbar_wait(&B->final_bar, 0, a.status);
+            if (resident) gb += KB;
         }
+        // Every MMA has completed once this barrier flips.
+        umma_commit_elect(&B->final_bar);
+        mbar_wait(&B->final_bar, 0, a.status);
         __syncwarp();
     }
     __syncthreads();
