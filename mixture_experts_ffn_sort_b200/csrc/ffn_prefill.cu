@@ -54,7 +54,10 @@ constexpr int kWRing = 64 * 1024;           // FP8 weight ring (128 reduction co
 constexpr int kOHalf = kNMax * 128;         // staging tile: two halves of 64 features (128-byte swizzled rows)
 constexpr int kOStoreRows = 32;             // rows per TMA store of the staging tile
 // Per mode: M-tiles (128 weight rows each) per step, weight stage bytes and
-// depths of the weight ring and of the bf16 A ring in TMEM.
+// depths of the weight ring and of the bf16 A ring in TMEM.  The A ring holds
+// kSA units of 32 columns (one M-tile's 64 reduction columns); a gate/up step
+// fills two units (one per M-tile, each released as soon as its own MMAs are
+// done), a down step one.
 template <int MODE> struct Cfg;
 // Warp roles (transform and epilogue warps sit on their TMEM lane quarter, warp % 4):
 // warps 2-3 load token rows.
@@ -76,7 +79,7 @@ enum Mode { kGateUp = 0, kDown = 1 };
 // A weight stage holds 128 reduction columns (128-byte rows) and feeds two
 // 64-column MMA steps.
 template <> struct Cfg<0> {
-    static constexpr int MT = 2, kWStage = 2 * 128 * 128, kSW = kWRing / kWStage, kSA = 2;
+    static constexpr int MT = 2, kWStage = 2 * 128 * 128, kSW = kWRing / kWStage, kSA = 4;
 };
 template <> struct Cfg<1> {
     static constexpr int MT = 1, kWStage = 128 * 128, kSW = kWRing / kWStage, kSA = 4;
@@ -271,7 +274,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&B->b_done[s], 1);
         }
         for (int s = 0; s < kSA; ++s) {
-            mbar_init(&B->a_full[s], kXformWarps);
+            // gate/up: the 4 transform warps of one M-tile fill a unit; down: all 8.
+            mbar_init(&B->a_full[s], MODE == kGateUp ? kXformWarps / 2 : kXformWarps);
             mbar_init(&B->a_done[s], 1);
         }
         for (int d = 0; d < 2; ++d) {
@@ -429,11 +433,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float* scr = sc_sm + (MODE == kGateUp ? (up_row ? KB128 : 0) : f * KB128);
                 for (int kb = 0; kb < KB; ++kb, ++g) {
                     const long gw = g >> 1;  // weight stage holding this step
-                    const int sw = static_cast<int>(gw % kSW), sa = static_cast<int>(g % kSA);
+                    const long u = MODE == kGateUp ? 2 * g + hi : g;  // A unit of this warp's work
+                    const int sw = static_cast<int>(gw % kSW), sa = static_cast<int>(u % kSA);
                     const bool ok1 = wait_bar(&B->w_full[sw], static_cast<uint32_t>((gw / kSW) & 1), B, a.status);
                     bool ok2 = true;
-                    if (g >= kSA)
-                        ok2 = wait_bar(&B->a_done[sa], static_cast<uint32_t>((g / kSA - 1) & 1), B, a.status);
+                    if (u >= kSA)
+                        ok2 = wait_bar(&B->a_done[sa], static_cast<uint32_t>((u / kSA - 1) & 1), B, a.status);
                     uint32_t v[NW];
                     if (ok1 && ok2) {
                         const float sc = scr[kb >> 1];
@@ -455,7 +460,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     __syncwarp();
                     if ((g & 1) && lane == 0) mbar_arrive(&B->w_empty[sw]);
-                    const uint32_t acol = kACol + sa * (MT * 32) + (MODE == kGateUp ? hi * 32 : hi * 16);
+                    const uint32_t acol = kACol + sa * 32 + (MODE == kGateUp ? 0 : hi * 16);
                     if constexpr (MODE == kGateUp)
                         tmem_st32(tmem + (static_cast<uint32_t>(32 * q) << 16) + acol, v);
                     else
@@ -625,26 +630,29 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t d_base = tmem + r0 * kDRegion;
                 for (int kb = 0; kb < KB; ++kb, ++ga) {
                     const long g_b = resident ? gb + kb : gb;  // token stage of this step
-                    const int sa = static_cast<int>(ga % kSA), sb = static_cast<int>(g_b % kSB);
-                    const bool ok =
-                        wait_bar(&B->a_full[sa], static_cast<uint32_t>((ga / kSA) & 1), B, a.status) &
-                        wait_bar(&B->b_full[sb], static_cast<uint32_t>((g_b / kSB) & 1), B, a.status);
+                    const int sb = static_cast<int>(g_b % kSB);
+                    const bool okb = wait_bar(&B->b_full[sb], static_cast<uint32_t>((g_b / kSB) & 1), B, a.status);
                     tc_fence_after();
                     // Token rows written by cp.async (generic proxy) are read by the MMA
                     // (async proxy).
                     if (MODE == kGateUp) fence_proxy_async_smem();
-                    if (ok) {
-                        const uint64_t bdesc = bdesc0 + static_cast<uint64_t>((sb * kBStage) >> 4);
-                        const uint32_t a_slot = a_base + sa * (MT * 32);
+                    const uint64_t bdesc = bdesc0 + static_cast<uint64_t>((sb * kBStage) >> 4);
 #pragma unroll
-                        for (int mt = 0; mt < MT; ++mt)
+                    for (int mt = 0; mt < MT; ++mt) {
+                        // A unit of M-tile mt of this step.
+                        const long u = ga * MT + mt;
+                        const int sa = static_cast<int>(u % kSA);
+                        const bool oka = wait_bar(&B->a_full[sa], static_cast<uint32_t>((u / kSA) & 1), B, a.status);
+                        tc_fence_after();
+                        if (okb && oka) {
 #pragma unroll
                             for (int k = 0; k < 4; ++k)
-                                umma_ts_f16_elect(d_base + mt * kDRegion, a_slot + mt * 32 + k * 8,
+                                umma_ts_f16_elect(d_base + mt * kDRegion, a_base + sa * 32 + k * 8,
                                                   bdesc + static_cast<uint64_t>(k * 2), idesc,
                                                   (kb > 0 || k > 0) ? 1u : 0u);
+                        }
+                        umma_commit_elect(&B->a_done[sa]);
                     }
-                    umma_commit_elect(&B->a_done[sa]);
                     if (!resident) {
                         umma_commit_elect(&B->b_done[sb]);
                         ++gb;
