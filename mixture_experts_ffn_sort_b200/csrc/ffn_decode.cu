@@ -9,14 +9,19 @@
 // device-side offsets (no host sync).
 //
 // Design (B200):
-//  * One CTA owns a slice of ONE expert's weights: 64 intermediate features
-//    (their gate and up rows) in the gate/up kernel, 128 output features in the
-//    down kernel.  CTAs whose expert received no route exit at once, so only
-//    the touched experts' weights are read, once per token group.
-//  * A producer warp streams the slice from HBM with TMA (evict-first L2
+//  * Persistent kernels (as many CTAs as the GPU holds at once).  Each CTA
+//    lists the experts that received rows (from the device-side offsets, no
+//    host sync) and takes a contiguous, equal share of the items (touched
+//    expert, token group, slice of weight rows): 64 intermediate features
+//    (their gate and up rows) in the gate/up kernel, 128 output features in
+//    the down kernel.  Every item streams the same weight bytes, so skewed
+//    expert loads stay balanced, and only the touched experts' weights are
+//    read, once per token group.  Consecutive items of a CTA share their token
+//    group, which is staged once.
+//  * A producer warp streams the slices from HBM with TMA (evict-first L2
 //    policy) in 16 KB stages of 128 reduction columns (one scale block),
 //    128-byte swizzled, through a 4-deep shared-memory ring (mbarrier
-//    full/empty pairs with bounded waits).
+//    full/empty pairs with bounded waits) that runs on across items.
 //  * Eight consumer warps each own 16 MMA rows.  They read the FP8 bytes with
 //    ldmatrix (conflict-free on the swizzled tile) and convert them with the
 //    one-instruction E4M3x2 -> f16x2 conversion, which is exact: the decoded
@@ -87,20 +92,19 @@ __device__ __forceinline__ bool expert_rows(const FfnArgs& a, int e, long& p0, l
     return true;
 }
 
-// Producer: stream `total` stages (cycling the slice's KB column blocks) into the ring.
-__device__ __forceinline__ void produce(const CUtensorMap* m0, const CUtensorMap* m1, int row,
-                                        int KB, long total, uint8_t* ring, uint64_t* full,
-                                        uint64_t* empty, volatile int* abort_flag, int32_t* status) {
-    tma_prefetch_desc(m0);
-    if (m1) tma_prefetch_desc(m1);
-    const uint64_t policy = l2_evict_first_policy();
-    for (long it = 0; it < total; ++it) {
+// Producer: stream `count` stages (cycling the slice's KB column blocks) into
+// the ring; `it` is the CTA's running stage counter.  Returns false once a
+// wait has expired.
+__device__ __forceinline__ bool produce(const CUtensorMap* m0, const CUtensorMap* m1, int row, int KB,
+                                        long count, long& it, uint8_t* ring, uint64_t* full, uint64_t* empty,
+                                        uint64_t policy, volatile int* abort_flag, int32_t* status) {
+    for (long j = 0; j < count; ++j, ++it) {
         const int s = static_cast<int>(it % kStages);
         if (it >= kStages &&
             !mbar_wait_or_abort(&empty[s], static_cast<uint32_t>((it / kStages - 1) & 1), abort_flag, status))
-            return;
+            return false;
         mbar_arrive_expect_tx(&full[s], kStageBytes);
-        const int kb = static_cast<int>(it % KB);
+        const int kb = static_cast<int>(j % KB);
         uint8_t* dst = ring + static_cast<size_t>(s) * kStageBytes;
         if (m1) {
             tma_load_2d_hint(dst, m0, &full[s], kb * 128, row, policy);
@@ -109,6 +113,7 @@ __device__ __forceinline__ void produce(const CUtensorMap* m0, const CUtensorMap
             tma_load_2d_hint(dst, m0, &full[s], kb * 128, row, policy);
         }
     }
+    return true;
 }
 
 // Largest |x| bit pattern (sign cleared) among the 8 bf16 of a 16-byte vector.
@@ -208,14 +213,17 @@ struct Smem {
     uint64_t* full;
     uint64_t* empty;
     volatile int* abort_flag;
+    int* touched;  // [E]: experts with at least one row
+    int* gpre;     // [E + 1]: exclusive prefix of their token groups
 };
 
-__host__ __device__ constexpr size_t smem_bytes(int NG, int row_stride, int otile_stride) {
+__host__ __device__ constexpr size_t smem_bytes(int NG, int row_stride, int otile_stride, int E) {
     return 1024 + static_cast<size_t>(kStages) * kStageBytes + static_cast<size_t>(NG) * row_stride +
-           static_cast<size_t>(NG) * otile_stride * 2 + 3 * NG * 4 + 2 * kStages * 8 + 16;
+           static_cast<size_t>(NG) * otile_stride * 2 + 3 * NG * 4 + 2 * kStages * 8 + 16 +
+           static_cast<size_t>(2 * E + 1) * 4;
 }
 
-__device__ __forceinline__ Smem carve(uint8_t* raw, int NG, int row_stride, int otile_stride) {
+__device__ __forceinline__ Smem carve(uint8_t* raw, int NG, int row_stride, int otile_stride, int E) {
     Smem s;
     uint8_t* p = align1024(raw);
     s.ring = p;
@@ -231,8 +239,111 @@ __device__ __forceinline__ Smem carve(uint8_t* raw, int NG, int row_stride, int 
     s.full = reinterpret_cast<uint64_t*>(p);
     s.empty = s.full + kStages;
     s.abort_flag = reinterpret_cast<volatile int*>(s.empty + kStages);
+    s.touched = reinterpret_cast<int*>(s.empty + kStages) + 4;
+    s.gpre = s.touched + E;
     return s;
 }
+
+// The experts of this call with at least one row, in increasing order, into
+// touched[0 .. count), and the exclusive prefix of their token groups (of NG
+// rows) into gpre[0 .. count]; returns the total number of groups.  Experts
+// whose offsets are corrupt are left out (and flagged); *ntouched = count.
+// Contains __syncthreads.
+__device__ long build_touched(const FfnArgs& a, int NG, int* touched, int* gpre, int* ntouched) {
+    const int E = a.identity ? 1 : a.ex.n;
+    __shared__ int warp_sums[32][2];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    const int per = (E + blockDim.x - 1) / blockDim.x;
+    const int e0 = min(E, static_cast<int>(threadIdx.x) * per), e1 = min(E, e0 + per);
+    int cnt = 0, grp = 0;
+    for (int e = e0; e < e1; ++e) {
+        long p0, n;
+        if (!expert_rows(a, e, p0, n)) {
+            report_status(a.status, MOE_STATUS_BAD_MAP);
+            continue;
+        }
+        cnt += n > 0;
+        grp += static_cast<int>((n + NG - 1) / NG);
+    }
+    int xc = cnt, xg = grp;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int yc = __shfl_up_sync(0xffffffffu, xc, off), yg = __shfl_up_sync(0xffffffffu, xg, off);
+        if (lane >= off) xc += yc, xg += yg;
+    }
+    if (lane == 31) warp_sums[warp][0] = xc, warp_sums[warp][1] = xg;
+    __syncthreads();
+    if (warp == 0) {
+        int vc = lane < nw ? warp_sums[lane][0] : 0, vg = lane < nw ? warp_sums[lane][1] : 0;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int yc = __shfl_up_sync(0xffffffffu, vc, off), yg = __shfl_up_sync(0xffffffffu, vg, off);
+            if (lane >= off) vc += yc, vg += yg;
+        }
+        warp_sums[lane][0] = vc, warp_sums[lane][1] = vg;
+    }
+    __syncthreads();
+    int pc = (warp ? warp_sums[warp - 1][0] : 0) + xc - cnt;
+    int pg = (warp ? warp_sums[warp - 1][1] : 0) + xg - grp;
+    for (int e = e0; e < e1; ++e) {
+        long p0, n;
+        if (expert_rows(a, e, p0, n) && n > 0) {
+            touched[pc] = e;
+            gpre[pc] = pg;
+            ++pc;
+            pg += static_cast<int>((n + NG - 1) / NG);
+        }
+    }
+    const int count = warp_sums[nw - 1][0], total = warp_sums[nw - 1][1];
+    if (threadIdx.x == 0) gpre[count] = total;
+    *ntouched = count;
+    __syncthreads();
+    return total;
+}
+
+// Walks a contiguous range of the balanced item list: (touched expert j,
+// token group of that expert, block of its weight rows), blocks fastest.
+// Every item streams the same weight bytes.  One search finds the start;
+// next() then advances without searching.
+struct ItemWalk {
+    long item, end;
+    int j, grp, blk;
+    int e;       // expert touched[j]
+    int ngrp;    // token groups of expert j
+    const Smem* s;
+    int bpe;
+
+    __device__ ItemWalk(const Smem& sm, long first, long last, int bpe_, int ntouched)
+        : item(first), end(last), s(&sm), bpe(bpe_) {
+        const int gi = static_cast<int>(first / bpe);
+        int lo = 0, hi = max(ntouched - 1, 0);  // last j with gpre[j] <= gi
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (sm.gpre[mid] <= gi)
+                lo = mid;
+            else
+                hi = mid - 1;
+        }
+        j = lo;
+        grp = gi - sm.gpre[lo];
+        blk = static_cast<int>(first % bpe);
+        load();
+    }
+    __device__ void load() {
+        e = s->touched[j];
+        ngrp = s->gpre[j + 1] - s->gpre[j];
+    }
+    __device__ bool valid() const { return item < end; }
+    __device__ void next() {
+        ++item;
+        if (++blk < bpe) return;
+        blk = 0;
+        if (++grp < ngrp) return;
+        grp = 0;
+        ++j;
+        if (item < end) load();
+    }
+};
 
 __device__ __forceinline__ void init_barriers(const Smem& s) {
     if (threadIdx.x == 0) {
@@ -255,26 +366,32 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr int NG = 8 * NT;  // tokens per group
     if (threadIdx.x == 0) grid_dependency_launch();  // the down kernel may start streaming
     extern __shared__ uint8_t smem_raw[];
-    const int e = blockIdx.y;
     const int H = a.H, I = a.ex.inter;
-    const int i0 = blockIdx.x * kGateUpFeat;
-    long p0, n;
-    if (!expert_rows(a, e, p0, n)) {
-        if (threadIdx.x == 0) report_status(a.status, MOE_STATUS_BAD_MAP);
-        return;
-    }
-    if (n == 0) return;
     const int KB = H / 128;
-    const int groups = static_cast<int>((n + NG - 1) / NG);
     const int xstride = 2 * H + 32;
-    const Smem s = carve(smem_raw, NG, xstride, kGuTile);
+    const int E = a.identity ? 1 : a.ex.n;
+    const Smem s = carve(smem_raw, NG, xstride, kGuTile, E);
     init_barriers(s);
+    // Items: (touched expert, token group, block of kGateUpFeat features); each
+    // CTA of the persistent grid takes a contiguous, equal share.
+    const int bpe = I / kGateUpFeat;
+    int ntouched = 0;
+    const long items = build_touched(a, NG, s.touched, s.gpre, &ntouched) * bpe;
+
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (warp == kConsumerWarps) {
-        if (lane == 0)
-            produce(&tm_gate, &tm_up, e * I + i0, KB, static_cast<long>(groups) * KB, s.ring, s.full,
-                    s.empty, s.abort_flag, a.status);
+        if (lane == 0) {
+            tma_prefetch_desc(&tm_gate);
+            tma_prefetch_desc(&tm_up);
+            const uint64_t policy = l2_evict_first_policy();
+            long it = 0;
+            for (ItemWalk w(s, items * blockIdx.x / gridDim.x, items * (blockIdx.x + 1) / gridDim.x, bpe, ntouched);
+                 w.valid(); w.next())
+                if (!produce(&tm_gate, &tm_up, w.e * I + w.blk * kGateUpFeat, KB, KB, it, s.ring, s.full, s.empty,
+                             policy, s.abort_flag, a.status))
+                    break;
+        }
         return;
     }
 
@@ -285,38 +402,49 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t chunk_sel = (mi >> 1) | ((mi & 1) << 1);  // bit 0: chunk j+1, bit 1: up tile
     const uint32_t ring_u32 = smem_u32(s.ring);
     const uint32_t b_lane = smem_u32(s.rows) + g * xstride + 8 * c;
-    const size_t sblk = (static_cast<size_t>(e) * (I / 128) + i0 / 128) * KB;
-    const float* sg = a.ex.s_gate + sblk;
-    const float* su = a.ex.s_up + sblk;
     const long R = static_cast<long>(a.T) * a.K;
 
     long it = 0;
-    for (int grp = 0; grp < groups; ++grp) {
-        const long gp0 = p0 + static_cast<long>(grp) * NG;
-        const int gn = static_cast<int>(min(static_cast<long>(NG), n - static_cast<long>(grp) * NG));
-        if (threadIdx.x < NG) {
-            int t = -1;
-            if (static_cast<int>(threadIdx.x) < gn) {
-                if (a.identity) {
-                    t = static_cast<int>(gp0 + threadIdx.x);
-                } else {
-                    const int r = a.sorted_route[gp0 + threadIdx.x];
-                    if (r >= 0 && r < R)
-                        t = r / a.K;
-                    else
-                        report_status(a.status, MOE_STATUS_BAD_MAP);
+    long staged = -1;  // token group (of the item list) staged in s.rows
+    for (ItemWalk w(s, items * blockIdx.x / gridDim.x, items * (blockIdx.x + 1) / gridDim.x, bpe, ntouched);
+         w.valid(); w.next()) {
+        const int e = w.e, i0 = w.blk * kGateUpFeat;
+        long p0, n;
+        expert_rows(a, e, p0, n);
+        const size_t sblk = (static_cast<size_t>(e) * (I / 128) + i0 / 128) * KB;
+        const float* sg = a.ex.s_gate + sblk;
+        const float* su = a.ex.s_up + sblk;
+        const long gp0 = p0 + static_cast<long>(w.grp) * NG;
+        const int gn = static_cast<int>(min(static_cast<long>(NG), n - static_cast<long>(w.grp) * NG));
+        // Consecutive items of a CTA share a token group for bpe items: its
+        // rows are staged once.
+        const bool restage = staged != w.item / bpe;
+        staged = w.item / bpe;
+        if (restage) {
+            if (threadIdx.x < NG) {
+                int t = -1;
+                if (static_cast<int>(threadIdx.x) < gn) {
+                    if (a.identity) {
+                        t = static_cast<int>(gp0 + threadIdx.x);
+                    } else {
+                        const int r = a.sorted_route[gp0 + threadIdx.x];
+                        if (r >= 0 && r < R)
+                            t = r / a.K;
+                        else
+                            report_status(a.status, MOE_STATUS_BAD_MAP);
+                    }
                 }
+                s.tok[threadIdx.x] = t;
             }
-            s.tok[threadIdx.x] = t;
+            named_barrier_sync(1, kConsumers);
+            stage_rows_f16<NG>(
+                [&](int q) -> const uint16_t* {
+                    const int t = s.tok[q];
+                    return t >= 0 ? a.x + static_cast<size_t>(t) * H : nullptr;
+                },
+                H, s.rows, xstride, s.inv);
+            named_barrier_sync(1, kConsumers);
         }
-        named_barrier_sync(1, kConsumers);
-        stage_rows_f16<NG>(
-            [&](int q) -> const uint16_t* {
-                const int t = s.tok[q];
-                return t >= 0 ? a.x + static_cast<size_t>(t) * H : nullptr;
-            },
-            H, s.rows, xstride, s.inv);
-        named_barrier_sync(1, kConsumers);
 
         float acc[NT][4];
         zero_acc<NT>(acc);
@@ -371,27 +499,31 @@ __global__ void __launch_bounds__(kThreads, 1)
     down_decode_kernel(const __grid_constant__ CUtensorMap tm_down, const FfnArgs a) {
     constexpr int NG = 8 * NT;
     extern __shared__ uint8_t smem_raw[];
-    const int e = blockIdx.y;
     const int H = a.H, I = a.ex.inter;
-    const int n0 = blockIdx.x * kDownRows;
-    // Offsets come from the sort, which finished before the gate/up grid began.
-    long p0, n;
-    if (!expert_rows(a, e, p0, n)) {
-        if (threadIdx.x == 0) report_status(a.status, MOE_STATUS_BAD_MAP);
-        return;
-    }
-    if (n == 0) return;
     const int KB = I / 128;
-    const int groups = static_cast<int>((n + NG - 1) / NG);
     const int hstride = 2 * I + 32;
-    const Smem s = carve(smem_raw, NG, hstride, kDnTile);
+    const int E = a.identity ? 1 : a.ex.n;
+    const Smem s = carve(smem_raw, NG, hstride, kDnTile, E);
     init_barriers(s);
+    // Items: (touched expert, token group, block of kDownRows output rows); each
+    // CTA of the persistent grid takes a contiguous, equal share.  Offsets come
+    // from the sort, which finished before the gate/up grid began.
+    const int bpe = H / kDownRows;
+    int ntouched = 0;
+    const long items = build_touched(a, NG, s.touched, s.gpre, &ntouched) * bpe;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (warp == kConsumerWarps) {
-        if (lane == 0)
-            produce(&tm_down, nullptr, e * H + n0, KB, static_cast<long>(groups) * KB, s.ring, s.full,
-                    s.empty, s.abort_flag, a.status);
+        if (lane == 0) {
+            tma_prefetch_desc(&tm_down);
+            const uint64_t policy = l2_evict_first_policy();
+            long it = 0;
+            for (ItemWalk w(s, items * blockIdx.x / gridDim.x, items * (blockIdx.x + 1) / gridDim.x, bpe, ntouched);
+                 w.valid(); w.next())
+                if (!produce(&tm_down, nullptr, w.e * H + w.blk * kDownRows, KB, KB, it, s.ring, s.full, s.empty,
+                             policy, s.abort_flag, a.status))
+                    break;
+        }
         return;
     }
     grid_dependency_wait();  // h is written by the gate/up grid
@@ -403,41 +535,50 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t chunk_sel = mi >> 1;
     const uint32_t ring_u32 = smem_u32(s.ring);
     const uint32_t b_lane = smem_u32(s.rows) + g * hstride + 8 * c;
-    const float* sd = a.ex.s_down + (static_cast<size_t>(e) * (H / 128) + n0 / 128) * KB;
     const long R = static_cast<long>(a.T) * a.K;
 
     long it = 0;
-    for (int grp = 0; grp < groups; ++grp) {
-        const long gp0 = p0 + static_cast<long>(grp) * NG;
-        const int gn = static_cast<int>(min(static_cast<long>(NG), n - static_cast<long>(grp) * NG));
-        if (threadIdx.x < NG) {
-            int t = -1;
-            float wv = 0.f;
-            if (static_cast<int>(threadIdx.x) < gn) {
-                const long p = gp0 + threadIdx.x;
-                if (a.identity) {
-                    t = static_cast<int>(p);
-                    wv = 1.f;
-                } else {
-                    const int r = a.sorted_route[p];
-                    if (r >= 0 && r < R) {
-                        t = r / a.K;
-                        wv = a.topk_w[r];
+    long staged = -1;  // token group (of the item list) staged in s.rows
+    for (ItemWalk w(s, items * blockIdx.x / gridDim.x, items * (blockIdx.x + 1) / gridDim.x, bpe, ntouched);
+         w.valid(); w.next()) {
+        const int e = w.e, n0 = w.blk * kDownRows;
+        long p0, n;
+        expert_rows(a, e, p0, n);
+        const float* sd = a.ex.s_down + (static_cast<size_t>(e) * (H / 128) + n0 / 128) * KB;
+        const long gp0 = p0 + static_cast<long>(w.grp) * NG;
+        const int gn = static_cast<int>(min(static_cast<long>(NG), n - static_cast<long>(w.grp) * NG));
+        const bool restage = staged != w.item / bpe;
+        staged = w.item / bpe;
+        if (restage) {
+            if (threadIdx.x < NG) {
+                int t = -1;
+                float wv = 0.f;
+                if (static_cast<int>(threadIdx.x) < gn) {
+                    const long p = gp0 + threadIdx.x;
+                    if (a.identity) {
+                        t = static_cast<int>(p);
+                        wv = 1.f;
                     } else {
-                        report_status(a.status, MOE_STATUS_BAD_MAP);
+                        const int r = a.sorted_route[p];
+                        if (r >= 0 && r < R) {
+                            t = r / a.K;
+                            wv = a.topk_w[r];
+                        } else {
+                            report_status(a.status, MOE_STATUS_BAD_MAP);
+                        }
                     }
                 }
+                s.tok[threadIdx.x] = t;
+                s.wr[threadIdx.x] = wv;
             }
-            s.tok[threadIdx.x] = t;
-            s.wr[threadIdx.x] = wv;
+            named_barrier_sync(1, kConsumers);
+            stage_rows_f16<NG>(
+                [&](int q) -> const uint16_t* {
+                    return (q < gn && s.tok[q] >= 0) ? a.h + static_cast<size_t>(gp0 + q) * I : nullptr;
+                },
+                I, s.rows, hstride, s.inv);
+            named_barrier_sync(1, kConsumers);
         }
-        named_barrier_sync(1, kConsumers);
-        stage_rows_f16<NG>(
-            [&](int q) -> const uint16_t* {
-                return (q < gn && s.tok[q] >= 0) ? a.h + static_cast<size_t>(gp0 + q) * I : nullptr;
-            },
-            I, s.rows, hstride, s.inv);
-        named_barrier_sync(1, kConsumers);
 
         float acc[NT][4];
         zero_acc<NT>(acc);
@@ -479,28 +620,51 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-size_t gateup_smem(int NT, int H) { return smem_bytes(8 * NT, 2 * H + 32, kGuTile); }
-size_t down_smem(int NT, int I) { return smem_bytes(8 * NT, 2 * I + 32, kDnTile); }
+size_t gateup_smem(int NT, int H, int E) { return smem_bytes(8 * NT, 2 * H + 32, kGuTile, E); }
+size_t down_smem(int NT, int I, int E) { return smem_bytes(8 * NT, 2 * I + 32, kDnTile, E); }
+
+int sm_count() {
+    static int sms = 0;
+    if (!sms) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (sms <= 0) sms = 148;
+    }
+    return sms;
+}
+
+// Persistent grid: every CTA the GPU holds at once, but no more than the items
+// of the call could use.
+template <class K>
+int persistent_grid(K kernel, size_t smem, long max_items) {
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kThreads, smem) != cudaSuccess || per_sm < 1)
+        per_sm = 1;
+    return static_cast<int>(std::max(1L, std::min(static_cast<long>(per_sm) * sm_count(), max_items)));
+}
 
 constexpr size_t kSmemLimit = 227 * 1024;
 
 template <int NT>
 cudaError_t launch_nt(const FfnArgs& a, const CUtensorMap& tg, const CUtensorMap& tu,
                       const CUtensorMap& td, cudaStream_t stream) {
-    const size_t s1 = gateup_smem(NT, a.H), s2 = down_smem(NT, a.ex.inter);
+    const int E = a.ex.n;
+    const size_t s1 = gateup_smem(NT, a.H, E), s2 = down_smem(NT, a.ex.inter, E);
     cudaError_t err = cudaFuncSetAttribute(gateup_decode_kernel<NT>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(s1));
     if (err != cudaSuccess) return err;
     err = cudaFuncSetAttribute(down_decode_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(s2));
     if (err != cudaSuccess) return err;
-    const int E = a.ex.n;
-    gateup_decode_kernel<NT><<<dim3(a.ex.inter / kGateUpFeat, E), kThreads, s1, stream>>>(tg, tu, a);
+    const int g1 = persistent_grid(gateup_decode_kernel<NT>, s1, static_cast<long>(E) * (a.ex.inter / kGateUpFeat));
+    const int g2 = persistent_grid(down_decode_kernel<NT>, s2, static_cast<long>(E) * (a.H / kDownRows));
+    gateup_decode_kernel<NT><<<g1, kThreads, s1, stream>>>(tg, tu, a);
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
 
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(a.H / kDownRows, E);
+    cfg.gridDim = dim3(g2);
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = s2;
     cfg.stream = stream;
@@ -515,8 +679,8 @@ cudaError_t launch_nt(const FfnArgs& a, const CUtensorMap& tg, const CUtensorMap
 }  // namespace
 
 bool ffn_decode_supported(int H, int I) {
-    return H % kDownRows == 0 && I % kGateUpFeat == 0 && gateup_smem(1, H) <= kSmemLimit &&
-           down_smem(1, I) <= kSmemLimit;
+    return H % kDownRows == 0 && I % kGateUpFeat == 0 && gateup_smem(1, H, MOE_MAX_E) <= kSmemLimit &&
+           down_smem(1, I, MOE_MAX_E) <= kSmemLimit;
 }
 
 cudaError_t launch_ffn_decode(const FfnArgs& a, cudaStream_t stream) {
@@ -528,7 +692,7 @@ cudaError_t launch_ffn_decode(const FfnArgs& a, cudaStream_t stream) {
     if (err != cudaSuccess) return err;
     // Token tile: the host only knows the average rows per expert.
     int NT = a.avg_rows > 12 ? 4 : (a.avg_rows > 6 ? 2 : 1);
-    while (NT > 1 && (gateup_smem(NT, a.H) > kSmemLimit || down_smem(NT, a.ex.inter) > kSmemLimit))
+    while (NT > 1 && (gateup_smem(NT, a.H, a.ex.n) > kSmemLimit || down_smem(NT, a.ex.inter, a.ex.n) > kSmemLimit))
         NT >>= 1;
     switch (NT) {
         case 4: return launch_nt<4>(a, tg, tu, td, stream);
