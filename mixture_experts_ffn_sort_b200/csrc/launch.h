@@ -14,7 +14,7 @@ cudaError_t launch_route(const float* logits, int T, int E, int K, const uint8_t
                          int32_t* ids, float* w, cudaStream_t stream);
 
 // ---------------------------------------------------------------- sort
-// Routes per warp-chunk of the multi-kernel sort, and the largest route count
+// Routes per tile (one thread block) of the multi-kernel sort, and the largest route count
 // handled by the single-block sort.
 constexpr int kSortChunk = 2048;
 constexpr long kSortSmallMaxRoutes = 16384;

@@ -4,13 +4,15 @@
 // (spark_model/layers/nemotron_moe.rs, `prefill` step 5), the NKI Permute
 // Routed Tokens kernel, and the sort with an inverse route map that the aiter
 // gfx950 prefill PR reuses.  A counting sort in three passes:
-//   1. each warp-chunk of routes builds an expert histogram;
+//   1. each chunk of routes builds an expert histogram;
 //   2. an exclusive scan in (expert, chunk) order gives every chunk the first
 //      sorted position of each of its experts, and the per-expert offsets;
-//   3. each warp-chunk walks its routes in order and scatters them, ranking
-//      equal experts within a 32-route step with __match_any_sync.
+//   3. each chunk walks its routes in order and scatters them, ranking equal
+//      experts within a 32-route step with __match_any_sync.
 // Order within an expert is therefore route order: the result is unique and
-// deterministic.  Small inputs run all three passes in one thread block.
+// deterministic.  Small inputs run all three passes in one thread block;
+// larger ones give each tile of kSortChunk routes a thread block (8 warps of
+// 256 routes) and scan per expert over the tiles.
 #include "device_common.cuh"
 #include "launch.h"
 
@@ -144,62 +146,94 @@ __global__ void __launch_bounds__(1024) sort_small_kernel(const int32_t* __restr
 }
 
 // ---------------------------------------------------------------- large: three kernels
+//
+// Tiles of kSortChunk routes, one thread block each; the block's 8 warps take
+// 256 consecutive routes apiece.  The workspace holds one counter per
+// (tile, expert), tile-major.
 
 constexpr int kSortWarpsPerBlock = 8;
+constexpr int kSortWarpRoutes = kSortChunk / kSortWarpsPerBlock;
 
-// counts[e * nchunks + c] = routes of chunk c with expert e.
-__global__ void __launch_bounds__(kSortWarpsPerBlock * 32)
-    sort_count_kernel(const int32_t* __restrict__ ids, long R, int E, int nchunks,
-                      int32_t* __restrict__ counts, int32_t* status) {
-    extern __shared__ int32_t sm[];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int c = blockIdx.x * kSortWarpsPerBlock + warp;
-    int32_t* hist = sm + warp * E;
-    for (int e = lane; e < E; e += 32) hist[e] = 0;
-    __syncwarp();
-    if (c >= nchunks) return;
-    const long rb = static_cast<long>(c) * kSortChunk, re = min(R, rb + kSortChunk);
-    if (count_chunk(ids, rb, re, E, hist) && lane == 0) report_status(status, MOE_STATUS_BAD_ID);
-    __syncwarp();
-    for (int e = lane; e < E; e += 32) counts[static_cast<size_t>(e) * nchunks + c] = hist[e];
+// Per-warp expert histograms of tile b into hist[warp][E] (shared memory).
+// Returns (in every thread of the warp) whether an id outside [0, E) was seen.
+__device__ __forceinline__ bool count_tile(const int32_t* __restrict__ ids, long R, int E, int32_t* hist) {
+    const int warp = threadIdx.x >> 5;
+    for (int i = threadIdx.x; i < kSortWarpsPerBlock * E; i += blockDim.x) hist[i] = 0;
+    __syncthreads();
+    const long rb = static_cast<long>(blockIdx.x) * kSortChunk + static_cast<long>(warp) * kSortWarpRoutes;
+    const bool bad = count_chunk(ids, min(R, rb), min(R, rb + kSortWarpRoutes), E, hist + warp * E);
+    __syncthreads();
+    return bad;
 }
 
-// In-place exclusive scan of counts[E * nchunks] (expert-major); offsets[e] is
-// the scan value at (e, chunk 0) and offsets[E] the total.
+// counts[b * E + e] = routes of tile b with expert e.
+__global__ void __launch_bounds__(kSortWarpsPerBlock * 32)
+    sort_count_kernel(const int32_t* __restrict__ ids, long R, int E, int32_t* __restrict__ counts,
+                      int32_t* status) {
+    extern __shared__ int32_t sm[];
+    if (count_tile(ids, R, E, sm) && (threadIdx.x & 31) == 0) report_status(status, MOE_STATUS_BAD_ID);
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        int c = 0;
+#pragma unroll
+        for (int w = 0; w < kSortWarpsPerBlock; ++w) c += sm[w * E + e];
+        counts[static_cast<size_t>(blockIdx.x) * E + e] = c;
+    }
+}
+
+// One thread per expert (E <= blockDim.x): the expert's total over the tiles,
+// offsets = exclusive scan of the totals, and counts[b * E + e] replaced by
+// tile b's first sorted position of expert e.
 __global__ void __launch_bounds__(1024)
-    sort_scan_kernel(int32_t* __restrict__ counts, int E, int nchunks, long R,
-                     int32_t* __restrict__ offsets, int32_t* __restrict__ sorted_route) {
+    sort_scan_kernel(int32_t* __restrict__ counts, int E, int ntiles, long R, int32_t* __restrict__ offsets,
+                     int32_t* __restrict__ sorted_route) {
     __shared__ int scratch[32];
-    const int N = E * nchunks;
-    const int per = (N + blockDim.x - 1) / blockDim.x;
-    const int i0 = min(N, static_cast<int>(threadIdx.x) * per), i1 = min(N, i0 + per);
-    int s = 0;
-    for (int i = i0; i < i1; ++i) s += counts[i];
+    const int e = threadIdx.x;
+    int tot = 0;
+    if (e < E) {
+        int part[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+        int b = 0;
+        for (; b + 8 <= ntiles; b += 8)
+#pragma unroll
+            for (int k = 0; k < 8; ++k) part[k] += counts[static_cast<size_t>(b + k) * E + e];
+        for (; b < ntiles; ++b) part[0] += counts[static_cast<size_t>(b) * E + e];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) tot += part[k];
+    }
     int total;
-    int prefix = block_exclusive_scan(s, scratch, &total);
-    for (int i = i0; i < i1; ++i) {
-        const int c = counts[i];
-        if (i % nchunks == 0) offsets[i / nchunks] = prefix;
-        counts[i] = prefix;
-        prefix += c;
+    int run = block_exclusive_scan(tot, scratch, &total);
+    if (e < E) {
+        offsets[e] = run;
+        for (int b = 0; b < ntiles; ++b) {
+            const size_t i = static_cast<size_t>(b) * E + e;
+            const int c = counts[i];
+            counts[i] = run;
+            run += c;
+        }
     }
     if (threadIdx.x == 0) offsets[E] = total;
     for (long p = total + threadIdx.x; p < R; p += blockDim.x) sorted_route[p] = -1;
 }
 
+// Tile b: recount per warp, turn the counts into per-warp cursors starting at
+// the tile's base positions, and scatter each warp's routes in order.
 __global__ void __launch_bounds__(kSortWarpsPerBlock * 32)
-    sort_scatter_kernel(const int32_t* __restrict__ ids, long R, int E, int nchunks,
-                        const int32_t* __restrict__ base, int32_t* __restrict__ sorted_route,
-                        int32_t* __restrict__ inv_route) {
+    sort_scatter_kernel(const int32_t* __restrict__ ids, long R, int E, const int32_t* __restrict__ base,
+                        int32_t* __restrict__ sorted_route, int32_t* __restrict__ inv_route) {
     extern __shared__ int32_t sm[];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int c = blockIdx.x * kSortWarpsPerBlock + warp;
-    if (c >= nchunks) return;
-    int32_t* cursor = sm + warp * E;
-    for (int e = lane; e < E; e += 32) cursor[e] = base[static_cast<size_t>(e) * nchunks + c];
-    __syncwarp();
-    const long rb = static_cast<long>(c) * kSortChunk, re = min(R, rb + kSortChunk);
-    scatter_chunk(ids, rb, re, E, cursor, sorted_route, inv_route);
+    count_tile(ids, R, E, sm);
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        int run = base[static_cast<size_t>(blockIdx.x) * E + e];
+#pragma unroll
+        for (int w = 0; w < kSortWarpsPerBlock; ++w) {
+            const int c = sm[w * E + e];
+            sm[w * E + e] = run;
+            run += c;
+        }
+    }
+    __syncthreads();
+    const int warp = threadIdx.x >> 5;
+    const long rb = static_cast<long>(blockIdx.x) * kSortChunk + static_cast<long>(warp) * kSortWarpRoutes;
+    scatter_chunk(ids, min(R, rb), min(R, rb + kSortWarpRoutes), E, sm + warp * E, sorted_route, inv_route);
 }
 
 int small_sort_warps(int E) {
@@ -225,15 +259,13 @@ cudaError_t launch_sort(const int32_t* ids, long R, int E, int32_t* offsets, int
                                                         status);
         return cudaGetLastError();
     }
-    const int nchunks = static_cast<int>((R + kSortChunk - 1) / kSortChunk);
+    const int ntiles = static_cast<int>((R + kSortChunk - 1) / kSortChunk);
     int32_t* counts = static_cast<int32_t*>(ws);
-    const int blocks = (nchunks + kSortWarpsPerBlock - 1) / kSortWarpsPerBlock;
     const size_t smem = static_cast<size_t>(kSortWarpsPerBlock) * E * sizeof(int32_t);
-    sort_count_kernel<<<blocks, kSortWarpsPerBlock * 32, smem, stream>>>(ids, R, E, nchunks, counts,
-                                                                         status);
-    sort_scan_kernel<<<1, 1024, 0, stream>>>(counts, E, nchunks, R, offsets, sorted_route);
-    sort_scatter_kernel<<<blocks, kSortWarpsPerBlock * 32, smem, stream>>>(
-        ids, R, E, nchunks, counts, sorted_route, inv_route);
+    sort_count_kernel<<<ntiles, kSortWarpsPerBlock * 32, smem, stream>>>(ids, R, E, counts, status);
+    sort_scan_kernel<<<1, 1024, 0, stream>>>(counts, E, ntiles, R, offsets, sorted_route);
+    sort_scatter_kernel<<<ntiles, kSortWarpsPerBlock * 32, smem, stream>>>(ids, R, E, counts, sorted_route,
+                                                                          inv_route);
     return cudaGetLastError();
 }
 
