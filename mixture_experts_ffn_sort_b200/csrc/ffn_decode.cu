@@ -360,7 +360,7 @@ __device__ __forceinline__ void init_barriers(const Smem& s) {
 // ------------------------------------------------------------------ gate/up + SwiGLU
 
 template <int NT>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
     gateup_decode_kernel(const __grid_constant__ CUtensorMap tm_gate,
                          const __grid_constant__ CUtensorMap tm_up, const FfnArgs a) {
     constexpr int NG = 8 * NT;  // tokens per group
@@ -495,7 +495,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ------------------------------------------------------------------ down + affinity
 
 template <int NT>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
     down_decode_kernel(const __grid_constant__ CUtensorMap tm_down, const FfnArgs a) {
     constexpr int NG = 8 * NT;
     extern __shared__ uint8_t smem_raw[];
