@@ -34,11 +34,23 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict
         const int t = static_cast<int>(idx / chunks);
         const int c = static_cast<int>(idx - static_cast<long>(t) * chunks);
         float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        for (int j = 0; j < K; ++j) {
-            const int32_t p = __ldg(inv_route + static_cast<size_t>(t) * K + j);
-            if (p < 0) continue;
-            const uint4 v = __ldg(reinterpret_cast<const uint4*>(y_sorted + static_cast<size_t>(p) * H) + c);
-            add_bf16x8(acc, v);
+        // Slots in batches of 8: all positions, then all rows, then the sums
+        // in slot order (independent loads overlap; the order of the fp32
+        // additions is unchanged).
+        for (int j0 = 0; j0 < K; j0 += 8) {
+            int32_t p[8];
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj)
+                p[jj] = j0 + jj < K ? __ldg(inv_route + static_cast<size_t>(t) * K + j0 + jj) : -1;
+            uint4 v[8];
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj)
+                v[jj] = p[jj] >= 0
+                            ? __ldg(reinterpret_cast<const uint4*>(y_sorted + static_cast<size_t>(p[jj]) * H) + c)
+                            : make_uint4(0, 0, 0, 0);
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj)
+                if (p[jj] >= 0) add_bf16x8(acc, v[jj]);
         }
         if (y_shared) {
             const uint4 v = __ldg(reinterpret_cast<const uint4*>(y_shared + static_cast<size_t>(t) * H) + c);

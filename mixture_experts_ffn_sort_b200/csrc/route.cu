@@ -3,8 +3,9 @@
 // Router of the FP8 MoE decode kernel page's serving contract ("softmax ->
 // top-8 -> norm", dstair/gated-deltanet-nki-trainium) and the NKI Router Top-K
 // kernel.  One warp per token: each lane holds ceil(E/32) logits in registers;
-// K rounds of a warp-wide arg-max (larger logit first, lower expert id on ties)
-// pick the experts in descending order.  Softmax is strictly increasing in the
+// K rounds of a warp-wide arg-max (larger logit first, lower expert id on ties;
+// two redux.sync reductions on an order-preserving key) pick the experts in
+// descending order.  Softmax is strictly increasing in the
 // logit, so this is the top-K of the probabilities; the weights are
 // exp(l_j - l_max) / sum_j' exp(l_j' - l_max), the full-softmax normaliser
 // cancelling in the renormalisation.
@@ -52,15 +53,14 @@ __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ lo
                 bi = e;
             }
         }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-            const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-            const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-            if (ov > bv || (ov == bv && oi < bi)) {
-                bv = ov;
-                bi = oi;
-            }
-        }
+        // Warp arg-max: the largest value, then the lowest expert id holding it,
+        // as two warp reductions on an order-preserving integer key.
+        const float bz = bv == 0.f ? 0.f : bv;  // -0 and +0 are the same logit
+        const uint32_t u = __float_as_uint(bz);
+        const uint32_t key = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+        const uint32_t kmax = __reduce_max_sync(0xffffffffu, key);
+        bi = static_cast<int>(__reduce_min_sync(0xffffffffu, key == kmax ? static_cast<uint32_t>(bi) : 0xffffffffu));
+        bv = __uint_as_float((kmax & 0x80000000u) ? (kmax & 0x7fffffffu) : ~kmax);
         if (bi >= E) bi = E - 1;  // only reachable with NaN logits (unspecified ids)
         if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
         if (j == 0) lmax = bv;

@@ -13,6 +13,8 @@
 // deterministic.  Small inputs run all three passes in one thread block;
 // larger ones give each tile of kSortChunk routes a thread block (8 warps of
 // 256 routes) and scan per expert over the tiles.
+#include <algorithm>
+
 #include "device_common.cuh"
 #include "launch.h"
 
@@ -27,11 +29,11 @@ __device__ __forceinline__ uint32_t lanemask_lt() {
 }
 
 // Scatter one warp-chunk [r_begin, r_end) given the chunk's start positions
-// `cursor[e]` (shared memory, advanced in place).
+// `cursor[e * stride]` (shared memory, advanced in place).
 __device__ __forceinline__ void scatter_chunk(const int32_t* __restrict__ ids, long r_begin,
                                               long r_end, int E, int32_t* cursor,
                                               int32_t* __restrict__ sorted_route,
-                                              int32_t* __restrict__ inv_route) {
+                                              int32_t* __restrict__ inv_route, int stride = 1) {
     const int lane = threadIdx.x & 31;
     const uint32_t lt = lanemask_lt();
     for (long r0 = r_begin; r0 < r_end; r0 += 32) {
@@ -41,10 +43,10 @@ __device__ __forceinline__ void scatter_chunk(const int32_t* __restrict__ ids, l
         const bool ok = in && e >= 0 && e < E;
         const uint32_t peers = __match_any_sync(0xffffffffu, ok ? e : (E + lane));
         int32_t pos = 0;
-        if (ok) pos = cursor[e] + __popc(peers & lt);
+        if (ok) pos = cursor[e * stride] + __popc(peers & lt);
         __syncwarp();
         // The highest lane of each group of equal experts advances the cursor.
-        if (ok && (peers >> lane) == 1u) cursor[e] += __popc(peers);
+        if (ok && (peers >> lane) == 1u) cursor[e * stride] += __popc(peers);
         __syncwarp();
         if (ok) {
             sorted_route[pos] = static_cast<int32_t>(r);
@@ -55,16 +57,16 @@ __device__ __forceinline__ void scatter_chunk(const int32_t* __restrict__ ids, l
     }
 }
 
-// Count one warp-chunk into hist[E] (shared memory, zeroed by the caller).
-// Returns true if an id outside [0, E) was seen.
+// Count one warp-chunk into hist[e * stride] (shared memory, zeroed by the
+// caller).  Returns true if an id outside [0, E) was seen.
 __device__ __forceinline__ bool count_chunk(const int32_t* __restrict__ ids, long r_begin,
-                                            long r_end, int E, int32_t* hist) {
+                                            long r_end, int E, int32_t* hist, int stride = 1) {
     const int lane = threadIdx.x & 31;
     bool bad = false;
     for (long r = r_begin + lane; r < r_end; r += 32) {
         const int e = ids[r];
         if (e >= 0 && e < E)
-            atomicAdd(&hist[e], 1);
+            atomicAdd(&hist[e * stride], 1);
         else
             bad = true;
     }
@@ -102,7 +104,8 @@ __device__ int block_exclusive_scan(int v, int* scratch /*[32]*/, int* total) {
 
 // ---------------------------------------------------------------- small: one block
 
-// smem: hist[NW][E] ints, then 32 ints of scan scratch.
+// smem: hist[E][NW] ints (expert-major, so the scan in (expert, warp) order
+// reads it contiguously), then 32 ints of scan scratch.
 __global__ void __launch_bounds__(1024) sort_small_kernel(const int32_t* __restrict__ ids, long R,
                                                           int E, int32_t* __restrict__ offsets,
                                                           int32_t* __restrict__ sorted_route,
@@ -111,14 +114,14 @@ __global__ void __launch_bounds__(1024) sort_small_kernel(const int32_t* __restr
     extern __shared__ int32_t sm[];
     const int NW = blockDim.x >> 5;
     const int warp = threadIdx.x >> 5;
-    int32_t* hist = sm;                      // [NW][E]
+    int32_t* hist = sm;                      // [E][NW]
     int32_t* scratch = sm + NW * E;          // [32]
     for (int i = threadIdx.x; i < NW * E; i += blockDim.x) hist[i] = 0;
     __syncthreads();
 
     const long chunk = ((R + NW - 1) / NW + 31) / 32 * 32;
     const long rb = min(R, warp * chunk), re = min(R, rb + chunk);
-    if (count_chunk(ids, rb, re, E, hist + warp * E) && (threadIdx.x & 31) == 0)
+    if (count_chunk(ids, rb, re, E, hist + warp, NW) && (threadIdx.x & 31) == 0)
         report_status(status, MOE_STATUS_BAD_ID);
     __syncthreads();
 
@@ -128,21 +131,20 @@ __global__ void __launch_bounds__(1024) sort_small_kernel(const int32_t* __restr
     const int per = (N + blockDim.x - 1) / blockDim.x;
     const int i0 = min(N, static_cast<int>(threadIdx.x) * per), i1 = min(N, i0 + per);
     int s = 0;
-    for (int i = i0; i < i1; ++i) s += hist[(i % NW) * E + i / NW];
+    for (int i = i0; i < i1; ++i) s += hist[i];
     int total;
     int prefix = block_exclusive_scan(s, scratch, &total);
     for (int i = i0; i < i1; ++i) {
-        const int idx = (i % NW) * E + i / NW;
-        const int c = hist[idx];
+        const int c = hist[i];
         if (i % NW == 0) offsets[i / NW] = prefix;
-        hist[idx] = prefix;
+        hist[i] = prefix;
         prefix += c;
     }
     if (threadIdx.x == 0) offsets[E] = total;
     for (long p = total + threadIdx.x; p < R; p += blockDim.x) sorted_route[p] = -1;
     __syncthreads();
 
-    scatter_chunk(ids, rb, re, E, hist + warp * E, sorted_route, inv_route);
+    scatter_chunk(ids, rb, re, E, hist + warp, sorted_route, inv_route, NW);
 }
 
 // ---------------------------------------------------------------- large: three kernels
@@ -253,7 +255,8 @@ size_t sort_workspace_bytes(long R, int E) {
 cudaError_t launch_sort(const int32_t* ids, long R, int E, int32_t* offsets, int32_t* sorted_route,
                         int32_t* inv_route, void* ws, int32_t* status, cudaStream_t stream) {
     if (R <= kSortSmallMaxRoutes) {
-        const int nw = small_sort_warps(E);
+        // As many warps as 32-route slices, up to what shared memory holds.
+        const int nw = static_cast<int>(std::min<long>(small_sort_warps(E), std::max<long>(1, (R + 31) / 32)));
         const size_t smem = (static_cast<size_t>(nw) * E + 32) * sizeof(int32_t);
         sort_small_kernel<<<1, nw * 32, smem, stream>>>(ids, R, E, offsets, sorted_route, inv_route,
                                                         status);
