@@ -213,7 +213,11 @@ def test_route_ties():
     np.testing.assert_allclose(wts.cpu().numpy(), ow, rtol=W_RTOL, atol=W_ATOL)
 
 
-@pytest.mark.parametrize("T,K,E", [(1024, 32, 1024), (700, 10, 512), (5000, 8, 3), (1, 1, 1)])
+# Single-block sort (R <= 16384) and tiled sort (2048-route tiles of 8 x 256):
+# exact tiles, a partial last tile, a partial last warp, R just above the
+# single-block limit, one expert, E = MOE_MAX_E.
+@pytest.mark.parametrize("T,K,E", [(1024, 32, 1024), (700, 10, 512), (5000, 8, 3), (1, 1, 1), (16384, 1, 64),
+                                   (16385, 1, 7), (4097, 4, 513), (20480, 1, 1), (2305, 8, 256), (512, 8, 256)])
 def test_sort_shapes(T, K, E):
     ids = wl.random_ids(T, K, E, seed=T, distinct=E >= K) if E >= K else \
         np.random.default_rng(0).integers(0, E, (T, K)).astype(np.int32)
@@ -224,7 +228,7 @@ def test_sort_shapes(T, K, E):
     assert np.array_equal(inv.cpu().numpy(), o[2])
 
 
-@pytest.mark.parametrize("T", [100, 4000])
+@pytest.mark.parametrize("T", [100, 4000, 6000])
 def test_sort_out_of_range_ids_are_skipped(T):
     K, E = 4, 16
     ids = wl.random_ids(T, K, E, seed=5)
