@@ -16,11 +16,12 @@
 //    so the FP8 decode writes tensor memory, not shared memory;
 //  * warp 0: the weight tile's FP8 bytes by TMA in stages of 128 reduction
 //    columns (128-byte rows, 128-byte swizzle), 64 KB ahead;
-//  * warps 2-3: the token rows into the 128-byte-swizzled K-major layout the
-//    MMA reads -- x rows gathered through sorted_route by cp.async (each
+//  * the token rows into the 128-byte-swizzled K-major layout the MMA reads:
+//    gate/up gathers x rows through sorted_route with cp.async on warps 2-7
+//    (the per-SM gather rate grows with the number of issuing warps; each
 //    thread keeps its rows' token indices in registers for the whole tile and
-//    arrives on the stage's mbarrier when its copies land) for gate/up,
-//    contiguous rows of h as one 2-D TMA tile for down -- up to 4 stages
+//    arrives on the stage's mbarrier when its copies land); down loads
+//    contiguous rows of h as one 2-D TMA tile from warp 2 -- up to 4 stages
 //    ahead;
 //  * transform warps 8-15: each thread owns one TMEM lane (one weight row)
 //    and half of a stage's columns, decodes its FP8 codes to
@@ -29,12 +30,14 @@
 //  * warp 1: one thread issues tcgen05.mma (kind::f16, A in TMEM, B in
 //    shared memory, fp32 accumulator D in TMEM, double-buffered so the
 //    epilogue of one tile overlaps the main loop of the next);
-//  * epilogue warps 4-7: tcgen05.ld of D; in each 32-lane quarter of a
-//    gate/up M-tile, lanes 0-15 hold the gate rows and lanes 16-31 the up
-//    rows of the same 16 features, so SwiGLU needs one shuffle; the down
-//    epilogue multiplies by the route weight.  bf16 results are staged in
-//    shared memory (one row per token) and leave as one 256-byte bulk async
-//    copy per token row.
+//  * epilogue warps 4-7 (in gate/up, between their gathers: after issuing the
+//    next item's first stages): tcgen05.ld 16x256b of D; in each 32-lane
+//    quarter of a gate/up M-tile, lanes 0-15 hold the gate rows and lanes
+//    16-31 the up rows of the same 16 features, so a thread receives gate and
+//    up of the same (feature, token) pairs and applies SwiGLU in place; the
+//    down epilogue multiplies by the route weight.  bf16 results go through
+//    a 128-byte-swizzled staging tile (stmatrix.trans, one row per token) and
+//    leave as 32-row TMA tensor stores, the last rows as 16-byte stores.
 // Every mbarrier wait is bounded; an expired wait sets a CTA-wide abort flag
 // and every role runs to the end without waiting, so the CTA always reaches
 // the TMEM de-allocation.
@@ -63,6 +66,9 @@ template <int MODE> struct Cfg;
 // warps 2-3 load token rows.
 constexpr int kWarpTma = 0, kWarpMma = 1, kWarpTok = 2, kWarpEpi = 4, kWarpXform = 8;
 constexpr int kTokThreads = 64;
+// gate/up: the token rows are gathered by warps 2-7 (the epilogue warps 4-7
+// gather too: one cp.async stream per warp caps the per-SM gather rate).
+constexpr int kGatherThreads = 192;
 constexpr int kNumWarps = 16;
 constexpr int kThreads = kNumWarps * 32;
 constexpr int kXformWarps = 8;
@@ -270,7 +276,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&B->w_empty[s], kXformWarps);
         }
         for (int s = 0; s < kSB; ++s) {
-            mbar_init(&B->b_full[s], MODE == kGateUp ? kTokThreads : 1);
+            mbar_init(&B->b_full[s], MODE == kGateUp ? kGatherThreads : 1);
             mbar_init(&B->b_done[s], 1);
         }
         for (int s = 0; s < kSA; ++s) {
@@ -330,159 +336,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
         }
-    } else if (warp == kWarpTok || warp == kWarpTok + 1) {
-        // ------------------------------------------------ token rows
+    } else if (warp >= kWarpTok && warp < kWarpXform) {
+        // ------------------------------------------------ token rows (warps 2-7) and epilogue (warps 4-7)
         // gate/up: rows of x gathered through sorted_route by cp.async (16 bytes
-        // per copy, 64 threads), each thread arriving on the stage barrier when
-        // its copies land; down: contiguous rows of h as one 2-D TMA tile.
+        // per copy) by warps 2-7, each thread arriving on the stage barrier when
+        // its copies land; warps 4-7 then run the item's epilogue.  down:
+        // contiguous rows of h as one 2-D TMA tile (warp 2), epilogue on warps 4-7.
         // Padding rows of the last MMA column group are left stale: column j of
         // D depends on token row j only, and the epilogue drops those columns.
-        const int lt = threadIdx.x - kWarpTok * 32;  // 0..63
-        // gate/up: thread lt copies 16-byte chunk ch of rows r0 + 8k, keeping
-        // those rows' token indices in registers for the whole tile; the
-        // 128-byte swizzle of those rows is the same for every k.
-        const int r0 = lt >> 3, ch = lt & 7;
-        const uint32_t cch = static_cast<uint32_t>((ch ^ (r0 & 7)) << 4);
-        constexpr int kRowsPerThread = kNMax / 8;
-        uint32_t tok[kRowsPerThread];
-        if (MODE == kDown) grid_dependency_wait();  // h comes from the gate/up grid
-        if (MODE == kDown && lt == 0)
-            for (int pt = 0; pt < (has_sh ? 2 : 1); ++pt) tma_prefetch_desc(&M.act[pt]);
-        long g = 0;
-        for (int item = blockIdx.x; item < total; item += gridDim.x) {
-            const Tile t = tile_of<MODE>(a, pre, item);
-            const PartCfg pc = part_cfg<MODE>(a, t.pt);
-            if (MODE == kGateUp) {
-                named_barrier_sync(2, kTokThreads);
-                bool bad = false;
-                for (int r = lt; r < t.n; r += kTokThreads) {
-                    int tk = 0;
-                    const long p = t.p0 + r;
-                    if (t.pt) {
-                        tk = static_cast<int>(p);
-                    } else {
-                        const int rt = a.sorted_route[p];
-                        if (rt >= 0 && rt < R)
-                            tk = rt / a.K;
-                        else
-                            bad = true;
-                    }
-                    row_tok[r] = tk;
-                }
-                if (bad) report_status(a.status, MOE_STATUS_BAD_MAP);
-                named_barrier_sync(2, kTokThreads);
-#pragma unroll
-                for (int k = 0; k < kRowsPerThread; ++k) tok[k] = r0 + 8 * k < t.n ? row_tok[r0 + 8 * k] : 0u;
-            }
-            for (int kb = 0; kb < pc.KB; ++kb, ++g) {
-                const int s = static_cast<int>(g % kSB);
-                if (g >= kSB) wait_bar(&B->b_done[s], static_cast<uint32_t>((g / kSB - 1) & 1), B, a.status);
-                uint8_t* dst = b_ring + s * kBStage;
-                if (MODE == kGateUp) {
-                    const uint32_t bdst = smem_u32(dst) + r0 * 128 + cch;
-                    const uint16_t* xs = a.x + kb * 64 + ch * 8;
-#pragma unroll
-                    for (int k = 0; k < kRowsPerThread; ++k)
-                        if (r0 + 8 * k < t.n)
-                            cp_async16(bdst + k * 1024, xs + static_cast<size_t>(tok[k]) * H, 16u);
-                    cp_async_arrive_noinc(&B->b_full[s]);
-                } else if (lt == 0) {
-                    mbar_arrive_expect_tx(&B->b_full[s], kBStage);
-                    tma_load_2d(dst, &M.act[t.pt], &B->b_full[s], kb * 64, static_cast<int>(t.p0));
-                }
-            }
-        }
-        if (MODE == kGateUp) cp_async_wait<0>();
-    } else if (warp >= kWarpXform) {
-        // ------------------------------------------------ transform: FP8 -> bf16 -> TMEM (A)
-        // gate/up: warp (q, mt) owns lane quarter q of M-tile mt and all 64 codes
-        // of a step; down: warp (q, hf) owns lane quarter q and half of the codes.
-        const int q = warp & 3, hi = (warp - kWarpXform) >> 2;
-        const int xt = threadIdx.x - kWarpXform * 32;           // 0..255
-        const int row = 32 * q + lane;  // TMEM lane = weight row of the M-tile
-        constexpr int NW = MODE == kGateUp ? 32 : 16;           // words (bf16 pairs) per thread per step
-        long g = 0;                                             // MMA steps (64 columns)
-        for (int item = blockIdx.x; item < total; item += gridDim.x) {
-            const Tile t = tile_of<MODE>(a, pre, item);
-            const PartCfg pc = part_cfg<MODE>(a, t.pt);
-            const ExpertsView& ev = t.pt ? a.sh : a.ex;
-            const int KB = pc.KB, KB128 = pc.KB128;
-            // Block scales of the item, staged once: gate/up -> [gate, up][KB128],
-            // down -> [output block][KB128].
-            named_barrier_sync(3, kXformWarps * 32);
-            if (MODE == kGateUp) {
-                const size_t off = (static_cast<size_t>(t.e) * (pc.I / 128) + t.fb0) * KB128;
-                for (int i = xt; i < 2 * KB128; i += kXformWarps * 32)
-                    sc_sm[i] = __ldg((i < KB128 ? ev.s_gate : ev.s_up) + off + (i % KB128));
-            } else {
-                for (int i = xt; i < t.nfb * KB128; i += kXformWarps * 32) {
-                    const int f = i / KB128, k = i - f * KB128;
-                    sc_sm[i] = __ldg(ev.s_down + (static_cast<size_t>(t.e) * (H / 128) + (t.fb0 + f)) * KB128 + k);
-                }
-            }
-            named_barrier_sync(3, kXformWarps * 32);
-            // Source row in the weight stage.  gate/up: in the lane quarter of
-            // warp q, lanes 0-15 hold the gate rows and lanes 16-31 the up rows
-            // of features 16q .. 16q+15 of the M-tile (so the eight lanes of a
-            // shared-memory phase read eight different rows).
-            const bool up_row = MODE == kGateUp && (lane & 16);
-            const int srow = MODE == kGateUp ? hi * 64 + 16 * q + (lane & 15) : row;
-            const int sub = up_row ? kWStage / 2 : 0;
-            const int c0 = MODE == kGateUp ? 0 : 2 * hi;  // first 16-byte chunk of this thread in a step
-            for (int f = 0; f < t.nfb; ++f) {
-                const float* scr = sc_sm + (MODE == kGateUp ? (up_row ? KB128 : 0) : f * KB128);
-                for (int kb = 0; kb < KB; ++kb, ++g) {
-                    const long gw = g >> 1;  // weight stage holding this step
-                    const long u = MODE == kGateUp ? 2 * g + hi : g;  // A unit of this warp's work
-                    const int sw = static_cast<int>(gw % kSW), sa = static_cast<int>(u % kSA);
-                    const bool ok1 = wait_bar(&B->w_full[sw], static_cast<uint32_t>((gw / kSW) & 1), B, a.status);
-                    bool ok2 = true;
-                    if (u >= kSA)
-                        ok2 = wait_bar(&B->a_done[sa], static_cast<uint32_t>((u / kSA - 1) & 1), B, a.status);
-                    uint32_t v[NW];
-                    if (ok1 && ok2) {
-                        const float sc = scr[kb >> 1];
-                        const uint8_t* base = w_ring + sw * kWStage + sub + srow * 128;
-#pragma unroll
-                        for (int c = 0; c < NW / 8; ++c) {
-                            const int chunk = (g & 1) * 4 + c0 + c;
-                            const uint4 w = *reinterpret_cast<const uint4*>(base + ((chunk ^ (srow & 7)) << 4));
-                            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-                            for (int k = 0; k < 4; ++k) {
-                                v[c * 8 + 2 * k] = decode_scaled(static_cast<uint16_t>(ws[k] & 0xFFFFu), sc);
-                                v[c * 8 + 2 * k + 1] = decode_scaled(static_cast<uint16_t>(ws[k] >> 16), sc);
-                            }
-                        }
-                    } else {
-#pragma unroll
-                        for (int k = 0; k < NW; ++k) v[k] = 0;
-                    }
-                    __syncwarp();
-                    if ((g & 1) && lane == 0) mbar_arrive(&B->w_empty[sw]);
-                    const uint32_t acol = kACol + sa * 32 + (MODE == kGateUp ? 0 : hi * 16);
-                    if constexpr (MODE == kGateUp)
-                        tmem_st32(tmem + (static_cast<uint32_t>(32 * q) << 16) + acol, v);
-                    else
-                        tmem_st16(tmem + (static_cast<uint32_t>(32 * q) << 16) + acol, v);
-                    tmem_st_wait();
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&B->a_full[sa]);
-                }
-            }
-        }
-    } else if (warp >= kWarpEpi) {
-        // ------------------------------------------------ epilogue
-        // bf16 results go through the staging tile (row = token column, 128
-        // features) and leave as 16-byte row-contiguous stores.
+        const bool epi_warp = warp >= kWarpEpi;
         const int q = warp & 3;
         const int et = threadIdx.x - kWarpEpi * 32;  // 0..127
         const uint32_t otile_u32 = smem_u32(otile);
         int uses[2] = {0, 0};
         int tc = 0;
-        for (int item = blockIdx.x; item < total; item += gridDim.x) {
-            const Tile t = tile_of<MODE>(a, pre, item);
+        // Epilogue of one item (warps 4-7).
+        auto epilogue = [&](const Tile& t) {
             const PartCfg pc = part_cfg<MODE>(a, t.pt);
             if (MODE == kDown) {
                 // Route weight of every column of the item, staged once (1 for
@@ -597,8 +466,167 @@ __global__ void __launch_bounds__(kThreads, 1)
                         *reinterpret_cast<const uint4*>(otile + hh * kOHalf + rr * 128 + ((c8 ^ (rr & 7)) << 4));
                 }
             }
+        };
+        if (MODE == kGateUp) {
+            // Thread lt copies 16-byte chunk ch of rows r0 + 24k, keeping those
+            // rows' token indices in registers for the whole tile; the 128-byte
+            // swizzle of those rows is the same for every k.
+            const int lt = threadIdx.x - kWarpTok * 32;  // 0..191
+            const int r0 = lt >> 3, ch = lt & 7;
+            const uint32_t cch = static_cast<uint32_t>((ch ^ (r0 & 7)) << 4);
+            constexpr int kRowsPerThread = kNMax / (kGatherThreads / 8);
+            uint32_t tok[kRowsPerThread];
+            long g = 0;
+            Tile prev{};
+            bool have_prev = false;
+            for (int item = blockIdx.x; item < total; item += gridDim.x) {
+                const Tile t = tile_of<MODE>(a, pre, item);
+                const PartCfg pc = part_cfg<MODE>(a, t.pt);
+                named_barrier_sync(2, kGatherThreads);
+                bool bad = false;
+                for (int r = lt; r < t.n; r += kGatherThreads) {
+                    int tk = 0;
+                    const long p = t.p0 + r;
+                    if (t.pt) {
+                        tk = static_cast<int>(p);
+                    } else {
+                        const int rt = a.sorted_route[p];
+                        if (rt >= 0 && rt < R)
+                            tk = rt / a.K;
+                        else
+                            bad = true;
+                    }
+                    row_tok[r] = tk;
+                }
+                if (bad) report_status(a.status, MOE_STATUS_BAD_MAP);
+                named_barrier_sync(2, kGatherThreads);
+#pragma unroll
+                for (int k = 0; k < kRowsPerThread; ++k)
+                    tok[k] = r0 + 24 * k < t.n ? row_tok[r0 + 24 * k] : 0u;
+                for (int kb = 0; kb < pc.KB; ++kb, ++g) {
+                    const int s = static_cast<int>(g % kSB);
+                    if (g >= kSB) wait_bar(&B->b_done[s], static_cast<uint32_t>((g / kSB - 1) & 1), B, a.status);
+                    const uint32_t bdst = smem_u32(b_ring + s * kBStage) + r0 * 128 + cch;
+                    const uint16_t* xs = a.x + kb * 64 + ch * 8;
+#pragma unroll
+                    for (int k = 0; k < kRowsPerThread; ++k)
+                        if (r0 + 24 * k < t.n)
+                            cp_async16(bdst + k * 24 * 128, xs + static_cast<size_t>(tok[k]) * H, 16u);
+                    cp_async_arrive_noinc(&B->b_full[s]);
+                    // The previous item's MMAs are done once the ring has turned
+                    // over: run its epilogue while these loads are in flight.
+                    if (epi_warp && have_prev && kb == min(kSB, pc.KB) - 1) {
+                        epilogue(prev);
+                        have_prev = false;
+                    }
+                }
+                prev = t;
+                have_prev = true;
+            }
+            if (epi_warp && have_prev) epilogue(prev);
+            cp_async_wait<0>();
+        } else if (!epi_warp) {
+            const int lt = threadIdx.x - kWarpTok * 32;  // 0..63
+            grid_dependency_wait();  // h comes from the gate/up grid
+            if (lt == 0)
+                for (int pt = 0; pt < (has_sh ? 2 : 1); ++pt) tma_prefetch_desc(&M.act[pt]);
+            long g = 0;
+            for (int item = blockIdx.x; item < total; item += gridDim.x) {
+                const Tile t = tile_of<MODE>(a, pre, item);
+                const PartCfg pc = part_cfg<MODE>(a, t.pt);
+                for (int kb = 0; kb < pc.KB; ++kb, ++g) {
+                    const int s = static_cast<int>(g % kSB);
+                    if (g >= kSB) wait_bar(&B->b_done[s], static_cast<uint32_t>((g / kSB - 1) & 1), B, a.status);
+                    if (lt == 0) {
+                        mbar_arrive_expect_tx(&B->b_full[s], kBStage);
+                        tma_load_2d(b_ring + s * kBStage, &M.act[t.pt], &B->b_full[s], kb * 64,
+                                    static_cast<int>(t.p0));
+                    }
+                }
+            }
+        } else {
+            for (int item = blockIdx.x; item < total; item += gridDim.x) epilogue(tile_of<MODE>(a, pre, item));
         }
-        bulk_wait0();
+        if (epi_warp) bulk_wait0();
+    } else if (warp >= kWarpXform) {
+        // ------------------------------------------------ transform: FP8 -> bf16 -> TMEM (A)
+        // gate/up: warp (q, mt) owns lane quarter q of M-tile mt and all 64 codes
+        // of a step; down: warp (q, hf) owns lane quarter q and half of the codes.
+        const int q = warp & 3, hi = (warp - kWarpXform) >> 2;
+        const int xt = threadIdx.x - kWarpXform * 32;           // 0..255
+        const int row = 32 * q + lane;  // TMEM lane = weight row of the M-tile
+        constexpr int NW = MODE == kGateUp ? 32 : 16;           // words (bf16 pairs) per thread per step
+        long g = 0;                                             // MMA steps (64 columns)
+        for (int item = blockIdx.x; item < total; item += gridDim.x) {
+            const Tile t = tile_of<MODE>(a, pre, item);
+            const PartCfg pc = part_cfg<MODE>(a, t.pt);
+            const ExpertsView& ev = t.pt ? a.sh : a.ex;
+            const int KB = pc.KB, KB128 = pc.KB128;
+            // Block scales of the item, staged once: gate/up -> [gate, up][KB128],
+            // down -> [output block][KB128].
+            named_barrier_sync(3, kXformWarps * 32);
+            if (MODE == kGateUp) {
+                const size_t off = (static_cast<size_t>(t.e) * (pc.I / 128) + t.fb0) * KB128;
+                for (int i = xt; i < 2 * KB128; i += kXformWarps * 32)
+                    sc_sm[i] = __ldg((i < KB128 ? ev.s_gate : ev.s_up) + off + (i % KB128));
+            } else {
+                for (int i = xt; i < t.nfb * KB128; i += kXformWarps * 32) {
+                    const int f = i / KB128, k = i - f * KB128;
+                    sc_sm[i] = __ldg(ev.s_down + (static_cast<size_t>(t.e) * (H / 128) + (t.fb0 + f)) * KB128 + k);
+                }
+            }
+            named_barrier_sync(3, kXformWarps * 32);
+            // Source row in the weight stage.  gate/up: in the lane quarter of
+            // warp q, lanes 0-15 hold the gate rows and lanes 16-31 the up rows
+            // of features 16q .. 16q+15 of the M-tile (so the eight lanes of a
+            // shared-memory phase read eight different rows).
+            const bool up_row = MODE == kGateUp && (lane & 16);
+            const int srow = MODE == kGateUp ? hi * 64 + 16 * q + (lane & 15) : row;
+            const int sub = up_row ? kWStage / 2 : 0;
+            const int c0 = MODE == kGateUp ? 0 : 2 * hi;  // first 16-byte chunk of this thread in a step
+            for (int f = 0; f < t.nfb; ++f) {
+                const float* scr = sc_sm + (MODE == kGateUp ? (up_row ? KB128 : 0) : f * KB128);
+                for (int kb = 0; kb < KB; ++kb, ++g) {
+                    const long gw = g >> 1;  // weight stage holding this step
+                    const long u = MODE == kGateUp ? 2 * g + hi : g;  // A unit of this warp's work
+                    const int sw = static_cast<int>(gw % kSW), sa = static_cast<int>(u % kSA);
+                    const bool ok1 = wait_bar(&B->w_full[sw], static_cast<uint32_t>((gw / kSW) & 1), B, a.status);
+                    bool ok2 = true;
+                    if (u >= kSA)
+                        ok2 = wait_bar(&B->a_done[sa], static_cast<uint32_t>((u / kSA - 1) & 1), B, a.status);
+                    uint32_t v[NW];
+                    if (ok1 && ok2) {
+                        const float sc = scr[kb >> 1];
+                        const uint8_t* base = w_ring + sw * kWStage + sub + srow * 128;
+#pragma unroll
+                        for (int c = 0; c < NW / 8; ++c) {
+                            const int chunk = (g & 1) * 4 + c0 + c;
+                            const uint4 w = *reinterpret_cast<const uint4*>(base + ((chunk ^ (srow & 7)) << 4));
+                            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                            for (int k = 0; k < 4; ++k) {
+                                v[c * 8 + 2 * k] = decode_scaled(static_cast<uint16_t>(ws[k] & 0xFFFFu), sc);
+                                v[c * 8 + 2 * k + 1] = decode_scaled(static_cast<uint16_t>(ws[k] >> 16), sc);
+                            }
+                        }
+                    } else {
+#pragma unroll
+                        for (int k = 0; k < NW; ++k) v[k] = 0;
+                    }
+                    __syncwarp();
+                    if ((g & 1) && lane == 0) mbar_arrive(&B->w_empty[sw]);
+                    const uint32_t acol = kACol + sa * 32 + (MODE == kGateUp ? 0 : hi * 16);
+                    if constexpr (MODE == kGateUp)
+                        tmem_st32(tmem + (static_cast<uint32_t>(32 * q) << 16) + acol, v);
+                    else
+                        tmem_st16(tmem + (static_cast<uint32_t>(32 * q) << 16) + acol, v);
+                    tmem_st_wait();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&B->a_full[sa]);
+                }
+            }
+        }
     } else if (warp == kWarpMma) {
         // ------------------------------------------------ MMA issuer
         // The whole warp runs the loop with warp-uniform operands; one elected
