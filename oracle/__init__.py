@@ -62,6 +62,9 @@ def lib():
             L.oracle_set_threads.restype = I
             L.oracle_get_threads.restype = I
             L.oracle_route.argtypes = [P, I, I, I, P, P, P]
+            L.oracle_route_ex.argtypes = [P, I, I, I, I, P, I, I, I, ctypes.c_double, P, P, P]
+            L.oracle_route_weights.argtypes = [P, I, I, I, I, I, ctypes.c_double, P, P]
+            L.oracle_route_select_scores.argtypes = [P, I, I, I, P, P]
             L.oracle_sort.argtypes = [P, I, I, I, P, P, P]
             L.oracle_sort.restype = I
             L.oracle_ffn_sorted.argtypes = [P, I, I, I, P, P, P, P, P]
@@ -132,6 +135,51 @@ def route(logits: np.ndarray, K: int, zero_mask: Optional[np.ndarray] = None):
     zm = None if zero_mask is None else _c(zero_mask, np.uint8)
     lib().oracle_route(_p(lg), T, E, K, _p(zm), _p(ids), _p(w))
     return ids, w
+
+
+SCORE_SOFTMAX, SCORE_SIGMOID = 0, 1
+
+
+def route_ex(logits: np.ndarray, K: int, score: int = SCORE_SOFTMAX, bias: Optional[np.ndarray] = None,
+             n_group: int = 1, topk_group: int = 1, renormalize: bool = True, scaling: float = 1.0,
+             zero_mask: Optional[np.ndarray] = None):
+    """Routing variants -> (ids int32 [T,K], w float64 [T,K])."""
+    lg = _c(logits, np.float32)
+    T, E = lg.shape
+    if n_group > 1:
+        assert E % n_group == 0 and n_group <= 64 and 1 <= topk_group <= n_group
+        assert topk_group * (E // n_group) >= K
+    ids = np.empty((T, K), np.int32)
+    w = np.empty((T, K), np.float64)
+    b = None if bias is None else _c(bias, np.float32)
+    zm = None if zero_mask is None else _c(zero_mask, np.uint8)
+    lib().oracle_route_ex(_p(lg), T, E, K, int(score), _p(b), int(n_group), int(topk_group),
+                          int(bool(renormalize)), float(scaling), _p(zm), _p(ids), _p(w))
+    return ids, w
+
+
+def route_weights(logits: np.ndarray, ids: np.ndarray, score: int = SCORE_SOFTMAX,
+                  renormalize: bool = True, scaling: float = 1.0) -> np.ndarray:
+    """float64 [T,K]: the routing variants' weights for the given expert choice."""
+    lg = _c(logits, np.float32)
+    T, E = lg.shape
+    idc = _c(ids, np.int32)
+    K = idc.shape[1]
+    w = np.empty((T, K), np.float64)
+    lib().oracle_route_weights(_p(lg), T, E, K, int(score), int(bool(renormalize)), float(scaling),
+                               _p(idc), _p(w))
+    return w
+
+
+def route_select_scores(logits: np.ndarray, score: int, bias: Optional[np.ndarray] = None) -> np.ndarray:
+    """float64 [T,E]: the selection score s_e + bias_e of every expert."""
+    lg = _c(logits, np.float32)
+    T, E = lg.shape
+    c = np.empty((T, E), np.float64)
+    b = None if bias is None else _c(bias, np.float32)
+    lib().oracle_route_select_scores(_p(lg), T, E, int(score), _p(b), _p(c))
+    return c
+
 
 
 def sort(ids: np.ndarray, E: int):

@@ -155,6 +155,128 @@ void oracle_route(const float* logits, int T, int E, int K, const uint8_t* zero_
     }
 }
 
+/* Routing variants named by the pages without a formula -- the Nemotron-H
+ * layer's "sigmoid topK routing" scaled by `routed_scaling_factor`
+ * (spark_model/layers/nemotron_moe.rs, module doc and `prefill`) and the NKI
+ * library's "DeepSeek-V3 group-limited noaux_tc routing" (NKI Library kernel
+ * reference, MoE kernels) -- taken in the published DeepSeek-V3 router's form:
+ *   s_e  = softmax(l)_e (score 0) or 1 / (1 + e^-l_e) (score 1)
+ *   c_e  = s_e + bias[e]                 (selection only; bias NULL -> 0)
+ *   with n_group > 1, expert e is in group e / (E / n_group); a group scores
+ *   the sum of its two largest c (its one c if it has one expert); the
+ *   topk_group best groups are kept (equal scores -> lower group index) and
+ *   only their experts may be chosen
+ *   ids  = the K eligible experts of largest c, descending, ties -> lower id
+ *   w_j  = scaling * s_{ids_j} / (renormalize ? sum_j' s_{ids_j'} : 1)
+ * With no bias and one group the ranking compares the fp32 logits themselves
+ * (both scores are strictly increasing in the logit); otherwise it compares
+ * the fp64 c.  zero_mask as in oracle_route. */
+static void route_scores(const float* l, int E, int score, double* s) {
+    if (score == 0) {
+        double lmax = -INFINITY, z = 0.0;
+        for (int e = 0; e < E; ++e)
+            if ((double)l[e] > lmax) lmax = (double)l[e];
+        for (int e = 0; e < E; ++e) {
+            s[e] = exp((double)l[e] - lmax);
+            z += s[e];
+        }
+        for (int e = 0; e < E; ++e) s[e] /= z;
+    } else {
+        for (int e = 0; e < E; ++e) s[e] = 1.0 / (1.0 + exp(-(double)l[e]));
+    }
+}
+
+void oracle_route_ex(const float* logits, int T, int E, int K, int score, const float* bias,
+                     int n_group, int topk_group, int renormalize, double scaling,
+                     const uint8_t* zero_mask, int32_t* ids, double* w) {
+    const int by_logit = bias == NULL && n_group <= 1;
+    const int G = n_group > 1 ? E / n_group : E;
+#pragma omp parallel for num_threads(g_threads) schedule(static)
+    for (int t = 0; t < T; ++t) {
+        const float* l = logits + (size_t)t * E;
+        double* s = (double*)malloc(sizeof(double) * (size_t)E);
+        double* c = (double*)malloc(sizeof(double) * (size_t)E);
+        unsigned char* ok = (unsigned char*)malloc((size_t)E);
+        route_scores(l, E, score, s);
+        for (int e = 0; e < E; ++e) {
+            c[e] = by_logit ? (double)l[e] : s[e] + (bias ? (double)bias[e] : 0.0);
+            ok[e] = 1;
+        }
+        if (n_group > 1) {
+            double gs[64];
+            unsigned char keep[64];
+            for (int g = 0; g < n_group; ++g) {
+                double a = -INFINITY, b = -INFINITY; /* two largest c of the group */
+                for (int e = g * G; e < (g + 1) * G; ++e) {
+                    if (c[e] > a) {
+                        b = a;
+                        a = c[e];
+                    } else if (c[e] > b) {
+                        b = c[e];
+                    }
+                }
+                gs[g] = G > 1 ? a + b : a;
+                keep[g] = 0;
+            }
+            for (int r = 0; r < topk_group; ++r) {
+                int best = -1;
+                for (int g = 0; g < n_group; ++g)
+                    if (!keep[g] && (best < 0 || gs[g] > gs[best])) best = g;
+                keep[best] = 1;
+            }
+            for (int e = 0; e < E; ++e) ok[e] = keep[e / G];
+        }
+        double sum = 0.0;
+        for (int j = 0; j < K; ++j) {
+            int best = -1;
+            for (int e = 0; e < E; ++e) {
+                if (!ok[e]) continue;
+                if (best < 0 || c[e] > c[best]) best = e; /* strict >: ties keep the lower id */
+            }
+            ok[best] = 0;
+            ids[(size_t)t * K + j] = best;
+            sum += s[best];
+        }
+        for (int j = 0; j < K; ++j) {
+            double v = scaling * s[ids[(size_t)t * K + j]] / (renormalize ? sum : 1.0);
+            if (zero_mask && zero_mask[(size_t)t * K + j]) v = 0.0;
+            w[(size_t)t * K + j] = v;
+        }
+        free(s);
+        free(c);
+        free(ok);
+    }
+}
+
+/* The weights the routing variants give a chosen set of experts: w[t, j] as in
+ * oracle_route_ex for ids[t, :] supplied by the caller (used to score a choice
+ * that differs from the oracle's only between experts whose selection scores
+ * tie to fp32 rounding). */
+void oracle_route_weights(const float* logits, int T, int E, int K, int score, int renormalize,
+                          double scaling, const int32_t* ids, double* w) {
+    double* s = (double*)malloc(sizeof(double) * (size_t)E);
+    for (int t = 0; t < T; ++t) {
+        route_scores(logits + (size_t)t * E, E, score, s);
+        double sum = 0.0;
+        for (int j = 0; j < K; ++j) sum += s[ids[(size_t)t * K + j]];
+        for (int j = 0; j < K; ++j)
+            w[(size_t)t * K + j] = scaling * s[ids[(size_t)t * K + j]] / (renormalize ? sum : 1.0);
+    }
+    free(s);
+}
+
+/* The selection score c of every expert (fp64), as oracle_route_ex ranks them
+ * when a bias or groups are present. */
+void oracle_route_select_scores(const float* logits, int T, int E, int score, const float* bias,
+                                double* c) {
+    for (int t = 0; t < T; ++t) {
+        double* ct = c + (size_t)t * E;
+        route_scores(logits + (size_t)t * E, E, score, ct);
+        if (bias)
+            for (int e = 0; e < E; ++e) ct[e] += (double)bias[e];
+    }
+}
+
 /* ---------------------------------------------------------------- sort */
 
 /* Sort the R = T*K routes (route r = t*K + j carries expert ids[r]) by expert,

@@ -134,6 +134,141 @@ def test_route_zero_mask_forces_zero_without_renormalising():
     assert np.array_equal(w1[mask == 0], w0[mask == 0])
 
 
+# ------------------------------------------------------------------ routing variants
+
+SIG = oracle.SCORE_SIGMOID
+
+
+def _sigmoid64(lg: np.ndarray) -> np.ndarray:
+    return scipy.special.expit(lg.astype(np.float64))
+
+
+def test_route_ex_default_is_route():
+    """Softmax, no bias, one group, renormalised, scale 1 is the plain router."""
+    lg = wl.tie_logits(60, 24, seed=6, levels=3)
+    ids0, w0 = oracle.route(lg, 5)
+    ids1, w1 = oracle.route_ex(lg, 5)
+    assert np.array_equal(ids0, ids1)
+    np.testing.assert_allclose(w1, w0, rtol=1e-15, atol=0)
+
+
+def test_route_ex_sigmoid_closed_forms():
+    """Sigmoid scores (scipy's expit): with K = E and renormalisation the weights
+    are sigmoid / sum(sigmoid); without it, scaling * sigmoid; the order is the
+    logit order, ties to the lower id (catches a softmax left in, a missing or
+    doubled scaling, a dropped renormalisation)."""
+    lg = np.random.default_rng(8).standard_normal((30, 10)).astype(np.float32) * 2
+    sg = _sigmoid64(lg)
+    ids, w = oracle.route_ex(lg, 10, score=SIG)
+    for t in range(30):
+        assert list(ids[t]) == _sorted_topk(lg[t], 10)
+    np.testing.assert_allclose(w, np.take_along_axis(sg / sg.sum(1, keepdims=True), ids, 1), rtol=1e-13)
+    ids, w = oracle.route_ex(lg, 4, score=SIG, renormalize=False, scaling=2.5)
+    np.testing.assert_allclose(w, 2.5 * np.take_along_axis(sg, ids, 1), rtol=1e-13)
+    ids, w = oracle.route_ex(lg, 4, score=SIG, scaling=2.5)
+    np.testing.assert_allclose(w.sum(1), 2.5, rtol=1e-14)
+
+
+def test_route_ex_bias_selects_but_does_not_weigh():
+    """A large selection bias on a set S forces S (ordered by score + bias),
+    while the weights stay the unbiased sigmoid scores of S, renormalised."""
+    rng = np.random.default_rng(9)
+    T, E, K = 40, 32, 4
+    lg = rng.standard_normal((T, E)).astype(np.float32)
+    S = np.array([3, 17, 22, 30])
+    bias = np.zeros(E, np.float32)
+    bias[S] = np.float32(10.0) + rng.random(K).astype(np.float32)
+    ids, w = oracle.route_ex(lg, K, score=SIG, bias=bias)
+    sg = _sigmoid64(lg)
+    for t in range(T):
+        order = sorted(S, key=lambda e: (-(sg[t, e] + float(bias[e])), e))
+        assert list(ids[t]) == order
+        np.testing.assert_allclose(w[t], sg[t, order] / sg[t, S].sum(), rtol=1e-13)
+
+
+def _brute_group_route(c: np.ndarray, n_group: int, topk_group: int, K: int):
+    """Exhaustive search: the group subset of largest total group score (a
+    group's score: sum of its two largest c), then the K-subset of its experts
+    of largest total c, listed by c descending."""
+    import itertools
+    E = c.size
+    G = E // n_group
+    gs = [sum(sorted(c[g * G:(g + 1) * G])[-2:]) for g in range(n_group)]
+    groups = max(itertools.combinations(range(n_group), topk_group), key=lambda gg: sum(gs[g] for g in gg))
+    pool = [e for g in groups for e in range(g * G, (g + 1) * G)]
+    best = max(itertools.combinations(pool, K), key=lambda ee: sum(c[e] for e in ee))
+    return sorted(best, key=lambda e: -c[e])
+
+
+@pytest.mark.parametrize("E,n_group,topk_group,K", [(12, 4, 2, 3), (16, 8, 3, 4), (18, 3, 1, 2), (8, 8, 5, 5)])
+def test_route_ex_groups_match_exhaustive_search(E, n_group, topk_group, K):
+    """Group-limited selection against an exhaustive search over group and
+    expert subsets on tiny, tie-free inputs (catches a top-1 group score, the
+    groups scored on the unbiased scores, experts taken outside the kept
+    groups)."""
+    rng = np.random.default_rng(E * 100 + K)
+    T = 25
+    lg = rng.standard_normal((T, E)).astype(np.float32)
+    bias = (rng.random(E) * 0.3 - 0.1).astype(np.float32)
+    ids, w = oracle.route_ex(lg, K, score=SIG, bias=bias, n_group=n_group, topk_group=topk_group)
+    c = _sigmoid64(lg) + bias.astype(np.float64)
+    for t in range(T):
+        assert list(ids[t]) == _brute_group_route(c[t], n_group, topk_group, K)
+
+
+def test_route_ex_all_groups_kept_is_no_group_limit():
+    lg = np.random.default_rng(11).standard_normal((50, 64)).astype(np.float32)
+    bias = (np.random.default_rng(12).random(64) * 0.2).astype(np.float32)
+    a = oracle.route_ex(lg, 8, score=SIG, bias=bias, n_group=8, topk_group=8, scaling=1.5)
+    b = oracle.route_ex(lg, 8, score=SIG, bias=bias, scaling=1.5)
+    assert np.array_equal(a[0], b[0])
+    np.testing.assert_array_equal(a[1], b[1])
+
+
+def test_route_ex_matches_transformers_deepseek_v3_router():
+    """The published DeepSeek-V3 router as the transformers library implements
+    it (sigmoid, selection-only correction bias, group-limited top-k,
+    renormalised, scaled), in float64 on tie-free inputs with a non-negative
+    bias (the library fills masked experts with 0, which only matters when an
+    eligible score is negative).  The library returns its picks unordered, so
+    sets and per-expert weights are compared."""
+    mod = pytest.importorskip("transformers.models.deepseek_v3.modeling_deepseek_v3")
+    from transformers import DeepseekV3Config
+    E, n_group, topk_group, K, scale = 64, 8, 4, 6, 2.5
+    cfg = DeepseekV3Config(hidden_size=32, intermediate_size=64, moe_intermediate_size=16,
+                           n_routed_experts=E, n_shared_experts=1, num_experts_per_tok=K,
+                           n_group=n_group, topk_group=topk_group, norm_topk_prob=True,
+                           routed_scaling_factor=scale, num_hidden_layers=1, num_attention_heads=4,
+                           num_key_value_heads=4)
+    moe = mod.DeepseekV3MoE(cfg).double()
+    rng = np.random.default_rng(13)
+    lg = rng.standard_normal((100, E)).astype(np.float32)
+    bias = (rng.random(E) * 0.05).astype(np.float32)
+    with torch.no_grad():
+        moe.gate.e_score_correction_bias.copy_(torch.from_numpy(bias.astype(np.float64)))
+        li, lw = moe.route_tokens_to_experts(torch.from_numpy(lg.astype(np.float64)))
+    ids, w = oracle.route_ex(lg, K, score=SIG, bias=bias, n_group=n_group, topk_group=topk_group,
+                             scaling=scale)
+    li, lw = li.numpy(), lw.numpy()
+    for t in range(100):
+        assert set(ids[t]) == set(li[t])
+        ref = dict(zip(li[t], lw[t]))
+        np.testing.assert_allclose(w[t], [ref[e] for e in ids[t]], rtol=1e-12)
+
+
+def test_route_ex_weights_and_scores_helpers():
+    """route_weights on the oracle's own choice reproduces its weights; the
+    selection scores are sigmoid + bias (scipy)."""
+    rng = np.random.default_rng(14)
+    lg = rng.standard_normal((20, 48)).astype(np.float32)
+    bias = (rng.random(48) * 0.1).astype(np.float32)
+    ids, w = oracle.route_ex(lg, 5, score=SIG, bias=bias, n_group=4, topk_group=2, scaling=3.0)
+    np.testing.assert_allclose(oracle.route_weights(lg, ids, score=SIG, scaling=3.0), w, rtol=1e-15)
+    np.testing.assert_allclose(oracle.route_select_scores(lg, SIG, bias), _sigmoid64(lg) + bias, rtol=1e-15)
+    p = scipy.special.softmax(lg.astype(np.float64), axis=1)
+    np.testing.assert_allclose(oracle.route_select_scores(lg, oracle.SCORE_SOFTMAX), p, rtol=1e-13)
+
+
 # ------------------------------------------------------------------ sort
 
 @pytest.mark.parametrize("T,K,E,distinct", [(0, 4, 8, True), (1, 1, 1, True), (37, 3, 5, True),
