@@ -129,6 +129,57 @@ MOE_API int moe_route(const float* logits, int T, int E, int K, const uint8_t* z
               int32_t* topk_ids, float* topk_w, moe_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * moe_route_ex -- routing variants: score function, selection-only bias,
+ * group-limited choice, optional renormalisation, routed scaling factor.
+ *
+ * The pages name these routers without giving their formulas: the Nemotron-H
+ * layer's "sigmoid topK routing" scaled by `routed_scaling_factor`
+ * (spark_model/layers/nemotron_moe.rs, module doc and `prefill`) and the NKI
+ * library's DeepSeek-V3 group-limited `noaux_tc` router (NKI Library kernel
+ * reference, MoE kernels).  Both are taken in the published DeepSeek-V3
+ * router's form.  Per token t, with l = logits[t, :]:
+ *   s_e = softmax(l)_e            (cfg->score == MOE_SCORE_SOFTMAX)
+ *       = 1 / (1 + exp(-l_e))     (cfg->score == MOE_SCORE_SIGMOID)
+ *   c_e = s_e + sel_bias[e]       (selection score; sel_bias NULL -> c = s)
+ *   n_group > 1: expert e is in group e / (E / n_group); a group's score is
+ *     the sum of its two largest c (its only c for one-expert groups); the
+ *     topk_group groups of largest score are kept, equal scores going to the
+ *     lower group index, and only their experts can be chosen;
+ *   topk_ids[t, :] = the K eligible experts of largest c, descending, equal c
+ *     going to the lower expert id;
+ *   topk_w[t, j]   = scaling * s_{ids[t,j]} / (renormalize ? sum_j' s_{ids[t,j']} : 1).
+ * The bias changes which experts are chosen, never their weights.  With
+ * MOE_SCORE_SOFTMAX, no bias, n_group = 1, renormalize = 1 and scaling = 1
+ * this is moe_route.
+ * Precision: with no bias and n_group = 1 experts are ranked by the fp32 logit
+ * (both scores are strictly increasing in it), exactly as moe_route; otherwise
+ * by the kernel's fp32 c (expf-based), so experts whose c differ by a few fp32
+ * ulps may be ranked either way.  Weights are computed in fp32.
+ *
+ *   cfg       host pointer (read during the call): score, sel_bias ([E] f32
+ *             device pointer or NULL), n_group (1..MOE_MAX_GROUPS, divides E),
+ *             topk_group (1..n_group, topk_group * (E / n_group) >= K),
+ *             renormalize (0 or 1), scaling (finite, > 0)
+ *   other arguments and limits as moe_route.
+ * Errors: MOE_ERR_INVALID_ARG for a NULL cfg or a field outside its range.
+ * ------------------------------------------------------------------------- */
+#define MOE_SCORE_SOFTMAX 0
+#define MOE_SCORE_SIGMOID 1
+#define MOE_MAX_GROUPS 32
+
+typedef struct moe_route_config {
+    int score;             /* MOE_SCORE_SOFTMAX or MOE_SCORE_SIGMOID */
+    const float* sel_bias; /* [E] f32 selection-only bias (device), or NULL */
+    int n_group;           /* expert groups; 1 = no group limit */
+    int topk_group;        /* groups kept per token (== n_group when n_group == 1) */
+    int renormalize;       /* 1: divide the K weights by their sum */
+    float scaling;         /* routed scaling factor applied to every weight */
+} moe_route_config;
+
+MOE_API int moe_route_ex(const float* logits, int T, int E, int K, const moe_route_config* cfg,
+                         const uint8_t* zero_mask, int32_t* topk_ids, float* topk_w, moe_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * moe_sort -- stable sort of the R = T*K routes by expert.
  *
  * The "sort tokens by expert" step of the Nemotron prefill path, the NKI

@@ -30,7 +30,7 @@ MOE_OUT_BF16, MOE_OUT_F32 = 0, 1
 MOE_STATUS_BAD_ID, MOE_STATUS_BAD_MAP, MOE_STATUS_TIMEOUT = 1, 2, 4
 MOE_MAX_E, MOE_MAX_K = 1024, 32
 
-EXPORTED = ("moe_last_error", "moe_abi_version", "moe_route", "moe_sort_workspace_bytes", "moe_sort",
+EXPORTED = ("moe_last_error", "moe_abi_version", "moe_route", "moe_route_ex", "moe_sort_workspace_bytes", "moe_sort",
             "moe_sort_static_ws", "moe_ffn_resolve_mode", "moe_ffn_workspace_bytes", "moe_expert_ffn", "moe_combine")
 
 
@@ -44,6 +44,11 @@ class _Experts(ctypes.Structure):
     _fields_ = [("w_gate", ctypes.c_void_p), ("w_up", ctypes.c_void_p), ("w_down", ctypes.c_void_p),
                 ("s_gate", ctypes.c_void_p), ("s_up", ctypes.c_void_p), ("s_down", ctypes.c_void_p),
                 ("n_experts", ctypes.c_int), ("inter", ctypes.c_int)]
+
+
+class _RouteConfig(ctypes.Structure):
+    _fields_ = [("score", ctypes.c_int), ("sel_bias", ctypes.c_void_p), ("n_group", ctypes.c_int),
+                ("topk_group", ctypes.c_int), ("renormalize", ctypes.c_int), ("scaling", ctypes.c_float)]
 
 
 _lock = threading.Lock()
@@ -63,6 +68,8 @@ def lib() -> ctypes.CDLL:
             L.moe_last_error.restype = ctypes.c_char_p
             L.moe_abi_version.restype = I
             L.moe_route.argtypes = [P, I, I, I, P, P, P, P]
+            L.moe_route_ex.argtypes = [P, I, I, I, ctypes.POINTER(_RouteConfig), P, P, P, P]
+            L.moe_route_ex.restype = I
             L.moe_route.restype = I
             L.moe_sort_workspace_bytes.argtypes = [I, I, I]
             L.moe_sort_workspace_bytes.restype = S
@@ -152,6 +159,28 @@ def moe_route(logits: torch.Tensor, K: int, zero_mask: Optional[torch.Tensor] = 
         topk_w = torch.empty((T, K), dtype=torch.float32, device=logits.device)
     _check(lib().moe_route(_ptr(logits), T, E, K, _ptr(zero_mask), _ptr(topk_ids), _ptr(topk_w),
                            _stream(stream)))
+    return topk_ids, topk_w
+
+
+MOE_SCORE_SOFTMAX, MOE_SCORE_SIGMOID = 0, 1
+
+
+def moe_route_ex(logits: torch.Tensor, K: int, score: int = MOE_SCORE_SOFTMAX,
+                 sel_bias: Optional[torch.Tensor] = None, n_group: int = 1, topk_group: Optional[int] = None,
+                 renormalize: bool = True, scaling: float = 1.0, zero_mask: Optional[torch.Tensor] = None,
+                 topk_ids: Optional[torch.Tensor] = None, topk_w: Optional[torch.Tensor] = None, stream=None):
+    """Routing variants: logits [T, E] f32 -> (topk_ids [T, K] i32, topk_w [T, K] f32).
+    sel_bias [E] f32 (selection only); n_group / topk_group: group-limited choice."""
+    _need_cuda(logits, zero_mask, sel_bias)
+    T, E = logits.shape
+    if topk_ids is None:
+        topk_ids = torch.empty((T, K), dtype=torch.int32, device=logits.device)
+    if topk_w is None:
+        topk_w = torch.empty((T, K), dtype=torch.float32, device=logits.device)
+    cfg = _RouteConfig(int(score), _ptr(sel_bias), int(n_group),
+                       int(n_group if topk_group is None else topk_group), int(bool(renormalize)), float(scaling))
+    _check(lib().moe_route_ex(_ptr(logits), T, E, K, ctypes.byref(cfg), _ptr(zero_mask), _ptr(topk_ids),
+                              _ptr(topk_w), _stream(stream)))
     return topk_ids, topk_w
 
 

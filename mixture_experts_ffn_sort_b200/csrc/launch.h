@@ -12,6 +12,17 @@ namespace moe {
 // ---------------------------------------------------------------- route
 cudaError_t launch_route(const float* logits, int T, int E, int K, const uint8_t* zero_mask,
                          int32_t* ids, float* w, cudaStream_t stream);
+// Routing variants (moe_route_ex); the fields as in moe_route_config.
+struct RouteCfg {
+    int score;
+    const float* bias;
+    int n_group;
+    int topk_group;
+    int renormalize;
+    float scaling;
+};
+cudaError_t launch_route_ex(const float* logits, int T, int E, int K, const RouteCfg& cfg,
+                            const uint8_t* zero_mask, int32_t* ids, float* w, cudaStream_t stream);
 
 // ---------------------------------------------------------------- sort
 // Routes per tile (one thread block) of the multi-kernel sort, and the largest route count

@@ -4,6 +4,7 @@
 // aiter gfx950 prefill PR, the launcher checks the tensor contracts; like the
 // Nemotron-H layer's constructor, an out-of-range top_k is reported with a
 // message naming the bound.
+#include <math.h>
 #include <stdarg.h>
 #include <stdio.h>
 
@@ -106,6 +107,38 @@ int moe_route(const float* logits, int T, int E, int K, const uint8_t* zero_mask
         return fail(MOE_ERR_MISALIGNED, "moe_route: tensor bases must be 16-byte aligned");
     cudaError_t e = moe::launch_route(logits, T, E, K, zero_mask, topk_ids, topk_w, stream);
     return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_route launch");
+}
+
+int moe_route_ex(const float* logits, int T, int E, int K, const moe_route_config* cfg, const uint8_t* zero_mask,
+                 int32_t* topk_ids, float* topk_w, moe_stream_t stream) {
+    g_err.clear();
+    int rc = check_topk(T, E, K);
+    if (rc) return rc;
+    if (!cfg) return fail(MOE_ERR_INVALID_ARG, "moe_route_ex: cfg must not be NULL");
+    if (cfg->score != MOE_SCORE_SOFTMAX && cfg->score != MOE_SCORE_SIGMOID)
+        return fail(MOE_ERR_INVALID_ARG, "moe_route_ex: unknown score function %d", cfg->score);
+    if (cfg->n_group < 1 || cfg->n_group > MOE_MAX_GROUPS || E % cfg->n_group)
+        return fail(MOE_ERR_INVALID_ARG, "moe_route_ex: n_group=%d must be in 1..%d and divide E=%d", cfg->n_group,
+                    MOE_MAX_GROUPS, E);
+    if (cfg->topk_group < 1 || cfg->topk_group > cfg->n_group ||
+        static_cast<long>(cfg->topk_group) * (E / cfg->n_group) < K)
+        return fail(MOE_ERR_INVALID_ARG, "moe_route_ex: topk_group=%d must be in 1..n_group and keep >= K=%d experts",
+                    cfg->topk_group, K);
+    if (cfg->renormalize != 0 && cfg->renormalize != 1)
+        return fail(MOE_ERR_INVALID_ARG, "moe_route_ex: renormalize must be 0 or 1");
+    if (!(cfg->scaling > 0.f) || !isfinite(cfg->scaling))
+        return fail(MOE_ERR_INVALID_ARG, "moe_route_ex: scaling must be finite and > 0");
+    if (T == 0) return MOE_OK;
+    if (!logits || !topk_ids || !topk_w)
+        return fail(MOE_ERR_INVALID_ARG, "moe_route_ex: logits, topk_ids and topk_w must not be NULL");
+    if (!aligned16(logits) || !aligned16(topk_ids) || !aligned16(topk_w))
+        return fail(MOE_ERR_MISALIGNED, "moe_route_ex: tensor bases must be 16-byte aligned");
+    if (reinterpret_cast<uintptr_t>(cfg->sel_bias) % 4)
+        return fail(MOE_ERR_MISALIGNED, "moe_route_ex: sel_bias must be 4-byte aligned");
+    const moe::RouteCfg rc_dev{cfg->score, cfg->sel_bias, cfg->n_group, cfg->topk_group, cfg->renormalize,
+                               cfg->scaling};
+    cudaError_t e = moe::launch_route_ex(logits, T, E, K, rc_dev, zero_mask, topk_ids, topk_w, stream);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_route_ex launch");
 }
 
 size_t moe_sort_workspace_bytes(int T, int K, int E) {

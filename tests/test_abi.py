@@ -108,6 +108,31 @@ def test_route_null_and_misaligned(L):
     assert L.moe_route(P(0x1008), 4, 8, 2, None, P(16), P(16), None) == moe.MOE_ERR_MISALIGNED
 
 
+def _rcfg(score=0, bias=None, n_group=1, topk_group=1, renorm=1, scaling=1.0):
+    return ctypes.byref(moe._RouteConfig(score, bias, n_group, topk_group, renorm, scaling))
+
+
+@pytest.mark.parametrize("cfg,why", [
+    (dict(score=2), "unknown score"), (dict(n_group=0), "n_group < 1"), (dict(n_group=33), "n_group > 32"),
+    (dict(n_group=3), "n_group does not divide E"), (dict(n_group=4, topk_group=0), "topk_group < 1"),
+    (dict(n_group=4, topk_group=5), "topk_group > n_group"),
+    (dict(n_group=8, topk_group=1), "kept groups hold fewer than K experts"),
+    (dict(renorm=2), "renormalize not 0/1"), (dict(scaling=0.0), "scaling 0"),
+    (dict(scaling=float("inf")), "scaling inf"), (dict(scaling=float("nan")), "scaling nan")])
+def test_route_ex_rejects_bad_config(L, cfg, why):
+    # E = 16, K = 4: n_group 8 with one kept group leaves 2 experts < K.
+    assert L.moe_route_ex(P(16), 4, 16, 4, _rcfg(**cfg), None, P(16), P(16), None) == moe.MOE_ERR_INVALID_ARG, why
+
+
+def test_route_ex_checks(L):
+    assert L.moe_route_ex(P(16), 4, 16, 4, None, None, P(16), P(16), None) == moe.MOE_ERR_INVALID_ARG
+    assert b"cfg" in L.moe_last_error()
+    assert L.moe_route_ex(P(16), 4, 16, 17, _rcfg(), None, P(16), P(16), None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_route_ex(None, 0, 16, 4, _rcfg(n_group=4, topk_group=2), None, None, None, None) == moe.MOE_OK
+    assert L.moe_route_ex(P(0x1008), 4, 16, 4, _rcfg(), None, P(16), P(16), None) == moe.MOE_ERR_MISALIGNED
+    assert L.moe_route_ex(P(16), 4, 16, 4, _rcfg(bias=0x1002), None, P(16), P(16), None) == moe.MOE_ERR_MISALIGNED
+
+
 def test_sort_checks(L):
     assert L.moe_sort(P(16), 4, 2, 8, None, P(16), P(16), None, 0, None, None) == moe.MOE_ERR_INVALID_ARG
     assert L.moe_sort(P(16), 4, 2, 8, P(20), P(16), P(16), None, 0, None, None) == moe.MOE_ERR_MISALIGNED
