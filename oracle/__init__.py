@@ -75,6 +75,7 @@ def lib():
             L.oracle_moe.restype = I
             L.oracle_moe_tokens.argtypes = [P, P, I, I, I, I, P, P, P, P, I, P]
             L.oracle_expert_rows.argtypes = [P, I, P, I, P, I, P]
+            L.oracle_moe_tokens_routed.argtypes = [P, I, I, P, P, P, P, P, I, P]
             L.oracle_swiglu.argtypes = [P, P, I, P]
             L.oracle_set_threads(int(os.environ.get("ORACLE_THREADS", os.cpu_count() or 1)))
             _lib = L
@@ -271,6 +272,23 @@ def moe_tokens(x, logits, K, routed, shared=None, zero_mask=None, tokens=None) -
     out = np.empty((n, H), np.float64)
     lib().oracle_moe_tokens(_p(x), _p(lg), T, H, E, K, _p(zm), r.ref(), s.ref() if s else None,
                             _p(tk), n, _p(out))
+    return out
+
+
+def moe_tokens_routed(x, ids, w, routed, shared=None, tokens=None) -> np.ndarray:
+    """Brute-force rows out[i] for token tokens[i] with the routing given:
+    ids / w [n, K] are token tokens[i]'s experts and weights (any router)."""
+    x = _c(x, np.uint16)
+    H = x.shape[1]
+    idc, wc = _c(ids, np.int32), _c(w, np.float64)
+    n, K = idc.shape
+    r = _ExpertsRef(routed)
+    s = _ExpertsRef(shared) if shared is not None else None
+    tk = None if tokens is None else _c(tokens, np.int32)
+    assert tk is None or tk.size == n
+    out = np.empty((n, H), np.float64)
+    lib().oracle_moe_tokens_routed(_p(x), H, K, _p(idc), _p(wc), r.ref(), s.ref() if s else None,
+                                   _p(tk), n, _p(out))
     return out
 
 

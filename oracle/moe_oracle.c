@@ -497,6 +497,40 @@ void oracle_moe_tokens(const uint16_t* x, const float* logits, int T, int H, int
     }
 }
 
+/* oracle_moe_tokens with the routing given: row i of ids / w ([n_tokens, K])
+ * holds the experts and weights of token tokens[i] (any router's choice). */
+void oracle_moe_tokens_routed(const uint16_t* x, int H, int K, const int32_t* ids, const double* w,
+                              const oracle_experts* routed, const oracle_experts* sh,
+                              const int32_t* tokens, int n_tokens, double* out) {
+    init_tables();
+    int I = routed->inter;
+    int Is = sh ? sh->inter : 0;
+    int Imax = I > Is ? I : Is;
+#pragma omp parallel for num_threads(g_threads) schedule(dynamic, 1)
+    for (int i = 0; i < n_tokens; ++i) {
+        int t = tokens ? tokens[i] : i;
+        double* xr = (double*)malloc(sizeof(double) * (size_t)H);
+        double* h = (double*)malloc(sizeof(double) * (size_t)Imax);
+        double* y = (double*)malloc(sizeof(double) * (size_t)H);
+        double* o = out + (size_t)i * H;
+        load_row(x, H, t, xr);
+        for (int n = 0; n < H; ++n) o[n] = 0.0;
+        for (int j = 0; j < K; ++j) {
+            const uint8_t *wg, *wu, *wd; const float *sg, *su, *sd;
+            expert_ptrs(routed, ids[(size_t)i * K + j], H, &wg, &sg, &wu, &su, &wd, &sd);
+            expert_row(xr, H, I, wg, sg, wu, su, wd, sd, h, y);
+            for (int n = 0; n < H; ++n) o[n] += w[(size_t)i * K + j] * y[n];
+        }
+        if (sh) {
+            const uint8_t *wg, *wu, *wd; const float *sg, *su, *sd;
+            expert_ptrs(sh, 0, H, &wg, &sg, &wu, &su, &wd, &sd);
+            expert_row(xr, H, Is, wg, sg, wu, su, wd, sd, h, y);
+            for (int n = 0; n < H; ++n) o[n] += y[n];
+        }
+        free(xr); free(h); free(y);
+    }
+}
+
 /* One expert FFN on explicit rows (no routing): y[i] = FFN_e(x[rows[i]]). */
 void oracle_expert_rows(const uint16_t* x, int H, const oracle_experts* ex, int e,
                         const int32_t* rows, int n_rows, double* y) {

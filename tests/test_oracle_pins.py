@@ -256,6 +256,17 @@ def test_route_ex_matches_transformers_deepseek_v3_router():
         np.testing.assert_allclose(w[t], [ref[e] for e in ids[t]], rtol=1e-12)
 
 
+def test_moe_tokens_routed_with_the_plain_router_is_moe_tokens(tiny):
+    """The FFN with a given routing, fed the plain router's choice, is the
+    routed brute-force oracle bit for bit."""
+    w = tiny
+    tk = np.arange(w.x.shape[0], dtype=np.int32)[::3]
+    ids, wt = oracle.route(w.logits, w.shape.K, w.zero_mask)
+    a = oracle.moe_tokens(w.x, w.logits, w.shape.K, w.routed, w.shared, w.zero_mask, tokens=tk)
+    b = oracle.moe_tokens_routed(w.x, ids[tk], wt[tk], w.routed, w.shared, tokens=tk)
+    np.testing.assert_array_equal(a, b)
+
+
 def test_route_ex_weights_and_scores_helpers():
     """route_weights on the oracle's own choice reproduces its weights; the
     selection scores are sigmoid + bias (scipy)."""
