@@ -122,18 +122,6 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
         : "memory");
 }
 
-// Four rows (r0..r3) of a 2-D tensor, columns [x, x + box), into shared
-// memory as consecutive rows (tile::gather4; the tensor map's box is one row
-// high).  x * elem_size must be a multiple of 16 bytes.
-__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int r0,
-                                            int r1, int r2, int r3) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
-        : "memory");
-}
-
 // Same load with an L2 cache-policy hint (see l2_evict_first_policy).
 __device__ __forceinline__ void tma_load_2d_hint(void* dst, const CUtensorMap* map, uint64_t* bar,
                                                  int x, int y, uint64_t policy) {
@@ -168,16 +156,6 @@ __device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t& r0, uint32_
                  : "r"(addr));
 }
 
-// D += A(16x16, row) * B(16x8, col), bf16 inputs, fp32 accumulators.
-__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
-                                               uint32_t a3, uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
-        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
 // D += A(16x16, row) * B(16x8, col), f16 inputs, fp32 accumulators.
 __device__ __forceinline__ void mma_f16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                               uint32_t a3, uint32_t b0, uint32_t b1) {
@@ -204,29 +182,6 @@ __device__ __forceinline__ void e4m3x4_to_f16(uint32_t w, uint32_t& lo, uint32_t
     hi = e4m3x2_to_f16x2(static_cast<uint16_t>(w >> 16));
 }
 
-// Two E4M3FN codes (low byte -> low half) to two BF16 values, exactly.
-// Every E4M3FN value is an f16 normal (or zero), so the hardware conversion to
-// f16x2 is exact.  Dropping the 7 low mantissa bits (always zero here) and
-// shifting the exponent into BF16's field gives |v| * 2^-112, a BF16 normal;
-// one BF16 multiply by 2^112 restores v with no rounding.  (NaN codes are not
-// valid weights; they decode to an unspecified value.)
-__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint16_t codes) {
-    uint32_t f;
-    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(f) : "h"(codes));
-    const uint32_t mag = (f & 0x7FFF7FFFu) >> 3;
-    const uint32_t b = (f & 0x80008000u) | mag;
-    __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(&b);
-    const __nv_bfloat162 k = __floats2bfloat162_rn(0x1p112f, 0x1p112f);
-    v = __hmul2(v, k);
-    return *reinterpret_cast<uint32_t*>(&v);
-}
-
-// Four codes (bytes 0..3 of w) -> lo = bf16x2(byte0, byte1), hi = bf16x2(byte2, byte3).
-__device__ __forceinline__ void e4m3x4_to_bf16(uint32_t w, uint32_t& lo, uint32_t& hi) {
-    lo = e4m3x2_to_bf16x2(static_cast<uint16_t>(w & 0xFFFFu));
-    hi = e4m3x2_to_bf16x2(static_cast<uint16_t>(w >> 16));
-}
-
 // ---------------------------------------------------------------- tcgen05 / TMEM
 
 // Allocate `ncols` TMEM columns (power of two >= 32); the base address is
@@ -250,20 +205,9 @@ __device__ __forceinline__ void tc_fence_after() {
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-// D[tmem] (+)= A[tmem] * B[smem desc], kind::f16 (bf16 inputs, fp32 accumulate).
-__device__ __forceinline__ void umma_ts_f16(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                            uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
-        ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
-// Arrive on `bar` once every tcgen05.mma issued so far by this thread has completed.
-// The same MMA issued by one elected lane of a warp that executes the call
-// warp-uniformly (all operands equal across the warp).
+// D[tmem] (+)= A[tmem] * B[smem desc], kind::f16 (bf16 inputs, fp32 accumulate),
+// issued by one elected lane of a warp that executes the call warp-uniformly
+// (all operands equal across the warp).
 __device__ __forceinline__ void umma_ts_f16_elect(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
                                                   uint32_t accumulate) {
     asm volatile(
@@ -275,6 +219,7 @@ __device__ __forceinline__ void umma_ts_f16_elect(uint32_t d_tmem, uint32_t a_tm
         : "memory");
 }
 
+// Arrive on `bar` once every tcgen05.mma issued so far has completed: a
 // tcgen05.commit from one elected lane of a warp executing it uniformly.
 __device__ __forceinline__ void umma_commit_elect(uint64_t* bar) {
     asm volatile(
@@ -283,11 +228,6 @@ __device__ __forceinline__ void umma_commit_elect(uint64_t* bar) {
         "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}"
         ::"r"(smem_u32(bar))
         : "memory");
-}
-
-__device__ __forceinline__ void umma_commit(uint64_t* bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
-                 : "memory");
 }
 
 // Store 32 consecutive 32-bit TMEM columns of this thread's lane (32x32b.x32).
@@ -312,20 +252,6 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16
 }
 
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
-
-// Load 32 consecutive 32-bit TMEM columns of this thread's lane (32x32b.x32).
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
-          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]),
-          "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]),
-          "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]),
-          "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
-        : "r"(taddr)
-        : "memory");
-}
 
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
@@ -358,7 +284,6 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32
 __device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
     asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
@@ -401,25 +326,11 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t sr
                  : "memory");
 }
 
-// Asynchronous copy of `bytes` (a multiple of 16, both addresses 16-byte
-// aligned) from shared to global memory, tracked by this thread's bulk group.
-// Generic-proxy writes to the source must be fenced (fence_proxy_async_smem)
-// before the copy is issued.
-__device__ __forceinline__ void bulk_store_s2g(void* dst, uint32_t src, uint32_t bytes) {
-    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(src), "r"(bytes)
-                 : "memory");
-}
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // Wait until every committed bulk copy of this thread has finished reading its source.
 __device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 // Wait until every committed bulk copy of this thread has completed.
 __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
-
-// 16-bit shared store with no compiler memory clobber: lets the compiler keep
-// unrelated shared loads ahead of it (callers order it with barriers).
-__device__ __forceinline__ void st_shared_u16(uint32_t addr, uint16_t v) {
-    asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"(v));
-}
 
 // ---------------------------------------------------------------- misc
 

@@ -63,9 +63,9 @@ constexpr int kOStoreRows = 32;             // rows per TMA store of the staging
 // done), a down step one.
 template <int MODE> struct Cfg;
 // Warp roles (transform and epilogue warps sit on their TMEM lane quarter, warp % 4):
-// warps 2-3 load token rows.
+// 0 weight TMA, 1 MMA, 2-7 token rows (gate/up) or 2 token TMA (down), 4-7
+// epilogue, 8-15 FP8 transform.
 constexpr int kWarpTma = 0, kWarpMma = 1, kWarpTok = 2, kWarpEpi = 4, kWarpXform = 8;
-constexpr int kTokThreads = 64;
 // gate/up: the token rows are gathered by warps 2-7 (the epilogue warps 4-7
 // gather too: one cp.async stream per warp caps the per-SM gather rate).
 constexpr int kGatherThreads = 192;
