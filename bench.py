@@ -135,6 +135,27 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- reference arm (CPU oracle)
 
+def oracle_route_kwargs(router, shape):
+    """The oracle's route_ex arguments for a router preset (None: plain router)."""
+    cfg = wl.ROUTERS[router]
+    if cfg is None:
+        return None
+    kw = {k: v for k, v in cfg.items() if k != "bias"}
+    kw["bias"] = wl.selection_bias(shape.E, shape.seed) if cfg.get("bias") else None
+    return kw
+
+
+def oracle_rows(w, shape, tk, router):
+    """Brute-force oracle rows of the sampled tokens tk, routed by `router`."""
+    import oracle
+    kw = oracle_route_kwargs(router, shape)
+    if kw is None:
+        return oracle.moe_tokens(w.x, w.logits, shape.K, w.routed, w.shared, w.zero_mask, tokens=tk)
+    zm = None if w.zero_mask is None else w.zero_mask[tk]
+    ids, wt = oracle.route_ex(w.logits[tk], shape.K, zero_mask=zm, **kw)
+    return oracle.moe_tokens_routed(w.x, ids, wt, w.routed, w.shared, tokens=tk)
+
+
 def run_reference(args, shape):
     import oracle
     w = wl.make_workload(shape.name)
@@ -143,7 +164,7 @@ def run_reference(args, shape):
 
     def one():
         t0 = time.perf_counter()
-        oracle.moe_tokens(w.x, w.logits, shape.K, w.routed, w.shared, w.zero_mask, tokens=tk)
+        oracle_rows(w, shape, tk, args.router)
         return time.perf_counter() - t0
 
     for _ in range(args.warmup):
@@ -155,19 +176,19 @@ def run_reference(args, shape):
     return {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": 1e3 * tot / len(ts), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "impl": "reference", "config": config_of(shape),
+            "impl": "reference", "config": config_of(shape, args.router),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
-def cpu_baseline(shape, budget_s=10.0):
+def cpu_baseline(shape, router="softmax", budget_s=10.0):
     """The oracle as it stands, on the host cores, on a bounded sample."""
     import oracle
     w = wl.make_workload(shape.name)
     tk = np.arange(min(shape.T, 64), dtype=np.int32)
     n, t0 = 0, time.perf_counter()
     while time.perf_counter() - t0 < budget_s or n == 0:
-        oracle.moe_tokens(w.x, w.logits, shape.K, w.routed, w.shared, w.zero_mask, tokens=tk)
+        oracle_rows(w, shape, tk, router)
         n += 1
     dt = time.perf_counter() - t0
     return {"value": n * len(tk) / dt, "unit": UNIT, "cores": oracle.threads(), "kind": "oracle",
@@ -199,11 +220,15 @@ def job_tokens_per_s(T, world, ms_per_step):
     return T * world / (ms_per_step * 1e-3)
 
 
-def config_of(shape):
-    return {"workload": shape.name, "T": shape.T, "H": shape.H, "I": shape.I, "E": shape.E, "K": shape.K,
-            "I_shared": shape.I_shared, "weights": "fp8 e4m3fn, fp32 scale per 128x128 block",
-            "activations": "bf16", "logit_bias": shape.bias, "zero_route_frac": shape.zero_frac,
-            "seed": shape.seed}
+def config_of(shape, router="softmax"):
+    c = {"workload": shape.name, "T": shape.T, "H": shape.H, "I": shape.I, "E": shape.E, "K": shape.K,
+         "I_shared": shape.I_shared, "weights": "fp8 e4m3fn, fp32 scale per 128x128 block",
+         "activations": "bf16", "logit_bias": shape.bias, "zero_route_frac": shape.zero_frac,
+         "seed": shape.seed, "router": router}
+    if wl.ROUTERS[router] is not None:
+        c["router_cfg"] = {k: v for k, v in wl.ROUTERS[router].items() if k != "bias"}
+        c["router_cfg"]["selection_bias"] = "N(0, 0.02) per expert" if wl.ROUTERS[router].get("bias") else None
+    return c
 
 
 # ---------------------------------------------------------------- our arm
@@ -216,6 +241,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="decode", choices=wl.SHAPE_ORDER)
     ap.add_argument("--mode", type=int, default=0, help="moe_expert_ffn mode: 0 AUTO, 1 DECODE, 2 PREFILL")
+    ap.add_argument("--router", default="softmax", choices=sorted(wl.ROUTERS),
+                    help="routing variant: softmax top-k (moe_route) or a moe_route_ex preset")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--eager", action="store_true",
                     help="launch every call directly instead of replaying CUDA graphs (for profilers)")
@@ -250,7 +277,13 @@ def main():
     zmask = torch.from_numpy(w.zero_mask).to(dev) if w.zero_mask is not None else None
     routed = moe.Experts.from_host(w.routed, dev)
     shared = moe.Experts.from_host(w.shared, dev) if w.shared is not None else None
-    layer = moe.MoEFFN(routed, T, K, shared, mode=args.mode, device=dev)
+    route_cfg = None
+    kw = wl.ROUTERS[args.router]
+    if kw is not None:
+        route_cfg = {k: v for k, v in kw.items() if k != "bias"}
+        route_cfg["sel_bias"] = (torch.from_numpy(wl.selection_bias(E, shape.seed)).to(dev)
+                                 if kw.get("bias") else None)
+    layer = moe.MoEFFN(routed, T, K, shared, mode=args.mode, device=dev, route_cfg=route_cfg)
     stream = torch.cuda.Stream(device=dev)
 
     def step():
@@ -272,7 +305,11 @@ def main():
 
     def instrumented():
         ev[0].record()
-        moe.moe_route(logits, K, zmask, layer.topk_ids, layer.topk_w)
+        if route_cfg is None:
+            moe.moe_route(logits, K, zmask, layer.topk_ids, layer.topk_w)
+        else:
+            moe.moe_route_ex(logits, K, zero_mask=zmask, topk_ids=layer.topk_ids, topk_w=layer.topk_w,
+                             **route_cfg)
         ev[1].record()
         moe.moe_sort(layer.topk_ids, E, layer.status, layer.offsets, layer.sorted_route, layer.inv_route,
                      layer.sort_ws)
@@ -375,7 +412,7 @@ def main():
     out = {"metric": METRIC, "value": job_tokens_per_s(T, world, t_max), "unit": UNIT, "n_gpus": world,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_max, "higher_is_better": True,
            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-           "config": dict(config_of(shape), parallelism="replicas x%d" % world,
+           "config": dict(config_of(shape, args.router), parallelism="replicas x%d" % world,
                           l2="inputs larger than L2 (touched expert weights %.2f GB > 126 MB)"
                              % (touched * expert_bytes(H, I) / 1e9) if decode_path else
                              "inputs larger than L2 (expert weights %.2f GB > 126 MB)" % (E * expert_bytes(H, I) / 1e9),
@@ -389,7 +426,7 @@ def main():
            "gpu_launches": n_launch * args.steps,
            "clocks": clk.summary()}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(shape)
+        out["cpu_baseline"] = cpu_baseline(shape, args.router)
     if rank == 0:
         print(json.dumps(out), flush=True)
     del g, g2

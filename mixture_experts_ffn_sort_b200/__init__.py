@@ -263,11 +263,16 @@ def moe_combine(y_sorted: torch.Tensor, inv_route: torch.Tensor, y_shared: Optio
 class MoEFFN:
     """The routed MoE FFN of one layer on fixed shapes: route -> sort -> expert
     FFN -> combine, with every buffer allocated once (no allocation per call,
-    so a call can be captured in a CUDA graph after the first one)."""
+    so a call can be captured in a CUDA graph after the first one).
+    route_cfg: keyword arguments of moe_route_ex (score, sel_bias, n_group,
+    topk_group, renormalize, scaling) for a routing variant; None routes with
+    moe_route."""
 
     def __init__(self, routed: Experts, T: int, K: int, shared: Optional[Experts] = None,
-                 mode: int = MOE_MODE_AUTO, out_dtype: int = MOE_OUT_BF16, device="cuda"):
+                 mode: int = MOE_MODE_AUTO, out_dtype: int = MOE_OUT_BF16, device="cuda",
+                 route_cfg: Optional[dict] = None):
         self.routed, self.shared, self.T, self.K = routed, shared, T, K
+        self.route_cfg = dict(route_cfg) if route_cfg else None
         self.E, self.I, self.H = routed.n, routed.inter, routed.w_gate.shape[2]
         self.mode, self.out_dtype = mode, out_dtype
         d = device
@@ -290,12 +295,19 @@ class MoEFFN:
     # Number of the library's kernel launches one forward makes.
     def launches(self) -> int:
         R = self.T * self.K
-        n = 1 + (1 if R <= 16384 else 3) + 2 + (2 if self.shared is not None else 0) + 1
-        return n
+        # The decode form runs the shared expert as a second kernel pair; the
+        # prefill form runs it inside its two kernels.
+        decode = moe_ffn_resolve_mode(self.T, self.K, self.E, self.mode) == MOE_MODE_DECODE
+        ffn = 2 + (2 if self.shared is not None and decode else 0)
+        return 1 + (1 if R <= 16384 else 3) + ffn + 1
 
     def forward(self, x: torch.Tensor, logits: torch.Tensor, zero_mask: Optional[torch.Tensor] = None,
                 stream=None) -> torch.Tensor:
-        moe_route(logits, self.K, zero_mask, self.topk_ids, self.topk_w, stream=stream)
+        if self.route_cfg is None:
+            moe_route(logits, self.K, zero_mask, self.topk_ids, self.topk_w, stream=stream)
+        else:
+            moe_route_ex(logits, self.K, zero_mask=zero_mask, topk_ids=self.topk_ids, topk_w=self.topk_w,
+                         stream=stream, **self.route_cfg)
         moe_sort(self.topk_ids, self.E, self.status, self.offsets, self.sorted_route, self.inv_route,
                  self.sort_ws, stream=stream)
         moe_expert_ffn(x, self.K, self.routed, self.offsets, self.sorted_route, self.topk_w, self.shared,

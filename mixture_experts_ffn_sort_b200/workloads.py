@@ -34,7 +34,7 @@ BLOCK = 128
 
 # Stream tags: one independent stream per tensor kind.
 _TAG_X, _TAG_LOGITS, _TAG_BIAS, _TAG_ROUTED, _TAG_SHARED, _TAG_MASK = 1, 2, 3, 4, 5, 6
-_TAG_IDS, _TAG_YS, _TAG_PROBE = 7, 8, 9
+_TAG_IDS, _TAG_YS, _TAG_PROBE, _TAG_SEL_BIAS = 7, 8, 9, 10
 
 
 def _rng(seed: int, tag: int, index: int = 0) -> np.random.Generator:
@@ -221,6 +221,22 @@ def make_workload(shape, seed: Optional[int] = None, threads: Optional[int] = No
 
 # ---------------------------------------------------------------------------
 # Probe inputs for single-step tests and edge cases.
+
+def selection_bias(E: int, seed: int = 0, std: float = 0.02) -> np.ndarray:
+    """float32 [E] selection-only router bias ~ N(0, std) (the learned
+    load-balancing correction of a DeepSeek-V3-style router, drawn)."""
+    return (_rng(seed, _TAG_SEL_BIAS).standard_normal(E) * std).astype(np.float32)
+
+
+# Router variants of the benchmark and the end-to-end tests, by name: keyword
+# arguments of moe_route_ex / oracle.route_ex (a selection bias, when used, is
+# selection_bias(E, seed)).  "softmax" is the plain router.
+ROUTERS = {
+    "softmax": None,
+    "sigmoid": dict(score=1, n_group=1, topk_group=1, renormalize=True, scaling=2.5),
+    "grouped": dict(score=1, n_group=8, topk_group=4, renormalize=True, scaling=2.5, bias=True),
+}
+
 
 def random_ids(T: int, K: int, E: int, seed: int = 0, distinct: bool = True) -> np.ndarray:
     """int32 [T, K] expert ids; distinct within a token unless distinct=False."""

@@ -133,3 +133,36 @@ def test_route_ex_large_bias_forces_the_set():
     ids, w, _, _ = _run(lg, K, score=SIG, bias=bias)
     assert all(set(r) == set(S) for r in ids)
     _check(lg, K, score=SIG, bias=bias)
+
+
+@pytest.mark.parametrize("router", ["sigmoid", "grouped"])
+@pytest.mark.parametrize("workload,mode", [("tiny", moe.MOE_MODE_AUTO), ("decode", moe.MOE_MODE_DECODE),
+                                           ("decode", moe.MOE_MODE_PREFILL)])
+def test_layer_with_router_variant(workload, mode, router):
+    """The whole path with a routing variant: the layer's expert choice agrees
+    with the oracle router (up to fp32 score ties) and its output equals the
+    brute-force oracle FFN for that choice and the oracle's weights."""
+    from _gpu_util import assert_moe_close, device_workload
+    shape = wl.SHAPES[workload]
+    dw = device_workload(workload)
+    w = dw.w
+    cfg = dict(wl.ROUTERS[router])
+    use_bias = cfg.pop("bias", False)
+    bias = wl.selection_bias(shape.E, shape.seed) if use_bias else None
+    dev = torch.device("cuda")
+    route_cfg = dict(cfg, sel_bias=None if bias is None else torch.from_numpy(bias).to(dev))
+    layer = moe.MoEFFN(dw.routed, shape.T, shape.K, dw.shared, mode=mode, device=dev, route_cfg=route_cfg)
+    out = layer(dw.x, dw.logits, dw.zero_mask)
+    torch.cuda.synchronize()
+    assert layer.status.item() == 0
+    ids = layer.topk_ids.cpu().numpy()
+    oid, _ = oracle.route_ex(w.logits, shape.K, bias=bias, zero_mask=w.zero_mask, **cfg)
+    differ = np.any(ids != oid, axis=1)
+    assert differ.mean() <= 0.01
+    wt = oracle.route_weights(w.logits, ids, score=cfg["score"], renormalize=cfg["renormalize"],
+                              scaling=cfg["scaling"])
+    if w.zero_mask is not None:
+        wt[w.zero_mask != 0] = 0.0
+    np.testing.assert_allclose(layer.topk_w.cpu().numpy(), wt, rtol=W_RTOL, atol=W_ATOL)
+    ref = oracle.moe_tokens_routed(w.x, ids, wt, w.routed, w.shared)
+    assert_moe_close(out, ref, "%s/%s" % (workload, router))
