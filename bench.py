@@ -393,7 +393,8 @@ def main():
     ffn_ms = statistics.median(parts["ffn"])
     R_nz = int(np.count_nonzero(layer.topk_w.cpu().numpy()))
     flops = (R_nz + (T if shape.I_shared else 0)) * 6 * H * I
-    decode_path = moe.moe_ffn_resolve_mode(T, K, E, args.mode) == moe.MOE_MODE_DECODE
+    form = moe.moe_ffn_resolve_mode(T, K, E, args.mode)
+    decode_path = form in (moe.MOE_MODE_DECODE, moe.MOE_MODE_HYBRID)  # bound by the touched weights
     if decode_path:
         algo = touched * expert_bytes(H, I) + (expert_bytes(H, shape.I_shared) if shape.I_shared else 0)
         ach = algo / (ffn_ms * 1e-3) / 1e9

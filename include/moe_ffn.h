@@ -90,6 +90,10 @@ typedef enum moe_status {
 #define MOE_MODE_AUTO 0     /* see moe_ffn_resolve_mode */
 #define MOE_MODE_DECODE 1   /* weight-streaming kernels (memory-bound regime) */
 #define MOE_MODE_PREFILL 2  /* tcgen05 / TMEM grouped GEMM kernels (compute-bound regime) */
+#define MOE_MODE_HYBRID 3   /* experts with <= MOE_HYBRID_ROW_SPLIT rows in the DECODE kernels, the rest
+                               (and the shared expert) in the PREFILL kernels */
+#define MOE_HYBRID_ROW_SPLIT 8
+#define MOE_HYBRID_MAX_ROWS_PER_EXPERT 32
 #define MOE_DECODE_MAX_ROUTES 8192
 #define MOE_DECODE_MAX_ROWS_PER_EXPERT 8
 
@@ -260,12 +264,17 @@ typedef struct moe_fp8_experts {
  *
  * No counterpart on the pages (they pick a kernel per serving phase: the NKI
  * library's MoE TKG for decode and MoE CTE for prefill).  Host-only, launches
- * nothing.  DECODE and PREFILL resolve to themselves; AUTO resolves from
- * host-known sizes alone (never from the device-side expert counts) to
+ * nothing.  DECODE, PREFILL and HYBRID resolve to themselves; AUTO resolves
+ * from host-known sizes alone (never from the device-side expert counts) to
  *   MOE_MODE_DECODE   when T*K <= MOE_DECODE_MAX_ROUTES and
  *                     T*K <= MOE_DECODE_MAX_ROWS_PER_EXPERT * E
  *                     (few rows per expert: streaming the touched weights
  *                     bounds the time),
+ *   MOE_MODE_HYBRID   otherwise when T*K <= MOE_HYBRID_MAX_ROWS_PER_EXPERT * E
+ *                     (a few tens of rows per expert on average: under a
+ *                     skewed load many experts have a few rows and a few have
+ *                     many, and each form takes the experts it is fast on; the
+ *                     split is made on the device from the expert offsets),
  *   MOE_MODE_PREFILL  otherwise (enough rows per expert for the tensor-core
  *                     grouped GEMM to win).
  * Returns the resolved mode, or MOE_ERR_INVALID_ARG for an unknown mode or
@@ -297,8 +306,10 @@ MOE_API int moe_ffn_resolve_mode(int T, int K, int E, int mode);
  *   topk_w         [T, K] f32 (read; route r's weight is topk_w[r])
  *   y_sorted       [T*K, H] bf16 (written for rows p < expert_offsets[E])
  *   y_shared       [T, H] bf16 (written) when shared != NULL, else ignored
- *   mode           MOE_MODE_AUTO | MOE_MODE_DECODE | MOE_MODE_PREFILL
- *                  (AUTO as moe_ffn_resolve_mode resolves it)
+ *   mode           MOE_MODE_AUTO | MOE_MODE_DECODE | MOE_MODE_PREFILL |
+ *                  MOE_MODE_HYBRID (AUTO as moe_ffn_resolve_mode resolves it;
+ *                  HYBRID launches both forms, each skipping the experts the
+ *                  other takes, so every row is written exactly once)
  *   workspace      moe_ffn_workspace_bytes(...) bytes of device scratch
  *   status         optional device int32: MOE_STATUS_BAD_MAP is OR-ed in when
  *                  offsets or route ids are out of range (those rows skipped)

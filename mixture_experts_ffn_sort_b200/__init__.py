@@ -25,7 +25,8 @@ MOE_ERR_UNSUPPORTED_SHAPE = -2
 MOE_ERR_MISALIGNED = -3
 MOE_ERR_WORKSPACE_TOO_SMALL = -4
 MOE_ERR_CUDA = -5
-MOE_MODE_AUTO, MOE_MODE_DECODE, MOE_MODE_PREFILL = 0, 1, 2
+MOE_MODE_AUTO, MOE_MODE_DECODE, MOE_MODE_PREFILL, MOE_MODE_HYBRID = 0, 1, 2, 3
+MOE_HYBRID_ROW_SPLIT = 8
 MOE_OUT_BF16, MOE_OUT_F32 = 0, 1
 MOE_STATUS_BAD_ID, MOE_STATUS_BAD_MAP, MOE_STATUS_TIMEOUT = 1, 2, 4
 MOE_MAX_E, MOE_MAX_K = 1024, 32
@@ -210,7 +211,7 @@ def moe_sort(topk_ids: torch.Tensor, E: int, status: Optional[torch.Tensor] = No
 
 
 def moe_ffn_resolve_mode(T: int, K: int, E: int, mode: int = MOE_MODE_AUTO) -> int:
-    """The FFN form (MOE_MODE_DECODE or MOE_MODE_PREFILL) moe_expert_ffn runs for `mode`."""
+    """The FFN form (MOE_MODE_DECODE, MOE_MODE_PREFILL or MOE_MODE_HYBRID) moe_expert_ffn runs for `mode`."""
     rc = int(lib().moe_ffn_resolve_mode(T, K, E, mode))
     _check(min(rc, 0))
     return rc
@@ -297,8 +298,9 @@ class MoEFFN:
         R = self.T * self.K
         # The decode form runs the shared expert as a second kernel pair; the
         # prefill form runs it inside its two kernels.
-        decode = moe_ffn_resolve_mode(self.T, self.K, self.E, self.mode) == MOE_MODE_DECODE
-        ffn = 2 + (2 if self.shared is not None and decode else 0)
+        form = moe_ffn_resolve_mode(self.T, self.K, self.E, self.mode)
+        ffn = {MOE_MODE_DECODE: 2 + (2 if self.shared is not None else 0), MOE_MODE_PREFILL: 2,
+               MOE_MODE_HYBRID: 4}[form]
         return 1 + (1 if R <= 16384 else 3) + ffn + 1
 
     def forward(self, x: torch.Tensor, logits: torch.Tensor, zero_mask: Optional[torch.Tensor] = None,

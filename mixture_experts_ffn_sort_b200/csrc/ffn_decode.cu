@@ -244,7 +244,8 @@ __device__ __forceinline__ Smem carve(uint8_t* raw, int NG, int row_stride, int 
     return s;
 }
 
-// The experts of this call with at least one row, in increasing order, into
+// The experts of this call with at least one row (and at most a.row_split
+// rows when a.row_split > 0), in increasing order, into
 // touched[0 .. count), and the exclusive prefix of their token groups (of NG
 // rows) into gpre[0 .. count]; returns the total number of groups.  Experts
 // whose offsets are corrupt are left out (and flagged); *ntouched = count.
@@ -262,6 +263,7 @@ __device__ long build_touched(const FfnArgs& a, int NG, int* touched, int* gpre,
             report_status(a.status, MOE_STATUS_BAD_MAP);
             continue;
         }
+        if (a.row_split > 0 && n > a.row_split) continue;  // left to the prefill form
         cnt += n > 0;
         grp += static_cast<int>((n + NG - 1) / NG);
     }
@@ -287,7 +289,7 @@ __device__ long build_touched(const FfnArgs& a, int NG, int* touched, int* gpre,
     int pg = (warp ? warp_sums[warp - 1][1] : 0) + xg - grp;
     for (int e = e0; e < e1; ++e) {
         long p0, n;
-        if (expert_rows(a, e, p0, n) && n > 0) {
+        if (expert_rows(a, e, p0, n) && n > 0 && (a.row_split <= 0 || n <= a.row_split)) {
             touched[pc] = e;
             gpre[pc] = pg;
             ++pc;

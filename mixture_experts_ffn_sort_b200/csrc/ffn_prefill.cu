@@ -166,6 +166,13 @@ __device__ __forceinline__ long expert_len(const FfnArgs& a, int e, long R, bool
     return f - b;
 }
 
+// Rows of expert e this launch processes: none for a routed expert left to
+// the decode form (at most a.row_split rows when a.row_split > 0).
+__device__ __forceinline__ long expert_rows_here(const FfnArgs& a, int e, long R, bool* bad) {
+    const long n = expert_len(a, e, R, bad);
+    return (a.row_split > 0 && e < a.ex.n && n <= a.row_split) ? 0 : n;
+}
+
 __device__ __forceinline__ int num_experts(const FfnArgs& a) { return a.ex.n + (a.sh.n ? 1 : 0); }
 
 // Item list over the routed experts then the shared one: pre[] holds the
@@ -177,7 +184,7 @@ __device__ int build_tiles(const FfnArgs& a, int groups_r, int groups_s, int* pr
     const int e0 = min(E, static_cast<int>(threadIdx.x) * per), e1 = min(E, e0 + per);
     int local = 0;
     bool bad = false;
-    for (int e = e0; e < e1; ++e) local += items_of(expert_len(a, e, R, &bad), e < a.ex.n ? groups_r : groups_s);
+    for (int e = e0; e < e1; ++e) local += items_of(expert_rows_here(a, e, R, &bad), e < a.ex.n ? groups_r : groups_s);
     if (bad) report_status(a.status, MOE_STATUS_BAD_MAP);
     // Block exclusive scan of `local`.
     __shared__ int warp_sums[32];
@@ -203,7 +210,7 @@ __device__ int build_tiles(const FfnArgs& a, int groups_r, int groups_s, int* pr
     int run = (warp ? warp_sums[warp - 1] : 0) + x - local;
     for (int e = e0; e < e1; ++e) {
         pre[e] = run;
-        run += items_of(expert_len(a, e, R, &bad), e < a.ex.n ? groups_r : groups_s);
+        run += items_of(expert_rows_here(a, e, R, &bad), e < a.ex.n ? groups_r : groups_s);
     }
     const int total = warp_sums[nw - 1];
     if (threadIdx.x == 0) pre[E] = total;

@@ -70,6 +70,10 @@ struct FfnArgs {
     ExpertsView sh;  // sh.n == 0: none
     uint16_t* h_sh;  // [T, sh.inter] bf16 scratch
     uint16_t* y_sh;  // [T, H] bf16 output
+    // Split of the routed experts between the two forms (MOE_MODE_HYBRID):
+    // when > 0, the decode form takes the experts with 1..row_split rows and
+    // the prefill form those with more; 0 = every expert.
+    int row_split;
 };
 
 cudaError_t launch_ffn_decode(const FfnArgs& a, cudaStream_t stream);

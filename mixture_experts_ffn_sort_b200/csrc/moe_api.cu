@@ -177,13 +177,13 @@ int moe_ffn_resolve_mode(int T, int K, int E, int mode) {
     g_err.clear();
     if (T < 0 || K < 1 || E < 1)
         return fail(MOE_ERR_INVALID_ARG, "moe_ffn_resolve_mode: T=%d, K=%d, E=%d out of range", T, K, E);
-    if (mode == MOE_MODE_DECODE || mode == MOE_MODE_PREFILL) return mode;
+    if (mode == MOE_MODE_DECODE || mode == MOE_MODE_PREFILL || mode == MOE_MODE_HYBRID) return mode;
     if (mode != MOE_MODE_AUTO)
-        return fail(MOE_ERR_INVALID_ARG, "moe_ffn_resolve_mode: mode=%d is not AUTO/DECODE/PREFILL", mode);
+        return fail(MOE_ERR_INVALID_ARG, "moe_ffn_resolve_mode: mode=%d is not AUTO/DECODE/PREFILL/HYBRID", mode);
     const long R = static_cast<long>(T) * K;
-    return R <= MOE_DECODE_MAX_ROUTES && R <= static_cast<long>(MOE_DECODE_MAX_ROWS_PER_EXPERT) * E
-               ? MOE_MODE_DECODE
-               : MOE_MODE_PREFILL;
+    if (R <= MOE_DECODE_MAX_ROUTES && R <= static_cast<long>(MOE_DECODE_MAX_ROWS_PER_EXPERT) * E)
+        return MOE_MODE_DECODE;
+    return R <= static_cast<long>(MOE_HYBRID_MAX_ROWS_PER_EXPERT) * E ? MOE_MODE_HYBRID : MOE_MODE_PREFILL;
 }
 
 size_t moe_ffn_workspace_bytes(int T, int K, int H, int E, int I, int I_shared, int mode) {
@@ -205,8 +205,8 @@ int moe_expert_ffn(const uint16_t* x, int T, int H, int K, const moe_fp8_experts
     const int E = routed->n_experts, I = routed->inter;
     int rc = check_sizes(T, E, K);
     if (rc) return rc;
-    if (mode != MOE_MODE_AUTO && mode != MOE_MODE_DECODE && mode != MOE_MODE_PREFILL)
-        return fail(MOE_ERR_INVALID_ARG, "moe_expert_ffn: mode=%d is not AUTO/DECODE/PREFILL", mode);
+    if (mode != MOE_MODE_AUTO && mode != MOE_MODE_DECODE && mode != MOE_MODE_PREFILL && mode != MOE_MODE_HYBRID)
+        return fail(MOE_ERR_INVALID_ARG, "moe_expert_ffn: mode=%d is not AUTO/DECODE/PREFILL/HYBRID", mode);
     if (H < 128 || H % MOE_BLOCK || H > 8192)
         return fail(MOE_ERR_UNSUPPORTED_SHAPE, "moe_expert_ffn: H=%d must be a multiple of 128 in 128..=8192", H);
     if ((rc = check_experts(routed, H, "routed"))) return rc;
@@ -227,7 +227,8 @@ int moe_expert_ffn(const uint16_t* x, int T, int H, int K, const moe_fp8_experts
     if (workspace_bytes < need || !workspace)
         return fail(MOE_ERR_WORKSPACE_TOO_SMALL, "moe_expert_ffn: workspace of %zu bytes, need %zu",
                     workspace_bytes, need);
-    const bool prefill = moe_ffn_resolve_mode(T, K, E, mode) == MOE_MODE_PREFILL;
+    const int form = moe_ffn_resolve_mode(T, K, E, mode);
+    const bool prefill = form == MOE_MODE_PREFILL || form == MOE_MODE_HYBRID;
     if (prefill && !moe::ffn_prefill_supported(H, I))
         return fail(MOE_ERR_UNSUPPORTED_SHAPE, "moe_expert_ffn: H=%d, inter=%d not supported by the PREFILL kernels", H, I);
 
@@ -253,12 +254,19 @@ int moe_expert_ffn(const uint16_t* x, int T, int H, int K, const moe_fp8_experts
             a.h_sh = reinterpret_cast<uint16_t*>(ws + ffn_h_bytes(R, I));
             a.y_sh = y_shared;
         }
+        // HYBRID: the experts with more than MOE_HYBRID_ROW_SPLIT rows here, the
+        // others in the decode form below.
+        a.row_split = form == MOE_MODE_HYBRID ? MOE_HYBRID_ROW_SPLIT : 0;
         const cudaError_t e = moe::launch_ffn_prefill(a, stream);
-        return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_expert_ffn launch");
+        if (e != cudaSuccess || form == MOE_MODE_PREFILL)
+            return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_expert_ffn launch");
+        // The decode form gets experts of at most MOE_HYBRID_ROW_SPLIT rows: its
+        // token group (8, 16 or 32 rows, from the average rows) covers them.
+        a.avg_rows = MOE_HYBRID_ROW_SPLIT / 2;
     }
     cudaError_t e = moe::launch_ffn_decode(a, stream);
     if (e != cudaSuccess) return cuda_fail(e, "moe_expert_ffn routed launch");
-    if (shared) {
+    if (shared && form == MOE_MODE_DECODE) {
         moe::FfnArgs s = a;
         s.ex = {shared->w_gate, shared->w_up, shared->w_down, shared->s_gate, shared->s_up, shared->s_down, 1, Is};
         s.identity = true;

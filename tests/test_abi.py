@@ -56,22 +56,26 @@ def test_workspace_queries(L):
 
 
 def test_ffn_resolve_mode(L):
-    D, PF = moe.MOE_MODE_DECODE, moe.MOE_MODE_PREFILL
+    D, PF, HY = moe.MOE_MODE_DECODE, moe.MOE_MODE_PREFILL, moe.MOE_MODE_HYBRID
     # Explicit modes resolve to themselves at any size.
     assert L.moe_ffn_resolve_mode(32768, 10, 512, D) == D
     assert L.moe_ffn_resolve_mode(1, 1, 8, PF) == PF
-    # AUTO: decode while routes per expert stay at most 8 and routes at most 8192.
+    assert L.moe_ffn_resolve_mode(1, 1, 8, HY) == HY
+    # AUTO: decode while routes per expert stay at most 8 and routes at most
+    # 8192; hybrid up to 32 routes per expert; prefill beyond.
     assert L.moe_ffn_resolve_mode(16, 2, 8, 0) == D          # 4 routes per expert
     assert L.moe_ffn_resolve_mode(64, 8, 256, 0) == D        # 2
     assert L.moe_ffn_resolve_mode(256, 8, 256, 0) == D       # 8: the limit
-    assert L.moe_ffn_resolve_mode(257, 8, 256, 0) == PF
-    assert L.moe_ffn_resolve_mode(512, 8, 256, 0) == PF      # 16
+    assert L.moe_ffn_resolve_mode(257, 8, 256, 0) == HY
+    assert L.moe_ffn_resolve_mode(512, 8, 256, 0) == HY      # 16
+    assert L.moe_ffn_resolve_mode(1024, 8, 256, 0) == HY     # 32: the limit
+    assert L.moe_ffn_resolve_mode(1025, 8, 256, 0) == PF
     assert L.moe_ffn_resolve_mode(1024, 8, 1024, 0) == D     # 8192 routes
-    assert L.moe_ffn_resolve_mode(1025, 8, 1024, 0) == PF    # 8200 routes
+    assert L.moe_ffn_resolve_mode(1025, 8, 1024, 0) == HY    # 8200 routes, 8.0 per expert
     assert L.moe_ffn_resolve_mode(8192, 10, 512, 0) == PF
     assert L.moe_ffn_resolve_mode(0, 8, 256, 0) == D
-    assert moe.moe_ffn_resolve_mode(512, 8, 256) == PF
-    for args in ((4, 2, 8, 3), (-1, 2, 8, 0), (4, 0, 8, 0), (4, 2, 0, 0)):
+    assert moe.moe_ffn_resolve_mode(512, 8, 256) == HY
+    for args in ((4, 2, 8, 4), (-1, 2, 8, 0), (4, 0, 8, 0), (4, 2, 0, 0)):
         assert L.moe_ffn_resolve_mode(*args) == moe.MOE_ERR_INVALID_ARG
         assert "moe_ffn_resolve_mode" in L.moe_last_error().decode()
     with pytest.raises(moe.MoEError):

@@ -22,7 +22,7 @@ pytestmark = pytest.mark.gpu
 ALL = wl.SHAPE_ORDER
 FULL = {"tiny", "decode", "decode_skew"}   # compared on every row
 SAMPLE_ROWS = 256
-MODES = [moe.MOE_MODE_DECODE, moe.MOE_MODE_PREFILL]
+MODES = [moe.MOE_MODE_DECODE, moe.MOE_MODE_PREFILL, moe.MOE_MODE_HYBRID]
 
 
 @pytest.fixture(scope="module", params=ALL)
