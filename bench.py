@@ -65,7 +65,8 @@ def profile_traffic(workload, kind):
 
 
 FFN_SOURCES = {"decode": ("ffn_decode.cu", "device_common.cuh", "launch.h"),
-               "prefill": ("ffn_prefill.cu", "device_common.cuh", "launch.h")}
+               "prefill": ("ffn_prefill.cu", "device_common.cuh", "launch.h"),
+               "hybrid": ("ffn_decode.cu", "ffn_prefill.cu", "device_common.cuh", "launch.h")}
 
 
 def sources_hash(kind="decode"):
@@ -398,7 +399,7 @@ def main():
     if decode_path:
         algo = touched * expert_bytes(H, I) + (expert_bytes(H, shape.I_shared) if shape.I_shared else 0)
         ach = algo / (ffn_ms * 1e-3) / 1e9
-        traffic = profile_traffic(shape.name, "decode")
+        traffic = profile_traffic(shape.name, "hybrid" if form == moe.MOE_MODE_HYBRID else "decode")
         roof = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm"], "unit": "GB/s",
                 "frac": ach / peaks["hbm"], "traffic": traffic,
                 "kernel": "moe_expert_ffn (gate/up + down kernels)", "algorithmic_bytes": algo,
