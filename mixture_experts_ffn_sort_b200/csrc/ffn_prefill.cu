@@ -598,11 +598,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const long u = MODE == kGateUp ? 2 * g + hi : g;  // A unit of this warp's work
                     const int sw = static_cast<int>(gw % kSW), sa = static_cast<int>(u % kSA);
                     const bool ok1 = wait_bar(&B->w_full[sw], static_cast<uint32_t>((gw / kSW) & 1), B, a.status);
-                    bool ok2 = true;
-                    if (u >= kSA)
-                        ok2 = wait_bar(&B->a_done[sa], static_cast<uint32_t>((u / kSA - 1) & 1), B, a.status);
                     uint32_t v[NW];
-                    if (ok1 && ok2) {
+                    if (ok1) {
                         const float sc = scr[kb >> 1];
                         const uint8_t* base = w_ring + sw * kWStage + sub + srow * 128;
 #pragma unroll
@@ -622,6 +619,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     __syncwarp();
                     if ((g & 1) && lane == 0) mbar_arrive(&B->w_empty[sw]);
+                    // The A slot is free once the MMAs that last read it have
+                    // completed; the decode above overlapped that wait.
+                    if (u >= kSA) wait_bar(&B->a_done[sa], static_cast<uint32_t>((u / kSA - 1) & 1), B, a.status);
+                    tc_fence_after();
                     const uint32_t acol = kACol + sa * 32 + (MODE == kGateUp ? 0 : hi * 16);
                     if constexpr (MODE == kGateUp)
                         tmem_st32(tmem + (static_cast<uint32_t>(32 * q) << 16) + acol, v);
