@@ -68,7 +68,7 @@ def test_prefill_shapes_with_shared(T, H, I, E, K, Is):
         assert_moe_close(ys, oracle.ffn_shared(x, sh), "y_shared")
 
 
-@pytest.mark.parametrize("mode", [moe.MOE_MODE_DECODE, moe.MOE_MODE_PREFILL])
+@pytest.mark.parametrize("mode", [moe.MOE_MODE_DECODE, moe.MOE_MODE_PREFILL, moe.MOE_MODE_HYBRID])
 def test_both_modes_full_pipeline(mode):
     T, H, I, E, K = 300, 512, 256, 16, 4
     ex = wl.draw_experts(5, 64, E, I, H, 0.05, threads=4)
