@@ -59,8 +59,9 @@ constexpr int kOStoreRows = 32;             // rows per TMA store of the staging
 // Per mode: M-tiles (128 weight rows each) per step, weight stage bytes and
 // depths of the weight ring and of the bf16 A ring in TMEM.  The A ring holds
 // kSA units of 32 columns (one M-tile's 64 reduction columns); a gate/up step
-// fills two units (one per M-tile, each released as soon as its own MMAs are
-// done), a down step one.
+// fills two units, a down step one, and the kSS = kSA / MT step slots each
+// have one full/done barrier pair (one wait and one commit per step for the
+// MMA warp, which shares its scheduler with transform warps).
 template <int MODE> struct Cfg;
 // Warp roles (transform and epilogue warps sit on their TMEM lane quarter, warp % 4):
 // 0 weight TMA, 1 MMA, 2-7 token rows (gate/up) or 2 token TMA (down), 4-7
@@ -85,10 +86,10 @@ enum Mode { kGateUp = 0, kDown = 1 };
 // A weight stage holds 128 reduction columns (128-byte rows) and feeds two
 // 64-column MMA steps.
 template <> struct Cfg<0> {
-    static constexpr int MT = 2, kWStage = 2 * 128 * 128, kSW = kWRing / kWStage, kSA = 4;
+    static constexpr int MT = 2, kWStage = 2 * 128 * 128, kSW = kWRing / kWStage, kSA = 4, kSS = kSA / MT;
 };
 template <> struct Cfg<1> {
-    static constexpr int MT = 1, kWStage = 128 * 128, kSW = kWRing / kWStage, kSA = 4;
+    static constexpr int MT = 1, kWStage = 128 * 128, kSW = kWRing / kWStage, kSA = 4, kSS = kSA / MT;
 };
 constexpr int kSWMax = 8, kSAMax = 4;
 
@@ -286,9 +287,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&B->b_full[s], MODE == kGateUp ? kGatherThreads : 1);
             mbar_init(&B->b_done[s], 1);
         }
-        for (int s = 0; s < kSA; ++s) {
-            // gate/up: the 4 transform warps of one M-tile fill a unit; down: all 8.
-            mbar_init(&B->a_full[s], MODE == kGateUp ? kXformWarps / 2 : kXformWarps);
+        for (int s = 0; s < C::kSS; ++s) {
+            // One barrier pair per step slot (the MT units of one step): all
+            // eight transform warps fill it, one commit frees it.
+            mbar_init(&B->a_full[s], kXformWarps);
             mbar_init(&B->a_done[s], 1);
         }
         for (int d = 0; d < 2; ++d) {
@@ -621,7 +623,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if ((g & 1) && lane == 0) mbar_arrive(&B->w_empty[sw]);
                     // The A slot is free once the MMAs that last read it have
                     // completed; the decode above overlapped that wait.
-                    if (u >= kSA) wait_bar(&B->a_done[sa], static_cast<uint32_t>((u / kSA - 1) & 1), B, a.status);
+                    const int ss = static_cast<int>(g % C::kSS);  // step slot of this step
+                    if (g >= C::kSS) wait_bar(&B->a_done[ss], static_cast<uint32_t>((g / C::kSS - 1) & 1), B, a.status);
                     tc_fence_after();
                     const uint32_t acol = kACol + sa * 32 + (MODE == kGateUp ? 0 : hi * 16);
                     if constexpr (MODE == kGateUp)
@@ -631,7 +634,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tmem_st_wait();
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&B->a_full[sa]);
+                    if (lane == 0) mbar_arrive(&B->a_full[ss]);
                 }
             }
         }
@@ -673,21 +676,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                     // (async proxy).
                     if (MODE == kGateUp) fence_proxy_async_smem();
                     const uint64_t bdesc = bdesc0 + static_cast<uint64_t>((sb * kBStage) >> 4);
+                    // The step's A units (one per M-tile) arrive together.
+                    const int ss = static_cast<int>(ga % C::kSS);
+                    const bool oka = wait_bar(&B->a_full[ss], static_cast<uint32_t>((ga / C::kSS) & 1), B, a.status);
+                    tc_fence_after();
+                    if (okb && oka) {
 #pragma unroll
-                    for (int mt = 0; mt < MT; ++mt) {
-                        // A unit of M-tile mt of this step.
-                        const long u = ga * MT + mt;
-                        const int sa = static_cast<int>(u % kSA);
-                        const bool oka = wait_bar(&B->a_full[sa], static_cast<uint32_t>((u / kSA) & 1), B, a.status);
-                        tc_fence_after();
-                        if (okb && oka) {
-#pragma unroll
-                            for (int k = 0; k < 4; ++k)
-                                umma_ts_f16_elect(d_base + mt * kDRegion, a_base + sa * 32 + k * 8,
-                                                  bdesc + static_cast<uint64_t>(k * 2), idesc,
-                                                  (kb > 0 || k > 0) ? 1u : 0u);
+                        for (int mt = 0; mt < MT; ++mt) {
+                            const int sa = static_cast<int>((ga * MT + mt) % kSA);  // TMEM slot of the unit
+                            if (mt == MT - 1)
+                                umma_ts_f16_x4_commit_elect(d_base + mt * kDRegion, a_base + sa * 32, bdesc, idesc,
+                                                            kb > 0 ? 1u : 0u, &B->a_done[ss]);
+                            else
+                                umma_ts_f16_x4_elect(d_base + mt * kDRegion, a_base + sa * 32, bdesc, idesc,
+                                                     kb > 0 ? 1u : 0u);
                         }
-                        umma_commit_elect(&B->a_done[sa]);
+                    } else {
+                        umma_commit_elect(&B->a_done[ss]);
                     }
                     if (!resident) {
                         umma_commit_elect(&B->b_done[sb]);
