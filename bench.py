@@ -70,13 +70,17 @@ FFN_SOURCES = {"decode": ("ffn_decode.cu", "device_common.cuh", "launch.h"),
 
 
 def sources_hash(kind="decode"):
-    """Hash of the sources of the FFN kernels a profile summary was taken on."""
+    """Hash of the code of the FFN kernels a profile summary was taken on
+    (comments and layout left out, so editing a comment keeps the summary)."""
     d = os.path.join(ROOT, "mixture_experts_ffn_sort_b200", "csrc")
     hs = hashlib.sha256()
     for f in FFN_SOURCES[kind]:
         path = os.path.join(d, f)
         if os.path.exists(path):
-            hs.update(open(path, "rb").read())
+            text = open(path).read()
+            text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+            text = re.sub(r"//[^\n]*", " ", text)
+            hs.update(" ".join(text.split()).encode())
     return hs.hexdigest()[:16]
 
 

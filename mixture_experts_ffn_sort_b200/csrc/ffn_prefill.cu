@@ -11,7 +11,9 @@
 //
 // One persistent kernel per GEMM (gate/up, then down); each CTA owns one SM
 // and walks a list of output tiles built on the device from the expert
-// offsets (no host sync).  A tile is 128 weight rows x up to 192 token rows:
+// offsets (no host sync; under MOE_MODE_HYBRID the experts with at most
+// FfnArgs::row_split rows are left to the weight-streaming kernels).  A tile
+// is 128 weight rows x up to 192 token rows:
 //  * swap-AB: the weights are the M=128 operand A, the tokens the N operand B,
 //    so the FP8 decode writes tensor memory, not shared memory;
 //  * warp 0: the weight tile's FP8 bytes by TMA in stages of 128 reduction
@@ -23,13 +25,18 @@
 //    arrives on the stage's mbarrier when its copies land); down loads
 //    contiguous rows of h as one 2-D TMA tile from warp 2 -- up to 4 stages
 //    ahead;
-//  * transform warps 8-15: each thread owns one TMEM lane (one weight row)
-//    and half of a stage's columns, decodes its FP8 codes to
-//    bf16(e4m3 * block scale) and stores them to TMEM with tcgen05.st (A
-//    operand, two bf16 per column), into a 4-deep A ring;
-//  * warp 1: one thread issues tcgen05.mma (kind::f16, A in TMEM, B in
-//    shared memory, fp32 accumulator D in TMEM, double-buffered so the
-//    epilogue of one tile overlaps the main loop of the next);
+//  * transform warps 8-15: each thread owns one TMEM lane (one weight row);
+//    gate/up: warps 8-11 decode M-tile 0 and 12-15 M-tile 1, all 64 columns
+//    of a step; down: two warps per lane quarter, half the columns each.  A
+//    thread decodes its FP8 codes to bf16(e4m3 * block scale) as soon as the
+//    weight stage lands, then waits for its A slot and stores them with
+//    tcgen05.st (A operand, two bf16 per column) into a ring of four 32-column
+//    units (two gate/up steps or four down steps, one barrier pair per step);
+//  * warp 1 issues tcgen05.mma warp-uniformly, one elected lane per four
+//    MMAs (kind::f16, A in TMEM, B in shared memory, fp32 accumulator D in
+//    TMEM: gate/up uses both 192-column regions for one tile's two M-tiles,
+//    down alternates between them so the epilogue of one output block
+//    overlaps the MMAs of the next);
 //  * epilogue warps 4-7 (in gate/up, between their gathers: after issuing the
 //    next item's first stages): tcgen05.ld 16x256b of D; in each 32-lane
 //    quarter of a gate/up M-tile, lanes 0-15 hold the gate rows and lanes
