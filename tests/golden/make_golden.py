@@ -1,4 +1,4 @@
-"""Writes tests/golden/tiny_oracle.txt from the CPU oracle alone.
+"""Writes tests/golden/tiny_oracle.txt and tiny_route_ex.txt from the CPU oracle alone.
 
 The source pages print no worked example of the MoE FFN, so the stored values
 here are the oracle's own output on the seeded "tiny" workload (T=16, H=256,
@@ -32,6 +32,17 @@ def main():
     for t in range(4):
         lines.append("out%d " % t + " ".join("%.17g" % v for v in o["out"][t, :16]))
     with open(os.path.join(HERE, "tiny_oracle.txt"), "w") as f:
+        f.write("\n".join(lines) + "\n")
+    # Routing variants on the tiny workload's logits: sigmoid scores, a
+    # selection-only bias, 4 groups of 2 experts with 2 kept, scaling 2.5.
+    bias = workloads.selection_bias(w.shape.E, seed=1, std=0.05)
+    ids, wt = oracle.route_ex(w.logits, w.shape.K, score=oracle.SCORE_SIGMOID, bias=bias, n_group=4,
+                              topk_group=2, scaling=2.5)
+    lines = ["# oracle route_ex, workload tiny logits; sigmoid, bias selection_bias(8, seed=1, std=0.05),",
+             "# 4 groups / 2 kept, renormalised, scaling 2.5; written by tests/golden/make_golden.py",
+             "ids " + " ".join(map(str, ids.ravel())),
+             "w " + " ".join("%.17g" % v for v in wt.ravel())]
+    with open(os.path.join(HERE, "tiny_route_ex.txt"), "w") as f:
         f.write("\n".join(lines) + "\n")
 
 

@@ -485,3 +485,19 @@ def test_oracle_matches_stored_golden(tiny):
     for t in range(4):
         np.testing.assert_allclose(np.array(rows["out%d" % t], float), o["out"][t, :16],
                                    rtol=1e-13, atol=1e-15)
+
+
+def test_route_ex_matches_stored_golden(tiny):
+    """The stored routing-variant output of the tiny workload (tests/golden/make_golden.py)."""
+    import os
+    path = os.path.join(os.path.dirname(__file__), "golden", "tiny_route_ex.txt")
+    rows = {}
+    for line in open(path):
+        if not line.startswith("#"):
+            key, *vals = line.split()
+            rows[key] = vals
+    bias = wl.selection_bias(tiny.shape.E, seed=1, std=0.05)
+    ids, w = oracle.route_ex(tiny.logits, tiny.shape.K, score=SIG, bias=bias, n_group=4, topk_group=2,
+                             scaling=2.5)
+    assert list(map(int, rows["ids"])) == list(ids.ravel())
+    np.testing.assert_allclose(np.array(rows["w"], float), w.ravel(), rtol=1e-15)
