@@ -34,7 +34,7 @@ BLOCK = 128
 
 # Stream tags: one independent stream per tensor kind.
 _TAG_X, _TAG_LOGITS, _TAG_BIAS, _TAG_ROUTED, _TAG_SHARED, _TAG_MASK = 1, 2, 3, 4, 5, 6
-_TAG_IDS, _TAG_YS, _TAG_PROBE, _TAG_SEL_BIAS = 7, 8, 9, 10
+_TAG_IDS, _TAG_YS, _TAG_PROBE, _TAG_SEL_BIAS, _TAG_ROUTER_W = 7, 8, 9, 10, 11
 
 
 def _rng(seed: int, tag: int, index: int = 0) -> np.random.Generator:
@@ -227,6 +227,14 @@ def selection_bias(E: int, seed: int = 0, std: float = 0.02) -> np.ndarray:
     load-balancing correction of a DeepSeek-V3-style router, drawn)."""
     return (_rng(seed, _TAG_SEL_BIAS).standard_normal(E) * std).astype(np.float32)
 
+
+
+def router_weight(E: int, H: int, seed: int = 0) -> np.ndarray:
+    """uint16 bf16 bits [E, H]: the router's gate vectors ~ N(0, 1/H), so that
+    for x ~ N(0, 1) the logits x . w_e are ~ N(0, 1), the logit distribution
+    the routing workloads draw directly."""
+    w = _rng(seed, _TAG_ROUTER_W).standard_normal((E, H), dtype=np.float32) * np.float32(1.0 / np.sqrt(H))
+    return to_bf16_bits(w)
 
 # Router variants of the benchmark and the end-to-end tests, by name: keyword
 # arguments of moe_route_ex / oracle.route_ex (a selection bias, when used, is

@@ -65,6 +65,7 @@ def lib():
             L.oracle_route_ex.argtypes = [P, I, I, I, I, P, I, I, I, ctypes.c_double, P, P, P]
             L.oracle_route_weights.argtypes = [P, I, I, I, I, I, ctypes.c_double, P, P]
             L.oracle_route_select_scores.argtypes = [P, I, I, I, P, P]
+            L.oracle_router_logits.argtypes = [P, P, I, I, I, P]
             L.oracle_sort.argtypes = [P, I, I, I, P, P, P]
             L.oracle_sort.restype = I
             L.oracle_ffn_sorted.argtypes = [P, I, I, I, P, P, P, P, P]
@@ -181,6 +182,27 @@ def route_select_scores(logits: np.ndarray, score: int, bias: Optional[np.ndarra
     lib().oracle_route_select_scores(_p(lg), T, E, int(score), _p(b), _p(c))
     return c
 
+
+def router_logits(x_bits: np.ndarray, w_router_bits: np.ndarray) -> np.ndarray:
+    """float64 [T,E]: the router's gate GEMM x . w_router^T of bf16 bit patterns
+    x [T,H] and w_router [E,H], in fp64."""
+    xb = _c(x_bits, np.uint16)
+    wb = _c(w_router_bits, np.uint16)
+    T, H = xb.shape
+    E = wb.shape[0]
+    assert wb.shape[1] == H
+    out = np.empty((T, E), np.float64)
+    lib().oracle_router_logits(_p(xb), _p(wb), T, H, E, _p(out))
+    return out
+
+
+def router(x_bits: np.ndarray, w_router_bits: np.ndarray, K: int, **route_kw):
+    """The fused router: fp64 gate GEMM, rounded to the route step's fp32 logit
+    type, then route_ex.  -> (logits64 [T,E], logits32 [T,E], ids [T,K], w [T,K])."""
+    l64 = router_logits(x_bits, w_router_bits)
+    l32 = l64.astype(np.float32)
+    ids, w = route_ex(l32, K, **route_kw)
+    return l64, l32, ids, w
 
 
 def sort(ids: np.ndarray, E: int):

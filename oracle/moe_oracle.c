@@ -14,6 +14,7 @@
  *   W[n, k]    = e4m3fn(q[n, k]) * s[n/128, k/128]                    (block-scaled FP8)
  *   FFN_e(x)   = Wd_e (silu(Wg_e x) * (Wu_e x)),  silu(z) = z / (1 + e^-z)
  *   out[t]     = sum_j w[t,j] FFN_{ids[t,j]}(x[t]) + FFN_shared(x[t])
+ *   logits[t]  = W_r x[t]   (the router's gate GEMM, when the logits are not given)
  *
  * Sources (page title, section):
  *  - dstair/gated-deltanet-nki-trainium, "FP8 MoE decode kernel
@@ -27,6 +28,8 @@
  *  - ROCm/aiter PR #5988 description: the sorted pipeline with an inverse
  *    route map and an FP32 route reduction; "10 routed experts plus one shared
  *    expert".
+ *  - spark_model/layers/nemotron_moe.rs, `prefill` step 2: the router's dense
+ *    gate GEMM [N, H] x [H, E]^T -> [N, E] logits.
  *  - NKI Library kernel reference, MoE kernels: Router Top-K, Permute Routed
  *    Tokens (sort by expert), Top-K Reduce.
  *
@@ -274,6 +277,25 @@ void oracle_route_select_scores(const float* logits, int T, int E, int score, co
         route_scores(logits + (size_t)t * E, E, score, ct);
         if (bias)
             for (int e = 0; e < E; ++e) ct[e] += (double)bias[e];
+    }
+}
+
+/* ---------------------------------------------------------------- router GEMM */
+
+/* The router's gate GEMM (spark_model/layers/nemotron_moe.rs, `prefill`, step
+ * 2: [N, H] x [H, E]^T -> [N, E] gate logits): for every token t and expert e,
+ *   logits[t, e] = sum_h x[t, h] * w_router[e, h],
+ * the bf16 inputs widened exactly, every product and the sum in fp64, h in
+ * increasing order.  The route step takes fp32 logits; the caller rounds. */
+void oracle_router_logits(const uint16_t* x, const uint16_t* w_router, int T, int H, int E, double* logits) {
+#pragma omp parallel for num_threads(g_threads) schedule(static)
+    for (int t = 0; t < T; ++t) {
+        for (int e = 0; e < E; ++e) {
+            double acc = 0.0;
+            for (int h = 0; h < H; ++h)
+                acc += oracle_bf16_value(x[(size_t)t * H + h]) * oracle_bf16_value(w_router[(size_t)e * H + h]);
+            logits[(size_t)t * E + e] = acc;
+        }
     }
 }
 

@@ -501,3 +501,52 @@ def test_route_ex_matches_stored_golden(tiny):
                              scaling=2.5)
     assert list(map(int, rows["ids"])) == list(ids.ravel())
     np.testing.assert_allclose(np.array(rows["w"], float), w.ravel(), rtol=1e-15)
+
+
+# ------------------------------------------------------------------ router gate GEMM
+
+def test_router_logits_match_library_matmul():
+    """The fp64 gate GEMM against numpy's matmul of torch's bf16 -> float64
+    widening: catches a transposed operand (T != E != H), a wrong stride or a
+    dropped term."""
+    x = wl.random_rows_bf16(37, 192, seed=3)
+    w = wl.router_weight(21, 192, seed=4)
+    got = oracle.router_logits(x, w)
+    ref = _x64(x).numpy() @ _x64(w).numpy().T
+    assert got.shape == (37, 21)
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_router_logits_closed_forms():
+    """One-hot tokens pick a column of w_router; small-integer inputs give
+    exact integer logits (every product and sum is exact in fp64)."""
+    H, E = 64, 5
+    w = wl.router_weight(E, H, seed=5)
+    x = np.zeros((3, H), np.uint16)
+    for t, h in enumerate((0, 17, 63)):
+        x[t, h] = 0x3F80  # 1.0
+    got = oracle.router_logits(x, w)
+    w64 = oracle.bf16_array(w)
+    for t, h in enumerate((0, 17, 63)):
+        assert np.array_equal(got[t], w64[:, h])
+    rng = np.random.default_rng(6)
+    xi = rng.integers(-8, 9, (4, H)).astype(np.float32)
+    wi = rng.integers(-8, 9, (E, H)).astype(np.float32)
+    got = oracle.router_logits(wl.to_bf16_bits(xi), wl.to_bf16_bits(wi))
+    exact = [[sum(int(a) * int(b) for a, b in zip(xi[t], wi[e])) for e in range(E)] for t in range(4)]
+    assert np.array_equal(got, np.array(exact, np.float64))
+
+
+def test_router_routes_the_rounded_logits():
+    """router() is the gate GEMM rounded to the fp32 logit type and then the
+    routing step: the plain router's ids are the K largest fp32 logits (ties to
+    the lower id, Python's sorted), and its weights the renormalised softmax."""
+    x = wl.random_rows_bf16(9, 128, seed=7)
+    w = wl.router_weight(16, 128, seed=8)
+    l64, l32, ids, wt = oracle.router(x, w, 4)
+    assert l32.dtype == np.float32 and np.array_equal(l32, l64.astype(np.float32))
+    for t in range(9):
+        order = sorted(range(16), key=lambda e: (-float(l32[t, e]), e))[:4]
+        assert list(ids[t]) == order
+        p = scipy.special.softmax(l32[t].astype(np.float64))
+        np.testing.assert_allclose(wt[t], p[order] / p[order].sum(), rtol=1e-12)
