@@ -85,6 +85,8 @@ typedef enum moe_status {
 /* Bits OR-ed into the optional device status word (int32) by the kernels. */
 #define MOE_STATUS_BAD_ID 1      /* an expert id outside [0, E) was skipped */
 #define MOE_STATUS_BAD_MAP 2     /* offsets / route map out of range: rows skipped */
+#define MOE_STATUS_TIMEOUT 4     /* a bounded wait inside a kernel expired (a copy or MMA that never
+                                    completed; never expected): that call's outputs are invalid */
 
 /* moe_expert_ffn `mode`. */
 #define MOE_MODE_AUTO 0     /* see moe_ffn_resolve_mode */
@@ -182,6 +184,38 @@ typedef struct moe_route_config {
 
 MOE_API int moe_route_ex(const float* logits, int T, int E, int K, const moe_route_config* cfg,
                          const uint8_t* zero_mask, int32_t* topk_ids, float* topk_w, moe_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * moe_router -- fused router: gate GEMM and top-K routing in one kernel.
+ *
+ * The Nemotron-H layer's router is a dense gate GEMM, [N, H] x [H, E]^T ->
+ * [N, E] logits (spark_model/layers/nemotron_moe.rs, `prefill`, step 2),
+ * followed by the top-K kernel; the NKI library fuses the two (NKI Library
+ * kernel reference, Router Top-K).  Per token t:
+ *   logits[t, e] = sum_h x[t, h] * w_router[e, h]   (bf16 inputs, fp32 result)
+ * then exactly what moe_route_ex computes from those fp32 logits (moe_route
+ * when cfg is NULL).  The products are summed by the tensor cores in fp32, so
+ * a logit differs from the exact sum by fp32 rounding; experts whose logits
+ * (or selection scores) lie that close may be ranked either way.
+ *
+ *   x         [T, H] bf16 (read)
+ *   w_router  [E, H] bf16 (read): row e = the gate vector of expert e
+ *   cfg       host pointer or NULL (NULL = softmax, no bias, no groups,
+ *             renormalised, scaling 1); fields and checks as moe_route_ex
+ *   zero_mask, topk_ids, topk_w   as moe_route
+ *   logits    [T, E] f32 (written) or NULL: a copy of the fp32 logits
+ *   status    optional device int32: MOE_STATUS_TIMEOUT is OR-ed in if a
+ *             bounded wait expired (never expected)
+ * Limits: H % 64 == 0, 64 <= H <= MOE_ROUTER_MAX_H, 1 <= E <= MOE_ROUTER_MAX_E,
+ *   1 <= K <= min(E, MOE_MAX_K), 0 <= T <= MOE_MAX_T; x and w_router 16-byte
+ *   aligned (MOE_ERR_UNSUPPORTED_SHAPE / MOE_ERR_INVALID_ARG /
+ *   MOE_ERR_MISALIGNED otherwise).  Allocates nothing; graph capturable.
+ * ------------------------------------------------------------------------- */
+#define MOE_ROUTER_MAX_E 512
+#define MOE_ROUTER_MAX_H 16384
+MOE_API int moe_router(const uint16_t* x, int T, int H, const uint16_t* w_router, int E, int K,
+                       const moe_route_config* cfg, const uint8_t* zero_mask, int32_t* topk_ids, float* topk_w,
+                       float* logits, int32_t* status, moe_stream_t stream);
 
 /* ---------------------------------------------------------------------------
  * moe_sort -- stable sort of the R = T*K routes by expert.

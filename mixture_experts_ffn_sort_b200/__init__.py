@@ -31,7 +31,8 @@ MOE_OUT_BF16, MOE_OUT_F32 = 0, 1
 MOE_STATUS_BAD_ID, MOE_STATUS_BAD_MAP, MOE_STATUS_TIMEOUT = 1, 2, 4
 MOE_MAX_E, MOE_MAX_K = 1024, 32
 
-EXPORTED = ("moe_last_error", "moe_abi_version", "moe_route", "moe_route_ex", "moe_sort_workspace_bytes", "moe_sort",
+EXPORTED = ("moe_last_error", "moe_abi_version", "moe_route", "moe_route_ex", "moe_router", "moe_sort_workspace_bytes",
+            "moe_sort",
             "moe_sort_static_ws", "moe_ffn_resolve_mode", "moe_ffn_workspace_bytes", "moe_expert_ffn", "moe_combine")
 
 
@@ -71,6 +72,8 @@ def lib() -> ctypes.CDLL:
             L.moe_route.argtypes = [P, I, I, I, P, P, P, P]
             L.moe_route_ex.argtypes = [P, I, I, I, ctypes.POINTER(_RouteConfig), P, P, P, P]
             L.moe_route_ex.restype = I
+            L.moe_router.argtypes = [P, I, I, P, I, I, ctypes.POINTER(_RouteConfig), P, P, P, P, P, P]
+            L.moe_router.restype = I
             L.moe_route.restype = I
             L.moe_sort_workspace_bytes.argtypes = [I, I, I]
             L.moe_sort_workspace_bytes.restype = S
@@ -185,6 +188,32 @@ def moe_route_ex(logits: torch.Tensor, K: int, score: int = MOE_SCORE_SOFTMAX,
     return topk_ids, topk_w
 
 
+
+MOE_ROUTER_MAX_E = 512
+MOE_STATUS_TIMEOUT = 4
+
+
+def moe_router(x: torch.Tensor, w_router: torch.Tensor, K: int, score: int = MOE_SCORE_SOFTMAX,
+               sel_bias: Optional[torch.Tensor] = None, n_group: int = 1, topk_group: Optional[int] = None,
+               renormalize: bool = True, scaling: float = 1.0, zero_mask: Optional[torch.Tensor] = None,
+               logits: Optional[torch.Tensor] = None, status: Optional[torch.Tensor] = None,
+               topk_ids: Optional[torch.Tensor] = None, topk_w: Optional[torch.Tensor] = None, stream=None):
+    """Fused router: x [T, H] bf16 and w_router [E, H] bf16 -> (topk_ids [T, K] i32, topk_w [T, K] f32),
+    the gate GEMM and the routing of moe_route_ex in one kernel.  logits [T, E] f32, if given,
+    receives the fp32 logits."""
+    _need_cuda(x, w_router, zero_mask, sel_bias, logits, status)
+    T, H = x.shape
+    E = w_router.shape[0]
+    if topk_ids is None:
+        topk_ids = torch.empty((T, K), dtype=torch.int32, device=x.device)
+    if topk_w is None:
+        topk_w = torch.empty((T, K), dtype=torch.float32, device=x.device)
+    cfg = _RouteConfig(int(score), _ptr(sel_bias), int(n_group),
+                       int(n_group if topk_group is None else topk_group), int(bool(renormalize)), float(scaling))
+    _check(lib().moe_router(_ptr(x), T, H, _ptr(w_router), E, K, ctypes.byref(cfg), _ptr(zero_mask),
+                            _ptr(topk_ids), _ptr(topk_w), _ptr(logits), _ptr(status), _stream(stream)))
+    return topk_ids, topk_w
+
 def moe_sort_workspace_bytes(T: int, K: int, E: int) -> int:
     return int(lib().moe_sort_workspace_bytes(T, K, E))
 
@@ -267,12 +296,14 @@ class MoEFFN:
     so a call can be captured in a CUDA graph after the first one).
     route_cfg: keyword arguments of moe_route_ex (score, sel_bias, n_group,
     topk_group, renormalize, scaling) for a routing variant; None routes with
-    moe_route."""
+    moe_route.  w_router: bf16 [E, H] gate vectors for forward_fused, which
+    routes with the fused router (moe_router) from x alone."""
 
     def __init__(self, routed: Experts, T: int, K: int, shared: Optional[Experts] = None,
                  mode: int = MOE_MODE_AUTO, out_dtype: int = MOE_OUT_BF16, device="cuda",
-                 route_cfg: Optional[dict] = None):
+                 route_cfg: Optional[dict] = None, w_router: Optional[torch.Tensor] = None):
         self.routed, self.shared, self.T, self.K = routed, shared, T, K
+        self.w_router = w_router
         self.route_cfg = dict(route_cfg) if route_cfg else None
         self.E, self.I, self.H = routed.n, routed.inter, routed.w_gate.shape[2]
         self.mode, self.out_dtype = mode, out_dtype
@@ -310,6 +341,17 @@ class MoEFFN:
         else:
             moe_route_ex(logits, self.K, zero_mask=zero_mask, topk_ids=self.topk_ids, topk_w=self.topk_w,
                          stream=stream, **self.route_cfg)
+        return self._experts(x, stream)
+
+    def forward_fused(self, x: torch.Tensor, zero_mask: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        """The same layer with the router's gate GEMM fused into the routing step."""
+        if self.w_router is None:
+            raise ValueError("forward_fused needs w_router")
+        moe_router(x, self.w_router, self.K, zero_mask=zero_mask, topk_ids=self.topk_ids, topk_w=self.topk_w,
+                   stream=stream, **(self.route_cfg or {}))
+        return self._experts(x, stream)
+
+    def _experts(self, x: torch.Tensor, stream) -> torch.Tensor:
         moe_sort(self.topk_ids, self.E, self.status, self.offsets, self.sorted_route, self.inv_route,
                  self.sort_ws, stream=stream)
         moe_expert_ffn(x, self.K, self.routed, self.offsets, self.sorted_route, self.topk_w, self.shared,

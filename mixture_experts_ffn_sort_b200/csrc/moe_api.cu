@@ -109,36 +109,83 @@ int moe_route(const float* logits, int T, int E, int K, const uint8_t* zero_mask
     return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_route launch");
 }
 
+namespace {
+
+// Range checks of a moe_route_config (messages prefixed with the caller's name).
+int check_route_cfg(const char* fn, const moe_route_config* cfg, int E, int K) {
+    if (cfg->score != MOE_SCORE_SOFTMAX && cfg->score != MOE_SCORE_SIGMOID)
+        return fail(MOE_ERR_INVALID_ARG, "%s: unknown score function %d", fn, cfg->score);
+    if (cfg->n_group < 1 || cfg->n_group > MOE_MAX_GROUPS || E % cfg->n_group)
+        return fail(MOE_ERR_INVALID_ARG, "%s: n_group=%d must be in 1..%d and divide E=%d", fn, cfg->n_group,
+                    MOE_MAX_GROUPS, E);
+    if (cfg->topk_group < 1 || cfg->topk_group > cfg->n_group ||
+        static_cast<long>(cfg->topk_group) * (E / cfg->n_group) < K)
+        return fail(MOE_ERR_INVALID_ARG, "%s: topk_group=%d must be in 1..n_group and keep >= K=%d experts", fn,
+                    cfg->topk_group, K);
+    if (cfg->renormalize != 0 && cfg->renormalize != 1)
+        return fail(MOE_ERR_INVALID_ARG, "%s: renormalize must be 0 or 1", fn);
+    if (!(cfg->scaling > 0.f) || !isfinite(cfg->scaling))
+        return fail(MOE_ERR_INVALID_ARG, "%s: scaling must be finite and > 0", fn);
+    if (reinterpret_cast<uintptr_t>(cfg->sel_bias) % 4)
+        return fail(MOE_ERR_MISALIGNED, "%s: sel_bias must be 4-byte aligned", fn);
+    return MOE_OK;
+}
+
+}  // namespace
+
 int moe_route_ex(const float* logits, int T, int E, int K, const moe_route_config* cfg, const uint8_t* zero_mask,
                  int32_t* topk_ids, float* topk_w, moe_stream_t stream) {
     g_err.clear();
     int rc = check_topk(T, E, K);
     if (rc) return rc;
     if (!cfg) return fail(MOE_ERR_INVALID_ARG, "moe_route_ex: cfg must not be NULL");
-    if (cfg->score != MOE_SCORE_SOFTMAX && cfg->score != MOE_SCORE_SIGMOID)
-        return fail(MOE_ERR_INVALID_ARG, "moe_route_ex: unknown score function %d", cfg->score);
-    if (cfg->n_group < 1 || cfg->n_group > MOE_MAX_GROUPS || E % cfg->n_group)
-        return fail(MOE_ERR_INVALID_ARG, "moe_route_ex: n_group=%d must be in 1..%d and divide E=%d", cfg->n_group,
-                    MOE_MAX_GROUPS, E);
-    if (cfg->topk_group < 1 || cfg->topk_group > cfg->n_group ||
-        static_cast<long>(cfg->topk_group) * (E / cfg->n_group) < K)
-        return fail(MOE_ERR_INVALID_ARG, "moe_route_ex: topk_group=%d must be in 1..n_group and keep >= K=%d experts",
-                    cfg->topk_group, K);
-    if (cfg->renormalize != 0 && cfg->renormalize != 1)
-        return fail(MOE_ERR_INVALID_ARG, "moe_route_ex: renormalize must be 0 or 1");
-    if (!(cfg->scaling > 0.f) || !isfinite(cfg->scaling))
-        return fail(MOE_ERR_INVALID_ARG, "moe_route_ex: scaling must be finite and > 0");
+    rc = check_route_cfg("moe_route_ex", cfg, E, K);
+    if (rc && rc != MOE_ERR_MISALIGNED) return rc;
     if (T == 0) return MOE_OK;
     if (!logits || !topk_ids || !topk_w)
         return fail(MOE_ERR_INVALID_ARG, "moe_route_ex: logits, topk_ids and topk_w must not be NULL");
     if (!aligned16(logits) || !aligned16(topk_ids) || !aligned16(topk_w))
         return fail(MOE_ERR_MISALIGNED, "moe_route_ex: tensor bases must be 16-byte aligned");
-    if (reinterpret_cast<uintptr_t>(cfg->sel_bias) % 4)
-        return fail(MOE_ERR_MISALIGNED, "moe_route_ex: sel_bias must be 4-byte aligned");
+    if (rc) return rc;
     const moe::RouteCfg rc_dev{cfg->score, cfg->sel_bias, cfg->n_group, cfg->topk_group, cfg->renormalize,
                                cfg->scaling};
     cudaError_t e = moe::launch_route_ex(logits, T, E, K, rc_dev, zero_mask, topk_ids, topk_w, stream);
     return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_route_ex launch");
+}
+
+int moe_router(const uint16_t* x, int T, int H, const uint16_t* w_router, int E, int K, const moe_route_config* cfg,
+               const uint8_t* zero_mask, int32_t* topk_ids, float* topk_w, float* logits, int32_t* status,
+               moe_stream_t stream) {
+    g_err.clear();
+    int rc = check_topk(T, E, K);
+    if (rc) return rc;
+    if (E > MOE_ROUTER_MAX_E)
+        return fail(MOE_ERR_UNSUPPORTED_SHAPE, "moe_router: num_experts=%d must be in 1..=%d", E, MOE_ROUTER_MAX_E);
+    if (H < 64 || H > MOE_ROUTER_MAX_H || H % 64)
+        return fail(MOE_ERR_UNSUPPORTED_SHAPE, "moe_router: H=%d must be a multiple of 64 in 64..=%d", H,
+                    MOE_ROUTER_MAX_H);
+    if (cfg) {
+        rc = check_route_cfg("moe_router", cfg, E, K);
+        if (rc) return rc;
+    }
+    if (T == 0) return MOE_OK;
+    if (!x || !w_router || !topk_ids || !topk_w)
+        return fail(MOE_ERR_INVALID_ARG, "moe_router: x, w_router, topk_ids and topk_w must not be NULL");
+    if (!aligned16(x) || !aligned16(w_router) || !aligned16(topk_ids) || !aligned16(topk_w) || !aligned16(logits) ||
+        (status && (reinterpret_cast<uintptr_t>(status) & 3)))
+        return fail(MOE_ERR_MISALIGNED, "moe_router: tensor bases must be 16-byte aligned");
+    const moe::RouteCfg rc_dev = cfg ? moe::RouteCfg{cfg->score, cfg->sel_bias, cfg->n_group, cfg->topk_group,
+                                                     cfg->renormalize, cfg->scaling}
+                                     : moe::RouteCfg{MOE_SCORE_SOFTMAX, nullptr, 1, 1, 1, 1.f};
+    const moe::RouterPlan plan = moe::plan_router(T, E);
+    CUtensorMap tx, tw;
+    cudaError_t e = moe::make_tmap_bf16_2d(&tx, x, static_cast<uint64_t>(T), static_cast<uint64_t>(H), 64, 128);
+    if (e == cudaSuccess)
+        e = moe::make_tmap_bf16_2d(&tw, w_router, static_cast<uint64_t>(E), static_cast<uint64_t>(H), 64,
+                                   static_cast<uint32_t>(plan.ne));
+    if (e != cudaSuccess) return cuda_fail(e, "moe_router tensor maps");
+    e = moe::launch_router(tx, tw, T, H, E, K, rc_dev, zero_mask, topk_ids, topk_w, logits, status, stream);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_router launch");
 }
 
 size_t moe_sort_workspace_bytes(int T, int K, int E) {

@@ -9,187 +9,21 @@
 // bias, groups scored by the sum of their two best experts, a kept-group
 // limit, optional renormalisation and a scaling factor.
 //
-// One warp per token.  Lane `lane` holds experts lane + 32 i as
-// order-preserving integer keys (larger key = larger value, -0 == +0; 0 marks
-// an expert that cannot be chosen).  The key is the fp32 logit itself when
-// there is neither a bias nor a group limit -- both scores are strictly
-// increasing in the logit, so ranking logits is exact -- and the fp32
-// selection score s + bias otherwise.  With groups, each group's score (the
-// sum of its two largest keys' values) comes from lane-local top-two lists
-// (groups of a multiple of 32 experts) or from two warp arg-max passes, and
-// topk_group arg-max passes over the lanes keep the best groups.  K rounds of
-// a warp arg-max (two redux.sync: largest key, then lowest expert id holding
-// it) pick the experts in descending order.  The chosen expert's score is
-// recomputed from its logit: softmax weights are exp(l_j - l_max) over their
-// sum (renormalised; the full-softmax normaliser cancels) or over the full
-// normaliser, sigmoid weights 1 / (1 + exp(-l_j)).
-#include <math.h>
-
-#include "device_common.cuh"
-#include "launch.h"
+// One warp per token (route_token, route_device.cuh).
+#include "route_device.cuh"
 
 namespace moe {
 
 namespace {
 
-// Order-preserving integer key of a float (larger float -> larger key; -0 and
-// +0 share a key; every key is nonzero) and its inverse.
-__device__ __forceinline__ uint32_t order_key(float v) {
-    const uint32_t u = __float_as_uint(v == 0.f ? 0.f : v);
-    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-__device__ __forceinline__ float key_value(uint32_t k) {
-    return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
-}
-
-__device__ __forceinline__ float sigmoid(float x) { return __frcp_rn(1.f + expf(-x)); }
-
-// COMPUTED: rank by s (+ bias) -- a bias or a group limit is present.
 template <int EPL, bool COMPUTED>
 __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ logits, int T, int E, int K,
                                                     const RouteCfg cfg, const uint8_t* __restrict__ zero_mask,
                                                     int32_t* __restrict__ ids, float* __restrict__ w) {
-    const int lane = threadIdx.x & 31;
     const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     if (t >= T) return;
-    const float* lg = logits + static_cast<size_t>(t) * E;
-    const uint32_t full = 0xffffffffu;
-    const bool softmax = cfg.score == MOE_SCORE_SOFTMAX;
-
-    float l[EPL];
-    float lmax = -INFINITY;
-#pragma unroll
-    for (int i = 0; i < EPL; ++i) {
-        const int e = lane + 32 * i;
-        l[i] = e < E ? __ldg(lg + e) : -INFINITY;
-        lmax = fmaxf(lmax, l[i]);
-    }
-    float z = 1.f;  // softmax normaliser (sum of exp(l - l_max))
-    if (softmax) {
-        lmax = key_value(__reduce_max_sync(full, order_key(lmax)));
-        if (COMPUTED || !cfg.renormalize) {
-            z = 0.f;
-#pragma unroll
-            for (int i = 0; i < EPL; ++i) z += lane + 32 * i < E ? expf(l[i] - lmax) : 0.f;
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(full, z, off);
-        }
-    }
-    uint32_t key[EPL];
-#pragma unroll
-    for (int i = 0; i < EPL; ++i) {
-        const int e = lane + 32 * i;
-        float c = l[i];
-        if (COMPUTED && e < E) {
-            c = softmax ? expf(l[i] - lmax) / z : sigmoid(l[i]);
-            if (cfg.bias) c += __ldg(cfg.bias + e);
-        }
-        key[i] = e < E ? order_key(c) : 0u;
-    }
-
-    if (COMPUTED && cfg.n_group > 1) {
-        const int G = E / cfg.n_group;
-        float gs = 0.f;  // lane g: score of group g
-        if (G % 32 == 0) {
-            // Group of register i: i / (G / 32).  Lane-local top two of each
-            // group, then the group's best (largest lane top) and second best
-            // (the winner lane's second or another lane's top).
-            const int rpg = G / 32;
-            for (int g = 0; g < cfg.n_group; ++g) {
-                uint32_t a = 0, b = 0;
-#pragma unroll
-                for (int i = 0; i < EPL; ++i) {
-                    if (i / rpg != g) continue;
-                    const uint32_t k = key[i];
-                    if (k > a) {
-                        b = a;
-                        a = k;
-                    } else if (k > b) {
-                        b = k;
-                    }
-                }
-                const uint32_t k1 = __reduce_max_sync(full, a);
-                const uint32_t win = __reduce_min_sync(full, a == k1 ? static_cast<uint32_t>(lane) : 32u);
-                const uint32_t k2 = __reduce_max_sync(full, lane == static_cast<int>(win) ? b : a);
-                if (lane == g) gs = key_value(k1) + key_value(k2);
-            }
-        } else {
-            // Any group size: two warp arg-max passes per group.
-            for (int g = 0; g < cfg.n_group; ++g) {
-                float top = 0.f;
-                int skip = -1;  // the group's best expert, excluded from the second pass
-                for (int pass = 0; pass < (G > 1 ? 2 : 1); ++pass) {
-                    uint32_t best = 0;
-                    int bi = 0x7fffffff;
-#pragma unroll
-                    for (int i = 0; i < EPL; ++i) {
-                        const int e = lane + 32 * i;
-                        if (e / G == g && e != skip && key[i] > best) {
-                            best = key[i];
-                            bi = e;
-                        }
-                    }
-                    const uint32_t kmax = __reduce_max_sync(full, best);
-                    skip = static_cast<int>(
-                        __reduce_min_sync(full, best == kmax ? static_cast<uint32_t>(bi) : 0xffffffffu));
-                    top += key_value(kmax);
-                }
-                if (lane == g) gs = top;
-            }
-        }
-        uint32_t keep = 0;
-        for (int r = 0; r < cfg.topk_group; ++r) {
-            const bool cand = lane < cfg.n_group && !((keep >> lane) & 1u);
-            const uint32_t k = cand ? order_key(gs) : 0u;
-            const uint32_t kmax = __reduce_max_sync(full, k);
-            keep |= 1u << __reduce_min_sync(full, cand && k == kmax ? static_cast<uint32_t>(lane) : 31u);
-        }
-#pragma unroll
-        for (int i = 0; i < EPL; ++i) {
-            const int g = (lane + 32 * i) / G;  // >= 32 only for padding, whose key is already 0
-            if (g >= 32 || !((keep >> g) & 1u)) key[i] = 0u;
-        }
-    }
-
-    float sum = 0.f, mine = 0.f;
-    int my_id = 0;
-    for (int j = 0; j < K; ++j) {
-        uint32_t best = 0;
-        int bi = 0;
-#pragma unroll
-        for (int i = 0; i < EPL; ++i) {
-            if (key[i] > best) {  // ascending i: equal keys keep the lower expert id
-                best = key[i];
-                bi = i;
-            }
-        }
-        const uint32_t kmax = __reduce_max_sync(full, best);
-        int e = static_cast<int>(
-            __reduce_min_sync(full, best == kmax && best ? static_cast<uint32_t>(lane + 32 * bi) : 0xffffffffu));
-        if (e >= E) e = E - 1;  // only reachable with NaN logits (unspecified ids)
-        const int slot = e >> 5;
-        // The chosen logit: the key itself when ranking by logit, else reloaded.
-        const float le = COMPUTED ? __ldg(lg + e) : key_value(kmax);
-        if (lane == (e & 31)) {
-#pragma unroll
-            for (int i = 0; i < EPL; ++i)
-                if (i == slot) key[i] = 0u;
-        }
-        const float s = softmax ? expf(le - lmax) : sigmoid(le);
-        sum += s;
-        if (lane == j) {
-            my_id = e;
-            mine = s;
-        }
-    }
-    if (lane < K) {
-        const size_t o = static_cast<size_t>(t) * K + lane;
-        float wv = cfg.renormalize ? mine / sum : mine / z;  // z = 1 for sigmoid scores
-        wv *= cfg.scaling;
-        if (zero_mask && zero_mask[o]) wv = 0.f;
-        ids[o] = my_id;
-        w[o] = wv;
-    }
+    route_token<EPL, COMPUTED, LoadGlobal>(logits + static_cast<size_t>(t) * E, t, E, K, cfg, zero_mask, ids, w,
+                                          nullptr);
 }
 
 }  // namespace

@@ -190,3 +190,29 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(moe, "_L", None)
     with pytest.raises(RuntimeError, match="missing"):
         moe.lib()
+
+
+def test_router_checks(L):
+    base = dict(x=P(16), T=4, H=128, w=P(16), E=16, K=4, cfg=None, zm=None, ids=P(16), wt=P(16), lg=None,
+                status=None)
+
+    def call(**kw):
+        a = dict(base, **kw)
+        return L.moe_router(a["x"], a["T"], a["H"], a["w"], a["E"], a["K"], a["cfg"], a["zm"], a["ids"], a["wt"],
+                            a["lg"], a["status"], None)
+
+    assert call(E=moe.MOE_ROUTER_MAX_E + 1) == moe.MOE_ERR_UNSUPPORTED_SHAPE
+    assert "moe_router" in _err(L)
+    for H in (0, 96, 16384 + 64):
+        assert call(H=H) == moe.MOE_ERR_UNSUPPORTED_SHAPE, H
+    assert call(K=17) == moe.MOE_ERR_INVALID_ARG
+    assert call(cfg=_rcfg(n_group=3)) == moe.MOE_ERR_INVALID_ARG
+    assert call(cfg=_rcfg(scaling=0.0)) == moe.MOE_ERR_INVALID_ARG
+    assert call(x=None) == moe.MOE_ERR_INVALID_ARG
+    assert call(ids=None) == moe.MOE_ERR_INVALID_ARG
+    assert call(x=P(24)) == moe.MOE_ERR_MISALIGNED
+    assert call(w=P(0x1008)) == moe.MOE_ERR_MISALIGNED
+    assert call(lg=P(0x1004)) == moe.MOE_ERR_MISALIGNED
+    assert call(status=P(0x1002)) == moe.MOE_ERR_MISALIGNED
+    assert call(T=0, x=None, w=None, ids=None, wt=None) == moe.MOE_OK
+    assert call(T=-1) == moe.MOE_ERR_INVALID_ARG
