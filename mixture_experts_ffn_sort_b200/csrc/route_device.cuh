@@ -12,7 +12,8 @@
 // (groups of a multiple of 32 experts) or from two warp arg-max passes, and
 // topk_group arg-max passes over the lanes keep the best groups.  K rounds of
 // a warp arg-max (two redux.sync: largest key, then lowest expert id holding
-// it) pick the experts in descending order.  The chosen experts' scores are
+// it) pick the experts in descending order, over the few candidate keys a
+// threshold leaves when it can (see the selection below).  The chosen experts' scores are
 // then recomputed from their logits, lane j taking choice j: softmax weights
 // are exp(l_j - l_max) over their sum (renormalised; the full-softmax
 // normaliser cancels) or over the full normaliser, sigmoid weights
@@ -163,30 +164,89 @@ __device__ __forceinline__ void route_token(const float* lg, int t, int E, int K
     // after the K rounds, one per lane, and summed across the warp.
     float my_l = 0.f;
     int my_id = 0;
-    for (int j = 0; j < K; ++j) {
-        uint32_t best = 0;
-        int bi = 0;
+    // theta = the K-th largest of the lanes' largest keys.  At least K keys
+    // are >= theta, so every chosen key is: the candidates (nonzero keys >=
+    // theta) are few.  Each lane keeps its four best candidates in order
+    // (key descending, then expert id ascending); when no lane has more than
+    // four, the K rounds take the best lane head and advance that lane,
+    // otherwise they scan every key.
+    uint32_t theta = 0;
+    {
+        uint32_t m = 0;
 #pragma unroll
-        for (int i = 0; i < EPL; ++i) {
-            if (key[i] > best) {  // ascending i: equal keys keep the lower expert id
-                best = key[i];
-                bi = i;
+        for (int i = 0; i < EPL; ++i) m = key[i] > m ? key[i] : m;
+        for (int j = 0; j < K; ++j) {
+            theta = __reduce_max_sync(full, m);
+            const uint32_t win = __reduce_min_sync(full, m == theta ? static_cast<uint32_t>(lane) : 32u);
+            if (lane == static_cast<int>(win)) m = 0;
+        }
+    }
+    uint32_t h0 = 0, h1 = 0, h2 = 0, h3 = 0;
+    int i0 = 0, i1 = 0, i2 = 0, i3 = 0, cnt = 0;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+        const uint32_t k = key[i];
+        if (k != 0u && k >= theta) {
+            ++cnt;
+            if (k > h3) {  // a key equal to one held goes after it (larger expert id)
+                if (k > h2) {
+                    h3 = h2; i3 = i2;
+                    if (k > h1) {
+                        h2 = h1; i2 = i1;
+                        if (k > h0) {
+                            h1 = h0; i1 = i0; h0 = k; i0 = i;
+                        } else {
+                            h1 = k; i1 = i;
+                        }
+                    } else {
+                        h2 = k; i2 = i;
+                    }
+                } else {
+                    h3 = k; i3 = i;
+                }
             }
         }
-        const uint32_t kmax = __reduce_max_sync(full, best);
-        int e = static_cast<int>(
-            __reduce_min_sync(full, best == kmax && best ? static_cast<uint32_t>(lane + 32 * bi) : 0xffffffffu));
-        if (e >= E) e = E - 1;  // only reachable with NaN logits (unspecified ids)
-        const int slot = e >> 5;
-        if (lane == (e & 31)) {
-#pragma unroll
-            for (int i = 0; i < EPL; ++i)
-                if (i == slot) key[i] = 0u;
+    }
+    if (__all_sync(full, cnt <= 4)) {
+        for (int j = 0; j < K; ++j) {
+            const uint32_t kmax = __reduce_max_sync(full, h0);
+            int e = static_cast<int>(
+                __reduce_min_sync(full, h0 == kmax && kmax ? static_cast<uint32_t>(lane + 32 * i0) : 0xffffffffu));
+            if (e >= E) e = E - 1;  // only reachable with NaN logits (unspecified ids)
+            if (lane == (e & 31)) {
+                h0 = h1; i0 = i1; h1 = h2; i1 = i2; h2 = h3; i2 = i3; h3 = 0u;
+            }
+            if (lane == j) {
+                my_id = e;
+                // The chosen logit: the key itself when ranking by logit, else reloaded.
+                my_l = COMPUTED ? ld(lg + e) : key_value(kmax);
+            }
         }
-        if (lane == j) {
-            my_id = e;
-            // The chosen logit: the key itself when ranking by logit, else reloaded.
-            my_l = COMPUTED ? ld(lg + e) : key_value(kmax);
+    } else {
+        for (int j = 0; j < K; ++j) {
+            uint32_t best = 0;
+            int bi = 0;
+#pragma unroll
+            for (int i = 0; i < EPL; ++i) {
+                if (key[i] > best) {  // ascending i: equal keys keep the lower expert id
+                    best = key[i];
+                    bi = i;
+                }
+            }
+            const uint32_t kmax = __reduce_max_sync(full, best);
+            int e = static_cast<int>(
+                __reduce_min_sync(full, best == kmax && best ? static_cast<uint32_t>(lane + 32 * bi) : 0xffffffffu));
+            if (e >= E) e = E - 1;
+            const int slot = e >> 5;
+            if (lane == (e & 31)) {
+#pragma unroll
+                for (int i = 0; i < EPL; ++i)
+                    if (i == slot) key[i] = 0u;
+            }
+            if (lane == j) {
+                my_id = e;
+                my_l = COMPUTED ? ld(lg + e) : key_value(kmax);
+            }
         }
     }
     const float mine = lane < K ? (softmax ? expf(my_l - lmax) : sigmoid(my_l)) : 0.f;
