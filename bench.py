@@ -150,14 +150,19 @@ def oracle_route_kwargs(router, shape):
     return kw
 
 
-def oracle_rows(w, shape, tk, router):
-    """Brute-force oracle rows of the sampled tokens tk, routed by `router`."""
+def oracle_rows(w, shape, tk, router, fused_router=False):
+    """Brute-force oracle rows of the sampled tokens tk, routed by `router`
+    (fused_router: the logits are the router's gate GEMM of x, computed here)."""
     import oracle
     kw = oracle_route_kwargs(router, shape)
-    if kw is None:
+    if kw is None and not fused_router:
         return oracle.moe_tokens(w.x, w.logits, shape.K, w.routed, w.shared, w.zero_mask, tokens=tk)
     zm = None if w.zero_mask is None else w.zero_mask[tk]
-    ids, wt = oracle.route_ex(w.logits[tk], shape.K, zero_mask=zm, **kw)
+    if fused_router:
+        lg = oracle.router_logits(w.x[tk], wl.router_weight(shape.E, shape.H, shape.seed)).astype(np.float32)
+    else:
+        lg = w.logits[tk]
+    ids, wt = oracle.route_ex(lg, shape.K, zero_mask=zm, **(kw or {}))
     return oracle.moe_tokens_routed(w.x, ids, wt, w.routed, w.shared, tokens=tk)
 
 
@@ -169,7 +174,7 @@ def run_reference(args, shape):
 
     def one():
         t0 = time.perf_counter()
-        oracle_rows(w, shape, tk, args.router)
+        oracle_rows(w, shape, tk, args.router, args.fused_router)
         return time.perf_counter() - t0
 
     for _ in range(args.warmup):
@@ -181,19 +186,19 @@ def run_reference(args, shape):
     return {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": 1e3 * tot / len(ts), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "impl": "reference", "config": config_of(shape, args.router),
+            "impl": "reference", "config": config_of(shape, args.router, args.fused_router),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
-def cpu_baseline(shape, router="softmax", budget_s=10.0):
+def cpu_baseline(shape, router="softmax", fused_router=False, budget_s=10.0):
     """The oracle as it stands, on the host cores, on a bounded sample."""
     import oracle
     w = wl.make_workload(shape.name)
     tk = np.arange(min(shape.T, 64), dtype=np.int32)
     n, t0 = 0, time.perf_counter()
     while time.perf_counter() - t0 < budget_s or n == 0:
-        oracle_rows(w, shape, tk, router)
+        oracle_rows(w, shape, tk, router, fused_router)
         n += 1
     dt = time.perf_counter() - t0
     return {"value": n * len(tk) / dt, "unit": UNIT, "cores": oracle.threads(), "kind": "oracle",
@@ -225,7 +230,7 @@ def job_tokens_per_s(T, world, ms_per_step):
     return T * world / (ms_per_step * 1e-3)
 
 
-def config_of(shape, router="softmax"):
+def config_of(shape, router="softmax", fused_router=False):
     c = {"workload": shape.name, "T": shape.T, "H": shape.H, "I": shape.I, "E": shape.E, "K": shape.K,
          "I_shared": shape.I_shared, "weights": "fp8 e4m3fn, fp32 scale per 128x128 block",
          "activations": "bf16", "logit_bias": shape.bias, "zero_route_frac": shape.zero_frac,
@@ -233,6 +238,10 @@ def config_of(shape, router="softmax"):
     if wl.ROUTERS[router] is not None:
         c["router_cfg"] = {k: v for k, v in wl.ROUTERS[router].items() if k != "bias"}
         c["router_cfg"]["selection_bias"] = "N(0, 0.02) per expert" if wl.ROUTERS[router].get("bias") else None
+    c["logits"] = ("x . W_r^T on the device (moe_router: gate GEMM fused with the routing; W_r bf16 "
+                   "[E, H] ~ N(0, 1/H))" if fused_router else "given, f32 [T, E]")
+    if fused_router:
+        c["logit_bias"] = None  # the router computes the logits; no drawn bias is added
     return c
 
 
@@ -249,6 +258,8 @@ def main():
     ap.add_argument("--router", default="softmax", choices=sorted(wl.ROUTERS),
                     help="routing variant: softmax top-k (moe_route) or a moe_route_ex preset")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--fused-router", action="store_true",
+                    help="route from x with the fused router (gate GEMM + top-K) instead of given logits")
     ap.add_argument("--eager", action="store_true",
                     help="launch every call directly instead of replaying CUDA graphs (for profilers)")
     args = ap.parse_args()
@@ -288,11 +299,19 @@ def main():
         route_cfg = {k: v for k, v in kw.items() if k != "bias"}
         route_cfg["sel_bias"] = (torch.from_numpy(wl.selection_bias(E, shape.seed)).to(dev)
                                  if kw.get("bias") else None)
-    layer = moe.MoEFFN(routed, T, K, shared, mode=args.mode, device=dev, route_cfg=route_cfg)
+    wr = (torch.from_numpy(wl.router_weight(E, H, shape.seed).view(np.int16)).view(torch.bfloat16).to(dev)
+          if args.fused_router else None)
+    layer = moe.MoEFFN(routed, T, K, shared, mode=args.mode, device=dev, route_cfg=route_cfg, w_router=wr)
     stream = torch.cuda.Stream(device=dev)
 
+    def run(lay, xx, ll):
+        if args.fused_router:
+            lay.forward_fused(xx, zmask)
+        else:
+            lay(xx, ll, zmask)
+
     def step():
-        layer(x, logits, zmask)
+        run(layer, x, logits)
 
     with torch.cuda.stream(stream):
         for _ in range(max(1, args.warmup)):
@@ -310,7 +329,10 @@ def main():
 
     def instrumented():
         ev[0].record()
-        if route_cfg is None:
+        if args.fused_router:
+            moe.moe_router(x, wr, K, zero_mask=zmask, topk_ids=layer.topk_ids, topk_w=layer.topk_w,
+                           **(route_cfg or {}))
+        elif route_cfg is None:
             moe.moe_route(logits, K, zmask, layer.topk_ids, layer.topk_w)
         else:
             moe.moe_route_ex(logits, K, zero_mask=zmask, topk_ids=layer.topk_ids, topk_w=layer.topk_w,
@@ -378,7 +400,8 @@ def main():
     xh = torch.from_numpy(w.x.view(np.int16)).view(torch.bfloat16).pin_memory()
     lh = torch.from_numpy(w.logits).pin_memory()
     oh = [torch.empty((T, H), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
-    layers = [layer, moe.MoEFFN(routed, T, K, shared, mode=args.mode, device=dev, route_cfg=route_cfg)]
+    layers = [layer, moe.MoEFFN(routed, T, K, shared, mode=args.mode, device=dev, route_cfg=route_cfg,
+                                w_router=wr)]
     xs, ls = [x, torch.empty_like(x)], [logits, torch.empty_like(logits)]
     h2d, d2h = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
     in_ready, in_free, out_ready, out_free = ([torch.cuda.Event(), torch.cuda.Event()] for _ in range(4))
@@ -387,7 +410,7 @@ def main():
     with torch.cuda.stream(stream):
         xs[1].copy_(xh)
         ls[1].copy_(lh)
-        layers[1](xs[1], ls[1], zmask)  # first call of the second layer outside the timed region
+        run(layers[1], xs[1], ls[1])  # first call of the second layer outside the timed region
     barrier()
     torch.cuda.synchronize(dev)
     e0.record(stream)
@@ -398,13 +421,14 @@ def main():
             if i >= 2:
                 h2d.wait_event(in_free[b])
             xs[b].copy_(xh, non_blocking=True)
-            ls[b].copy_(lh, non_blocking=True)
+            if not args.fused_router:  # the fused router computes the logits from x
+                ls[b].copy_(lh, non_blocking=True)
             in_ready[b].record(h2d)
         with torch.cuda.stream(stream):
             stream.wait_event(in_ready[b])
             if i >= 2:
                 stream.wait_event(out_free[b])
-            layers[b](xs[b], ls[b], zmask)
+            run(layers[b], xs[b], ls[b])
             in_free[b].record(stream)
             out_ready[b].record(stream)
         with torch.cuda.stream(d2h):
@@ -442,11 +466,20 @@ def main():
         roof = {"bound": "tensor", "achieved": ach, "peak": pk, "unit": "TFLOP/s", "frac": ach / pk,
                 "traffic": profile_traffic(shape.name, "prefill"), "kernel": "moe_expert_ffn", "flops": flops,
                 "peak_source": peaks["src"] + " sustained"}
+    if args.fused_router:
+        # The fused router's own roofline: a bf16 GEMM of 2 T H E flops (its
+        # top-K epilogue adds no HBM traffic beyond the ids and weights).
+        r_ms = statistics.median(parts["route"])
+        r_flops = 2.0 * T * H * E
+        r_ach = r_flops / (r_ms * 1e-3) / 1e12
+        roof["router"] = {"kernel": "moe_router (gate GEMM + top-K)", "bound": "tensor", "flops": r_flops,
+                          "achieved": r_ach, "peak": peaks["bf16_sus"], "unit": "TFLOP/s",
+                          "frac": r_ach / peaks["bf16_sus"]}
     n_launch = layer.launches()
     out = {"metric": METRIC, "value": job_tokens_per_s(T, world, t_max), "unit": UNIT, "n_gpus": world,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_max, "higher_is_better": True,
            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-           "config": dict(config_of(shape, args.router), parallelism="replicas x%d" % world,
+           "config": dict(config_of(shape, args.router, args.fused_router), parallelism="replicas x%d" % world,
                           l2="inputs larger than L2 (touched expert weights %.2f GB > 126 MB)"
                              % (touched * expert_bytes(H, I) / 1e9) if decode_path else
                              "inputs larger than L2 (expert weights %.2f GB > 126 MB)" % (E * expert_bytes(H, I) / 1e9),
@@ -455,12 +488,12 @@ def main():
            "roofline": roof,
            "breakdown_ms": {k: statistics.median(v) for k, v in parts.items()},
            "e2e": {"value": job_tokens_per_s(T, world, e2e_ms), "unit": UNIT,
-                   "h2d_bytes_per_step": x.numel() * 2 + logits.numel() * 4,
+                   "h2d_bytes_per_step": x.numel() * 2 + (0 if args.fused_router else logits.numel() * 4),
                    "d2h_bytes_per_step": layer.out.numel() * 2},
            "gpu_launches": n_launch * args.steps,
            "clocks": clk.summary()}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(shape, args.router)
+        out["cpu_baseline"] = cpu_baseline(shape, args.router, args.fused_router)
     if rank == 0:
         print(json.dumps(out), flush=True)
     del g, g2
