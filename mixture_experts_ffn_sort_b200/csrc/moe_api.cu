@@ -12,6 +12,7 @@
 
 #include "../../include/moe_ffn.h"
 #include "launch.h"
+#include "router.h"
 
 namespace moe {
 bool ffn_decode_supported(int H, int I);
@@ -179,7 +180,8 @@ int moe_router(const uint16_t* x, int T, int H, const uint16_t* w_router, int E,
                                      : moe::RouteCfg{MOE_SCORE_SOFTMAX, nullptr, 1, 1, 1, 1.f};
     const moe::RouterPlan plan = moe::plan_router(T, E);
     CUtensorMap tx, tw;
-    cudaError_t e = moe::make_tmap_bf16_2d(&tx, x, static_cast<uint64_t>(T), static_cast<uint64_t>(H), 64, 128);
+    cudaError_t e = moe::make_tmap_bf16_2d(&tx, x, static_cast<uint64_t>(T), static_cast<uint64_t>(H), 64,
+                                           static_cast<uint32_t>(plan.xrows));
     if (e == cudaSuccess)
         e = moe::make_tmap_bf16_2d(&tw, w_router, static_cast<uint64_t>(E), static_cast<uint64_t>(H), 64,
                                    static_cast<uint32_t>(plan.ne));

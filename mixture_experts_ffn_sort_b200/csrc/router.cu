@@ -28,16 +28,20 @@
 // MMAs have read their stages by then).  Waits on mbarriers are bounded; an
 // expired wait records MOE_STATUS_TIMEOUT and the kernel runs to its end.
 #include "route_device.cuh"
+#include "router.h"
+#include "router_common.cuh"
 
 namespace moe {
 
 namespace {
 
+static_assert(kStatusTimeout == MOE_STATUS_TIMEOUT, "timeout status bit of the bounded waits");
+
 constexpr int kRouterThreads = 512;
 constexpr int kTileM = 128;             // tokens per tile (TMEM lanes)
 constexpr int kKStage = 64;             // bf16 columns per stage: one 128-byte swizzle row
 constexpr int kXStageBytes = kTileM * 128;
-constexpr int kMaxStages = 8;
+constexpr int kMaxStages = 16;
 
 struct RouterArgs {
     int T, H, E, K;
@@ -46,6 +50,7 @@ struct RouterArgs {
     int stages;     // K stages in the ring
     int tmem_cols;  // allocated TMEM columns (power of two >= max(32, NE))
     int S;          // row stride (floats) of the staging rows
+    int xrows;      // token rows a stage loads (128, or T rounded up to 8 when T < 128)
     RouteCfg cfg;
     const uint8_t* zero_mask;
     int32_t* ids;
@@ -69,7 +74,10 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
     RouterBars* B = reinterpret_cast<RouterBars*>(smem);
     uint8_t* ring = smem + 1024;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int stage_bytes = kXStageBytes + a.NE * 128;
+    // A stage: the x rows (xrows x 128 B), then the expert slice (NE x 128 B).
+    const int x_bytes = a.xrows * 128;
+    const int stage_bytes = x_bytes + a.NE * 128;
+    const uint32_t tx_bytes = static_cast<uint32_t>(stage_bytes);
     const uint32_t rank = cluster_ctarank();
     const int m0 = static_cast<int>(blockIdx.x / a.CN) * kTileM;
     const int e0 = static_cast<int>(rank) * a.NE;
@@ -102,9 +110,9 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
                     mbar_wait_or_abort(&B->empty[s], static_cast<uint32_t>((k / a.stages - 1) & 1), abort_flag,
                                        a.status);
                 uint8_t* st = ring + s * stage_bytes;
-                mbar_arrive_expect_tx(&B->full[s], static_cast<uint32_t>(stage_bytes));
+                mbar_arrive_expect_tx(&B->full[s], tx_bytes);
                 tma_load_2d(st, &tm_x, &B->full[s], k * kKStage, m0);
-                tma_load_2d(st + kXStageBytes, &tm_w, &B->full[s], k * kKStage, e0);
+                tma_load_2d(st + x_bytes, &tm_w, &B->full[s], k * kKStage, e0);
             }
         }
         __syncwarp();
@@ -117,7 +125,7 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
             mbar_wait_or_abort(&B->full[s], static_cast<uint32_t>((k / a.stages) & 1), abort_flag, a.status);
             tc_fence_after();
             const uint32_t st = ring_u32 + static_cast<uint32_t>(s * stage_bytes);
-            umma_ss_f16_x4_commit_elect(tmem, umma_desc_sw128(st), umma_desc_sw128(st + kXStageBytes), idesc,
+            umma_ss_f16_x4_commit_elect(tmem, umma_desc_sw128(st), umma_desc_sw128(st + x_bytes), idesc,
                                         k > 0 ? 1u : 0u, &B->empty[s]);
         }
         umma_commit_elect(&B->done);
@@ -202,13 +210,17 @@ RouterPlan plan_router(int T, int E) {
     p.cn = cn;
     p.ne = ((E + cn - 1) / cn + 15) / 16 * 16;
     p.tiles = tiles;
-    const int stage_bytes = kXStageBytes + p.ne * 128;
+    // A batch smaller than a tile loads only its rows (the MMA's other rows
+    // read whatever shared memory follows and produce accumulator rows nobody
+    // reads; the allocation keeps a full x tile of slack after the ring).
+    p.xrows = T < kTileM ? (T + 7) / 8 * 8 : kTileM;
+    const int stage_bytes = (p.xrows + p.ne) * 128;
     p.stages = 200 * 1024 / stage_bytes;
     if (p.stages > kMaxStages) p.stages = kMaxStages;
     p.tmem_cols = 32;
     while (p.tmem_cols < p.ne) p.tmem_cols *= 2;
     p.S = (E + 15) / 16 * 16 + 4;
-    const size_t ring = static_cast<size_t>(p.stages) * stage_bytes;
+    const size_t ring = static_cast<size_t>(p.stages) * stage_bytes + kXStageBytes;
     const size_t staging = static_cast<size_t>(kTileM / cn) * p.S * sizeof(float);
     p.smem = 2048 + (ring > staging ? ring : staging);
     return p;
@@ -228,6 +240,7 @@ cudaError_t launch_router(const CUtensorMap& tx, const CUtensorMap& tw, int T, i
     a.stages = p.stages;
     a.tmem_cols = p.tmem_cols;
     a.S = p.S;
+    a.xrows = p.xrows;
     a.cfg = cfg;
     a.zero_mask = zero_mask;
     a.ids = ids;
