@@ -1,4 +1,5 @@
-"""Expert-parallel decode over a process group (NCCL on GPUs).
+"""Expert parallelism over a process group (NCCL on GPUs): decode with an
+all-reduce of partial outputs, prefill with all-to-all dispatch and combine.
 
 The pages' decode kernel shards the experts across devices: every device
 routes all tokens the same way, applies only the experts it holds, and the
@@ -22,8 +23,8 @@ from typing import Optional, Tuple
 
 import torch
 
-from . import (MOE_MODE_DECODE, MOE_OUT_F32, Experts, moe_combine, moe_expert_ffn, moe_ffn_workspace_bytes,
-               moe_route, moe_sort, moe_sort_workspace_bytes)
+from . import (MOE_MODE_AUTO, MOE_MODE_DECODE, MOE_OUT_BF16, MOE_OUT_F32, Experts, moe_combine, moe_expert_ffn,
+               moe_ffn_workspace_bytes, moe_route, moe_sort, moe_sort_workspace_bytes)
 
 
 def expert_range(E: int, rank: int, world: int) -> Tuple[int, int]:
@@ -101,5 +102,120 @@ class ExpertParallelMoE:
     def forward(self, x: torch.Tensor, logits: torch.Tensor, zero_mask: Optional[torch.Tensor] = None,
                 stream=None) -> torch.Tensor:
         return reduce_partials(self.partial(x, logits, zero_mask, stream), self.group)
+
+    __call__ = forward
+
+
+# ---------------------------------------------------------------- prefill: all-to-all dispatch and combine
+
+def all_to_all_rows(send: torch.Tensor, send_rows, recv_rows, group=None) -> torch.Tensor:
+    """Exchange row blocks: block d of `send` (send_rows[d] rows) goes to rank
+    d; the result holds recv_rows[s] rows from each rank s, in rank order."""
+    import torch.distributed as dist
+    out = torch.empty((int(sum(recv_rows)),) + tuple(send.shape[1:]), dtype=send.dtype, device=send.device)
+    dist.all_to_all_single(out, send.contiguous(), output_split_sizes=[int(v) for v in recv_rows],
+                           input_split_sizes=[int(v) for v in send_rows], group=group)
+    return out
+
+
+class ExpertParallelPrefill:
+    """One rank of a token-sharded, expert-parallel MoE FFN (the all-to-all-v
+    dispatch and combine of the NKI library's MoE kernels: Build All2All
+    Dispatch Metadata, Permute / Unpermute Routed Tokens).
+
+    Every rank routes and sorts its own T tokens over all E experts, sends each
+    route's x row and weight to the rank holding its expert (rows of one
+    destination are contiguous in the sorted order), runs its experts on the
+    rows it receives (as tokens with K = 1: sort by local expert, expert FFN
+    with the route weight in the down epilogue, un-permute), sends the
+    results back, where they arrive in the sender's sorted order -- its
+    y_sorted -- and combines them through its inverse route map, adding its
+    own shared expert.  The library's kernels do all of that but the
+    exchanges (all_to_all_single) and the bookkeeping of counts (integer
+    tensors; the row counts are read back to the host to size the exchange).
+
+    The steps are also callable one by one (dispatch, expert_rows, finish),
+    which is how one process can stand in for several ranks.
+    """
+
+    def __init__(self, routed: Experts, E: int, T: int, K: int, rank: int, world: int,
+                 shared: Optional[Experts] = None, mode: int = MOE_MODE_AUTO, device="cuda", group=None):
+        self.e_begin, self.e_end = expert_range(E, rank, world)
+        if routed.n != self.e_end - self.e_begin:
+            raise ValueError("rank %d holds %d experts, expected %d" % (rank, routed.n, self.e_end - self.e_begin))
+        self.routed, self.shared, self.E, self.T, self.K = routed, shared, E, T, K
+        self.rank, self.world, self.mode, self.group, self.dev = rank, world, mode, group, device
+        self.El = E // world
+        self.H = routed.w_gate.shape[2]
+        d = device
+        R = T * K
+        self.topk_ids = torch.empty((T, K), dtype=torch.int32, device=d)
+        self.topk_w = torch.empty((T, K), dtype=torch.float32, device=d)
+        self.offsets = torch.empty(E + 1, dtype=torch.int32, device=d)
+        self.sorted_route = torch.empty(R, dtype=torch.int32, device=d)
+        self.inv_route = torch.empty(R, dtype=torch.int32, device=d)
+        self.sort_ws = torch.empty(max(16, moe_sort_workspace_bytes(T, K, E)), dtype=torch.uint8, device=d)
+        self.no_rows = torch.zeros(self.El + 1, dtype=torch.int32, device=d)  # offsets of an empty routed set
+        self.status = torch.zeros(1, dtype=torch.int32, device=d)
+
+    def dispatch(self, x: torch.Tensor, logits: torch.Tensor, zero_mask: Optional[torch.Tensor] = None):
+        """Route and sort this rank's tokens.  Returns (rows [R, H] bf16 and
+        weights [R] f32 in sorted order, per-expert route counts [world, El]
+        i32 on the device, rows per destination rank as a host list)."""
+        moe_route(logits, self.K, zero_mask, self.topk_ids, self.topk_w)
+        moe_sort(self.topk_ids, self.E, self.status, self.offsets, self.sorted_route, self.inv_route, self.sort_ws)
+        R = self.T * self.K
+        # Row p of the sorted order is route sorted_route[p] = t * K + j: token t.
+        src_token = torch.div(self.sorted_route, self.K, rounding_mode="floor").to(torch.int32)
+        rows = moe_combine(x, src_token, None, R, 1, MOE_OUT_BF16)  # a gather: one term per output row
+        wts = self.topk_w.view(-1)[self.sorted_route.long()]
+        counts = (self.offsets[1:] - self.offsets[:-1]).view(self.world, self.El).contiguous()
+        ends = self.offsets[::self.El].cpu().tolist()  # dispatch metadata: one read-back
+        send_rows = [ends[d + 1] - ends[d] for d in range(self.world)]
+        return rows, wts, counts, send_rows
+
+    def expert_rows(self, recv_x: torch.Tensor, recv_w: torch.Tensor, recv_counts: torch.Tensor) -> torch.Tensor:
+        """Run this rank's experts on the rows it received (recv_counts
+        [world, El]: rows per source rank and local expert, the rows of each
+        source grouped by expert in that order).  Returns the weighted output
+        rows [Rr, H] bf16 in the received order."""
+        Rr = recv_x.shape[0]
+        H, El = self.H, self.El
+        if Rr == 0:
+            return torch.empty((0, H), dtype=torch.bfloat16, device=recv_x.device)
+        dev = recv_x.device
+        local = torch.arange(El, dtype=torch.int32, device=dev).repeat(self.world)
+        ids = torch.repeat_interleave(local, recv_counts.reshape(-1).long()).view(Rr, 1)
+        offs = torch.empty(El + 1, dtype=torch.int32, device=dev)
+        srt = torch.empty(Rr, dtype=torch.int32, device=dev)
+        inv = torch.empty(Rr, dtype=torch.int32, device=dev)
+        ws = torch.empty(max(16, moe_sort_workspace_bytes(Rr, 1, El)), dtype=torch.uint8, device=dev)
+        moe_sort(ids, El, self.status, offs, srt, inv, ws)
+        y, _ = moe_expert_ffn(recv_x, 1, self.routed, offs, srt, recv_w.contiguous().view(Rr, 1), None, self.mode,
+                              self.status)
+        return moe_combine(y, inv, None, Rr, 1, MOE_OUT_BF16)  # back to the received order
+
+    def finish(self, y_back: torch.Tensor, x: torch.Tensor, out_dtype: int = MOE_OUT_BF16) -> torch.Tensor:
+        """Combine the returned rows (this rank's y_sorted) through the inverse
+        route map, with this rank's shared expert on its own tokens."""
+        y_shared = None
+        if self.shared is not None:
+            # The shared expert alone: an expert set with no routed rows.
+            _, y_shared = moe_expert_ffn(x, self.K, self.routed, self.no_rows, self.sorted_route, self.topk_w,
+                                         self.shared, self.mode, self.status)
+        return moe_combine(y_back, self.inv_route, y_shared, self.T, self.K, out_dtype)
+
+    def forward(self, x: torch.Tensor, logits: torch.Tensor, zero_mask: Optional[torch.Tensor] = None,
+                out_dtype: int = MOE_OUT_BF16) -> torch.Tensor:
+        import torch.distributed as dist
+        rows, wts, counts, send_rows = self.dispatch(x, logits, zero_mask)
+        recv_counts = torch.empty_like(counts)
+        dist.all_to_all_single(recv_counts, counts, group=self.group)
+        recv_rows = recv_counts.sum(dim=1).cpu().tolist()
+        recv_x = all_to_all_rows(rows, send_rows, recv_rows, self.group)
+        recv_w = all_to_all_rows(wts, send_rows, recv_rows, self.group)
+        y = self.expert_rows(recv_x, recv_w, recv_counts)
+        y_back = all_to_all_rows(y, recv_rows, send_rows, self.group)
+        return self.finish(y_back, x, out_dtype)
 
     __call__ = forward

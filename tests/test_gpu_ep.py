@@ -67,3 +67,55 @@ def test_ep_with_shared_expert(world, mode):
     torch.testing.assert_close(total, single, rtol=1e-5, atol=1e-5)
     ref = oracle.moe(w.x, w.logits, K, w.routed, w.shared)["out"]
     assert_moe_close(total.double().cpu().numpy(), ref, "ep shared x%d" % world)
+
+
+def _exchange_emulated(layers, xs, lgs, zms):
+    """Run the prefill ranks in one process: each exchange is a concatenation
+    of the senders' row blocks in rank order, as all_to_all_single lays them out."""
+    G = len(layers)
+    disp = [layers[r].dispatch(xs[r], lgs[r], zms[r]) for r in range(G)]
+    starts = [np.concatenate([[0], np.cumsum(d[3])]) for d in disp]  # rank s: first row for each destination
+    ys = []
+    for d in range(G):
+        rx = torch.cat([disp[s][0][starts[s][d]:starts[s][d + 1]] for s in range(G)])
+        rw = torch.cat([disp[s][1][starts[s][d]:starts[s][d + 1]] for s in range(G)])
+        rc = torch.stack([disp[s][2][d] for s in range(G)])
+        ys.append((layers[d].expert_rows(rx, rw, rc), [disp[s][3][d] for s in range(G)]))
+    outs = []
+    for s in range(G):
+        back = []
+        for d in range(G):
+            y, from_each = ys[d]
+            b = int(sum(from_each[:s]))
+            back.append(y[b:b + from_each[s]])
+        outs.append(layers[s].finish(torch.cat(back), xs[s], moe.MOE_OUT_F32))
+    torch.cuda.synchronize()
+    return outs
+
+
+@pytest.mark.parametrize("world", [1, 2, 4])
+def test_ep_prefill_all_to_all(world):
+    """Token-sharded expert parallelism: every rank's output equals the
+    single-device layer on its tokens and the oracle."""
+    H, I, E, K, Is = 256, 128, 16, 3, 128
+    Ts = [40, 33, 57, 21][:world]
+    dev = torch.device("cuda")
+    routed = wl.draw_experts(11, 4, E, I, H)
+    shared = wl.draw_experts(11, 5, 1, Is, H)
+    full = moe.Experts.from_host(routed, dev)
+    sh = moe.Experts.from_host(shared, dev)
+    xs_np = [wl.random_rows_bf16(T, H, seed=30 + r) for r, T in enumerate(Ts)]
+    lg_np = [np.random.default_rng(40 + r).standard_normal((T, E)).astype(np.float32) for r, T in enumerate(Ts)]
+    zm_np = [(np.random.default_rng(50 + r).random((T, K)) < 0.05).astype(np.uint8) for r, T in enumerate(Ts)]
+    layers = [ep.ExpertParallelPrefill(ep.local_experts(full, r, world), E, Ts[r], K, r, world, sh, device=dev)
+              for r in range(world)]
+    outs = _exchange_emulated(layers, [bf16_tensor(a) for a in xs_np], [torch.from_numpy(a).to(dev) for a in lg_np],
+                              [torch.from_numpy(a).to(dev) for a in zm_np])
+    for r in range(world):
+        assert layers[r].status.item() == 0
+        single = moe.MoEFFN(full, Ts[r], K, sh, out_dtype=moe.MOE_OUT_F32, device=dev)(
+            bf16_tensor(xs_np[r]), torch.from_numpy(lg_np[r]).to(dev), torch.from_numpy(zm_np[r]).to(dev))
+        torch.cuda.synchronize()
+        torch.testing.assert_close(outs[r], single, rtol=2e-2, atol=2e-3)
+        ref = oracle.moe(xs_np[r], lg_np[r], K, routed, shared, zero_mask=zm_np[r])["out"]
+        assert_moe_close(outs[r].double().cpu().numpy(), ref, "ep prefill rank %d of %d" % (r, world))
