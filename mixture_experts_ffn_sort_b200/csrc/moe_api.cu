@@ -178,15 +178,30 @@ int moe_router(const uint16_t* x, int T, int H, const uint16_t* w_router, int E,
     const moe::RouteCfg rc_dev = cfg ? moe::RouteCfg{cfg->score, cfg->sel_bias, cfg->n_group, cfg->topk_group,
                                                      cfg->renormalize, cfg->scaling}
                                      : moe::RouteCfg{MOE_SCORE_SOFTMAX, nullptr, 1, 1, 1, 1.f};
-    const moe::RouterPlan plan = moe::plan_router(T, E);
+    // Stages of several 64-column chunks (3-D boxes); one chunk if the
+    // driver declines the 3-D view.
+    moe::RouterPlan plan = moe::plan_router(T, H, E, 4);
     CUtensorMap tx, tw;
-    cudaError_t e = moe::make_tmap_bf16_2d(&tx, x, static_cast<uint64_t>(T), static_cast<uint64_t>(H), 64,
-                                           static_cast<uint32_t>(plan.xrows));
-    if (e == cudaSuccess)
-        e = moe::make_tmap_bf16_2d(&tw, w_router, static_cast<uint64_t>(E), static_cast<uint64_t>(H), 64,
-                                   static_cast<uint32_t>(plan.ne));
+    cudaError_t e = cudaSuccess;
+    for (int attempt = 0; attempt < 2; ++attempt) {
+        if (plan.kch == 1) {
+            e = moe::make_tmap_bf16_2d(&tx, x, static_cast<uint64_t>(T), static_cast<uint64_t>(H), 64,
+                                       static_cast<uint32_t>(plan.xrows));
+            if (e == cudaSuccess)
+                e = moe::make_tmap_bf16_2d(&tw, w_router, static_cast<uint64_t>(E), static_cast<uint64_t>(H), 64,
+                                           static_cast<uint32_t>(plan.ne));
+        } else {
+            e = moe::make_tmap_bf16_kchunks(&tx, x, static_cast<uint64_t>(T), static_cast<uint64_t>(H),
+                                            static_cast<uint32_t>(plan.xrows), static_cast<uint32_t>(plan.kch));
+            if (e == cudaSuccess)
+                e = moe::make_tmap_bf16_kchunks(&tw, w_router, static_cast<uint64_t>(E), static_cast<uint64_t>(H),
+                                                static_cast<uint32_t>(plan.ne), static_cast<uint32_t>(plan.kch));
+        }
+        if (e == cudaSuccess || plan.kch == 1) break;
+        plan = moe::plan_router(T, H, E, 1);
+    }
     if (e != cudaSuccess) return cuda_fail(e, "moe_router tensor maps");
-    e = moe::launch_router(tx, tw, T, H, E, K, rc_dev, zero_mask, topk_ids, topk_w, logits, status, stream);
+    e = moe::launch_router(plan, tx, tw, T, H, E, K, rc_dev, zero_mask, topk_ids, topk_w, logits, status, stream);
     return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_router launch");
 }
 

@@ -51,6 +51,7 @@ struct RouterArgs {
     int tmem_cols;  // allocated TMEM columns (power of two >= max(32, NE))
     int S;          // row stride (floats) of the staging rows
     int xrows;      // token rows a stage loads (128, or T rounded up to 8 when T < 128)
+    int kch;        // 64-column chunks per stage
     RouteCfg cfg;
     const uint8_t* zero_mask;
     int32_t* ids;
@@ -74,14 +75,16 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
     RouterBars* B = reinterpret_cast<RouterBars*>(smem);
     uint8_t* ring = smem + 1024;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    // A stage: the x rows (xrows x 128 B), then the expert slice (NE x 128 B).
-    const int x_bytes = a.xrows * 128;
-    const int stage_bytes = x_bytes + a.NE * 128;
+    // A stage: kch chunks of the x rows (xrows x 128 B each), then kch chunks
+    // of the expert slice (NE x 128 B each), every chunk a 64-column K slice.
+    const int xc_bytes = a.xrows * 128, wc_bytes = a.NE * 128;
+    const int x_bytes = a.kch * xc_bytes;
+    const int stage_bytes = a.kch * (xc_bytes + wc_bytes);
     const uint32_t tx_bytes = static_cast<uint32_t>(stage_bytes);
     const uint32_t rank = cluster_ctarank();
     const int m0 = static_cast<int>(blockIdx.x / a.CN) * kTileM;
     const int e0 = static_cast<int>(rank) * a.NE;
-    const int nk = a.H / kKStage;
+    const int nk = a.H / (kKStage * a.kch);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < a.stages; ++s) {
@@ -111,8 +114,13 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
                                        a.status);
                 uint8_t* st = ring + s * stage_bytes;
                 mbar_arrive_expect_tx(&B->full[s], tx_bytes);
-                tma_load_2d(st, &tm_x, &B->full[s], k * kKStage, m0);
-                tma_load_2d(st + x_bytes, &tm_w, &B->full[s], k * kKStage, e0);
+                if (a.kch == 1) {  // 2-D maps: box 64 columns x rows
+                    tma_load_2d(st, &tm_x, &B->full[s], k * kKStage, m0);
+                    tma_load_2d(st + x_bytes, &tm_w, &B->full[s], k * kKStage, e0);
+                } else {  // 3-D maps: box 64 columns x rows x kch chunks
+                    tma_load_3d(st, &tm_x, &B->full[s], 0, m0, k * a.kch);
+                    tma_load_3d(st + x_bytes, &tm_w, &B->full[s], 0, e0, k * a.kch);
+                }
             }
         }
         __syncwarp();
@@ -125,8 +133,13 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
             mbar_wait_or_abort(&B->full[s], static_cast<uint32_t>((k / a.stages) & 1), abort_flag, a.status);
             tc_fence_after();
             const uint32_t st = ring_u32 + static_cast<uint32_t>(s * stage_bytes);
-            umma_ss_f16_x4_commit_elect(tmem, umma_desc_sw128(st), umma_desc_sw128(st + x_bytes), idesc,
-                                        k > 0 ? 1u : 0u, &B->empty[s]);
+            for (int j = 0; j < a.kch - 1; ++j)
+                umma_ss_f16_x4_elect(tmem, umma_desc_sw128(st + j * xc_bytes),
+                                     umma_desc_sw128(st + x_bytes + j * wc_bytes), idesc, k > 0 || j > 0 ? 1u : 0u);
+            const int j = a.kch - 1;
+            umma_ss_f16_x4_commit_elect(tmem, umma_desc_sw128(st + j * xc_bytes),
+                                        umma_desc_sw128(st + x_bytes + j * wc_bytes), idesc,
+                                        k > 0 || j > 0 ? 1u : 0u, &B->empty[s]);
         }
         umma_commit_elect(&B->done);
     }
@@ -200,7 +213,7 @@ cudaError_t launch_router_t(const CUtensorMap& tx, const CUtensorMap& tw, const 
 
 }  // namespace
 
-RouterPlan plan_router(int T, int E) {
+RouterPlan plan_router(int T, int H, int E, int kch_max) {
     RouterPlan p{};
     const int tiles = (T + kTileM - 1) / kTileM;
     int cn = E > 256 ? 2 : 1;
@@ -214,7 +227,12 @@ RouterPlan plan_router(int T, int E) {
     // read whatever shared memory follows and produce accumulator rows nobody
     // reads; the allocation keeps a full x tile of slack after the ring).
     p.xrows = T < kTileM ? (T + 7) / 8 * 8 : kTileM;
-    const int stage_bytes = (p.xrows + p.ne) * 128;
+    // Chunks per stage: as many (up to kch_max) as keep a stage within 48 KB,
+    // so that at least four stages fit; fewer, larger TMA boxes per stage.
+    p.kch = 1;
+    while (p.kch * 2 <= kch_max && (H / 64) % (p.kch * 2) == 0 && p.kch * 2 * (p.xrows + p.ne) * 128 <= 48 * 1024)
+        p.kch *= 2;
+    const int stage_bytes = p.kch * (p.xrows + p.ne) * 128;
     p.stages = 200 * 1024 / stage_bytes;
     if (p.stages > kMaxStages) p.stages = kMaxStages;
     p.tmem_cols = 32;
@@ -226,10 +244,9 @@ RouterPlan plan_router(int T, int E) {
     return p;
 }
 
-cudaError_t launch_router(const CUtensorMap& tx, const CUtensorMap& tw, int T, int H, int E, int K,
-                          const RouteCfg& cfg, const uint8_t* zero_mask, int32_t* ids, float* w, float* logits,
-                          int32_t* status, cudaStream_t stream) {
-    const RouterPlan p = plan_router(T, E);
+cudaError_t launch_router(const RouterPlan& p, const CUtensorMap& tx, const CUtensorMap& tw, int T, int H, int E,
+                          int K, const RouteCfg& cfg, const uint8_t* zero_mask, int32_t* ids, float* w,
+                          float* logits, int32_t* status, cudaStream_t stream) {
     RouterArgs a{};
     a.T = T;
     a.H = H;
@@ -241,6 +258,7 @@ cudaError_t launch_router(const CUtensorMap& tx, const CUtensorMap& tw, int T, i
     a.tmem_cols = p.tmem_cols;
     a.S = p.S;
     a.xrows = p.xrows;
+    a.kch = p.kch;
     a.cfg = cfg;
     a.zero_mask = zero_mask;
     a.ids = ids;

@@ -7,6 +7,35 @@
 
 namespace moe {
 
+// 3-D tiled load into shared memory (coordinates innermost first), completion
+// counted on `bar` (bytes).  The innermost coordinate is 0 here.
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y, int z) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
+        : "memory");
+}
+
+// Four K=16 steps of D[tmem] (+)= A[smem desc] * B[smem desc] without a
+// commit (see umma_ss_f16_x4_commit_elect).
+__device__ __forceinline__ void umma_ss_f16_x4_elect(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                                     uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred e, p, t;\n\t.reg .b64 a1, a2, a3, b1, b2, b3;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "setp.ne.b32 p, %3, 0;\n\t"
+        "setp.eq.b32 t, 0, 0;\n\t"
+        "add.u64 a1, %1, 2;\n\tadd.u64 a2, %1, 4;\n\tadd.u64 a3, %1, 6;\n\t"
+        "add.u64 b1, %2, 2;\n\tadd.u64 b2, %2, 4;\n\tadd.u64 b3, %2, 6;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %4, p;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a1, b1, %4, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a2, b2, %4, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a3, b3, %4, t;\n\t}"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(accumulate), "r"(idesc)
+        : "memory");
+}
+
 // Four consecutive K=16 steps of D[tmem] (+)= A[smem desc] * B[smem desc]
 // (kind::f16, both operands from shared memory, K-major), both descriptors
 // 32 bytes further along K per step, then a commit to `bar`; one elected lane.
