@@ -158,3 +158,35 @@ def test_router_feeds_the_path():
     ref = oracle.moe_tokens_routed(wk.x, oid, ow, wk.routed)
     rel = np.linalg.norm(out - ref) / np.linalg.norm(ref)
     assert rel < 5e-3, rel
+
+
+def test_router_graph_replay_with_changing_tokens():
+    """The layer's fused-router forward captured once in a CUDA graph and
+    replayed on new token rows: the routing follows x (the oracle's router on
+    each new batch) and the output matches the oracle's method."""
+    T, H, I, E, K = 64, 512, 256, 32, 4
+    ex = wl.draw_experts(3, 55, E, I, H, 0.05, threads=4)
+    wr = wl.router_weight(E, H, seed=56)
+    layer = moe.MoEFFN(moe.Experts.from_host(ex), T, K, w_router=torch.from_numpy(wr.view(np.int16)).cuda())
+    x_s = torch.zeros(T, H, dtype=torch.int16, device="cuda")
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        layer.forward_fused(x_s)          # first call outside capture (one-time set-up)
+    torch.cuda.current_stream().wait_stream(s)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        layer.forward_fused(x_s)
+    # Batches whose oracle top-K+1 logits are at least 1e-3 apart (a margin far
+    # above the fp32 accumulation error), so the choice is unique.
+    for it, seed in enumerate((402, 409, 412)):
+        x = wl.random_rows_bf16(T, H, seed=seed)
+        x_s.copy_(torch.from_numpy(x.view(np.int16)).cuda())
+        g.replay()
+        torch.cuda.synchronize()
+        _, _, oid, ow = oracle.router(x, wr, K)
+        assert np.array_equal(layer.topk_ids.cpu().numpy(), oid), "replay %d: ids" % it
+        ref = oracle.moe_tokens_routed(x, oid, ow, ex)
+        got = layer.out.double().cpu().numpy()
+        rel = np.linalg.norm(got - ref) / np.linalg.norm(ref)
+        assert rel < 5e-3, (it, rel)
