@@ -218,6 +218,21 @@ MOE_API int moe_router(const uint16_t* x, int T, int H, const uint16_t* w_router
                        float* logits, int32_t* status, moe_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * moe_selftest_bounded_wait -- a diagnostic with no counterpart in the pages:
+ * it makes the kernels' bounded wait run out on purpose, without a fault.
+ *
+ * One CTA of the library's wait mechanism: two threads wait on mbarriers that
+ * nothing completes.  Each wait gives up after the library's wait limit (2 s
+ * of the GPU's global timer), ORs MOE_STATUS_TIMEOUT into *status and returns;
+ * the kernel ends normally and the context stays usable.  Takes about 2 s.
+ *   status      device int32 (required; the caller clears it)
+ *   elapsed_ns  device uint64[2] (required): how long each wait took
+ * Errors: MOE_ERR_INVALID_ARG for a NULL pointer, MOE_ERR_MISALIGNED for a
+ * misaligned one.
+ * ------------------------------------------------------------------------- */
+MOE_API int moe_selftest_bounded_wait(int32_t* status, uint64_t* elapsed_ns, moe_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * moe_sort -- stable sort of the R = T*K routes by expert.
  *
  * The "sort tokens by expert" step of the Nemotron prefill path, the NKI

@@ -32,7 +32,7 @@ MOE_STATUS_BAD_ID, MOE_STATUS_BAD_MAP, MOE_STATUS_TIMEOUT = 1, 2, 4
 MOE_MAX_E, MOE_MAX_K = 1024, 32
 
 EXPORTED = ("moe_last_error", "moe_abi_version", "moe_route", "moe_route_ex", "moe_router", "moe_sort_workspace_bytes",
-            "moe_sort",
+            "moe_sort", "moe_selftest_bounded_wait",
             "moe_sort_static_ws", "moe_ffn_resolve_mode", "moe_ffn_workspace_bytes", "moe_expert_ffn", "moe_combine")
 
 
@@ -74,6 +74,8 @@ def lib() -> ctypes.CDLL:
             L.moe_route_ex.restype = I
             L.moe_router.argtypes = [P, I, I, P, I, I, ctypes.POINTER(_RouteConfig), P, P, P, P, P, P]
             L.moe_router.restype = I
+            L.moe_selftest_bounded_wait.argtypes = [P, P, P]
+            L.moe_selftest_bounded_wait.restype = I
             L.moe_route.restype = I
             L.moe_sort_workspace_bytes.argtypes = [I, I, I]
             L.moe_sort_workspace_bytes.restype = S
@@ -190,7 +192,6 @@ def moe_route_ex(logits: torch.Tensor, K: int, score: int = MOE_SCORE_SOFTMAX,
 
 
 MOE_ROUTER_MAX_E = 512
-MOE_STATUS_TIMEOUT = 4
 
 
 def moe_router(x: torch.Tensor, w_router: torch.Tensor, K: int, score: int = MOE_SCORE_SOFTMAX,
@@ -213,6 +214,16 @@ def moe_router(x: torch.Tensor, w_router: torch.Tensor, K: int, score: int = MOE
     _check(lib().moe_router(_ptr(x), T, H, _ptr(w_router), E, K, ctypes.byref(cfg), _ptr(zero_mask),
                             _ptr(topk_ids), _ptr(topk_w), _ptr(logits), _ptr(status), _stream(stream)))
     return topk_ids, topk_w
+
+
+def moe_selftest_bounded_wait(stream=None):
+    """Make the library's bounded wait run out on purpose (about 2 s): returns
+    (status word, [elapsed ns of the two waits]) after a synchronize."""
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    elapsed = torch.zeros(2, dtype=torch.int64, device="cuda")
+    _check(lib().moe_selftest_bounded_wait(_ptr(status), _ptr(elapsed), _stream(stream)))
+    torch.cuda.synchronize()
+    return int(status.item()), [int(v) for v in elapsed.cpu().tolist()]
 
 def moe_sort_workspace_bytes(T: int, K: int, E: int) -> int:
     return int(lib().moe_sort_workspace_bytes(T, K, E))

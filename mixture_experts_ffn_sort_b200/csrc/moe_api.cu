@@ -90,6 +90,11 @@ int api_error(int code, const char* msg) {
 void api_clear_error() { g_err.clear(); }
 }  // namespace moe
 
+namespace moe {
+// selftest.cu
+cudaError_t launch_bounded_wait_probe(int32_t* status, unsigned long long* elapsed_ns, cudaStream_t stream);
+}  // namespace moe
+
 extern "C" {
 
 const char* moe_last_error(void) { return g_err.c_str(); }
@@ -152,6 +157,16 @@ int moe_route_ex(const float* logits, int T, int E, int K, const moe_route_confi
                                cfg->scaling};
     cudaError_t e = moe::launch_route_ex(logits, T, E, K, rc_dev, zero_mask, topk_ids, topk_w, stream);
     return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_route_ex launch");
+}
+
+int moe_selftest_bounded_wait(int32_t* status, uint64_t* elapsed_ns, moe_stream_t stream) {
+    g_err.clear();
+    if (!status || !elapsed_ns)
+        return fail(MOE_ERR_INVALID_ARG, "moe_selftest_bounded_wait: status and elapsed_ns must not be NULL");
+    if ((reinterpret_cast<uintptr_t>(status) & 3) || (reinterpret_cast<uintptr_t>(elapsed_ns) & 7))
+        return fail(MOE_ERR_MISALIGNED, "moe_selftest_bounded_wait: misaligned pointer");
+    cudaError_t e = moe::launch_bounded_wait_probe(status, reinterpret_cast<unsigned long long*>(elapsed_ns), stream);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_selftest_bounded_wait launch");
 }
 
 int moe_router(const uint16_t* x, int T, int H, const uint16_t* w_router, int E, int K, const moe_route_config* cfg,

@@ -216,3 +216,10 @@ def test_router_checks(L):
     assert call(status=P(0x1002)) == moe.MOE_ERR_MISALIGNED
     assert call(T=0, x=None, w=None, ids=None, wt=None) == moe.MOE_OK
     assert call(T=-1) == moe.MOE_ERR_INVALID_ARG
+
+
+def test_selftest_bounded_wait_checks(L):
+    assert L.moe_selftest_bounded_wait(None, P(16), None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_selftest_bounded_wait(P(16), None, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_selftest_bounded_wait(P(0x1002), P(16), None) == moe.MOE_ERR_MISALIGNED
+    assert L.moe_selftest_bounded_wait(P(16), P(0x1004), None) == moe.MOE_ERR_MISALIGNED
