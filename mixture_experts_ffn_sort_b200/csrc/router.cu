@@ -11,13 +11,18 @@
 // tile: CTA c computes the logits of experts [c NE, (c+1) NE) (NE a multiple
 // of 16, at most 256: the MMA's N) for all 128 tokens, so small batches still
 // spread over CN SMs.  Per CTA:
-//   warp 0      TMA: 64-column K stages of the x tile (128 x 128 B) and of the
-//               expert slice of W_r (NE x 128 B), both 128-byte swizzled,
-//               into a ring of `stages` stages;
+//   warp 0      TMA: K stages of kch 64-column chunks of the x tile (128
+//               rows, or the batch's rows when T < 128, x 128 B per chunk)
+//               and of the expert slice of W_r (NE x 128 B per chunk), each
+//               chunk a 128-byte-swizzled tile, into a ring of `stages`
+//               stages.  kch = 1 loads one chunk per 2-D box; small batches
+//               load up to four per 3-D box (64 columns x rows x chunks),
+//               because the producer issues boxes at a fixed rate whatever
+//               their size;
 //   warp 1      TMEM allocation and the MMA issuer: tcgen05.mma kind::f16,
-//               A = x stage, B = W_r stage (both from shared memory), fp32
-//               accumulators in TMEM columns 0..NE-1, four K=16 steps and a
-//               commit that frees the stage, per stage;
+//               A = x chunk, B = W_r chunk (both from shared memory), fp32
+//               accumulators in TMEM columns 0..NE-1, four K=16 steps per
+//               chunk and a commit that frees the stage;
 //   all warps   (16) once every MMA has completed: the accumulators go from
 //               TMEM to the shared memory of the CTA that routes each token
 //               (token rows split evenly over the cluster, written through
