@@ -37,6 +37,12 @@ UNIT = "tokens/s"
 # Bytes of one expert's FP8 weights and fp32 block scales, used for the decode roofline.
 
 
+# Nominal B200 figures, reported beside the measured-peak fractions: HBM3e
+# bandwidth and dense bf16 tensor-core throughput.
+SPEC_HBM_GBS = 8000.0
+SPEC_BF16_TFLOPS = 2250.0
+
+
 def expert_bytes(H, I):
     return 3 * H * I + 3 * (H // 128) * (I // 128) * 4
 
@@ -459,13 +465,15 @@ def main():
         roof = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm"], "unit": "GB/s",
                 "frac": ach / peaks["hbm"], "traffic": traffic,
                 "kernel": "moe_expert_ffn (gate/up + down kernels)", "algorithmic_bytes": algo,
-                "touched_experts": touched, "peak_source": peaks["src"]}
+                "touched_experts": touched, "peak_source": peaks["src"],
+                "spec_peak": SPEC_HBM_GBS, "frac_of_spec": ach / SPEC_HBM_GBS}
     else:
         ach = flops / (ffn_ms * 1e-3) / 1e12
         pk = peaks["bf16_sus"]
         roof = {"bound": "tensor", "achieved": ach, "peak": pk, "unit": "TFLOP/s", "frac": ach / pk,
                 "traffic": profile_traffic(shape.name, "prefill"), "kernel": "moe_expert_ffn", "flops": flops,
-                "peak_source": peaks["src"] + " sustained"}
+                "peak_source": peaks["src"] + " sustained",
+                "spec_peak": SPEC_BF16_TFLOPS, "frac_of_spec": ach / SPEC_BF16_TFLOPS}
     if args.fused_router:
         # The fused router's own roofline: a bf16 GEMM of 2 T H E flops (its
         # top-K epilogue adds no HBM traffic beyond the ids and weights).
