@@ -144,6 +144,27 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+def ffn_roofline(shape, form_kind, touched, flops, ffn_ms, peaks):
+    """The roofline object of the FFN call: touched-expert bytes against HBM
+    for the weight-streaming and hybrid forms (form_kind "decode" / "hybrid"),
+    bf16 FLOPs against the tensor cores for the prefill form."""
+    H, I = shape.H, shape.I
+    if form_kind in ("decode", "hybrid"):
+        algo = touched * expert_bytes(H, I) + (expert_bytes(H, shape.I_shared) if shape.I_shared else 0)
+        ach = algo / (ffn_ms * 1e-3) / 1e9
+        return {"bound": "hbm", "achieved": ach, "peak": peaks["hbm"], "unit": "GB/s",
+                "frac": ach / peaks["hbm"], "traffic": profile_traffic(shape.name, form_kind),
+                "kernel": "moe_expert_ffn (gate/up + down kernels)", "algorithmic_bytes": algo,
+                "touched_experts": touched, "peak_source": peaks["src"],
+                "spec_peak": SPEC_HBM_GBS, "frac_of_spec": ach / SPEC_HBM_GBS}
+    ach = flops / (ffn_ms * 1e-3) / 1e12
+    pk = peaks["bf16_sus"]
+    return {"bound": "tensor", "achieved": ach, "peak": pk, "unit": "TFLOP/s", "frac": ach / pk,
+            "traffic": profile_traffic(shape.name, "prefill"), "kernel": "moe_expert_ffn", "flops": flops,
+            "peak_source": peaks["src"] + " sustained",
+            "spec_peak": SPEC_BF16_TFLOPS, "frac_of_spec": ach / SPEC_BF16_TFLOPS}
+
+
 # ---------------------------------------------------------------- reference arm (CPU oracle)
 
 def oracle_route_kwargs(router, shape):
@@ -458,22 +479,9 @@ def main():
     flops = (R_nz + (T if shape.I_shared else 0)) * 6 * H * I
     form = moe.moe_ffn_resolve_mode(T, K, E, args.mode)
     decode_path = form in (moe.MOE_MODE_DECODE, moe.MOE_MODE_HYBRID)  # bound by the touched weights
-    if decode_path:
-        algo = touched * expert_bytes(H, I) + (expert_bytes(H, shape.I_shared) if shape.I_shared else 0)
-        ach = algo / (ffn_ms * 1e-3) / 1e9
-        traffic = profile_traffic(shape.name, "hybrid" if form == moe.MOE_MODE_HYBRID else "decode")
-        roof = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm"], "unit": "GB/s",
-                "frac": ach / peaks["hbm"], "traffic": traffic,
-                "kernel": "moe_expert_ffn (gate/up + down kernels)", "algorithmic_bytes": algo,
-                "touched_experts": touched, "peak_source": peaks["src"],
-                "spec_peak": SPEC_HBM_GBS, "frac_of_spec": ach / SPEC_HBM_GBS}
-    else:
-        ach = flops / (ffn_ms * 1e-3) / 1e12
-        pk = peaks["bf16_sus"]
-        roof = {"bound": "tensor", "achieved": ach, "peak": pk, "unit": "TFLOP/s", "frac": ach / pk,
-                "traffic": profile_traffic(shape.name, "prefill"), "kernel": "moe_expert_ffn", "flops": flops,
-                "peak_source": peaks["src"] + " sustained",
-                "spec_peak": SPEC_BF16_TFLOPS, "frac_of_spec": ach / SPEC_BF16_TFLOPS}
+    roof = ffn_roofline(shape, form_kind="hybrid" if form == moe.MOE_MODE_HYBRID else
+                        ("decode" if decode_path else "prefill"), touched=touched, flops=flops, ffn_ms=ffn_ms,
+                        peaks=peaks)
     if args.fused_router:
         # The fused router's own roofline: a bf16 GEMM of 2 T H E flops (its
         # top-K epilogue adds no HBM traffic beyond the ids and weights).
