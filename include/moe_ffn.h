@@ -12,6 +12,11 @@
  *                  weight fused in; optional always-on shared expert
  *   moe_combine    top-K reduce back to token order (+ shared expert)
  *
+ * plus the routing variants (moe_route_ex), the fused router that computes the
+ * logits from the token rows and routes in one kernel (moe_router), a sort
+ * with library-owned scratch (moe_sort_static_ws) and a diagnostic of the
+ * kernels' bounded waits (moe_selftest_bounded_wait).
+ *
  * Sources (page title, section):
  *  - dstair/gated-deltanet-nki-trainium, "FP8 MoE decode kernel
  *    (moe_fused_w8_35b)": the fused chain gate/up GEMM -> SwiGLU -> down GEMM
@@ -19,10 +24,11 @@
  *    block scales decoded to BF16 tile by tile; "Interface" (hidden, gate_up,
  *    down, scales, affinities -> [B, H] f32); "Serving contract" (softmax ->
  *    top-8 -> norm router; the shared expert is added after the routed sum).
- *  - spark_model/layers/nemotron_moe.rs: module doc ("all expert dispatch is
- *    device-side ... zero D2H sync"), `new` (top_k bounds checked with an error
- *    message), `prefill` step 5 (sort by expert, grouped GEMM, unpermute-reduce,
- *    ids and weights as [N, top_k] 4-byte arrays).
+ *  - spark_model/layers/nemotron_moe.rs: module doc (expert dispatch stays on the
+ *    device, with no device-to-host synchronisation), `new` (top_k bounds checked with an error
+ *    message), `prefill` step 2 (the router's dense gate GEMM) and step 5 (sort
+ *    by expert, grouped GEMM, unpermute-reduce, ids and weights as [N, top_k]
+ *    4-byte arrays).
  *  - ROCm/aiter PR #5988: ctypes C-ABI entry point whose launcher validates the
  *    tensor contracts; reuse of a sort with an inverse route map; FP32 route
  *    reduction; zero routing weights and caller-provided output buffers.
@@ -139,7 +145,7 @@ MOE_API int moe_route(const float* logits, int T, int E, int K, const uint8_t* z
  * group-limited choice, optional renormalisation, routed scaling factor.
  *
  * The pages name these routers without giving their formulas: the Nemotron-H
- * layer's "sigmoid topK routing" scaled by `routed_scaling_factor`
+ * layer's sigmoid top-K routing scaled by `routed_scaling_factor`
  * (spark_model/layers/nemotron_moe.rs, module doc and `prefill`) and the NKI
  * library's DeepSeek-V3 group-limited `noaux_tc` router (NKI Library kernel
  * reference, MoE kernels).  Both are taken in the published DeepSeek-V3
@@ -235,7 +241,7 @@ MOE_API int moe_selftest_bounded_wait(int32_t* status, uint64_t* elapsed_ns, moe
 /* ---------------------------------------------------------------------------
  * moe_sort -- stable sort of the R = T*K routes by expert.
  *
- * The "sort tokens by expert" step of the Nemotron prefill path, the NKI
+ * The step of the Nemotron prefill path that sorts the tokens by expert, the NKI
  * Permute Routed Tokens kernel, and the aiter pipeline's sort with inverse
  * route map.  A counting sort: per-chunk expert histograms, an expert-major
  * exclusive scan, and an in-order scatter, so the result is deterministic.
@@ -342,7 +348,7 @@ MOE_API int moe_ffn_resolve_mode(int T, int K, int E, int mode);
  *   y_shared[t, :] = bf16( Wd_s (silu(Wg_s x[t]) * (Wu_s x[t])) )
  * This is the decode kernel page's fused chain (gate/up -> SwiGLU -> down ->
  * affinity scale) over the Nemotron page's sorted grouped-GEMM order; the
- * shared expert is the "one shared expert" of the aiter PR, weight 1.
+ * shared expert is the single always-on expert of the aiter PR, weight 1.
  * Numerics: bf16 x bf16 products accumulated in fp32; weights decoded from
  * E4M3FN to BF16 (DECODE mode: the exact E4M3 value, its block scale applied to
  * each 128-wide fp32 partial sum; PREFILL mode: bf16(e4m3 * scale));

@@ -1,7 +1,7 @@
 // route.cu -- top-K routing (moe_route, moe_route_ex).
 //
 // moe_route is the router of the FP8 MoE decode kernel page's serving
-// contract ("softmax -> top-8 -> norm", dstair/gated-deltanet-nki-trainium)
+// contract (softmax, top-8, renormalise; dstair/gated-deltanet-nki-trainium)
 // and the NKI Router Top-K kernel; moe_route_ex adds the variants the pages
 // name (the Nemotron-H layer's sigmoid top-K with a routed scaling factor,
 // spark_model/layers/nemotron_moe.rs; the NKI library's DeepSeek-V3

@@ -26,8 +26,8 @@
  *  - spark_model/layers/nemotron_moe.rs, module doc and `prefill` step 5: sort
  *    tokens by expert, grouped GEMM over each expert's rows, unpermute-reduce.
  *  - ROCm/aiter PR #5988 description: the sorted pipeline with an inverse
- *    route map and an FP32 route reduction; "10 routed experts plus one shared
- *    expert".
+ *    route map and an FP32 route reduction; ten routed experts and one shared
+ *    expert per token.
  *  - spark_model/layers/nemotron_moe.rs, `prefill` step 2: the router's dense
  *    gate GEMM [N, H] x [H, E]^T -> [N, E] logits.
  *  - NKI Library kernel reference, MoE kernels: Router Top-K, Permute Routed
@@ -70,7 +70,7 @@ int oracle_get_threads(void) { return g_threads; }
 
 /* ---------------------------------------------------------------- formats */
 
-/* OCP FP8 E4M3FN (the "official E4M3FN" weights of the decode kernel page):
+/* OCP FP8 E4M3FN (the weight format the decode kernel page names):
  * 1 sign bit, 4 exponent bits with bias 7, 3 mantissa bits.
  * exponent 0: subnormal, value (m/8) * 2^-6.  exponent 1..15: (1 + m/8) * 2^(e-7).
  * S.1111.111 is NaN; there is no infinity (so S.1111.110 = 448 is the maximum). */
@@ -159,7 +159,7 @@ void oracle_route(const float* logits, int T, int E, int K, const uint8_t* zero_
 }
 
 /* Routing variants named by the pages without a formula -- the Nemotron-H
- * layer's "sigmoid topK routing" scaled by `routed_scaling_factor`
+ * layer's sigmoid top-K routing scaled by `routed_scaling_factor`
  * (spark_model/layers/nemotron_moe.rs, module doc and `prefill`) and the NKI
  * library's "DeepSeek-V3 group-limited noaux_tc routing" (NKI Library kernel
  * reference, MoE kernels) -- taken in the published DeepSeek-V3 router's form:
@@ -303,7 +303,7 @@ void oracle_router_logits(const uint16_t* x, const uint16_t* w_router, int T, in
 
 /* Sort the R = T*K routes (route r = t*K + j carries expert ids[r]) by expert,
  * keeping route order within an expert (a stable counting sort: count, exclusive
- * scan, scatter in route order).  This is the "sort tokens by expert" step of the
+ * scan, scatter in route order).  This is the step that sorts the tokens by expert in the
  * Nemotron prefill path and the NKI "Permute Routed Tokens" kernel.
  *   offsets[e]       = number of valid routes with id < e; offsets[E] = valid routes
  *   sorted_route[p]  = the route at sorted position p (p < offsets[E]); -1 after
@@ -380,7 +380,7 @@ static void load_row(const uint16_t* x, int H, int t, double* xr) {
     for (int k = 0; k < H; ++k) xr[k] = oracle_bf16_value(x[(size_t)t * H + k]);
 }
 
-/* Grouped expert FFN over the sorted routes (the "sorted grouped GEMM" of the
+/* Grouped expert FFN over the sorted routes (the grouped GEMM over expert-sorted rows of the
  * Nemotron prefill path): for each expert e and each sorted position p in
  * [offsets[e], offsets[e+1]), route r = sorted_route[p], token t = r / K:
  *     y_sorted[p] = w[r] * FFN_e(x[t])
