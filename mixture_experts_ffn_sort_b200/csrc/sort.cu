@@ -1,6 +1,6 @@
 // sort.cu -- stable sort of the routes by expert (moe_sort).
 //
-// The "sort tokens by expert" step of the Nemotron-H sorted prefill path
+// The step of the Nemotron-H sorted prefill path that orders tokens by expert
 // (spark_model/layers/nemotron_moe.rs, `prefill` step 5), the NKI Permute
 // Routed Tokens kernel, and the sort with an inverse route map that the aiter
 // gfx950 prefill PR reuses.  A counting sort in three passes:
