@@ -550,3 +550,18 @@ def test_router_routes_the_rounded_logits():
         assert list(ids[t]) == order
         p = scipy.special.softmax(l32[t].astype(np.float64))
         np.testing.assert_allclose(wt[t], p[order] / p[order].sum(), rtol=1e-12)
+
+
+def test_router_logits_permutations_and_linearity():
+    """Permuting tokens permutes logit rows, permuting experts permutes
+    columns (bit-identical), and the GEMM is linear in x: logits of a
+    power-of-two multiple of x are that multiple (exact in fp64)."""
+    x = wl.random_rows_bf16(11, 128, seed=9)
+    w = wl.router_weight(7, 128, seed=10)
+    base = oracle.router_logits(x, w)
+    pt = np.random.default_rng(1).permutation(11)
+    pe = np.random.default_rng(2).permutation(7)
+    assert np.array_equal(oracle.router_logits(x[pt], w), base[pt])
+    assert np.array_equal(oracle.router_logits(x, w[pe]), base[:, pe])
+    x4 = wl.to_bf16_bits(oracle.bf16_array(x).astype(np.float32) * np.float32(4.0))
+    assert np.array_equal(oracle.router_logits(x4, w), 4.0 * base)
