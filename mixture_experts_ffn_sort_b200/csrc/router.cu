@@ -270,6 +270,13 @@ cudaError_t launch_router(const RouterPlan& p, const CUtensorMap& tx, const CUte
     a.w = w;
     a.logits = logits;
     a.status = status;
+    // The plan's invariants, which the kernel's indexing relies on: a cluster
+    // of at most 8 CTAs splitting 128 tokens evenly, an MMA N of 16..256 in
+    // steps of 16 within the TMEM allocation, at least two stages, chunks that
+    // divide H, and shared memory within one CTA's limit.
+    if (p.cn < 1 || p.cn > 8 || kTileM % p.cn || p.ne < 16 || p.ne > 256 || p.ne % 16 || p.ne > p.tmem_cols ||
+        p.stages < 2 || p.stages > kMaxStages || p.kch < 1 || (H / kKStage) % p.kch || p.smem > 227 * 1024)
+        return cudaErrorInvalidConfiguration;
     const int grid = p.tiles * p.cn;
     const bool computed = cfg.bias != nullptr || cfg.n_group > 1;
 #define MOE_ROUTER_CASE(EPL)                                                                    \
