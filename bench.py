@@ -56,10 +56,10 @@ def load_peaks():
     return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
 
 
-def profile_traffic(workload, kind):
+def profile_traffic(workload, kind, root=ROOT):
     """DRAM bytes per FFN call from the committed ncu summary of this workload,
     if the kernel sources it was taken on are unchanged (else None)."""
-    path = os.path.join(ROOT, "profiles", "ffn_%s_%s.md" % (kind, workload))
+    path = os.path.join(root, "profiles", "ffn_%s_%s.md" % (kind, workload))
     if not os.path.exists(path):
         return None
     text = open(path).read()
@@ -91,19 +91,20 @@ def sources_hash(kind="decode"):
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons every 100 ms while running."""
+    """nvidia-smi clocks and throttle reasons every 50 ms while running; the
+    samples are time-stamped so that each timed region gets its own summary."""
 
     Q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
          "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
          "clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, index):
-        self.index, self.lines, self.proc = index, [], None
+    def __init__(self, index, period_ms=50):
+        self.index, self.period_ms, self.lines, self.proc = index, period_ms, [], None
 
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.Q,
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                          "--format=csv,noheader,nounits", "-lms", str(self.period_ms)],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
@@ -113,7 +114,7 @@ class ClockSampler:
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.monotonic(), line.strip()))
 
     def __exit__(self, *a):
         if self.proc is not None:
@@ -123,16 +124,21 @@ class ClockSampler:
             except subprocess.TimeoutExpired:
                 self.proc.kill()
 
-    def summary(self):
-        sm, mx, reasons = [], [], set()
+    def summary(self, t0=None, t1=None):
+        """Median SM clock, max clock and throttle reasons of the samples taken
+        in [t0, t1] (all samples when no interval is given)."""
+        sm, mx, pw, reasons = [], [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for l in self.lines:
+        for ts, l in list(self.lines):
+            if (t0 is not None and ts < t0) or (t1 is not None and ts > t1):
+                continue
             f = [x.strip() for x in l.split(",")]
             if len(f) < 8:
                 continue
             try:
                 sm.append(float(f[0]))
                 mx.append(float(f[1]))
+                pw.append(float(f[2]))
             except ValueError:
                 continue
             for n, v in zip(names, f[4:8]):
@@ -140,29 +146,46 @@ class ClockSampler:
                     reasons.add(n)
         if not sm:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "power_w_max": max(pw),
+                "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def ffn_roofline(shape, form_kind, touched, flops, ffn_ms, peaks):
+def ffn_roofline(shape, form_kind, touched, flops, ffn_ms, peaks, root=ROOT):
     """The roofline object of the FFN call: touched-expert bytes against HBM
     for the weight-streaming and hybrid forms (form_kind "decode" / "hybrid"),
-    bf16 FLOPs against the tensor cores for the prefill form."""
+    bf16 FLOPs against the tensor cores for the prefill form.  The FFN time is
+    a median of single synchronised replays, a kernel timed on its own, so
+    the tensor-core fraction is against the burst bf16 peak (the sustained
+    one, for a kernel inside a seconds-long loop, is reported beside it)."""
     H, I = shape.H, shape.I
     if form_kind in ("decode", "hybrid"):
         algo = touched * expert_bytes(H, I) + (expert_bytes(H, shape.I_shared) if shape.I_shared else 0)
         ach = algo / (ffn_ms * 1e-3) / 1e9
         return {"bound": "hbm", "achieved": ach, "peak": peaks["hbm"], "unit": "GB/s",
-                "frac": ach / peaks["hbm"], "traffic": profile_traffic(shape.name, form_kind),
+                "frac": ach / peaks["hbm"], "traffic": profile_traffic(shape.name, form_kind, root),
                 "kernel": "moe_expert_ffn (gate/up + down kernels)", "algorithmic_bytes": algo,
-                "touched_experts": touched, "peak_source": peaks["src"],
+                "touched_experts": touched, "peak_source": peaks["src"] + " copy bandwidth",
                 "spec_peak": SPEC_HBM_GBS, "frac_of_spec": ach / SPEC_HBM_GBS}
     ach = flops / (ffn_ms * 1e-3) / 1e12
-    pk = peaks["bf16_sus"]
+    pk = peaks["bf16"]
     return {"bound": "tensor", "achieved": ach, "peak": pk, "unit": "TFLOP/s", "frac": ach / pk,
-            "traffic": profile_traffic(shape.name, "prefill"), "kernel": "moe_expert_ffn", "flops": flops,
-            "peak_source": peaks["src"] + " sustained",
+            "traffic": profile_traffic(shape.name, "prefill", root), "kernel": "moe_expert_ffn", "flops": flops,
+            "peak_source": peaks["src"] + " burst bf16",
+            "peak_sustained": peaks["bf16_sus"], "frac_of_sustained": ach / peaks["bf16_sus"],
             "spec_peak": SPEC_BF16_TFLOPS, "frac_of_spec": ach / SPEC_BF16_TFLOPS}
+
+
+# The arithmetic each FFN form computes in ("dtype" of the line and its description).
+ARITHMETIC = {
+    "decode": ("f16", "E4M3 weights taken exactly as f16 MMA operands, activations as f16 after an exact "
+                      "power-of-two row scale, fp32 accumulate, fp32 block scale per 128-column partial; "
+                      "bf16 h, y_sorted and out"),
+    "prefill": ("bf16", "weights decoded to bf16(e4m3 x block scale), bf16 activations, fp32 accumulate in "
+                        "TMEM; bf16 h, y_sorted and out"),
+    "hybrid": ("f16+bf16", "experts with few rows as the decode form (f16 MMA on exact E4M3), the others as the "
+                           "prefill form (bf16 MMA on bf16(e4m3 x scale)); fp32 accumulate; bf16 h, y_sorted "
+                           "and out"),
+}
 
 
 # ---------------------------------------------------------------- reference arm (CPU oracle)
@@ -274,44 +297,33 @@ def config_of(shape, router="softmax", fused_router=False):
 
 # ---------------------------------------------------------------- our arm
 
-def main():
-    ap = argparse.ArgumentParser()
-    ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=None)
-    ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="decode", choices=wl.SHAPE_ORDER)
-    ap.add_argument("--mode", type=int, default=0, help="moe_expert_ffn mode: 0 AUTO, 1 DECODE, 2 PREFILL")
-    ap.add_argument("--router", default="softmax", choices=sorted(wl.ROUTERS),
-                    help="routing variant: softmax top-k (moe_route) or a moe_route_ex preset")
-    ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--fused-router", action="store_true",
-                    help="route from x with the fused router (gate GEMM + top-K) instead of given logits")
-    ap.add_argument("--eager", action="store_true",
-                    help="launch every call directly instead of replaying CUDA graphs (for profilers)")
-    args = ap.parse_args()
-    shape = wl.SHAPES[args.workload]
-    rank, world, local = dist_env()
+# Windows of `steps` replays timed one by one; the step time is their median.
+N_WINDOWS = 7
+# Workloads timed after the headline one with the same protocol (the line's
+# "workloads" object): the skewed high-batch decode and both prefills.
+EXTRA_WORKLOADS = ("decode_skew", "prefill", "prefill_large")
+DEFAULT_STEPS = {"tiny": 500, "decode": 500, "decode_skew": 200, "prefill": 30, "prefill_large": 10}
 
-    if args.impl == "reference":
-        if args.steps is None:
-            args.steps = 3
-        if rank == 0:
-            print(json.dumps(run_reference(args, shape)), flush=True)
-        return
 
+class Eager:
+    """Stands in for a CUDA graph: replay() launches every call directly."""
+
+    def __init__(self, fn):
+        self.fn = fn
+
+    def replay(self):
+        self.fn()
+
+
+def measure(args, shape, steps, dev, world, clk, want_e2e):
+    """One workload: build the layer, capture a step in a CUDA graph, warm up,
+    time N_WINDOWS windows of `steps` replays (barrier and synchronize around
+    each, max over ranks), then the per-call breakdown from an instrumented
+    graph.  Returns the workload's record, plus the end-to-end measurement
+    through the public API when want_e2e."""
     import torch
     import torch.distributed as dist
     import mixture_experts_ffn_sort_b200 as moe
-
-    if args.steps is None:
-        args.steps = {"tiny": 2000, "decode": 5000, "decode_skew": 2000, "prefill": 200,
-                      "prefill_large": 30}[shape.name]
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if world > 1:
-        from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
 
     w = wl.make_workload(shape.name)
     T, K, E, H, I = shape.T, shape.K, shape.E, shape.H, shape.I
@@ -340,19 +352,13 @@ def main():
     def step():
         run(layer, x, logits)
 
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
     with torch.cuda.stream(stream):
-        for _ in range(max(1, args.warmup)):
-            step()
+        step()  # first call outside any capture (one-time set-up)
     stream.synchronize()
-    if layer.status.item() != 0:
-        raise RuntimeError("status word %d after warm-up" % layer.status.item())
-
-    class Eager:
-        def __init__(self, fn):
-            self.fn = fn
-
-        def replay(self):
-            self.fn()
 
     def instrumented():
         ev[0].record()
@@ -371,11 +377,12 @@ def main():
         moe.moe_expert_ffn(x, K, routed, layer.offsets, layer.sorted_route, layer.topk_w, shared, args.mode,
                            layer.status, layer.y_sorted, layer.y_shared, layer.ffn_ws)
         ev[3].record()
-        moe.moe_combine(layer.y_sorted, layer.inv_route, layer.y_shared, T, K, moe.MOE_OUT_BF16, layer.out)
+        moe.moe_combine(layer.y_sorted, layer.inv_route, layer.y_shared, T, K, moe.MOE_OUT_BF16, layer.out,
+                        status=layer.status)
         ev[4].record()
 
-    # Graph of one step; the timed region replays it K times.  A second graph
-    # records events around each call, for the per-call breakdown.
+    # Graph of one step; the timed windows replay it.  A second graph records
+    # events around each call, for the per-call breakdown.
     ev = [torch.cuda.Event(enable_timing=True, external=not args.eager) for _ in range(5)]
     if args.eager:
         g, g2 = Eager(step), Eager(instrumented)
@@ -386,44 +393,95 @@ def main():
         g2 = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g2, stream=stream):
             instrumented()
+    t_warm = time.monotonic()
     with torch.cuda.stream(stream):
-        for _ in range(3):
+        for _ in range(max(3, args.warmup)):
             g.replay()
-            g2.replay()
+        g2.replay()
     stream.synchronize()
+    if layer.status.item() != 0:
+        raise RuntimeError("%s: status word %d after warm-up" % (shape.name, layer.status.item()))
 
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
+    windows = []
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local) as clk:
+    t_timed = time.monotonic()
+    for _ in range(N_WINDOWS):
         barrier()
         torch.cuda.synchronize(dev)
         start.record(stream)
         with torch.cuda.stream(stream):
-            for _ in range(args.steps):
+            for _ in range(steps):
                 g.replay()
         end.record(stream)
         torch.cuda.synchronize(dev)
         barrier()
-    ms = start.elapsed_time(end)
-    t_local = ms / args.steps
-    # Per-call breakdown from the instrumented graph (same stream, after the timed region).
+        windows.append(start.elapsed_time(end) / steps)
+    t_done = time.monotonic()
+    t_local = statistics.median(windows)
+    # Per-call breakdown from the instrumented graph (same stream, after the timed windows).
     parts = {k: [] for k in ("route", "sort", "ffn", "combine")}
     with torch.cuda.stream(stream):
-        for _ in range(min(args.steps, 200)):
+        for _ in range(min(max(steps, 20), 200)):
             g2.replay()
             stream.synchronize()
             for i, k in enumerate(parts):
                 parts[k].append(ev[i].elapsed_time(ev[i + 1]))
     t_max = max_over_ranks(t_local, dev)
+    if layer.status.item() != 0:
+        raise RuntimeError("%s: status word %d after the timed windows" % (shape.name, layer.status.item()))
 
-    # End to end through the public API with host buffers: every step copies
-    # its x and logits in from pinned host memory and its output back out.
-    # Two sets of device buffers (a second layer object over the same
-    # weights) let step i+1's input copy and step i-1's output copy overlap
-    # step i's compute: copy-in, compute and copy-out streams ordered by events.
+    peaks = load_peaks()
+    off = layer.offsets.cpu().numpy()
+    touched = int(np.count_nonzero(np.diff(off)))
+    ffn_ms = statistics.median(parts["ffn"])
+    R_nz = int(np.count_nonzero(layer.topk_w.cpu().numpy()))
+    flops = (R_nz + (T if shape.I_shared else 0)) * 6 * H * I
+    form = moe.moe_ffn_resolve_mode(T, K, E, args.mode)
+    form_kind = {moe.MOE_MODE_DECODE: "decode", moe.MOE_MODE_PREFILL: "prefill",
+                 moe.MOE_MODE_HYBRID: "hybrid"}[form]
+    roof = ffn_roofline(shape, form_kind, touched=touched, flops=flops, ffn_ms=ffn_ms, peaks=peaks)
+    if form_kind == "hybrid":
+        # The tensor-core share of the same call, for reference.
+        roof["flops"] = flops
+        roof["tflops"] = flops / (ffn_ms * 1e-3) / 1e12
+    if args.fused_router:
+        # The fused router's own roofline: a bf16 GEMM of 2 T H E flops (its
+        # top-K epilogue adds no HBM traffic beyond the ids and weights).
+        r_ms = statistics.median(parts["route"])
+        r_flops = 2.0 * T * H * E
+        r_ach = r_flops / (r_ms * 1e-3) / 1e12
+        roof["router"] = {"kernel": "moe_router (gate GEMM + top-K)", "bound": "tensor", "flops": r_flops,
+                          "achieved": r_ach, "peak": peaks["bf16"], "unit": "TFLOP/s",
+                          "frac": r_ach / peaks["bf16"]}
+    weights_gb = (touched if form_kind != "prefill" else E) * expert_bytes(H, I) / 1e9
+    rec = {"workload": shape.name, "value": job_tokens_per_s(T, world, t_max), "unit": UNIT,
+           "ms_per_step": t_max, "steps": steps, "windows": N_WINDOWS,
+           "window_ms_per_step": {"min": min(windows), "median": t_local, "max": max(windows)},
+           "spread": (max(windows) - min(windows)) / t_local,
+           "form": form_kind, "dtype": ARITHMETIC[form_kind][0], "arithmetic": ARITHMETIC[form_kind][1],
+           "l2": "inputs larger than L2 (%s expert weights %.2f GB > 126 MB)"
+                 % ("touched" if form_kind != "prefill" else "all", weights_gb),
+           "roofline": roof, "breakdown_ms": {k: statistics.median(v) for k, v in parts.items()},
+           "gpu_launches": layer.launches() * steps * N_WINDOWS,
+           "clocks": clk.summary(t_timed, t_done) if clk.summary(t_timed, t_done)["samples"]
+           else dict(clk.summary(t_warm, time.monotonic()), note="no sample inside the timed windows; "
+                     "samples from warm-up to the breakdown")}
+    e2e = None
+    if want_e2e:
+        e2e = measure_e2e(args, w, shape, layer, routed, shared, route_cfg, wr, x, logits, run, dev, world, stream)
+    del g, g2
+    return rec, e2e
+
+
+def measure_e2e(args, w, shape, layer, routed, shared, route_cfg, wr, x, logits, run, dev, world, stream):
+    """End to end through the public API with host buffers: every step copies
+    its x and logits in from pinned host memory and its output back out.  Two
+    sets of device buffers (a second layer object over the same weights) let
+    step i+1's input copy and step i-1's output copy overlap step i's compute:
+    copy-in, compute and copy-out streams ordered by events."""
+    import torch
+    import mixture_experts_ffn_sort_b200 as moe
+    T, K, H = shape.T, shape.K, shape.H
     xh = torch.from_numpy(w.x.view(np.int16)).view(torch.bfloat16).pin_memory()
     lh = torch.from_numpy(w.logits).pin_memory()
     oh = [torch.empty((T, H), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
@@ -433,12 +491,14 @@ def main():
     h2d, d2h = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
     in_ready, in_free, out_ready, out_free = ([torch.cuda.Event(), torch.cuda.Event()] for _ in range(4))
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    n_e2e = min(args.steps, 500)
+    n_e2e = min(args.steps * N_WINDOWS, 500)
     with torch.cuda.stream(stream):
         xs[1].copy_(xh)
         ls[1].copy_(lh)
         run(layers[1], xs[1], ls[1])  # first call of the second layer outside the timed region
-    barrier()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
     torch.cuda.synchronize(dev)
     e0.record(stream)
     h2d.wait_event(e0)
@@ -469,50 +529,82 @@ def main():
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / n_e2e, dev)
     for lay in layers:
         if lay.status.item() != 0:
-            raise RuntimeError("status word %d after the timed region" % lay.status.item())
+            raise RuntimeError("status word %d after the end-to-end run" % lay.status.item())
+    return {"value": job_tokens_per_s(T, world, e2e_ms), "unit": UNIT,
+            "h2d_bytes_per_step": x.numel() * 2 + (0 if args.fused_router else logits.numel() * 4),
+            "d2h_bytes_per_step": layer.out.numel() * 2, "steps": n_e2e}
 
-    peaks = load_peaks()
-    off = layer.offsets.cpu().numpy()
-    touched = int(np.count_nonzero(np.diff(off)))
-    ffn_ms = statistics.median(parts["ffn"])
-    R_nz = int(np.count_nonzero(layer.topk_w.cpu().numpy()))
-    flops = (R_nz + (T if shape.I_shared else 0)) * 6 * H * I
-    form = moe.moe_ffn_resolve_mode(T, K, E, args.mode)
-    decode_path = form in (moe.MOE_MODE_DECODE, moe.MOE_MODE_HYBRID)  # bound by the touched weights
-    roof = ffn_roofline(shape, form_kind="hybrid" if form == moe.MOE_MODE_HYBRID else
-                        ("decode" if decode_path else "prefill"), touched=touched, flops=flops, ffn_ms=ffn_ms,
-                        peaks=peaks)
-    if args.fused_router:
-        # The fused router's own roofline: a bf16 GEMM of 2 T H E flops (its
-        # top-K epilogue adds no HBM traffic beyond the ids and weights).
-        r_ms = statistics.median(parts["route"])
-        r_flops = 2.0 * T * H * E
-        r_ach = r_flops / (r_ms * 1e-3) / 1e12
-        roof["router"] = {"kernel": "moe_router (gate GEMM + top-K)", "bound": "tensor", "flops": r_flops,
-                          "achieved": r_ach, "peak": peaks["bf16_sus"], "unit": "TFLOP/s",
-                          "frac": r_ach / peaks["bf16_sus"]}
-    n_launch = layer.launches()
-    out = {"metric": METRIC, "value": job_tokens_per_s(T, world, t_max), "unit": UNIT, "n_gpus": world,
-           "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_max, "higher_is_better": True,
-           "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-           "config": dict(config_of(shape, args.router, args.fused_router), parallelism="replicas x%d" % world,
-                          l2="inputs larger than L2 (touched expert weights %.2f GB > 126 MB)"
-                             % (touched * expert_bytes(H, I) / 1e9) if decode_path else
-                             "inputs larger than L2 (expert weights %.2f GB > 126 MB)" % (E * expert_bytes(H, I) / 1e9),
-                          timing="CUDA events around %d %s of one step" % (
-                              args.steps, "eager launches" if args.eager else "CUDA-graph replays")),
-           "roofline": roof,
-           "breakdown_ms": {k: statistics.median(v) for k, v in parts.items()},
-           "e2e": {"value": job_tokens_per_s(T, world, e2e_ms), "unit": UNIT,
-                   "h2d_bytes_per_step": x.numel() * 2 + (0 if args.fused_router else logits.numel() * 4),
-                   "d2h_bytes_per_step": layer.out.numel() * 2},
-           "gpu_launches": n_launch * args.steps,
-           "clocks": clk.summary()}
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=None, help="replays per timed window (7 windows)")
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="decode", choices=wl.SHAPE_ORDER)
+    ap.add_argument("--extra-workloads", default=",".join(EXTRA_WORKLOADS),
+                    help="comma-separated workloads timed after the headline one (\"none\" for none)")
+    ap.add_argument("--mode", type=int, default=0, help="moe_expert_ffn mode: 0 AUTO, 1 DECODE, 2 PREFILL, 3 HYBRID")
+    ap.add_argument("--router", default="softmax", choices=sorted(wl.ROUTERS),
+                    help="routing variant: softmax top-k (moe_route) or a moe_route_ex preset")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--fused-router", action="store_true",
+                    help="route from x with the fused router (gate GEMM + top-K) instead of given logits")
+    ap.add_argument("--eager", action="store_true",
+                    help="launch every call directly instead of replaying CUDA graphs (for profilers)")
+    args = ap.parse_args()
+    shape = wl.SHAPES[args.workload]
+    rank, world, local = dist_env()
+
+    if args.impl == "reference":
+        if args.steps is None:
+            args.steps = 3
+        if rank == 0:
+            print(json.dumps(run_reference(args, shape)), flush=True)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    extras = [n for n in args.extra_workloads.split(",") if n and n != "none" and n != shape.name]
+    for n in extras:
+        if n not in wl.SHAPES:
+            raise SystemExit("unknown workload %r" % n)
+    steps_given = args.steps is not None
+    if not steps_given:
+        args.steps = DEFAULT_STEPS[shape.name]
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    with ClockSampler(local) as clk:
+        head, e2e = measure(args, shape, args.steps, dev, world, clk, want_e2e=True)
+        others = {}
+        for n in extras:
+            torch.cuda.empty_cache()
+            rec, _ = measure(args, wl.SHAPES[n], args.steps if steps_given else DEFAULT_STEPS[n], dev, world, clk,
+                             want_e2e=False)
+            others[n] = rec
+    out = {"metric": METRIC, "value": head["value"], "unit": UNIT, "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms_per_step"],
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": head["dtype"],
+           "data": "synthetic",
+           "config": config_of(shape, args.router, args.fused_router),
+           "parallelism": "replicas x%d" % world, "l2": head["l2"],
+           "timing": "median of %d windows of %d %s of one step (CUDA events on the launching stream, "
+                     "barrier and synchronize around each window, max over ranks)"
+                     % (N_WINDOWS, args.steps, "eager launches" if args.eager else "CUDA-graph replays"),
+           "window_ms_per_step": head["window_ms_per_step"], "spread": head["spread"],
+           "arithmetic": head["arithmetic"], "form": head["form"],
+           "roofline": head["roofline"], "breakdown_ms": head["breakdown_ms"],
+           "e2e": e2e, "gpu_launches": head["gpu_launches"], "clocks": head["clocks"],
+           "workloads": others}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(shape, args.router, args.fused_router)
     if rank == 0:
         print(json.dumps(out), flush=True)
-    del g, g2
     if world > 1:
         dist.destroy_process_group()
 

@@ -43,7 +43,8 @@
  *    default stream), never synchronises the host, and reads no device value
  *    back.  The first call of a process also does one-time host set-up (kernel
  *    attributes, driver entry points); make one call before capturing a CUDA
- *    graph, after which the calls may be captured.
+ *    graph, after which moe_route, moe_route_ex, moe_router, moe_sort,
+ *    moe_expert_ffn and moe_combine may be captured.
  *  - Return value: MOE_OK (0) or a negative moe_status.  On error nothing has
  *    been launched and moe_last_error() holds a message (thread-local, valid
  *    until the next call on the same thread).  MOE_ERR_CUDA reports a launch
@@ -112,8 +113,9 @@ typedef enum moe_status {
 /* Thread-local message describing the last error on this thread ("" if none). */
 MOE_API const char* moe_last_error(void);
 
-/* ABI version of this header (incremented on incompatible changes). */
-#define MOE_ABI_VERSION 1
+/* ABI version of this header (incremented on incompatible changes; 2: moe_combine
+ * takes a status word). */
+#define MOE_ABI_VERSION 2
 MOE_API int moe_abi_version(void);
 
 /* ---------------------------------------------------------------------------
@@ -224,6 +226,22 @@ MOE_API int moe_router(const uint16_t* x, int T, int H, const uint16_t* w_router
                        float* logits, int32_t* status, moe_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * moe_router_plan_check -- a host-only diagnostic with no counterpart in the
+ * pages: the launch plan moe_router would use for T tokens, width H and E
+ * experts (with at most kch_max 64-column chunks per pipeline stage), checked
+ * against the invariants the router kernel's indexing relies on.  Launches
+ * nothing and touches no GPU.
+ *   fields  host int32[9] or NULL: tiles, CTAs per cluster, experts per CTA,
+ *           stages, TMEM columns, staging row stride (floats), x rows per
+ *           tile, chunks per stage, dynamic shared memory bytes
+ * Returns MOE_OK, MOE_ERR_INVALID_ARG for arguments outside moe_router's
+ * limits (kch_max must be 1, 2 or 4), or MOE_ERR_UNSUPPORTED_SHAPE when the
+ * plan breaks an invariant (moe_last_error names the field); moe_router
+ * refuses such a plan the same way before launching.
+ * ------------------------------------------------------------------------- */
+MOE_API int moe_router_plan_check(int T, int H, int E, int kch_max, int32_t* fields);
+
+/* ---------------------------------------------------------------------------
  * moe_selftest_bounded_wait -- a diagnostic with no counterpart in the pages:
  * it makes the kernels' bounded wait run out on purpose, without a fault.
  *
@@ -266,23 +284,23 @@ MOE_API int moe_sort(const int32_t* topk_ids, int T, int K, int E, int32_t* expe
 /* ---------------------------------------------------------------------------
  * moe_sort_static_ws -- moe_sort for callers that cannot allocate device memory.
  *
- * The source paper has no counterpart of this call; it exists for callers that
- * may not call cudaMalloc or any allocating routine: plugins whose host
- * framework owns every device allocation, code that runs while a stream is
- * being captured into a CUDA graph (where allocation is not allowed), and
+ * The source paper has no counterpart of this call.  It exists for callers
+ * that may not call cudaMalloc or any allocating routine: plugins whose host
+ * framework owns every device allocation and hands out no scratch, and
  * processes held to a fixed device-memory budget.  It computes exactly what
  * moe_sort computes (same arguments, same outputs, bit for bit) but takes no
  * workspace: the scratch its multi-kernel path needs (one int32 counter per
  * expert per 2048-route chunk) lives in a statically allocated device array of
  * MOE_SORT_STATIC_WS_BYTES bytes inside the library, which every GPU that
  * loads the library holds until the process exits.  The call itself allocates
- * nothing.
+ * nothing (no cudaMalloc, cudaFree or allocating library routine).
  *  - Sizes whose scratch would exceed the array (E * ceil(T*K / 2048) * 4 >
  *    MOE_SORT_STATIC_WS_BYTES) are rejected with MOE_ERR_UNSUPPORTED_SHAPE and a
  *    message naming both byte counts; use moe_sort with a workspace for them.
  *  - The first call on a device looks up the array's device address (a host
- *    set-up step, with that device current).  Make that first call before
- *    capturing a stream into a CUDA graph.
+ *    set-up step, with that device current); so does the first call after the
+ *    device's context changed (a cudaDeviceReset, another context made
+ *    current).  Make that first call before any stream capture.
  *  - Every call shares the one array and leaves its contents behind.  Nothing
  *    in it needs to start at zero: each call overwrites every counter it reads.
  *    Calls that overlap on the GPU (on different streams without ordering, or
@@ -391,10 +409,13 @@ MOE_API int moe_expert_ffn(const uint16_t* x, int T, int H, int K, const moe_fp8
  * at the end.  Routes with inv_route = -1 add nothing.
  *   y_sorted  [T*K, H] bf16; inv_route [T*K] i32; y_shared [T, H] bf16 or NULL
  *   out       [T, H], bf16 (out_dtype MOE_OUT_BF16) or f32 (MOE_OUT_F32)
+ *   status    optional device int32 (4-byte aligned, may be NULL): an
+ *             inv_route entry outside [0, T*K) other than -1 is skipped (never
+ *             read out of bounds) and sets MOE_STATUS_BAD_MAP
  * Limits: H % 8 == 0, 1 <= K <= MOE_MAX_K.
  * ------------------------------------------------------------------------- */
 MOE_API int moe_combine(const uint16_t* y_sorted, const int32_t* inv_route, const uint16_t* y_shared,
-                int T, int K, int H, void* out, int out_dtype, moe_stream_t stream);
+                int T, int K, int H, void* out, int out_dtype, int32_t* status, moe_stream_t stream);
 
 #ifdef __cplusplus
 }

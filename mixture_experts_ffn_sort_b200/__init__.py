@@ -32,7 +32,7 @@ MOE_STATUS_BAD_ID, MOE_STATUS_BAD_MAP, MOE_STATUS_TIMEOUT = 1, 2, 4
 MOE_MAX_E, MOE_MAX_K = 1024, 32
 
 EXPORTED = ("moe_last_error", "moe_abi_version", "moe_route", "moe_route_ex", "moe_router", "moe_sort_workspace_bytes",
-            "moe_sort", "moe_selftest_bounded_wait",
+            "moe_sort", "moe_selftest_bounded_wait", "moe_router_plan_check",
             "moe_sort_static_ws", "moe_ffn_resolve_mode", "moe_ffn_workspace_bytes", "moe_expert_ffn", "moe_combine")
 
 
@@ -74,6 +74,8 @@ def lib() -> ctypes.CDLL:
             L.moe_route_ex.restype = I
             L.moe_router.argtypes = [P, I, I, P, I, I, ctypes.POINTER(_RouteConfig), P, P, P, P, P, P]
             L.moe_router.restype = I
+            L.moe_router_plan_check.argtypes = [I, I, I, I, P]
+            L.moe_router_plan_check.restype = I
             L.moe_selftest_bounded_wait.argtypes = [P, P, P]
             L.moe_selftest_bounded_wait.restype = I
             L.moe_route.restype = I
@@ -89,7 +91,7 @@ def lib() -> ctypes.CDLL:
             L.moe_ffn_workspace_bytes.restype = S
             L.moe_expert_ffn.argtypes = [P, I, I, I, P, P, P, P, P, P, P, I, P, S, P, P]
             L.moe_expert_ffn.restype = I
-            L.moe_combine.argtypes = [P, P, P, I, I, I, P, I, P]
+            L.moe_combine.argtypes = [P, P, P, I, I, I, P, I, P, P]
             L.moe_combine.restype = I
             _L = L
     return _L
@@ -287,15 +289,17 @@ def moe_expert_ffn(x: torch.Tensor, K: int, routed: Experts, expert_offsets: tor
 
 
 def moe_combine(y_sorted: torch.Tensor, inv_route: torch.Tensor, y_shared: Optional[torch.Tensor],
-                T: int, K: int, out_dtype: int = MOE_OUT_BF16, out=None, stream=None):
-    """-> out [T, H] (bf16 or f32)."""
-    _need_cuda(y_sorted, inv_route, y_shared)
+                T: int, K: int, out_dtype: int = MOE_OUT_BF16, out=None, stream=None,
+                status: Optional[torch.Tensor] = None):
+    """-> out [T, H] (bf16 or f32).  status: optional int32 device word that
+    receives MOE_STATUS_BAD_MAP for an out-of-range inv_route entry."""
+    _need_cuda(y_sorted, inv_route, y_shared, status)
     H = y_sorted.shape[1]
     if out is None:
         dt = torch.bfloat16 if out_dtype == MOE_OUT_BF16 else torch.float32
         out = torch.empty((T, H), dtype=dt, device=y_sorted.device)
     _check(lib().moe_combine(_ptr(y_sorted), _ptr(inv_route), _ptr(y_shared), T, K, H, _ptr(out),
-                             out_dtype, _stream(stream)))
+                             out_dtype, _ptr(status), _stream(stream)))
     return out
 
 
@@ -368,7 +372,7 @@ class MoEFFN:
         moe_expert_ffn(x, self.K, self.routed, self.offsets, self.sorted_route, self.topk_w, self.shared,
                        self.mode, self.status, self.y_sorted, self.y_shared, self.ffn_ws, stream=stream)
         moe_combine(self.y_sorted, self.inv_route, self.y_shared, self.T, self.K, self.out_dtype, self.out,
-                    stream=stream)
+                    stream=stream, status=self.status)
         return self.out
 
     __call__ = forward

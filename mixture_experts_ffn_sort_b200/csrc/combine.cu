@@ -5,7 +5,9 @@
 // FP32 route reduction of the aiter gfx950 prefill PR and the NKI Top-K Reduce
 // kernel: out[t] = sum_j y_sorted[inv_route[t*K + j]] (+ y_shared[t]), summed
 // in fp32 in slot order, rounded once.  Each thread owns 8 consecutive
-// columns of one token and reads them with 16-byte loads.
+// columns of one token and reads them with 16-byte loads.  A position outside
+// [0, T*K) other than -1 is a corrupt map: that term is skipped (never read
+// out of bounds) and MOE_STATUS_BAD_MAP is OR-ed into the status word.
 #include "device_common.cuh"
 #include "launch.h"
 
@@ -26,9 +28,12 @@ template <bool OUT_F32>
 __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict__ y_sorted,
                                                       const int32_t* __restrict__ inv_route,
                                                       const uint16_t* __restrict__ y_shared,
-                                                      int T, int K, int H, void* __restrict__ out) {
+                                                      int T, int K, int H, void* __restrict__ out,
+                                                      int32_t* __restrict__ status) {
     const int chunks = H >> 3;
     const long total = static_cast<long>(T) * chunks;
+    const long R = static_cast<long>(T) * K;
+    bool bad = false;
     for (long idx = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
          idx += static_cast<long>(gridDim.x) * blockDim.x) {
         const int t = static_cast<int>(idx / chunks);
@@ -40,8 +45,13 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict
         for (int j0 = 0; j0 < K; j0 += 8) {
             int32_t p[8];
 #pragma unroll
-            for (int jj = 0; jj < 8; ++jj)
+            for (int jj = 0; jj < 8; ++jj) {
                 p[jj] = j0 + jj < K ? __ldg(inv_route + static_cast<size_t>(t) * K + j0 + jj) : -1;
+                if (p[jj] >= R || p[jj] < -1) {
+                    bad = true;
+                    p[jj] = -1;
+                }
+            }
             uint4 v[8];
 #pragma unroll
             for (int jj = 0; jj < 8; ++jj)
@@ -69,23 +79,24 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict
             reinterpret_cast<uint4*>(static_cast<uint16_t*>(out) + static_cast<size_t>(t) * H)[c] = r;
         }
     }
+    if (bad) report_status(status, MOE_STATUS_BAD_MAP);
 }
 
 }  // namespace
 
 cudaError_t launch_combine(const uint16_t* y_sorted, const int32_t* inv_route,
                            const uint16_t* y_shared, int T, int K, int H, void* out, int out_f32,
-                           cudaStream_t stream) {
+                           int32_t* status, cudaStream_t stream) {
     const long total = static_cast<long>(T) * (H >> 3);
     const int threads = 256;
     long blocks = (total + threads - 1) / threads;
     if (blocks > 148L * 64) blocks = 148L * 64;
     if (out_f32)
         combine_kernel<true><<<static_cast<int>(blocks), threads, 0, stream>>>(y_sorted, inv_route,
-                                                                                y_shared, T, K, H, out);
+                                                                                y_shared, T, K, H, out, status);
     else
         combine_kernel<false><<<static_cast<int>(blocks), threads, 0, stream>>>(y_sorted, inv_route,
-                                                                                 y_shared, T, K, H, out);
+                                                                                 y_shared, T, K, H, out, status);
     return cudaGetLastError();
 }
 

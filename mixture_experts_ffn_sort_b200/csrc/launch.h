@@ -36,7 +36,7 @@ cudaError_t launch_sort(const int32_t* ids, long R, int E, int32_t* offsets, int
 // ---------------------------------------------------------------- combine
 cudaError_t launch_combine(const uint16_t* y_sorted, const int32_t* inv_route,
                            const uint16_t* y_shared, int T, int K, int H, void* out, int out_f32,
-                           cudaStream_t stream);
+                           int32_t* status, cudaStream_t stream);
 
 // ---------------------------------------------------------------- expert FFN (decode)
 // One projection set of experts as the kernels see it.

@@ -189,13 +189,17 @@ int moe_router(const uint16_t* x, int T, int H, const uint16_t* w_router, int E,
         return fail(MOE_ERR_INVALID_ARG, "moe_router: x, w_router, topk_ids and topk_w must not be NULL");
     if (!aligned16(x) || !aligned16(w_router) || !aligned16(topk_ids) || !aligned16(topk_w) || !aligned16(logits) ||
         (status && (reinterpret_cast<uintptr_t>(status) & 3)))
-        return fail(MOE_ERR_MISALIGNED, "moe_router: tensor bases must be 16-byte aligned");
+        return fail(MOE_ERR_MISALIGNED, "moe_router: tensor bases must be 16-byte aligned and status 4-byte aligned");
     const moe::RouteCfg rc_dev = cfg ? moe::RouteCfg{cfg->score, cfg->sel_bias, cfg->n_group, cfg->topk_group,
                                                      cfg->renormalize, cfg->scaling}
                                      : moe::RouteCfg{MOE_SCORE_SOFTMAX, nullptr, 1, 1, 1, 1.f};
     // Stages of several 64-column chunks (3-D boxes); one chunk if the
     // driver declines the 3-D view.
     moe::RouterPlan plan = moe::plan_router(T, H, E, 4);
+    if (const char* field = moe::router_plan_violation(plan, H, E))
+        return fail(MOE_ERR_UNSUPPORTED_SHAPE,
+                    "moe_router: the launch plan for T=%d, H=%d, E=%d breaks the kernel's invariant on '%s'", T, H,
+                    E, field);
     CUtensorMap tx, tw;
     cudaError_t e = cudaSuccess;
     for (int attempt = 0; attempt < 2; ++attempt) {
@@ -214,10 +218,31 @@ int moe_router(const uint16_t* x, int T, int H, const uint16_t* w_router, int E,
         }
         if (e == cudaSuccess || plan.kch == 1) break;
         plan = moe::plan_router(T, H, E, 1);
+        if (const char* field = moe::router_plan_violation(plan, H, E))
+            return fail(MOE_ERR_UNSUPPORTED_SHAPE,
+                        "moe_router: the launch plan for T=%d, H=%d, E=%d breaks the kernel's invariant on '%s'", T,
+                        H, E, field);
     }
     if (e != cudaSuccess) return cuda_fail(e, "moe_router tensor maps");
     e = moe::launch_router(plan, tx, tw, T, H, E, K, rc_dev, zero_mask, topk_ids, topk_w, logits, status, stream);
     return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_router launch");
+}
+
+int moe_router_plan_check(int T, int H, int E, int kch_max, int32_t* fields) {
+    g_err.clear();
+    if (T < 1 || H < 64 || H % 64 || E < 1 || E > MOE_ROUTER_MAX_E || (kch_max != 1 && kch_max != 2 && kch_max != 4))
+        return fail(MOE_ERR_INVALID_ARG, "moe_router_plan_check: T=%d, H=%d, E=%d, kch_max=%d out of range", T, H, E,
+                    kch_max);
+    const moe::RouterPlan p = moe::plan_router(T, H, E, kch_max);
+    if (fields) {
+        const int32_t v[9] = {p.tiles, p.cn, p.ne, p.stages, p.tmem_cols, p.S, p.xrows, p.kch,
+                              static_cast<int32_t>(p.smem)};
+        for (int i = 0; i < 9; ++i) fields[i] = v[i];
+    }
+    if (const char* field = moe::router_plan_violation(p, H, E))
+        return fail(MOE_ERR_UNSUPPORTED_SHAPE, "moe_router_plan_check: T=%d, H=%d, E=%d: invariant on '%s' broken", T,
+                    H, E, field);
+    return MOE_OK;
 }
 
 size_t moe_sort_workspace_bytes(int T, int K, int E) {
@@ -236,7 +261,7 @@ int moe_sort(const int32_t* topk_ids, int T, int K, int E, int32_t* expert_offse
         return fail(MOE_ERR_INVALID_ARG, "moe_sort: topk_ids, sorted_route and inv_route must not be NULL");
     if (!aligned16(topk_ids) || !aligned16(expert_offsets) || !aligned16(sorted_route) ||
         !aligned16(inv_route) || !aligned16(workspace) || (status && (reinterpret_cast<uintptr_t>(status) & 3)))
-        return fail(MOE_ERR_MISALIGNED, "moe_sort: tensor bases must be 16-byte aligned");
+        return fail(MOE_ERR_MISALIGNED, "moe_sort: tensor bases must be 16-byte aligned and status 4-byte aligned");
     const long R = static_cast<long>(T) * K;
     const size_t need = moe::sort_workspace_bytes(R, E);
     if (workspace_bytes < need || (need && !workspace))
@@ -362,7 +387,7 @@ int moe_expert_ffn(const uint16_t* x, int T, int H, int K, const moe_fp8_experts
 }
 
 int moe_combine(const uint16_t* y_sorted, const int32_t* inv_route, const uint16_t* y_shared, int T,
-                int K, int H, void* out, int out_dtype, moe_stream_t stream) {
+                int K, int H, void* out, int out_dtype, int32_t* status, moe_stream_t stream) {
     g_err.clear();
     if (T < 0 || T > MOE_MAX_T) return fail(MOE_ERR_INVALID_ARG, "moe_combine: T=%d out of range", T);
     if (K < 1 || K > MOE_MAX_K) return fail(MOE_ERR_INVALID_ARG, "moe_combine: K=%d must be in 1..=%d", K, MOE_MAX_K);
@@ -372,10 +397,12 @@ int moe_combine(const uint16_t* y_sorted, const int32_t* inv_route, const uint16
     if (T == 0) return MOE_OK;
     if (!y_sorted || !inv_route || !out)
         return fail(MOE_ERR_INVALID_ARG, "moe_combine: y_sorted, inv_route and out must not be NULL");
-    if (!aligned16(y_sorted) || !aligned16(inv_route) || !aligned16(y_shared) || !aligned16(out))
-        return fail(MOE_ERR_MISALIGNED, "moe_combine: tensor bases must be 16-byte aligned");
+    if (!aligned16(y_sorted) || !aligned16(inv_route) || !aligned16(y_shared) || !aligned16(out) ||
+        (reinterpret_cast<uintptr_t>(status) & 3))
+        return fail(MOE_ERR_MISALIGNED,
+                    "moe_combine: tensor bases must be 16-byte aligned and status 4-byte aligned");
     cudaError_t e = moe::launch_combine(y_sorted, inv_route, y_shared, T, K, H, out,
-                                        out_dtype == MOE_OUT_F32, stream);
+                                        out_dtype == MOE_OUT_F32, status, stream);
     return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_combine launch");
 }
 

@@ -212,7 +212,10 @@ __device__ __forceinline__ void route_token(const float* lg, int t, int E, int K
             const uint32_t kmax = __reduce_max_sync(full, h0);
             int e = static_cast<int>(
                 __reduce_min_sync(full, h0 == kmax && kmax ? static_cast<uint32_t>(lane + 32 * i0) : 0xffffffffu));
-            if (e >= E) e = E - 1;  // only reachable with NaN logits (unspecified ids)
+            // With no candidate left (kmax == 0) the min's sentinel casts to -1.
+            // That needs fewer than K nonzero keys, i.e. NaN logits whose key is 0
+            // (sign bit set); such a token's ids are unspecified but stay in [0, E).
+            if (e < 0 || e >= E) e = E - 1;
             if (lane == (e & 31)) {
                 h0 = h1; i0 = i1; h1 = h2; i1 = i2; h2 = h3; i2 = i3; h3 = 0u;
             }
@@ -236,7 +239,7 @@ __device__ __forceinline__ void route_token(const float* lg, int t, int E, int K
             const uint32_t kmax = __reduce_max_sync(full, best);
             int e = static_cast<int>(
                 __reduce_min_sync(full, best == kmax && best ? static_cast<uint32_t>(lane + 32 * bi) : 0xffffffffu));
-            if (e >= E) e = E - 1;
+            if (e < 0 || e >= E) e = E - 1;
             const int slot = e >> 5;
             if (lane == (e & 31)) {
 #pragma unroll

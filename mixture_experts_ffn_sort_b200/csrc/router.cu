@@ -249,6 +249,25 @@ RouterPlan plan_router(int T, int H, int E, int kch_max) {
     return p;
 }
 
+// The plan's invariants, which the kernel's indexing relies on: a cluster of
+// at most 8 CTAs splitting 128 tokens evenly, an MMA N of 16..256 in steps of
+// 16 within the TMEM allocation that covers the cluster's share of E, at
+// least two stages, chunks that divide H, x rows a multiple of 8 within a
+// tile, and shared memory within one CTA's limit.  Returns the name of the
+// first field that breaks one, or nullptr.
+const char* router_plan_violation(const RouterPlan& p, int H, int E) {
+    if (p.cn < 1 || p.cn > 8 || kTileM % p.cn) return "cn";
+    if (p.ne < 16 || p.ne > 256 || p.ne % 16 || static_cast<long>(p.ne) * p.cn < E) return "ne";
+    if (p.tmem_cols < 32 || p.tmem_cols > 512 || (p.tmem_cols & (p.tmem_cols - 1)) || p.ne > p.tmem_cols)
+        return "tmem_cols";
+    if (p.stages < 2 || p.stages > kMaxStages) return "stages";
+    if (p.kch < 1 || (H / kKStage) % p.kch) return "kch";
+    if (p.xrows < 8 || p.xrows > kTileM || p.xrows % 8) return "xrows";
+    if (p.S < E + 4 || p.S % 4) return "S";
+    if (p.smem > 227 * 1024) return "smem";
+    return nullptr;
+}
+
 cudaError_t launch_router(const RouterPlan& p, const CUtensorMap& tx, const CUtensorMap& tw, int T, int H, int E,
                           int K, const RouteCfg& cfg, const uint8_t* zero_mask, int32_t* ids, float* w,
                           float* logits, int32_t* status, cudaStream_t stream) {
@@ -270,13 +289,7 @@ cudaError_t launch_router(const RouterPlan& p, const CUtensorMap& tx, const CUte
     a.w = w;
     a.logits = logits;
     a.status = status;
-    // The plan's invariants, which the kernel's indexing relies on: a cluster
-    // of at most 8 CTAs splitting 128 tokens evenly, an MMA N of 16..256 in
-    // steps of 16 within the TMEM allocation, at least two stages, chunks that
-    // divide H, and shared memory within one CTA's limit.
-    if (p.cn < 1 || p.cn > 8 || kTileM % p.cn || p.ne < 16 || p.ne > 256 || p.ne % 16 || p.ne > p.tmem_cols ||
-        p.stages < 2 || p.stages > kMaxStages || p.kch < 1 || (H / kKStage) % p.kch || p.smem > 227 * 1024)
-        return cudaErrorInvalidConfiguration;
+    if (router_plan_violation(p, H, E)) return cudaErrorInvalidConfiguration;
     const int grid = p.tiles * p.cn;
     const bool computed = cfg.bias != nullptr || cfg.n_group > 1;
 #define MOE_ROUTER_CASE(EPL)                                                                    \

@@ -14,6 +14,8 @@ struct RouterPlan {
 };
 // kch: 64-column chunks per K stage (1, 2 or 4; H / 64 a multiple of it).
 RouterPlan plan_router(int T, int H, int E, int kch_max);
+// Name of the first plan field that breaks the kernel's indexing invariants, or nullptr.
+const char* router_plan_violation(const RouterPlan& p, int H, int E);
 // x [rows, cols] bf16 viewed as (64 columns, rows, cols / 64 chunks), box
 // 64 x box_rows x box_chunks, 128-byte swizzle (cols a multiple of 64).
 cudaError_t make_tmap_bf16_kchunks(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,

@@ -4,8 +4,10 @@
 // For callers that cannot allocate device memory, the sort's scratch (the
 // per-chunk expert counters of its multi-kernel path) lives in a file-scope
 // __device__ array instead of a caller-provided workspace.  Its device address
-// is looked up once per device with cudaGetSymbolAddress; the array's host-side
-// name is only a stand-in and is never passed to a kernel.
+// is looked up with cudaGetSymbolAddress once per device and context (the
+// first call on a device, or the first after that device's context was
+// replaced, e.g. by cudaDeviceReset); the array's host-side name is only a
+// stand-in and is never passed to a kernel.
 #include <stdio.h>
 
 #include <mutex>
@@ -25,7 +27,12 @@ __device__ __align__(256) unsigned char g_sort_scratch[kScratchBytes];
 
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
-void* g_scratch_ptr[kMaxDevices];
+// Per device: the context the address was looked up in, and the address.
+struct ScratchSlot {
+    CUcontext ctx;
+    void* ptr;
+};
+ScratchSlot g_slot[kMaxDevices];
 
 int err(int code, const char* fmt, long a = 0, long b = 0) {
     char buf[256];
@@ -33,22 +40,49 @@ int err(int code, const char* fmt, long a = 0, long b = 0) {
     return moe::api_error(code, buf);
 }
 
-// Device address of g_sort_scratch on the current device (set up on first use).
+// The driver's cuCtxGetCurrent, fetched through the runtime (the library does
+// not link libcuda); NULL if the driver does not provide it.
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+CtxGetCurrentFn ctx_get_current() {
+    static std::once_flag once;
+    static CtxGetCurrentFn fn = nullptr;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<CtxGetCurrentFn>(p);
+    });
+    return fn;
+}
+
+CUcontext current_context() {
+    CUcontext c = nullptr;
+    CtxGetCurrentFn fn = ctx_get_current();
+    if (!fn || fn(&c) != CUDA_SUCCESS) return nullptr;
+    return c;
+}
+
+// Device address of g_sort_scratch on the current device, looked up again
+// whenever the current context is not the one of the cached address.
 int scratch_address(void** out) {
     int dev = -1;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return moe::api_error(MOE_ERR_CUDA, cudaGetErrorString(e));
     if (dev < 0 || dev >= kMaxDevices) return err(MOE_ERR_CUDA, "moe_sort_static_ws: device %ld out of range", dev);
     std::lock_guard<std::mutex> lock(g_mu);
-    if (!g_scratch_ptr[dev]) {
+    ScratchSlot& slot = g_slot[dev];
+    const CUcontext ctx = current_context();
+    if (!slot.ptr || !ctx || slot.ctx != ctx) {
         void* p = nullptr;
         e = cudaGetSymbolAddress(&p, g_sort_scratch);
         if (e != cudaSuccess || !p)
             return moe::api_error(MOE_ERR_CUDA, e != cudaSuccess ? cudaGetErrorString(e)
                                                                  : "cudaGetSymbolAddress returned NULL");
-        g_scratch_ptr[dev] = p;
+        slot.ptr = p;
+        slot.ctx = current_context();  // the lookup has made the device's context current
     }
-    *out = g_scratch_ptr[dev];
+    *out = slot.ptr;
     return MOE_OK;
 }
 
@@ -68,7 +102,8 @@ extern "C" MOE_API int moe_sort_static_ws(const int32_t* topk_ids, int T, int K,
     const uintptr_t mis = reinterpret_cast<uintptr_t>(topk_ids) | reinterpret_cast<uintptr_t>(expert_offsets) |
                           reinterpret_cast<uintptr_t>(sorted_route) | reinterpret_cast<uintptr_t>(inv_route);
     if ((mis & 15u) || (reinterpret_cast<uintptr_t>(status) & 3u))
-        return err(MOE_ERR_MISALIGNED, "moe_sort_static_ws: tensor bases must be 16-byte aligned");
+        return err(MOE_ERR_MISALIGNED,
+                   "moe_sort_static_ws: tensor bases must be 16-byte aligned and status 4-byte aligned");
     const long R = static_cast<long>(T) * K;
     const size_t need = moe::sort_workspace_bytes(R, E);
     if (need > kScratchBytes)

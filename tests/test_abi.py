@@ -44,7 +44,7 @@ def test_no_other_symbols_exported(L):
 
 
 def test_abi_version(L):
-    assert L.moe_abi_version() == 1
+    assert L.moe_abi_version() == 2
 
 
 def test_workspace_queries(L):
@@ -179,10 +179,11 @@ def test_expert_ffn_checks(L):
 
 
 def test_combine_checks(L):
-    assert L.moe_combine(P(16), P(16), None, 4, 2, 12, P(16), 0, None) == moe.MOE_ERR_UNSUPPORTED_SHAPE
-    assert L.moe_combine(P(16), P(16), None, 4, 2, 16, P(16), 3, None) == moe.MOE_ERR_INVALID_ARG
-    assert L.moe_combine(P(16), P(16), P(40), 4, 2, 16, P(16), 0, None) == moe.MOE_ERR_MISALIGNED
-    assert L.moe_combine(None, None, None, 0, 2, 16, None, 0, None) == moe.MOE_OK
+    assert L.moe_combine(P(16), P(16), None, 4, 2, 12, P(16), 0, None, None) == moe.MOE_ERR_UNSUPPORTED_SHAPE
+    assert L.moe_combine(P(16), P(16), None, 4, 2, 16, P(16), 3, None, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_combine(P(16), P(16), P(40), 4, 2, 16, P(16), 0, None, None) == moe.MOE_ERR_MISALIGNED
+    assert L.moe_combine(P(16), P(16), None, 4, 2, 16, P(16), 0, P(18), None) == moe.MOE_ERR_MISALIGNED
+    assert L.moe_combine(None, None, None, 0, 2, 16, None, 0, None, None) == moe.MOE_OK
 
 
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
@@ -223,3 +224,33 @@ def test_selftest_bounded_wait_checks(L):
     assert L.moe_selftest_bounded_wait(P(16), None, None) == moe.MOE_ERR_INVALID_ARG
     assert L.moe_selftest_bounded_wait(P(0x1002), P(16), None) == moe.MOE_ERR_MISALIGNED
     assert L.moe_selftest_bounded_wait(P(16), P(0x1004), None) == moe.MOE_ERR_MISALIGNED
+
+
+def test_router_plan_invariants_hold_over_a_wide_grid(L):
+    """moe_router's launch plan satisfies the kernel's indexing invariants for
+    every valid size: H in steps of 64 up to the limit, E from 1 to 512, batch
+    sizes below, at and above one 128-token tile and up to a full wave, and
+    both chunking limits.  Host only: the plan is computed and checked, nothing
+    is launched."""
+    fields = (ctypes.c_int32 * 9)()
+    bad = []
+    for kch in (1, 4):
+        for T in (1, 7, 8, 100, 127, 128, 129, 1000, 8192, 32768):
+            for H in range(64, 16384 + 1, 64):
+                for E in range(1, 513):
+                    if L.moe_router_plan_check(T, H, E, kch, fields) != moe.MOE_OK:
+                        bad.append((T, H, E, kch, L.moe_last_error().decode()))
+                        if len(bad) > 5:
+                            break
+    assert not bad, bad
+    # The fields are what the kernel is launched with.
+    assert L.moe_router_plan_check(8192, 4096, 512, 1, fields) == moe.MOE_OK
+    tiles, cn, ne = fields[0], fields[1], fields[2]
+    assert tiles == 64 and cn * ne >= 512 and ne % 16 == 0
+
+
+def test_router_plan_check_rejects_bad_arguments(L):
+    assert L.moe_router_plan_check(0, 128, 8, 1, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_router_plan_check(4, 100, 8, 1, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_router_plan_check(4, 128, 513, 1, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_router_plan_check(4, 128, 8, 3, None) == moe.MOE_ERR_INVALID_ARG

@@ -3,8 +3,10 @@
 Routing ids and the sort maps must match bit for bit; route weights within
 1e-5 relative; FFN outputs within rel-L2 <= 5e-3 and max-abs <= 1e-2 *
 max|oracle| + 1e-3.  The five workloads run in the launch configuration the
-benchmark uses (AUTO mode) and the FFN in both of its forms; the two largest
-compare a seeded sample of rows.
+benchmark uses (AUTO mode) and the FFN in each of its forms; the first four
+are compared on every row and token, the largest (32768 tokens at width
+8192) on every routing and sort output and on a seeded sample of 2048 tokens
+and 2048 sorted rows plus every expert's first row.
 """
 import numpy as np
 import pytest
@@ -20,8 +22,8 @@ from _gpu_util import (W_ATOL, W_RTOL, DeviceWorkload, assert_moe_close, bf16_nu
 pytestmark = pytest.mark.gpu
 
 ALL = wl.SHAPE_ORDER
-FULL = {"tiny", "decode", "decode_skew"}   # compared on every row
-SAMPLE_ROWS = 256
+FULL = {"tiny", "decode", "decode_skew", "prefill"}   # compared on every row
+SAMPLE_ROWS = 2048
 MODES = [moe.MOE_MODE_DECODE, moe.MOE_MODE_PREFILL, moe.MOE_MODE_HYBRID]
 
 
@@ -96,12 +98,13 @@ def test_expert_ffn(cfg, mode):
     if cfg in FULL:
         ref = oracle_full(cfg)["y_sorted"]
         assert_moe_close(y, ref, "y_sorted")
+        if w.shared is not None:
+            assert_moe_close(ys, oracle_full(cfg)["y_shared"], "y_shared")
     else:
-        pos = np.unique(np.concatenate([sample_tokens(R, SAMPLE_ROWS, seed=1), m["offsets"][1:-1].clip(0, R - 1)]))
-        pos = pos[:SAMPLE_ROWS * 2]
+        pos = np.unique(np.concatenate([sample_tokens(R, SAMPLE_ROWS, seed=1), m["offsets"][:-1].clip(0, R - 1)]))
         assert_moe_close(to_f64(y[torch.from_numpy(pos).long().cuda()]), oracle_y_rows(w, m, pos), "y_sorted rows")
         if w.shared is not None:
-            tk = sample_tokens(w.shape.T, 64, seed=2)
+            tk = sample_tokens(w.shape.T, 256, seed=2)
             ref = oracle.expert_rows(w.x, w.shared, 0, tk)
             assert_moe_close(to_f64(ys[torch.from_numpy(tk).long().cuda()]), ref, "y_shared rows")
 
@@ -115,7 +118,7 @@ def test_pipeline(cfg):
     if cfg in FULL:
         assert_moe_close(out, oracle_full(cfg)["out"], "out")
     else:
-        tk = sample_tokens(w.shape.T, 128, seed=3)
+        tk = sample_tokens(w.shape.T, SAMPLE_ROWS, seed=3)
         ref = oracle.moe_tokens(w.x, w.logits, w.shape.K, w.routed, w.shared, w.zero_mask, tokens=tk)
         assert_moe_close(to_f64(out[torch.from_numpy(tk).long().cuda()]), ref, "out rows")
 
@@ -274,6 +277,32 @@ def test_combine_step(K, shared):
     assert np.all(np.abs(g32 - ref) <= bound)
     g16 = to_f64(o16)
     assert np.all(np.abs(g16 - ref) <= 2.0 ** -8 * np.abs(ref) + 2 * bound)
+
+
+def test_combine_skips_and_flags_corrupt_positions():
+    """inv_route entries outside [0, T*K) (other than -1) are skipped, never
+    read, and set MOE_STATUS_BAD_MAP; the rest sums as if they were -1."""
+    T, K, E, H = 100, 4, 8, 64
+    ids = wl.random_ids(T, K, E, seed=31)
+    off, sr, inv, _ = oracle.sort(ids, E)
+    ys = wl.random_rows_bf16(T * K, H, seed=31)
+    bad = inv.copy()
+    bad[5] = T * K                 # one past the end
+    bad[17] = 1 << 30              # far out of range
+    bad[42] = -3                   # negative, not the skip marker
+    clean = bad.copy()
+    clean[[5, 17, 42]] = -1
+    ref = oracle.combine(oracle.bf16_array(ys), clean, None, T, K)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    o32 = moe.moe_combine(bf16_tensor(ys), dev(bad), None, T, K, moe.MOE_OUT_F32, status=status)
+    torch.cuda.synchronize()
+    assert status.item() & moe.MOE_STATUS_BAD_MAP
+    terms = oracle.combine(np.abs(oracle.bf16_array(ys)), clean, None, T, K)
+    assert np.all(np.abs(to_f64(o32) - ref) <= (K + 2) * 2.0 ** -24 * terms)
+    status.zero_()
+    moe.moe_combine(bf16_tensor(ys), dev(inv), None, T, K, moe.MOE_OUT_F32, status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
 
 
 def test_outputs_fully_written():

@@ -1,6 +1,8 @@
 """Parity of the tcgen05 (PREFILL) expert-FFN kernels with the CPU oracle on
-small inputs: tile boundaries of the 256-row token tiles, several H and I,
-the shared expert, and agreement of both modes with the oracle."""
+small inputs: boundaries of the 192-row token tiles (one expert receiving
+exactly 191, 192, 193, 383, 384, 385, ... rows) in the PREFILL and HYBRID
+forms, several H and I, the shared expert, and agreement of every form with
+the oracle."""
 import numpy as np
 import pytest
 import torch
@@ -40,15 +42,24 @@ def test_prefill_tiny_single_expert():
     assert_moe_close(y, oracle.ffn_sorted(x, K, ex, off, sr, wt), "y_sorted")
 
 
-@pytest.mark.parametrize("n_hot", [1, 15, 16, 17, 255, 256, 257, 300, 513])
-def test_prefill_token_tile_boundaries(n_hot):
+# The prefill kernels' token tile is 192 rows (the MMA's N); an expert's rows
+# are split into tiles of 192 and a ragged last tile.
+TILE_ROWS = 192
+
+
+@pytest.mark.parametrize("n_hot", [1, 15, 16, 17, 31, 32, 33, TILE_ROWS - 1, TILE_ROWS, TILE_ROWS + 1, 255, 256, 257,
+                                   2 * TILE_ROWS - 1, 2 * TILE_ROWS, 2 * TILE_ROWS + 1, 513, 3 * TILE_ROWS + 1])
+@pytest.mark.parametrize("mode", [moe.MOE_MODE_PREFILL, moe.MOE_MODE_HYBRID])
+def test_prefill_token_tile_boundaries(n_hot, mode):
+    """The hot expert receives exactly n_hot rows (slot 0 of every token)."""
     T, H, I, E, K = n_hot, 256, 128, 5, 2
     ex = wl.draw_experts(3, 61, E, I, H, 0.05, threads=2)
     x = wl.random_rows_bf16(T, H, seed=n_hot)
     ids = wl.skewed_ids(T, K, E, hot=1, seed=n_hot)
     off, sr, inv, _ = oracle.sort(ids, E)
+    assert off[2] - off[1] == n_hot
     wt = np.random.default_rng(n_hot).random((T, K)).astype(np.float32).astype(np.float64)
-    y, _ = _ffn(x, K, ex, off, sr, wt, moe.MOE_MODE_PREFILL)
+    y, _ = _ffn(x, K, ex, off, sr, wt, mode)
     assert_moe_close(y, oracle.ffn_sorted(x, K, ex, off, sr, wt), "y_sorted")
 
 

@@ -1,12 +1,14 @@
 """moe_sort_static_ws: the route sort for callers that cannot allocate.
 
 Some callers may not allocate device memory at all: a plugin whose host
-framework owns every allocation, code running while a stream is captured into
-a CUDA graph, or a process held to a fixed memory budget.  moe_sort_static_ws
-serves them by keeping the sort's scratch in a device array inside the library.
-These tests call it through the C ABI and check that it returns exactly what
-moe_sort (with a caller-provided workspace) returns, on two calls in a row,
-with sizes that use the scratch (more than 16384 routes) and one that does not.
+framework owns every device allocation and hands out no scratch, or a process
+held to a fixed device-memory budget.  moe_sort_static_ws serves them by
+keeping the sort's scratch in a device array inside the library.  These tests
+call it through the C ABI, on two calls in a row, with sizes that use the
+scratch (more than 16384 routes) and one that does not, and check that it
+returns exactly what moe_sort (with a caller-provided workspace) and the
+oracle's counting sort return, and that a call changes neither torch's
+allocated bytes nor the device's free memory.
 """
 import ctypes
 
@@ -15,6 +17,7 @@ import pytest
 import torch
 
 import mixture_experts_ffn_sort_b200 as moe
+import oracle
 from mixture_experts_ffn_sort_b200 import workloads as wl
 
 pytestmark = pytest.mark.gpu
@@ -24,11 +27,16 @@ def _p(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-def static_sort(ids: torch.Tensor, E: int, status: torch.Tensor):
-    T, K = ids.shape
+def _buffers(T, K, E):
     off = torch.full((E + 1,), -7, dtype=torch.int32, device="cuda")
     sr = torch.full((T * K,), -7, dtype=torch.int32, device="cuda")
     inv = torch.full((T * K,), -7, dtype=torch.int32, device="cuda")
+    return off, sr, inv
+
+
+def static_sort(ids: torch.Tensor, E: int, status: torch.Tensor, bufs):
+    T, K = ids.shape
+    off, sr, inv = bufs
     rc = moe.lib().moe_sort_static_ws(_p(ids), T, K, E, _p(off), _p(sr), _p(inv), _p(status),
                                       ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
     assert rc == moe.MOE_OK, moe.lib().moe_last_error().decode()
@@ -36,16 +44,34 @@ def static_sort(ids: torch.Tensor, E: int, status: torch.Tensor):
 
 
 @pytest.mark.parametrize("T,K,E", [(4096, 8, 256), (40000, 10, 512), (100, 4, 16)])
-def test_static_scratch_sort_matches_moe_sort(T, K, E):
+def test_static_scratch_sort_matches_moe_sort_and_oracle(T, K, E):
     for call in range(2):                       # two calls in a row share the scratch array
-        ids = torch.from_numpy(wl.random_ids(T, K, E, seed=1000 * call + T)).cuda()
+        ids_h = wl.random_ids(T, K, E, seed=1000 * call + T)
+        ids = torch.from_numpy(ids_h).cuda()
         status = torch.zeros(1, dtype=torch.int32, device="cuda")
-        got = static_sort(ids, E, status)
+        got = static_sort(ids, E, status, _buffers(T, K, E))
         ref = moe.moe_sort(ids, E)
         torch.cuda.synchronize()
         assert status.item() == 0
-        for name, a, b in zip(("offsets", "sorted_route", "inv_route"), got, ref):
-            assert torch.equal(a, b), "call %d: %s differs" % (call, name)
+        o = oracle.sort(ids_h, E)
+        for name, a, b, c in zip(("offsets", "sorted_route", "inv_route"), got, ref, o):
+            assert torch.equal(a, b), "call %d: %s differs from moe_sort" % (call, name)
+            assert np.array_equal(a.cpu().numpy(), c), "call %d: %s differs from the oracle" % (call, name)
+
+
+def test_static_scratch_sort_allocates_nothing():
+    T, K, E = 40000, 10, 512
+    ids = torch.from_numpy(wl.random_ids(T, K, E, seed=7)).cuda()
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    bufs = _buffers(T, K, E)
+    static_sort(ids, E, status, bufs)           # first call: address set-up and module load
+    torch.cuda.synchronize()
+    alloc0, free0 = torch.cuda.memory_allocated(), torch.cuda.mem_get_info()[0]
+    static_sort(ids, E, status, bufs)
+    torch.cuda.synchronize()
+    assert torch.cuda.memory_allocated() == alloc0
+    assert torch.cuda.mem_get_info()[0] == free0
+    assert status.item() == 0
 
 
 def test_static_scratch_sort_rejects_sizes_beyond_its_array():
