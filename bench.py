@@ -91,32 +91,84 @@ def sources_hash(kind="decode"):
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons every 50 ms while running; the
-    samples are time-stamped so that each timed region gets its own summary."""
+    """SM clock, power and clock-event (throttle) reasons of one GPU, sampled
+    every 5 ms by a thread through NVML (read-only queries; nvidia-smi every
+    50 ms if NVML is unavailable).  Samples are time-stamped, so each timed
+    region gets its own summary."""
 
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
     Q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
          "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
          "clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, index, period_ms=50):
-        self.index, self.period_ms, self.lines, self.proc = index, period_ms, [], None
+    def __init__(self, index, pci_bus_id=None, period_s=0.005):
+        self.index, self.pci, self.period = index, pci_bus_id, period_s
+        self.samples = []  # (time, sm MHz, max MHz, power W, {reason names})
+        self.proc, self.stop, self.source = None, threading.Event(), None
 
     def __enter__(self):
         try:
+            import pynvml
+            pynvml.nvmlInit()
+            try:
+                h = pynvml.nvmlDeviceGetHandleByPciBusId(self.pci) if self.pci else None
+            except pynvml.NVMLError:
+                h = None
+            if h is None:
+                h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            self.nvml, self.h = pynvml, h
+            bits = (pynvml.nvmlClocksEventReasonHwSlowdown, pynvml.nvmlClocksEventReasonHwThermalSlowdown,
+                    pynvml.nvmlClocksEventReasonSwThermalSlowdown, pynvml.nvmlClocksEventReasonSwPowerCap)
+            self.bits = list(zip(self.NAMES, bits))
+            self.source = "nvml, %.0f ms" % (self.period * 1e3)
+            self.t = threading.Thread(target=self._nvml_loop, daemon=True)
+            self.t.start()
+            return self
+        except Exception:
+            pass
+        try:
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.Q,
-                                          "--format=csv,noheader,nounits", "-lms", str(self.period_ms)],
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.t = threading.Thread(target=self._read, daemon=True)
+            self.source = "nvidia-smi, 50 ms"
+            self.t = threading.Thread(target=self._smi_loop, daemon=True)
             self.t.start()
         except (OSError, FileNotFoundError):
             self.proc = None
         return self
 
-    def _read(self):
+    def _nvml_loop(self):
+        n = self.nvml
+        mx = n.nvmlDeviceGetMaxClockInfo(self.h, n.NVML_CLOCK_SM)
+        while not self.stop.is_set():
+            try:
+                sm = n.nvmlDeviceGetClockInfo(self.h, n.NVML_CLOCK_SM)
+                pw = n.nvmlDeviceGetPowerUsage(self.h) / 1000.0
+                r = n.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((time.monotonic(), float(sm), float(mx), pw,
+                                     {name for name, b in self.bits if r & b}))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def _smi_loop(self):
         for line in self.proc.stdout:
-            self.lines.append((time.monotonic(), line.strip()))
+            f = [x.strip() for x in line.strip().split(",")]
+            if len(f) < 8:
+                continue
+            try:
+                self.samples.append((time.monotonic(), float(f[0]), float(f[1]), float(f[2]),
+                                     {n for n, v in zip(self.NAMES, f[4:8]) if v.lower().startswith("active")}))
+            except ValueError:
+                continue
+
+    def wait_first(self, timeout_s=3.0):
+        t0 = time.monotonic()
+        while not self.samples and time.monotonic() - t0 < timeout_s and self.source:
+            time.sleep(0.01)
 
     def __exit__(self, *a):
+        self.stop.set()
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -128,26 +180,17 @@ class ClockSampler:
         """Median SM clock, max clock and throttle reasons of the samples taken
         in [t0, t1] (all samples when no interval is given)."""
         sm, mx, pw, reasons = [], [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ts, l in list(self.lines):
+        for ts, c, m, p, rs in list(self.samples):
             if (t0 is not None and ts < t0) or (t1 is not None and ts > t1):
                 continue
-            f = [x.strip() for x in l.split(",")]
-            if len(f) < 8:
-                continue
-            try:
-                sm.append(float(f[0]))
-                mx.append(float(f[1]))
-                pw.append(float(f[2]))
-            except ValueError:
-                continue
-            for n, v in zip(names, f[4:8]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
+            sm.append(c)
+            mx.append(m)
+            pw.append(p)
+            reasons |= rs
         if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "source": self.source}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "power_w_max": max(pw),
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm), "source": self.source}
 
 
 def ffn_roofline(shape, form_kind, touched, flops, ffn_ms, peaks, root=ROOT):
@@ -579,7 +622,11 @@ def main():
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
 
-    with ClockSampler(local) as clk:
+    props = torch.cuda.get_device_properties(dev)
+    pci = ("%08x:%02x:%02x.0" % (props.pci_domain_id, props.pci_bus_id, props.pci_device_id)
+           if hasattr(props, "pci_bus_id") else None)
+    with ClockSampler(local, pci) as clk:
+        clk.wait_first()
         head, e2e = measure(args, shape, args.steps, dev, world, clk, want_e2e=True)
         others = {}
         for n in extras:

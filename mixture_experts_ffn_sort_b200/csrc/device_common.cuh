@@ -314,6 +314,12 @@ __host__ __device__ constexpr uint32_t umma_idesc_bf16(int M, int N) {
            (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// Instruction descriptor of kind::f16 with f16 A and B (both K-major), fp32
+// accumulator, shape M x N.
+__host__ __device__ constexpr uint32_t umma_idesc_f16(int M, int N) {
+    return (1u << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
 // ---------------------------------------------------------------- cp.async
 
 // 16-byte global -> shared copy; src_bytes < 16 zero-fills the rest (0 = all zeros).

@@ -7,7 +7,18 @@
 // (spark_model/layers/nemotron_moe.rs, `prefill` step 5) and the fused
 // prefill producer of the aiter gfx950 PR (gate/up, SiLU, down and the
 // routing-weight multiply in one pipeline), with the block-scaled E4M3FN
-// weights of the FP8 MoE decode kernel page decoded to BF16 tile by tile.
+// weights of the FP8 MoE decode kernel page decoded tile by tile to 16-bit
+// MMA operands: f16 in the gate/up GEMM, bf16 in the down GEMM.
+//
+// gate/up runs on f16 operands, which take one conversion instruction and one
+// f16x2 multiply per code pair.  A pre-pass (x16_kernel) copies x to f16 with
+// each row scaled by a power of two 2^k_t that puts its largest magnitude in
+// [2^14, 2^15) (exact: f16 has 11 significant bits to bf16's 8); the weights
+// become f16(e4m3 * s * 2^ka), ka a power of two per row block chosen from its
+// largest block scale so that every product is an f16 normal.  The epilogue
+// multiplies the accumulators by 2^-ka * 2^-k_t before SwiGLU.  Both
+// roundings (s * 2^ka to f16, the product to f16) are of 2^-12 relative, finer
+// than the bf16(e4m3 * s) of the down GEMM.
 //
 // One persistent kernel per GEMM (gate/up, then down); each CTA owns one SM
 // and walks a list of output tiles built on the device from the expert
@@ -19,7 +30,8 @@
 //  * warp 0: the weight tile's FP8 bytes by TMA in stages of 128 reduction
 //    columns (128-byte rows, 128-byte swizzle), 64 KB ahead;
 //  * the token rows into the 128-byte-swizzled K-major layout the MMA reads:
-//    gate/up gathers x rows through sorted_route with cp.async on warps 2-7
+//    gate/up gathers rows of the f16 copy of x through sorted_route with
+//    cp.async on warps 2-7
 //    (the per-SM gather rate grows with the number of issuing warps; each
 //    thread keeps its rows' token indices in registers for the whole tile and
 //    arrives on the stage's mbarrier when its copies land); down loads
@@ -28,9 +40,10 @@
 //  * transform warps 8-15: each thread owns one TMEM lane (one weight row);
 //    gate/up: warps 8-11 decode M-tile 0 and 12-15 M-tile 1, all 64 columns
 //    of a step; down: two warps per lane quarter, half the columns each.  A
-//    thread decodes its FP8 codes to bf16(e4m3 * block scale) as soon as the
-//    weight stage lands, then waits for its A slot and stores them with
-//    tcgen05.st (A operand, two bf16 per column) into a ring of four 32-column
+//    thread decodes its FP8 codes (gate/up: f16(e4m3 * s * 2^ka); down:
+//    bf16(e4m3 * s)) as soon as the weight stage lands, then waits for its A
+//    slot and stores them with tcgen05.st (A operand, two 16-bit values per
+//    column) into a ring of four 32-column
 //    units (two gate/up steps or four down steps, one barrier pair per step);
 //  * warp 1 issues tcgen05.mma warp-uniformly, one elected lane per four
 //    MMAs (kind::f16, A in TMEM, B in shared memory, fp32 accumulator D in
@@ -257,11 +270,82 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, Barrier
     return mbar_wait_or_abort(bar, parity, &B->abort_flag, status);
 }
 
-// bf16(e4m3 * s) for two codes.
+// bf16(e4m3 * s) for two codes (down GEMM).
 __device__ __forceinline__ uint32_t decode_scaled(uint16_t codes, float s) {
     const uint32_t h = e4m3x2_to_f16x2(codes);
     const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h));
     return pack_bf16x2(f.x * s, f.y * s);
+}
+
+// f16(e4m3 * s2) for two codes (gate/up GEMM): the exact conversion of the
+// codes to f16, then one f16x2 multiply by the scale pair s2 (a power-of-two
+// multiple of the block scale, so every product is an f16 normal).
+__device__ __forceinline__ uint32_t decode_scaled_f16(uint16_t codes, uint32_t s2) {
+    const uint32_t h = e4m3x2_to_f16x2(codes);
+    __half2 r = __hmul2(*reinterpret_cast<const __half2*>(&h), *reinterpret_cast<const __half2*>(&s2));
+    return *reinterpret_cast<uint32_t*>(&r);
+}
+
+// Power-of-two exponent ka of a gate/up weight row block whose largest block
+// scale is smax: 448 * smax * 2^ka lies in [2^14, 2^15), so the f16 operands
+// e4m3 * s * 2^ka of every block stay below the f16 maximum, and those of
+// blocks whose scale is at least 2^-10 smax stay f16 normals (the smallest
+// nonzero E4M3FN magnitude is 2^-9, the largest 448).  The transform and the
+// epilogue compute it from the same scales, so they agree exactly.
+__device__ __forceinline__ int f16_row_exponent(float smax) {
+    const float m = 448.f * smax;
+    if (!(m > 0.f) || !(m < INFINITY)) return 0;
+    const int e = (__float_as_int(m) >> 23) & 0xFF;  // biased exponent (0 for a subnormal m)
+    return max(-120, min(120, 141 - e));
+}
+
+__device__ __forceinline__ float exp2_int(int k) {  // 2^k for -126 <= k <= 127
+    return __uint_as_float(static_cast<uint32_t>(k + 127) << 23);
+}
+
+// Largest |x| bit pattern (sign cleared) among the 8 bf16 of a 16-byte vector.
+__device__ __forceinline__ uint32_t absmax_bf16x8_bits(const uint4& v) {
+    const uint32_t m = __vmaxu2(__vmaxu2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu),
+                                __vmaxu2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu));
+    return max(m & 0xFFFFu, m >> 16);
+}
+
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2_times(uint32_t w, float up) {
+    __half2 h = __floats2half2_rn(__uint_as_float(w << 16) * up, __uint_as_float(w & 0xFFFF0000u) * up);
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// x16[t] = f16(x[t] * 2^k_t), xinv[t] = 2^-k_t, with k_t putting the row's
+// largest magnitude in [2^14, 2^15) (k_t = 0 for an all-zero row).  f16 has
+// 11 significant bits to bf16's 8, so every element within 2^-28 of its
+// row's largest is copied exactly; the gate/up epilogue multiplies by xinv.
+// One warp per row, 16-byte loads and stores.
+__global__ void __launch_bounds__(256) x16_kernel(const uint16_t* __restrict__ x, int T, int H,
+                                                  uint16_t* __restrict__ x16, float* __restrict__ xinv) {
+    const int t = static_cast<int>((static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5);
+    const int lane = threadIdx.x & 31;
+    if (t >= T) return;
+    const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * H);
+    uint4* dst = reinterpret_cast<uint4*>(x16 + static_cast<size_t>(t) * H);
+    const int nv = H >> 3;
+    uint32_t amax = 0;
+    for (int v = lane; v < nv; v += 32) amax = max(amax, absmax_bf16x8_bits(__ldg(src + v)));
+    amax = __reduce_max_sync(0xffffffffu, amax);
+    int k = 0;
+    if (amax) {
+        const int eb = static_cast<int>(amax >> 7);  // biased exponent of the largest magnitude (0: subnormal)
+        k = min(127, 14 - (eb ? eb - 127 : -127));
+    }
+    const float up = exp2_int(k);
+    if (lane == 0) xinv[t] = ldexpf(1.f, -k);
+    for (int v = lane; v < nv; v += 32) {
+        uint4 w = __ldg(src + v);
+        w.x = bf16x2_to_f16x2_times(w.x, up);
+        w.y = bf16x2_to_f16x2_times(w.y, up);
+        w.z = bf16x2_to_f16x2_times(w.z, up);
+        w.w = bf16x2_to_f16x2_times(w.w, up);
+        dst[v] = w;
+    }
 }
 
 template <int MODE>
@@ -369,6 +453,38 @@ __global__ void __launch_bounds__(kThreads, 1)
         // Epilogue of one item (warps 4-7).
         auto epilogue = [&](const Tile& t) {
             const PartCfg pc = part_cfg<MODE>(a, t.pt);
+            // gate/up: D of a gate (up) row is 2^ka_g (2^ka_u) x 2^k_t times the
+            // true sum (scaled weights, scaled x rows): fg, fu undo the first,
+            // col_w[c] = xinv of column c's token the second.
+            float fg = 1.f, fu = 1.f;
+            if (MODE == kGateUp) {
+                const ExpertsView& ev = t.pt ? a.sh : a.ex;
+                const size_t off = (static_cast<size_t>(t.e) * (pc.I / 128) + t.fb0) * pc.KB128;
+                float mg = 0.f, mu = 0.f;
+                for (int i = lane; i < pc.KB128; i += 32) {
+                    mg = fmaxf(mg, __ldg(ev.s_gate + off + i));
+                    mu = fmaxf(mu, __ldg(ev.s_up + off + i));
+                }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    mg = fmaxf(mg, __shfl_xor_sync(0xffffffffu, mg, o));
+                    mu = fmaxf(mu, __shfl_xor_sync(0xffffffffu, mu, o));
+                }
+                fg = exp2_int(-f16_row_exponent(mg));
+                fu = exp2_int(-f16_row_exponent(mu));
+                named_barrier_sync(4, 128);
+                for (int c = et; c < t.n; c += 128) {
+                    int tk = 0;
+                    if (t.pt) {
+                        tk = static_cast<int>(t.p0 + c);
+                    } else {
+                        const int rt = a.sorted_route[t.p0 + c];
+                        tk = (rt >= 0 && rt < R) ? rt / a.K : 0;
+                    }
+                    col_w[c] = __ldg(a.xinv + tk);
+                }
+                named_barrier_sync(4, 128);
+            }
             if (MODE == kDown) {
                 // Route weight of every column of the item, staged once (1 for
                 // the shared expert).
@@ -406,14 +522,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                             tmem_ld16x256b_x4(tl + (16u << 16) + c0, uv);
                             tmem_ld_wait();
                             if (!ok) continue;
+                            // Column scales of this thread's tokens c0 + 8g + 2(t%4) + {0, 1}.
+                            float2 cs[4];
+#pragma unroll
+                            for (int gq = 0; gq < 4; ++gq)
+                                cs[gq] = *reinterpret_cast<const float2*>(col_w + c0 + 8 * gq + 2 * (lane & 3));
                             uint32_t pk[8];
 #pragma unroll
                             for (int k = 0; k < 8; ++k) {
                                 float hv[2];
 #pragma unroll
                                 for (int j = 0; j < 2; ++j) {
-                                    const float z = __uint_as_float(gv[2 * k + j]);
-                                    hv[j] = __fdividef(z, 1.0f + __expf(-z)) * __uint_as_float(uv[2 * k + j]);
+                                    const float cc = j ? cs[k >> 1].y : cs[k >> 1].x;
+                                    const float z = __uint_as_float(gv[2 * k + j]) * (fg * cc);
+                                    const float u = __uint_as_float(uv[2 * k + j]) * (fu * cc);
+                                    hv[j] = __fdividef(z, 1.0f + __expf(-z)) * u;
                                 }
                                 pk[k] = pack_bf16x2(hv[0], hv[1]);
                             }
@@ -523,7 +646,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int s = static_cast<int>(g % kSB);
                     if (g >= kSB) wait_bar(&B->b_done[s], static_cast<uint32_t>((g / kSB - 1) & 1), B, a.status);
                     const uint32_t bdst = smem_u32(b_ring + s * kBStage) + r0 * 128 + cch;
-                    const uint16_t* xs = a.x + kb * 64 + ch * 8;
+                    const uint16_t* xs = a.x16 + kb * 64 + ch * 8;
 #pragma unroll
                     for (int k = 0; k < kRowsPerThread; ++k)
                         if (r0 + 24 * k < t.n)
@@ -600,6 +723,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int srow = MODE == kGateUp ? hi * 64 + 16 * q + (lane & 15) : row;
             const int sub = up_row ? kWStage / 2 : 0;
             const int c0 = MODE == kGateUp ? 0 : 2 * hi;  // first 16-byte chunk of this thread in a step
+            // gate/up: the f16 operands of this row are e4m3 * s * 2^ka, with ka
+            // from the largest block scale of the row's block row (gate or up).
+            float pa = 1.f;
+            if (MODE == kGateUp) {
+                const float* sr = sc_sm + (up_row ? KB128 : 0);
+                float m = 0.f;
+                for (int i = 0; i < KB128; ++i) m = fmaxf(m, sr[i]);
+                pa = exp2_int(f16_row_exponent(m));
+            }
             for (int f = 0; f < t.nfb; ++f) {
                 const float* scr = sc_sm + (MODE == kGateUp ? (up_row ? KB128 : 0) : f * KB128);
                 for (int kb = 0; kb < KB; ++kb, ++g) {
@@ -610,6 +742,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     uint32_t v[NW];
                     if (ok1) {
                         const float sc = scr[kb >> 1];
+                        __half2 s2h = __float2half2_rn(sc * pa);
+                        const uint32_t s2 = *reinterpret_cast<uint32_t*>(&s2h);
                         const uint8_t* base = w_ring + sw * kWStage + sub + srow * 128;
 #pragma unroll
                         for (int c = 0; c < NW / 8; ++c) {
@@ -618,8 +752,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                             const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
                             for (int k = 0; k < 4; ++k) {
-                                v[c * 8 + 2 * k] = decode_scaled(static_cast<uint16_t>(ws[k] & 0xFFFFu), sc);
-                                v[c * 8 + 2 * k + 1] = decode_scaled(static_cast<uint16_t>(ws[k] >> 16), sc);
+                                if (MODE == kGateUp) {
+                                    v[c * 8 + 2 * k] = decode_scaled_f16(static_cast<uint16_t>(ws[k] & 0xFFFFu), s2);
+                                    v[c * 8 + 2 * k + 1] = decode_scaled_f16(static_cast<uint16_t>(ws[k] >> 16), s2);
+                                } else {
+                                    v[c * 8 + 2 * k] = decode_scaled(static_cast<uint16_t>(ws[k] & 0xFFFFu), sc);
+                                    v[c * 8 + 2 * k + 1] = decode_scaled(static_cast<uint16_t>(ws[k] >> 16), sc);
+                                }
                             }
                         }
                     } else {
@@ -661,7 +800,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int KB = pc.KB;
             const bool resident = pc.resident;
             const int N = (t.n + 15) & ~15;
-            const uint32_t idesc = umma_idesc_bf16(128, N);
+            // gate/up: f16 operands (decoded weights and the f16 copy of x); down: bf16.
+            const uint32_t idesc = MODE == kGateUp ? umma_idesc_f16(128, N) : umma_idesc_bf16(128, N);
             for (int f = 0; f < t.nfb; ++f, ++tc) {
                 // Accumulator regions of this output block: both (gate/up) or one (down).
                 const int r0 = MODE == kGateUp ? 0 : (tc & 1);
@@ -745,7 +885,7 @@ int num_sms() {
 bool ffn_prefill_supported(int H, int I) { return H % 128 == 0 && I % 128 == 0 && prefill_smem(MOE_MAX_E) <= 227 * 1024; }
 
 cudaError_t launch_ffn_prefill(const FfnArgs& a, cudaStream_t stream) {
-    if (a.identity) return cudaErrorInvalidValue;
+    if (a.identity || !a.x16 || !a.xinv) return cudaErrorInvalidValue;
     const uint64_t E = static_cast<uint64_t>(a.ex.n), I = a.ex.inter, H = a.H;
     const uint64_t R = static_cast<uint64_t>(a.T) * a.K, T = static_cast<uint64_t>(a.T);
     PrefillMaps mg, md;  // gate/up and down launches
@@ -773,6 +913,10 @@ cudaError_t launch_ffn_prefill(const FfnArgs& a, cudaStream_t stream) {
         err = cudaFuncSetAttribute(prefill_kernel<kDown>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (err != cudaSuccess) return err;
     const int grid = num_sms();
+    x16_kernel<<<static_cast<unsigned>((static_cast<long>(a.T) * 32 + 255) / 256), 256, 0, stream>>>(a.x, a.T, a.H,
+                                                                                                   a.x16, a.xinv);
+    err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
     prefill_kernel<kGateUp><<<grid, kThreads, smem, stream>>>(mg, a);
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;

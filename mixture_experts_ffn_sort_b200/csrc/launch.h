@@ -74,7 +74,16 @@ struct FfnArgs {
     // when > 0, the decode form takes the experts with 1..row_split rows and
     // the prefill form those with more; 0 = every expert.
     int row_split;
+    // Prefill form only: scratch for the f16 copy of x ([T, H], each row
+    // scaled by a power of two, see launch_ffn_prefill) and the inverse row
+    // scales ([T] f32).
+    uint16_t* x16;
+    float* xinv;
 };
+
+// Bytes of the prefill form's f16 activation copy and its row scales (256-byte aligned).
+inline size_t ffn_x16_bytes(long T, int H) { return (static_cast<size_t>(T) * H * 2 + 255) & ~size_t(255); }
+inline size_t ffn_xinv_bytes(long T) { return (static_cast<size_t>(T) * 4 + 255) & ~size_t(255); }
 
 cudaError_t launch_ffn_decode(const FfnArgs& a, cudaStream_t stream);
 

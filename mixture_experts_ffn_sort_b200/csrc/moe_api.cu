@@ -291,12 +291,15 @@ int moe_ffn_resolve_mode(int T, int K, int E, int mode) {
 }
 
 size_t moe_ffn_workspace_bytes(int T, int K, int H, int E, int I, int I_shared, int mode) {
-    (void)H;
-    (void)E;
-    (void)mode;
-    if (T < 0 || K < 1 || I < 0 || I_shared < 0) return 0;
+    if (T < 0 || K < 1 || I < 0 || I_shared < 0 || H < 0) return 0;
     const long R = static_cast<long>(T) * K;
-    return ffn_h_bytes(R, I) + ffn_h_bytes(T, I_shared);
+    size_t b = ffn_h_bytes(R, I) + ffn_h_bytes(T, I_shared);
+    // The tensor-core form also keeps an f16 copy of x and its row scales.
+    const std::string saved = g_err;
+    const int form = moe_ffn_resolve_mode(T, K, E < 1 ? 1 : E, mode);
+    g_err = saved;
+    if (form != MOE_MODE_DECODE) b += moe::ffn_x16_bytes(T, H) + moe::ffn_xinv_bytes(T);
+    return b;
 }
 
 int moe_expert_ffn(const uint16_t* x, int T, int H, int K, const moe_fp8_experts* routed,
@@ -361,6 +364,8 @@ int moe_expert_ffn(const uint16_t* x, int T, int H, int K, const moe_fp8_experts
         // HYBRID: the experts with more than MOE_HYBRID_ROW_SPLIT rows here, the
         // others in the decode form below.
         a.row_split = form == MOE_MODE_HYBRID ? MOE_HYBRID_ROW_SPLIT : 0;
+        a.x16 = reinterpret_cast<uint16_t*>(ws + ffn_h_bytes(R, I) + ffn_h_bytes(T, Is));
+        a.xinv = reinterpret_cast<float*>(ws + ffn_h_bytes(R, I) + ffn_h_bytes(T, Is) + moe::ffn_x16_bytes(T, H));
         const cudaError_t e = moe::launch_ffn_prefill(a, stream);
         if (e != cudaSuccess || form == MOE_MODE_PREFILL)
             return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_expert_ffn launch");

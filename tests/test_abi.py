@@ -52,7 +52,11 @@ def test_workspace_queries(L):
     assert L.moe_sort_workspace_bytes(32768, 10, 512) == 160 * 512 * 4
     assert L.moe_ffn_workspace_bytes(64, 8, 2048, 256, 512, 0, 0) == 512 * 512 * 2
     assert L.moe_ffn_workspace_bytes(16, 2, 256, 8, 128, 0, 0) == 8192
-    assert L.moe_ffn_workspace_bytes(8192, 10, 4096, 512, 256, 256, 0) == 81920 * 512 + 8192 * 512
+    # The tensor-core forms add the f16 copy of x and its row scales.
+    assert L.moe_ffn_workspace_bytes(8192, 10, 4096, 512, 256, 256, 0) == \
+        81920 * 512 + 8192 * 512 + 8192 * 4096 * 2 + 8192 * 4
+    assert L.moe_ffn_workspace_bytes(64, 8, 2048, 256, 512, 0, moe.MOE_MODE_PREFILL) == \
+        512 * 512 * 2 + 64 * 2048 * 2 + 256
 
 
 def test_ffn_resolve_mode(L):
