@@ -260,6 +260,38 @@ __device__ __forceinline__ void umma_ts_f16_x4_elect(uint32_t d_tmem, uint32_t a
         : "memory");
 }
 
+// One gate/up step from one elected lane: four K=16 MMAs into each of two
+// accumulators (d0 with A columns a0[k], d1 with a1[k], both against B
+// descriptors b[k]), then commits to bar0 and bar1.  Every operand comes in a
+// register computed ahead of time, so the issuing warp -- which shares its
+// scheduler with busy warps and waits its turn for every instruction --
+// executes as few instructions as possible.  `accumulate` applies to the
+// first K step of each accumulator; the others add.
+__device__ __forceinline__ void umma_ts_step2_commit2_elect(uint32_t d0, uint32_t d1, const uint32_t (&a0)[4],
+                                                            const uint32_t (&a1)[4], const uint64_t (&b)[4],
+                                                            uint32_t idesc, uint32_t accumulate, uint64_t* bar0,
+                                                            uint64_t* bar1) {
+    asm volatile(
+        "{\n\t.reg .pred e, p, t;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "setp.ne.b32 p, %15, 0;\n\t"
+        "setp.eq.b32 t, 0, 0;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%2], %10, %14, p;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%3], %11, %14, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%4], %12, %14, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%5], %13, %14, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%1], [%6], %10, %14, p;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%1], [%7], %11, %14, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%1], [%8], %12, %14, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%1], [%9], %13, %14, t;\n\t"
+        "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%16];\n\t"
+        "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%17];\n\t}"
+        ::"r"(d0), "r"(d1), "r"(a0[0]), "r"(a0[1]), "r"(a0[2]), "r"(a0[3]), "r"(a1[0]), "r"(a1[1]), "r"(a1[2]),
+        "r"(a1[3]), "l"(b[0]), "l"(b[1]), "l"(b[2]), "l"(b[3]), "r"(idesc), "r"(accumulate), "r"(smem_u32(bar0)),
+        "r"(smem_u32(bar1))
+        : "memory");
+}
+
 // Arrive on `bar` once every tcgen05.mma issued so far has completed: a
 // tcgen05.commit from one elected lane of a warp executing it uniformly.
 __device__ __forceinline__ void umma_commit_elect(uint64_t* bar) {

@@ -27,8 +27,9 @@
 // is 128 weight rows x up to 192 token rows:
 //  * swap-AB: the weights are the M=128 operand A, the tokens the N operand B,
 //    so the FP8 decode writes tensor memory, not shared memory;
-//  * warp 0: the weight tile's FP8 bytes by TMA in stages of 128 reduction
-//    columns (128-byte rows, 128-byte swizzle), 64 KB ahead;
+//  * warp 0: the weight tile's FP8 bytes by TMA into a 64 KB ring of four
+//    stages: 64 reduction columns for gate/up (64-byte rows and swizzle), 128
+//    for down (128-byte rows and swizzle);
 //  * the token rows into the 128-byte-swizzled K-major layout the MMA reads:
 //    gate/up gathers rows of the f16 copy of x through sorted_route with
 //    cp.async on warps 2-7
@@ -105,13 +106,20 @@ enum Mode { kGateUp = 0, kDown = 1 };
 // accumulator regions); down: one M-tile per step, regions double-buffered.
 // A weight stage holds 128 reduction columns (128-byte rows) and feeds two
 // 64-column MMA steps.
+// kWCols: reduction columns (bytes of a row) per weight stage.  gate/up uses
+// 64-column stages (one MMA step each, 64-byte swizzle), so that three of the
+// ring's four stages are in flight while one is decoded: the weights of a
+// gate/up step are consumed at twice the rate of a down step.
 template <> struct Cfg<0> {
-    static constexpr int MT = 2, kWStage = 2 * 128 * 128, kSW = kWRing / kWStage, kSA = 4, kSS = kSA / MT;
+    static constexpr int MT = 2, kWCols = 64, kWStage = 2 * 128 * kWCols, kSW = kWRing / kWStage, kSA = 4,
+                         kSS = kSA / MT;
 };
 template <> struct Cfg<1> {
-    static constexpr int MT = 1, kWStage = 128 * 128, kSW = kWRing / kWStage, kSA = 4, kSS = kSA / MT;
+    static constexpr int MT = 1, kWCols = 128, kWStage = 128 * kWCols, kSW = kWRing / kWStage, kSA = 4,
+                         kSS = kSA / MT;
 };
 constexpr int kSWMax = 8, kSAMax = 4;
+static_assert(Cfg<0>::kSW <= kSWMax && Cfg<1>::kSW <= kSWMax, "weight ring depth");
 
 struct Barriers {
     uint64_t w_full[kSWMax], w_empty[kSWMax];
@@ -139,7 +147,7 @@ struct PrefillMaps {
 struct PartCfg {
     int I;         // intermediate size
     int KB;        // MMA steps (64 columns) per output block
-    int KB128;     // scale blocks = weight TMA stages per output block
+    int KB128;     // 128-column scale blocks per output block
     int FB;        // output blocks of 128 features (gate/up: their gate and up rows)
     int GFB;       // output blocks per item
     bool resident; // down: the token tile stays in the ring across the item
@@ -420,17 +428,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const PartCfg pc = part_cfg<MODE>(a, t.pt);
                 for (int f = 0; f < t.nfb; ++f) {
                     const int fb = t.fb0 + f;
-                    for (int kw = 0; kw < pc.KB128; ++kw, ++g) {
+                    const int nstages = (MODE == kGateUp ? H : pc.I) / C::kWCols;
+                    for (int kw = 0; kw < nstages; ++kw, ++g) {
                         const int s = static_cast<int>(g % kSW);
                         if (g >= kSW) wait_bar(&B->w_empty[s], static_cast<uint32_t>((g / kSW - 1) & 1), B, a.status);
                         uint8_t* dst = w_ring + s * kWStage;
                         mbar_arrive_expect_tx(&B->w_full[s], kWStage);
                         if (MODE == kGateUp) {
                             const int row = t.e * pc.I + fb * 128;  // 128 gate rows, 128 up rows
-                            tma_load_2d_hint(dst, &M.w0[t.pt], &B->w_full[s], kw * 128, row, policy);
-                            tma_load_2d_hint(dst + kWStage / 2, &M.w1[t.pt], &B->w_full[s], kw * 128, row, policy);
+                            tma_load_2d_hint(dst, &M.w0[t.pt], &B->w_full[s], kw * C::kWCols, row, policy);
+                            tma_load_2d_hint(dst + kWStage / 2, &M.w1[t.pt], &B->w_full[s], kw * C::kWCols, row,
+                                             policy);
                         } else {
-                            tma_load_2d_hint(dst, &M.w0[t.pt], &B->w_full[s], kw * 128, t.e * H + fb * 128, policy);
+                            tma_load_2d_hint(dst, &M.w0[t.pt], &B->w_full[s], kw * C::kWCols, t.e * H + fb * 128,
+                                             policy);
                         }
                     }
                 }
@@ -735,7 +746,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int f = 0; f < t.nfb; ++f) {
                 const float* scr = sc_sm + (MODE == kGateUp ? (up_row ? KB128 : 0) : f * KB128);
                 for (int kb = 0; kb < KB; ++kb, ++g) {
-                    const long gw = g >> 1;  // weight stage holding this step
+                    constexpr int kSPS = C::kWCols / 64;  // MMA steps per weight stage
+                    const long gw = g / kSPS;  // weight stage holding this step
                     const long u = MODE == kGateUp ? 2 * g + hi : g;  // A unit of this warp's work
                     const int sw = static_cast<int>(gw % kSW), sa = static_cast<int>(u % kSA);
                     const bool ok1 = wait_bar(&B->w_full[sw], static_cast<uint32_t>((gw / kSW) & 1), B, a.status);
@@ -744,11 +756,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const float sc = scr[kb >> 1];
                         __half2 s2h = __float2half2_rn(sc * pa);
                         const uint32_t s2 = *reinterpret_cast<uint32_t*>(&s2h);
-                        const uint8_t* base = w_ring + sw * kWStage + sub + srow * 128;
+                        const uint8_t* base = w_ring + sw * kWStage + sub + srow * C::kWCols;
 #pragma unroll
                         for (int c = 0; c < NW / 8; ++c) {
-                            const int chunk = (g & 1) * 4 + c0 + c;
-                            const uint4 w = *reinterpret_cast<const uint4*>(base + ((chunk ^ (srow & 7)) << 4));
+                            // 16-byte chunk of this thread's row in the stage, placed by
+                            // the TMA swizzle of the stage's row width (128 or 64 bytes).
+                            const int chunk = static_cast<int>(g % kSPS) * 4 + c0 + c;
+                            const int phys = C::kWCols == 128 ? (chunk ^ (srow & 7)) : (chunk ^ ((srow >> 1) & 3));
+                            const uint4 w = *reinterpret_cast<const uint4*>(base + (phys << 4));
                             const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
                             for (int k = 0; k < 4; ++k) {
@@ -766,7 +781,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int k = 0; k < NW; ++k) v[k] = 0;
                     }
                     __syncwarp();
-                    if ((g & 1) && lane == 0) mbar_arrive(&B->w_empty[sw]);
+                    if (g % kSPS == kSPS - 1 && lane == 0) mbar_arrive(&B->w_empty[sw]);
                     // The A slot is free once the MMAs that last read it have
                     // completed; the decode above overlapped that wait.
                     const int ss = static_cast<int>(g % C::kSS);  // step slot of this step
@@ -791,6 +806,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         // once plus per-slot offsets.
         const uint64_t bdesc0 = umma_desc_sw128(smem_u32(b_ring));
         const uint32_t a_base = tmem + kACol;
+        // gate/up: the operands of every ring position, computed once.
+        uint64_t bq[kSB][4];   // B descriptor of token stage s, K=16 step k
+        uint32_t aq[kSAMax][4];  // A column of unit u, K=16 step k
+#pragma unroll
+        for (int s2 = 0; s2 < kSB; ++s2)
+#pragma unroll
+            for (int k = 0; k < 4; ++k) bq[s2][k] = bdesc0 + static_cast<uint64_t>((s2 * kBStage) >> 4) + 2 * k;
+#pragma unroll
+        for (int u = 0; u < kSAMax; ++u)
+#pragma unroll
+            for (int k = 0; k < 4; ++k) aq[u][k] = a_base + u * 32 + 8 * k;
         long ga = 0, gb = 0;
         int uses[2] = {0, 0};
         int tc = 0;
@@ -814,19 +840,51 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_after();
                 const bool last = f == t.nfb - 1;
                 const uint32_t d_base = tmem + r0 * kDRegion;
+                bool grouped = false;
+                if constexpr (MODE == kGateUp) grouped = KB % kSB == 0 && (ga % kSB) == 0;
+                if constexpr (MODE == kGateUp) if (grouped) {
+                    // gate/up in groups of kSB steps aligned with the token ring
+                    // (so also with the two A step slots): every ring index and
+                    // barrier parity of a group is a compile-time function of
+                    // one value, and each step is two waits, two fences and one
+                    // issue of eight MMAs with two commits.
+                    static_assert(kSB == 4 && C::kSS == 2 && kSA == 4, "ring layout of the grouped gate/up issue");
+                    for (int kb = 0; kb < KB; kb += kSB, ga += kSB, gb += kSB) {
+                        const uint32_t pb = static_cast<uint32_t>((ga / kSB) & 1);
+                        const uint32_t pa = static_cast<uint32_t>((ga / C::kSS) & 1);
+#pragma unroll
+                        for (int j = 0; j < kSB; ++j) {
+                            const int ss = j & 1;
+                            const bool okb = wait_bar(&B->b_full[j], pb, B, a.status);
+                            const bool oka = wait_bar(&B->a_full[ss], pa ^ static_cast<uint32_t>(j >> 1), B, a.status);
+                            tc_fence_after();
+                            // Token rows written by cp.async (generic proxy) are read by the MMA
+                            // (async proxy).
+                            fence_proxy_async_smem();
+                            if (okb && oka) {
+                                umma_ts_step2_commit2_elect(d_base, d_base + kDRegion, aq[2 * ss], aq[2 * ss + 1],
+                                                            bq[j], idesc, (kb | j) ? 1u : 0u, &B->a_done[ss],
+                                                            &B->b_done[j]);
+                            } else {
+                                umma_commit_elect(&B->a_done[ss]);
+                                umma_commit_elect(&B->b_done[j]);
+                            }
+                        }
+                    }
+                }
+                if (!grouped)
                 for (int kb = 0; kb < KB; ++kb, ++ga) {
                     const long g_b = resident ? gb + kb : gb;  // token stage of this step
                     const int sb = static_cast<int>(g_b % kSB);
                     const bool okb = wait_bar(&B->b_full[sb], static_cast<uint32_t>((g_b / kSB) & 1), B, a.status);
-                    tc_fence_after();
-                    // Token rows written by cp.async (generic proxy) are read by the MMA
-                    // (async proxy).
-                    if (MODE == kGateUp) fence_proxy_async_smem();
                     const uint64_t bdesc = bdesc0 + static_cast<uint64_t>((sb * kBStage) >> 4);
                     // The step's A units (one per M-tile) arrive together.
                     const int ss = static_cast<int>(ga % C::kSS);
                     const bool oka = wait_bar(&B->a_full[ss], static_cast<uint32_t>((ga / C::kSS) & 1), B, a.status);
                     tc_fence_after();
+                    // Token rows written by cp.async (generic proxy) are read by the MMA
+                    // (async proxy).
+                    if (MODE == kGateUp) fence_proxy_async_smem();
                     if (okb && oka) {
 #pragma unroll
                         for (int mt = 0; mt < MT; ++mt) {
@@ -891,16 +949,16 @@ cudaError_t launch_ffn_prefill(const FfnArgs& a, cudaStream_t stream) {
     PrefillMaps mg, md;  // gate/up and down launches
     memset(&mg, 0, sizeof(mg));
     memset(&md, 0, sizeof(md));
-    cudaError_t err = make_tmap_u8_2d(&mg.w0[0], a.ex.w_gate, E * I, H, 128, 128);
-    if (err == cudaSuccess) err = make_tmap_u8_2d(&mg.w1[0], a.ex.w_up, E * I, H, 128, 128);
+    cudaError_t err = make_tmap_u8_2d(&mg.w0[0], a.ex.w_gate, E * I, H, Cfg<0>::kWCols, 128, Cfg<0>::kWCols);
+    if (err == cudaSuccess) err = make_tmap_u8_2d(&mg.w1[0], a.ex.w_up, E * I, H, Cfg<0>::kWCols, 128, Cfg<0>::kWCols);
     if (err == cudaSuccess) err = make_tmap_bf16_2d(&mg.out[0], a.h, R, I, 64, kOStoreRows);
     if (err == cudaSuccess) err = make_tmap_u8_2d(&md.w0[0], a.ex.w_down, E * H, I, 128, 128);
     if (err == cudaSuccess) err = make_tmap_bf16_2d(&md.act[0], a.h, R, I, 64, kNMax);
     if (err == cudaSuccess) err = make_tmap_bf16_2d(&md.out[0], a.y, R, H, 64, kOStoreRows);
     if (a.sh.n) {
         const uint64_t Is = a.sh.inter;
-        if (err == cudaSuccess) err = make_tmap_u8_2d(&mg.w0[1], a.sh.w_gate, Is, H, 128, 128);
-        if (err == cudaSuccess) err = make_tmap_u8_2d(&mg.w1[1], a.sh.w_up, Is, H, 128, 128);
+        if (err == cudaSuccess) err = make_tmap_u8_2d(&mg.w0[1], a.sh.w_gate, Is, H, Cfg<0>::kWCols, 128, Cfg<0>::kWCols);
+        if (err == cudaSuccess) err = make_tmap_u8_2d(&mg.w1[1], a.sh.w_up, Is, H, Cfg<0>::kWCols, 128, Cfg<0>::kWCols);
         if (err == cudaSuccess) err = make_tmap_bf16_2d(&mg.out[1], a.h_sh, T, Is, 64, kOStoreRows);
         if (err == cudaSuccess) err = make_tmap_u8_2d(&md.w0[1], a.sh.w_down, H, Is, 128, 128);
         if (err == cudaSuccess) err = make_tmap_bf16_2d(&md.act[1], a.h_sh, T, Is, 64, kNMax);
