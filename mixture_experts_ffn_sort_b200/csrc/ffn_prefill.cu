@@ -96,7 +96,8 @@ constexpr int kThreads = kNumWarps * 32;
 constexpr int kXformWarps = 8;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kDRegion = kNMax;        // two accumulator regions of kNMax columns
-constexpr uint32_t kACol = 2 * kNMax;       // A ring: 128 columns
+constexpr uint32_t kACol = 2 * kNMax;       // A ring: the remaining columns
+constexpr int kARing = (kTmemCols - kACol) / 32;  // A units of 32 columns (4 with 192-row tiles)
 constexpr int kDownGroup = 16;                  // output blocks sharing a resident token tile (down)
 constexpr int kScales = 512;                    // staged block scales per item (floats)
 
@@ -111,14 +112,14 @@ enum Mode { kGateUp = 0, kDown = 1 };
 // ring's four stages are in flight while one is decoded: the weights of a
 // gate/up step are consumed at twice the rate of a down step.
 template <> struct Cfg<0> {
-    static constexpr int MT = 2, kWCols = 64, kWStage = 2 * 128 * kWCols, kSW = kWRing / kWStage, kSA = 4,
+    static constexpr int MT = 2, kWCols = 64, kWStage = 2 * 128 * kWCols, kSW = kWRing / kWStage, kSA = kARing,
                          kSS = kSA / MT;
 };
 template <> struct Cfg<1> {
-    static constexpr int MT = 1, kWCols = 128, kWStage = 128 * kWCols, kSW = kWRing / kWStage, kSA = 4,
+    static constexpr int MT = 1, kWCols = 128, kWStage = 128 * kWCols, kSW = kWRing / kWStage, kSA = kARing,
                          kSS = kSA / MT;
 };
-constexpr int kSWMax = 8, kSAMax = 4;
+constexpr int kSWMax = 8, kSAMax = kARing;
 static_assert(Cfg<0>::kSW <= kSWMax && Cfg<1>::kSW <= kSWMax, "weight ring depth");
 
 struct Barriers {
@@ -624,7 +625,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int lt = threadIdx.x - kWarpTok * 32;  // 0..191
             const int r0 = lt >> 3, ch = lt & 7;
             const uint32_t cch = static_cast<uint32_t>((ch ^ (r0 & 7)) << 4);
-            constexpr int kRowsPerThread = kNMax / (kGatherThreads / 8);
+            constexpr int kRowsPerThread = (kNMax + kGatherThreads / 8 - 1) / (kGatherThreads / 8);
             uint32_t tok[kRowsPerThread];
             long g = 0;
             Tile prev{};
@@ -841,14 +842,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const bool last = f == t.nfb - 1;
                 const uint32_t d_base = tmem + r0 * kDRegion;
                 bool grouped = false;
-                if constexpr (MODE == kGateUp) grouped = KB % kSB == 0 && (ga % kSB) == 0;
-                if constexpr (MODE == kGateUp) if (grouped) {
+                constexpr bool kGroupable = MODE == kGateUp && kSB == 4 && C::kSS == 2 && kSA == 4;
+                if constexpr (kGroupable) grouped = KB % kSB == 0 && (ga % kSB) == 0;
+                if constexpr (kGroupable) if (grouped) {
                     // gate/up in groups of kSB steps aligned with the token ring
                     // (so also with the two A step slots): every ring index and
                     // barrier parity of a group is a compile-time function of
                     // one value, and each step is two waits, two fences and one
                     // issue of eight MMAs with two commits.
-                    static_assert(kSB == 4 && C::kSS == 2 && kSA == 4, "ring layout of the grouped gate/up issue");
                     for (int kb = 0; kb < KB; kb += kSB, ga += kSB, gb += kSB) {
                         const uint32_t pb = static_cast<uint32_t>((ga / kSB) & 1);
                         const uint32_t pa = static_cast<uint32_t>((ga / C::kSS) & 1);

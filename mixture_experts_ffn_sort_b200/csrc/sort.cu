@@ -28,6 +28,32 @@ __device__ __forceinline__ uint32_t lanemask_lt() {
     return m;
 }
 
+// Scatter the 32 routes r0 .. r0 + 31 of a warp (lane's route r0 + lane, its
+// expert e, `in` false past the chunk's end) given the chunk's start
+// positions `cursor[e * stride]` (shared memory, advanced in place): equal
+// experts are ranked by lane with __match_any_sync.
+__device__ __forceinline__ void scatter32(long r0, bool in, int e, int E, int32_t* cursor,
+                                          int32_t* __restrict__ sorted_route, int32_t* __restrict__ inv_route,
+                                          int stride) {
+    const int lane = threadIdx.x & 31;
+    const uint32_t lt = lanemask_lt();
+    const long r = r0 + lane;
+    const bool ok = in && e >= 0 && e < E;
+    const uint32_t peers = __match_any_sync(0xffffffffu, ok ? e : (E + lane));
+    int32_t pos = 0;
+    if (ok) pos = cursor[e * stride] + __popc(peers & lt);
+    __syncwarp();
+    // The highest lane of each group of equal experts advances the cursor.
+    if (ok && (peers >> lane) == 1u) cursor[e * stride] += __popc(peers);
+    __syncwarp();
+    if (ok) {
+        sorted_route[pos] = static_cast<int32_t>(r);
+        inv_route[r] = pos;
+    } else if (in) {
+        inv_route[r] = -1;
+    }
+}
+
 // Scatter one warp-chunk [r_begin, r_end) given the chunk's start positions
 // `cursor[e * stride]` (shared memory, advanced in place).
 __device__ __forceinline__ void scatter_chunk(const int32_t* __restrict__ ids, long r_begin,
@@ -35,25 +61,10 @@ __device__ __forceinline__ void scatter_chunk(const int32_t* __restrict__ ids, l
                                               int32_t* __restrict__ sorted_route,
                                               int32_t* __restrict__ inv_route, int stride = 1) {
     const int lane = threadIdx.x & 31;
-    const uint32_t lt = lanemask_lt();
     for (long r0 = r_begin; r0 < r_end; r0 += 32) {
         const long r = r0 + lane;
         const bool in = r < r_end;
-        const int e = in ? ids[r] : -1;
-        const bool ok = in && e >= 0 && e < E;
-        const uint32_t peers = __match_any_sync(0xffffffffu, ok ? e : (E + lane));
-        int32_t pos = 0;
-        if (ok) pos = cursor[e * stride] + __popc(peers & lt);
-        __syncwarp();
-        // The highest lane of each group of equal experts advances the cursor.
-        if (ok && (peers >> lane) == 1u) cursor[e * stride] += __popc(peers);
-        __syncwarp();
-        if (ok) {
-            sorted_route[pos] = static_cast<int32_t>(r);
-            inv_route[r] = pos;
-        } else if (in) {
-            inv_route[r] = -1;
-        }
+        scatter32(r0, in, in ? ids[r] : -1, E, cursor, sorted_route, inv_route, stride);
     }
 }
 
@@ -105,7 +116,11 @@ __device__ int block_exclusive_scan(int v, int* scratch /*[32]*/, int* total) {
 // ---------------------------------------------------------------- small: one block
 
 // smem: hist[E][NW] ints (expert-major, so the scan in (expert, warp) order
-// reads it contiguously), then 32 ints of scan scratch.
+// reads it contiguously), then 32 ints of scan scratch.  PER > 0: each lane
+// keeps its PER ids of the warp's chunk (routes rb + lane + 32 i) in registers
+// from one round of loads, for the count and the scatter alike (a warp's chunk
+// is at most 32 PER routes); PER = 0 reads them from global memory twice.
+template <int PER>
 __global__ void __launch_bounds__(1024) sort_small_kernel(const int32_t* __restrict__ ids, long R,
                                                           int E, int32_t* __restrict__ offsets,
                                                           int32_t* __restrict__ sorted_route,
@@ -113,16 +128,39 @@ __global__ void __launch_bounds__(1024) sort_small_kernel(const int32_t* __restr
                                                           int32_t* status) {
     extern __shared__ int32_t sm[];
     const int NW = blockDim.x >> 5;
-    const int warp = threadIdx.x >> 5;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     int32_t* hist = sm;                      // [E][NW]
     int32_t* scratch = sm + NW * E;          // [32]
+    const long chunk = ((R + NW - 1) / NW + 31) / 32 * 32;
+    const long rb = min(R, warp * chunk), re = min(R, rb + chunk);
+    int myid[PER > 0 ? PER : 1];
+    if constexpr (PER > 0) {
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+            const long r = rb + lane + 32 * i;
+            myid[i] = r < re ? __ldg(ids + r) : -1;
+        }
+    }
     for (int i = threadIdx.x; i < NW * E; i += blockDim.x) hist[i] = 0;
     __syncthreads();
 
-    const long chunk = ((R + NW - 1) / NW + 31) / 32 * 32;
-    const long rb = min(R, warp * chunk), re = min(R, rb + chunk);
-    if (count_chunk(ids, rb, re, E, hist + warp, NW) && (threadIdx.x & 31) == 0)
-        report_status(status, MOE_STATUS_BAD_ID);
+    bool bad;
+    if constexpr (PER > 0) {
+        bool b = false;
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+            if (rb + lane + 32 * i >= re) continue;
+            const int e = myid[i];
+            if (e >= 0 && e < E)
+                atomicAdd(&hist[e * NW + warp], 1);
+            else
+                b = true;
+        }
+        bad = __any_sync(0xffffffffu, b);
+    } else {
+        bad = count_chunk(ids, rb, re, E, hist + warp, NW);
+    }
+    if (bad && lane == 0) report_status(status, MOE_STATUS_BAD_ID);
     __syncthreads();
 
     // Exclusive scan over (expert, warp) order; each thread owns a contiguous
@@ -144,7 +182,16 @@ __global__ void __launch_bounds__(1024) sort_small_kernel(const int32_t* __restr
     for (long p = total + threadIdx.x; p < R; p += blockDim.x) sorted_route[p] = -1;
     __syncthreads();
 
-    scatter_chunk(ids, rb, re, E, hist + warp, sorted_route, inv_route, NW);
+    if constexpr (PER > 0) {
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+            const long r0 = rb + 32 * i;
+            if (r0 >= re) break;  // warp-uniform
+            scatter32(r0, r0 + lane < re, myid[i], E, hist + warp, sorted_route, inv_route, NW);
+        }
+    } else {
+        scatter_chunk(ids, rb, re, E, hist + warp, sorted_route, inv_route, NW);
+    }
 }
 
 // ---------------------------------------------------------------- large: three kernels
@@ -258,8 +305,22 @@ cudaError_t launch_sort(const int32_t* ids, long R, int E, int32_t* offsets, int
         // As many warps as 32-route slices, up to what shared memory holds.
         const int nw = static_cast<int>(std::min<long>(small_sort_warps(E), std::max<long>(1, (R + 31) / 32)));
         const size_t smem = (static_cast<size_t>(nw) * E + 32) * sizeof(int32_t);
-        sort_small_kernel<<<1, nw * 32, smem, stream>>>(ids, R, E, offsets, sorted_route, inv_route,
-                                                        status);
+        const long per = ((R + nw - 1) / nw + 31) / 32;  // ids per lane of a warp's chunk
+#define MOE_SORT_SMALL(P) \
+    sort_small_kernel<P><<<1, nw * 32, smem, stream>>>(ids, R, E, offsets, sorted_route, inv_route, status)
+        if (per <= 1)
+            MOE_SORT_SMALL(1);
+        else if (per <= 2)
+            MOE_SORT_SMALL(2);
+        else if (per <= 4)
+            MOE_SORT_SMALL(4);
+        else if (per <= 8)
+            MOE_SORT_SMALL(8);
+        else if (per <= 16)
+            MOE_SORT_SMALL(16);
+        else
+            MOE_SORT_SMALL(0);
+#undef MOE_SORT_SMALL
         return cudaGetLastError();
     }
     const int ntiles = static_cast<int>((R + kSortChunk - 1) / kSortChunk);
