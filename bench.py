@@ -383,7 +383,8 @@ def measure(args, shape, steps, dev, world, clk, want_e2e):
                                  if kw.get("bias") else None)
     wr = (torch.from_numpy(wl.router_weight(E, H, shape.seed).view(np.int16)).view(torch.bfloat16).to(dev)
           if args.fused_router else None)
-    layer = moe.MoEFFN(routed, T, K, shared, mode=args.mode, device=dev, route_cfg=route_cfg, w_router=wr)
+    layer = moe.MoEFFN(routed, T, K, shared, mode=args.mode, device=dev, route_cfg=route_cfg, w_router=wr,
+                       fused_combine=args.fused_combine)
     stream = torch.cuda.Stream(device=dev)
 
     def run(lay, xx, ll):
@@ -417,11 +418,16 @@ def measure(args, shape, steps, dev, world, clk, want_e2e):
         moe.moe_sort(layer.topk_ids, E, layer.status, layer.offsets, layer.sorted_route, layer.inv_route,
                      layer.sort_ws)
         ev[2].record()
-        moe.moe_expert_ffn(x, K, routed, layer.offsets, layer.sorted_route, layer.topk_w, shared, args.mode,
-                           layer.status, layer.y_sorted, layer.y_shared, layer.ffn_ws)
-        ev[3].record()
-        moe.moe_combine(layer.y_sorted, layer.inv_route, layer.y_shared, T, K, moe.MOE_OUT_BF16, layer.out,
-                        status=layer.status)
+        if args.fused_combine:
+            moe.moe_expert_ffn_combine(x, K, routed, layer.offsets, layer.sorted_route, layer.topk_w, shared,
+                                       moe.MOE_OUT_BF16, layer.status, layer.out, layer.ffn_ws)
+            ev[3].record()
+        else:
+            moe.moe_expert_ffn(x, K, routed, layer.offsets, layer.sorted_route, layer.topk_w, shared, args.mode,
+                               layer.status, layer.y_sorted, layer.y_shared, layer.ffn_ws)
+            ev[3].record()
+            moe.moe_combine(layer.y_sorted, layer.inv_route, layer.y_shared, T, K, moe.MOE_OUT_BF16, layer.out,
+                            status=layer.status)
         ev[4].record()
 
     # Graph of one step; the timed windows replay it.  A second graph records
@@ -479,7 +485,7 @@ def measure(args, shape, steps, dev, world, clk, want_e2e):
     ffn_ms = statistics.median(parts["ffn"])
     R_nz = int(np.count_nonzero(layer.topk_w.cpu().numpy()))
     flops = (R_nz + (T if shape.I_shared else 0)) * 6 * H * I
-    form = moe.moe_ffn_resolve_mode(T, K, E, args.mode)
+    form = moe.MOE_MODE_PREFILL if args.fused_combine else moe.moe_ffn_resolve_mode(T, K, E, args.mode)
     form_kind = {moe.MOE_MODE_DECODE: "decode", moe.MOE_MODE_PREFILL: "prefill",
                  moe.MOE_MODE_HYBRID: "hybrid"}[form]
     roof = ffn_roofline(shape, form_kind, touched=touched, flops=flops, ffn_ms=ffn_ms, peaks=peaks)
@@ -501,7 +507,9 @@ def measure(args, shape, steps, dev, world, clk, want_e2e):
            "ms_per_step": t_max, "steps": steps, "windows": N_WINDOWS,
            "window_ms_per_step": {"min": min(windows), "median": t_local, "max": max(windows)},
            "spread": (max(windows) - min(windows)) / t_local,
-           "form": form_kind, "dtype": ARITHMETIC[form_kind][0], "arithmetic": ARITHMETIC[form_kind][1],
+           "form": form_kind + ("+combine (moe_expert_ffn_combine: fp32 reductions, unordered)"
+                                if args.fused_combine else ""),
+           "dtype": ARITHMETIC[form_kind][0], "arithmetic": ARITHMETIC[form_kind][1],
            "l2": "inputs larger than L2 (%s expert weights %.2f GB > 126 MB)"
                  % ("touched" if form_kind != "prefill" else "all", weights_gb),
            "roofline": roof, "breakdown_ms": {k: statistics.median(v) for k, v in parts.items()},
@@ -529,7 +537,7 @@ def measure_e2e(args, w, shape, layer, routed, shared, route_cfg, wr, x, logits,
     lh = torch.from_numpy(w.logits).pin_memory()
     oh = [torch.empty((T, H), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
     layers = [layer, moe.MoEFFN(routed, T, K, shared, mode=args.mode, device=dev, route_cfg=route_cfg,
-                                w_router=wr)]
+                                w_router=wr, fused_combine=args.fused_combine)]
     xs, ls = [x, torch.empty_like(x)], [logits, torch.empty_like(logits)]
     h2d, d2h = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
     in_ready, in_free, out_ready, out_free = ([torch.cuda.Event(), torch.cuda.Event()] for _ in range(4))
@@ -595,6 +603,8 @@ def main():
                     help="route from x with the fused router (gate GEMM + top-K) instead of given logits")
     ap.add_argument("--eager", action="store_true",
                     help="launch every call directly instead of replaying CUDA graphs (for profilers)")
+    ap.add_argument("--fused-combine", action="store_true",
+                    help="expert FFN and combine in one call (moe_expert_ffn_combine; tensor-core form)")
     args = ap.parse_args()
     shape = wl.SHAPES[args.workload]
     rank, world, local = dist_env()

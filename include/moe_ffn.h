@@ -400,6 +400,33 @@ MOE_API int moe_expert_ffn(const uint16_t* x, int T, int H, int K, const moe_fp8
                    int32_t* status, moe_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * moe_expert_ffn_combine -- the expert FFN and the combine in one call
+ * (tensor-core form), without the sorted rows.
+ *
+ * out[t, :] = sum_j topk_w[t*K+j] * FFN_{e(t,j)}(x[t])  (+ FFN_shared(x[t]))
+ * -- what moe_expert_ffn followed by moe_combine computes, the reduction of
+ * the aiter PR's fused producer and the Nemotron-H page's unpermute-reduce
+ * (spark_model/layers/nemotron_moe.rs, `prefill` step 5) -- with the down
+ * GEMM's epilogue adding each sorted row (bf16, route weight applied, as the
+ * row moe_expert_ffn would store) into its token's fp32 output row with vector
+ * fp32 reductions at L2, instead of writing y_sorted for moe_combine to read
+ * back.  The order of the fp32 additions is not fixed: results may differ
+ * from run to run by fp32 rounding (moe_expert_ffn + moe_combine is the
+ * deterministic form).  Always runs the PREFILL kernels.
+ *   x, routed, shared, expert_offsets, sorted_route, topk_w   as moe_expert_ffn
+ *   out        [T, H], bf16 (out_dtype MOE_OUT_BF16) or f32 (MOE_OUT_F32)
+ *   workspace  moe_ffn_combine_workspace_bytes(...) bytes (bf16 output: it
+ *              also holds the [T, H] f32 accumulator)
+ *   status     optional device int32, as moe_expert_ffn
+ * Limits and errors as moe_expert_ffn.
+ * ------------------------------------------------------------------------- */
+MOE_API size_t moe_ffn_combine_workspace_bytes(int T, int K, int H, int E, int I, int I_shared, int out_dtype);
+MOE_API int moe_expert_ffn_combine(const uint16_t* x, int T, int H, int K, const moe_fp8_experts* routed,
+                                   const moe_fp8_experts* shared, const int32_t* expert_offsets,
+                                   const int32_t* sorted_route, const float* topk_w, void* out, int out_dtype,
+                                   void* workspace, size_t workspace_bytes, int32_t* status, moe_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * moe_combine -- top-K reduce back to token order.
  *
  * The Nemotron unpermute-reduce, the aiter FP32 route reduction and the NKI

@@ -33,7 +33,8 @@ MOE_MAX_E, MOE_MAX_K = 1024, 32
 
 EXPORTED = ("moe_last_error", "moe_abi_version", "moe_route", "moe_route_ex", "moe_router", "moe_sort_workspace_bytes",
             "moe_sort", "moe_selftest_bounded_wait", "moe_router_plan_check",
-            "moe_sort_static_ws", "moe_ffn_resolve_mode", "moe_ffn_workspace_bytes", "moe_expert_ffn", "moe_combine")
+            "moe_sort_static_ws", "moe_ffn_resolve_mode", "moe_ffn_workspace_bytes", "moe_expert_ffn", "moe_combine",
+            "moe_ffn_combine_workspace_bytes", "moe_expert_ffn_combine")
 
 
 class MoEError(RuntimeError):
@@ -91,6 +92,10 @@ def lib() -> ctypes.CDLL:
             L.moe_ffn_workspace_bytes.restype = S
             L.moe_expert_ffn.argtypes = [P, I, I, I, P, P, P, P, P, P, P, I, P, S, P, P]
             L.moe_expert_ffn.restype = I
+            L.moe_ffn_combine_workspace_bytes.argtypes = [I, I, I, I, I, I, I]
+            L.moe_ffn_combine_workspace_bytes.restype = S
+            L.moe_expert_ffn_combine.argtypes = [P, I, I, I, P, P, P, P, P, P, I, P, S, P, P]
+            L.moe_expert_ffn_combine.restype = I
             L.moe_combine.argtypes = [P, P, P, I, I, I, P, I, P, P]
             L.moe_combine.restype = I
             _L = L
@@ -288,6 +293,34 @@ def moe_expert_ffn(x: torch.Tensor, K: int, routed: Experts, expert_offsets: tor
     return y_sorted, (y_shared if shared is not None else None)
 
 
+def moe_ffn_combine_workspace_bytes(T, K, H, E, I, I_shared=0, out_dtype=MOE_OUT_BF16) -> int:
+    return int(lib().moe_ffn_combine_workspace_bytes(T, K, H, E, I, I_shared, out_dtype))
+
+
+def moe_expert_ffn_combine(x: torch.Tensor, K: int, routed: Experts, expert_offsets: torch.Tensor,
+                           sorted_route: torch.Tensor, topk_w: torch.Tensor, shared: Optional[Experts] = None,
+                           out_dtype: int = MOE_OUT_BF16, status: Optional[torch.Tensor] = None, out=None,
+                           workspace=None, stream=None):
+    """x [T, H] bf16 -> out [T, H] (bf16 or f32): the expert FFN and the combine
+    in one call (tensor-core kernels; fp32 reductions in no fixed order)."""
+    _need_cuda(x, expert_offsets, sorted_route, topk_w, status)
+    T, H = x.shape
+    dev = x.device
+    if out is None:
+        dt = torch.bfloat16 if out_dtype == MOE_OUT_BF16 else torch.float32
+        out = torch.empty((T, H), dtype=dt, device=dev)
+    need = moe_ffn_combine_workspace_bytes(T, K, H, routed.n, routed.inter, shared.inter if shared else 0, out_dtype)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    rs = routed.struct()
+    ss = shared.struct() if shared is not None else None
+    _check(lib().moe_expert_ffn_combine(_ptr(x), T, H, K, ctypes.byref(rs),
+                                        ctypes.byref(ss) if ss is not None else None, _ptr(expert_offsets),
+                                        _ptr(sorted_route), _ptr(topk_w), _ptr(out), out_dtype, _ptr(workspace),
+                                        workspace.numel(), _ptr(status), _stream(stream)))
+    return out
+
+
 def moe_combine(y_sorted: torch.Tensor, inv_route: torch.Tensor, y_shared: Optional[torch.Tensor],
                 T: int, K: int, out_dtype: int = MOE_OUT_BF16, out=None, stream=None,
                 status: Optional[torch.Tensor] = None):
@@ -312,12 +345,16 @@ class MoEFFN:
     route_cfg: keyword arguments of moe_route_ex (score, sel_bias, n_group,
     topk_group, renormalize, scaling) for a routing variant; None routes with
     moe_route.  w_router: bf16 [E, H] gate vectors for forward_fused, which
-    routes with the fused router (moe_router) from x alone."""
+    routes with the fused router (moe_router) from x alone.  fused_combine:
+    run the expert FFN and the combine as one call (moe_expert_ffn_combine:
+    tensor-core kernels, no y_sorted, fp32 reductions in no fixed order)."""
 
     def __init__(self, routed: Experts, T: int, K: int, shared: Optional[Experts] = None,
                  mode: int = MOE_MODE_AUTO, out_dtype: int = MOE_OUT_BF16, device="cuda",
-                 route_cfg: Optional[dict] = None, w_router: Optional[torch.Tensor] = None):
+                 route_cfg: Optional[dict] = None, w_router: Optional[torch.Tensor] = None,
+                 fused_combine: bool = False):
         self.routed, self.shared, self.T, self.K = routed, shared, T, K
+        self.fused_combine = fused_combine
         self.w_router = w_router
         self.route_cfg = dict(route_cfg) if route_cfg else None
         self.E, self.I, self.H = routed.n, routed.inter, routed.w_gate.shape[2]
@@ -330,11 +367,16 @@ class MoEFFN:
         self.sorted_route = torch.empty(R, dtype=torch.int32, device=d)
         self.inv_route = torch.empty(R, dtype=torch.int32, device=d)
         self.sort_ws = torch.empty(max(16, moe_sort_workspace_bytes(T, K, self.E)), dtype=torch.uint8, device=d)
-        self.ffn_ws = torch.empty(max(16, moe_ffn_workspace_bytes(T, K, self.H, self.E, self.I,
-                                                                  shared.inter if shared else 0, mode)),
-                                  dtype=torch.uint8, device=d)
-        self.y_sorted = torch.empty((R, self.H), dtype=torch.bfloat16, device=d)
-        self.y_shared = torch.empty((T, self.H), dtype=torch.bfloat16, device=d) if shared else None
+        if fused_combine:
+            self.ffn_ws = torch.empty(max(16, moe_ffn_combine_workspace_bytes(
+                T, K, self.H, self.E, self.I, shared.inter if shared else 0, out_dtype)), dtype=torch.uint8, device=d)
+            self.y_sorted, self.y_shared = None, None
+        else:
+            self.ffn_ws = torch.empty(max(16, moe_ffn_workspace_bytes(T, K, self.H, self.E, self.I,
+                                                                      shared.inter if shared else 0, mode)),
+                                      dtype=torch.uint8, device=d)
+            self.y_sorted = torch.empty((R, self.H), dtype=torch.bfloat16, device=d)
+            self.y_shared = torch.empty((T, self.H), dtype=torch.bfloat16, device=d) if shared else None
         dt = torch.bfloat16 if out_dtype == MOE_OUT_BF16 else torch.float32
         self.out = torch.empty((T, self.H), dtype=dt, device=d)
         self.status = torch.zeros(1, dtype=torch.int32, device=d)
@@ -344,10 +386,15 @@ class MoEFFN:
         R = self.T * self.K
         # The decode form runs the shared expert as a second kernel pair; the
         # prefill form runs it inside its two kernels.
+        sort = 1 if R <= 16384 else 3
+        if self.fused_combine:
+            # f16 copy of x, gate/up, down with the reductions, fp32 -> bf16.
+            return 1 + sort + 3 + (1 if self.out_dtype == MOE_OUT_BF16 else 0)
         form = moe_ffn_resolve_mode(self.T, self.K, self.E, self.mode)
-        ffn = {MOE_MODE_DECODE: 2 + (2 if self.shared is not None else 0), MOE_MODE_PREFILL: 2,
-               MOE_MODE_HYBRID: 4}[form]
-        return 1 + (1 if R <= 16384 else 3) + ffn + 1
+        # The tensor-core form also launches the f16 copy of x.
+        ffn = {MOE_MODE_DECODE: 2 + (2 if self.shared is not None else 0), MOE_MODE_PREFILL: 3,
+               MOE_MODE_HYBRID: 5}[form]
+        return 1 + sort + ffn + 1
 
     def forward(self, x: torch.Tensor, logits: torch.Tensor, zero_mask: Optional[torch.Tensor] = None,
                 stream=None) -> torch.Tensor:
@@ -369,6 +416,10 @@ class MoEFFN:
     def _experts(self, x: torch.Tensor, stream) -> torch.Tensor:
         moe_sort(self.topk_ids, self.E, self.status, self.offsets, self.sorted_route, self.inv_route,
                  self.sort_ws, stream=stream)
+        if self.fused_combine:
+            return moe_expert_ffn_combine(x, self.K, self.routed, self.offsets, self.sorted_route, self.topk_w,
+                                          self.shared, self.out_dtype, self.status, self.out, self.ffn_ws,
+                                          stream=stream)
         moe_expert_ffn(x, self.K, self.routed, self.offsets, self.sorted_route, self.topk_w, self.shared,
                        self.mode, self.status, self.y_sorted, self.y_shared, self.ffn_ws, stream=stream)
         moe_combine(self.y_sorted, self.inv_route, self.y_shared, self.T, self.K, self.out_dtype, self.out,

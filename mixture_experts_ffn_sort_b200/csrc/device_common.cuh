@@ -431,6 +431,13 @@ __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_
 
 // ---------------------------------------------------------------- misc
 
+// Four fp32 additions into global memory (one vector reduction, relaxed,
+// performed at L2; the order of concurrent additions is unspecified).
+__device__ __forceinline__ void red_add_f32x4(float* p, float a, float b, float c, float d) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d)
+                 : "memory");
+}
+
 __device__ __forceinline__ float silu_f32(float z) { return z / (1.0f + __expf(-z)); }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {

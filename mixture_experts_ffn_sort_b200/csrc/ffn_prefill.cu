@@ -369,6 +369,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t* otile = b_ring + kSB * kBStage;           // 2 x [kNMax][128 B] bf16 output staging
     Barriers* B = reinterpret_cast<Barriers*>(otile + 2 * kOHalf);
     int* row_tok = reinterpret_cast<int*>(B + 1);      // [kNMax] activation row of each tile row
+                                                       // (down with out_acc: token of each column)
     float* col_w = reinterpret_cast<float*>(row_tok + kNMax);  // [kNMax] route weight of each column (down)
     float* sc_sm = col_w + kNMax;                              // [kScales] block scales of the item
     int* pre = reinterpret_cast<int*>(sc_sm + kScales);        // [E + 2]
@@ -503,11 +504,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 named_barrier_sync(4, 128);
                 for (int c = et; c < t.n; c += 128) {
                     float wv = 1.f;
+                    int tk = static_cast<int>(t.p0 + c);
                     if (!t.pt) {
                         const int rt = a.sorted_route[t.p0 + c];
-                        wv = (rt >= 0 && rt < R) ? a.topk_w[rt] : 0.f;
+                        const bool okr = rt >= 0 && rt < R;
+                        wv = okr ? a.topk_w[rt] : 0.f;
+                        tk = okr ? rt / a.K : -1;
                     }
                     col_w[c] = wv;
+                    if (a.out_acc) row_tok[c] = tk;
                 }
                 named_barrier_sync(4, 128);
             }
@@ -596,11 +601,30 @@ __global__ void __launch_bounds__(kThreads, 1)
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&B->d_empty[r]);
                 }
+                const int fb = t.fb0 + f;
+                if (MODE == kDown && a.out_acc) {
+                    // Fused combine: each row's 128 features (bf16, route weight
+                    // applied) are added into its token's fp32 output row, 8
+                    // features per thread as two vector reductions.
+                    named_barrier_sync(4, 128);
+                    for (int i = et; i < t.n * 16; i += 128) {
+                        const int rr = i >> 4, hh = (i >> 3) & 1, c8 = i & 7;
+                        const int tk = row_tok[rr];
+                        if (tk < 0) continue;
+                        const uint4 v =
+                            *reinterpret_cast<const uint4*>(otile + hh * kOHalf + rr * 128 + ((c8 ^ (rr & 7)) << 4));
+                        float* dst = a.out_acc + static_cast<size_t>(tk) * H + fb * 128 + hh * 64 + c8 * 8;
+                        red_add_f32x4(dst, __uint_as_float(v.x << 16), __uint_as_float(v.x & 0xFFFF0000u),
+                                      __uint_as_float(v.y << 16), __uint_as_float(v.y & 0xFFFF0000u));
+                        red_add_f32x4(dst + 4, __uint_as_float(v.z << 16), __uint_as_float(v.z & 0xFFFF0000u),
+                                      __uint_as_float(v.w << 16), __uint_as_float(v.w & 0xFFFF0000u));
+                    }
+                    continue;  // the next block's barrier orders these reads before its staging writes
+                }
                 // Staging tile -> global: TMA tensor stores of 32 rows x 64 features,
                 // and 16-byte thread stores for the rows past the last full group.
                 fence_proxy_async_smem();
                 named_barrier_sync(4, 128);
-                const int fb = t.fb0 + f;
                 const int n32 = t.n / kOStoreRows;
                 if (et < 2 * n32) {
                     const int hh = et & 1, k = et >> 1;
@@ -923,6 +947,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
+__global__ void __launch_bounds__(256) acc_to_bf16_kernel(const float* __restrict__ acc, long n8,
+                                                          uint16_t* __restrict__ out) {
+    for (long i = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
+         i += static_cast<long>(gridDim.x) * blockDim.x) {
+        const float4 a0 = reinterpret_cast<const float4*>(acc)[2 * i];
+        const float4 a1 = reinterpret_cast<const float4*>(acc)[2 * i + 1];
+        uint4 r;
+        r.x = pack_bf16x2(a0.x, a0.y);
+        r.y = pack_bf16x2(a0.z, a0.w);
+        r.z = pack_bf16x2(a1.x, a1.y);
+        r.w = pack_bf16x2(a1.z, a1.w);
+        reinterpret_cast<uint4*>(out)[i] = r;
+    }
+}
+
 size_t prefill_smem(int E) {
     return 1024 + kWRing + kSB * kBStage + 2 * kOHalf + sizeof(Barriers) + 2 * kNMax * 4 + kScales * 4 +
            (E + 2) * 4 + 64;
@@ -941,6 +980,15 @@ int num_sms() {
 
 }  // namespace
 
+cudaError_t launch_acc_to_bf16(const float* acc, long n, uint16_t* out, cudaStream_t stream) {
+    const long n8 = n / 8;
+    long blocks = (n8 + 255) / 256;
+    if (blocks > 148L * 32) blocks = 148L * 32;
+    if (blocks < 1) return cudaSuccess;
+    acc_to_bf16_kernel<<<static_cast<int>(blocks), 256, 0, stream>>>(acc, n8, out);
+    return cudaGetLastError();
+}
+
 bool ffn_prefill_supported(int H, int I) { return H % 128 == 0 && I % 128 == 0 && prefill_smem(MOE_MAX_E) <= 227 * 1024; }
 
 cudaError_t launch_ffn_prefill(const FfnArgs& a, cudaStream_t stream) {
@@ -955,7 +1003,7 @@ cudaError_t launch_ffn_prefill(const FfnArgs& a, cudaStream_t stream) {
     if (err == cudaSuccess) err = make_tmap_bf16_2d(&mg.out[0], a.h, R, I, 64, kOStoreRows);
     if (err == cudaSuccess) err = make_tmap_u8_2d(&md.w0[0], a.ex.w_down, E * H, I, 128, 128);
     if (err == cudaSuccess) err = make_tmap_bf16_2d(&md.act[0], a.h, R, I, 64, kNMax);
-    if (err == cudaSuccess) err = make_tmap_bf16_2d(&md.out[0], a.y, R, H, 64, kOStoreRows);
+    if (err == cudaSuccess && !a.out_acc) err = make_tmap_bf16_2d(&md.out[0], a.y, R, H, 64, kOStoreRows);
     if (a.sh.n) {
         const uint64_t Is = a.sh.inter;
         if (err == cudaSuccess) err = make_tmap_u8_2d(&mg.w0[1], a.sh.w_gate, Is, H, Cfg<0>::kWCols, 128, Cfg<0>::kWCols);
@@ -963,7 +1011,7 @@ cudaError_t launch_ffn_prefill(const FfnArgs& a, cudaStream_t stream) {
         if (err == cudaSuccess) err = make_tmap_bf16_2d(&mg.out[1], a.h_sh, T, Is, 64, kOStoreRows);
         if (err == cudaSuccess) err = make_tmap_u8_2d(&md.w0[1], a.sh.w_down, H, Is, 128, 128);
         if (err == cudaSuccess) err = make_tmap_bf16_2d(&md.act[1], a.h_sh, T, Is, 64, kNMax);
-        if (err == cudaSuccess) err = make_tmap_bf16_2d(&md.out[1], a.y_sh, T, H, 64, kOStoreRows);
+        if (err == cudaSuccess && !a.out_acc) err = make_tmap_bf16_2d(&md.out[1], a.y_sh, T, H, 64, kOStoreRows);
     }
     if (err != cudaSuccess) return err;
     const size_t smem = prefill_smem(a.ex.n);

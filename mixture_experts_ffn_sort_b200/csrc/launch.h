@@ -79,6 +79,10 @@ struct FfnArgs {
     // scales ([T] f32).
     uint16_t* x16;
     float* xinv;
+    // Prefill form only: when not null, the down epilogue adds each row's
+    // bf16 result (route weight applied) into out_acc[token] ([T, H] f32, zeroed
+    // by the caller) with fp32 reductions instead of storing y / y_sh.
+    float* out_acc;
 };
 
 // Bytes of the prefill form's f16 activation copy and its row scales (256-byte aligned).
@@ -100,5 +104,7 @@ cudaError_t make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows,
 // Routed rows (a.identity must be false) plus the optional shared expert a.sh.
 cudaError_t launch_ffn_prefill(const FfnArgs& a, cudaStream_t stream);
 bool ffn_prefill_supported(int H, int I);
+// out[T, H] = bf16(acc[T, H]) (the last step of the fused down + combine).
+cudaError_t launch_acc_to_bf16(const float* acc, long n, uint16_t* out, cudaStream_t stream);
 
 }  // namespace moe

@@ -391,6 +391,85 @@ int moe_expert_ffn(const uint16_t* x, int T, int H, int K, const moe_fp8_experts
     return MOE_OK;
 }
 
+size_t moe_ffn_combine_workspace_bytes(int T, int K, int H, int E, int I, int I_shared, int out_dtype) {
+    (void)E;
+    if (T < 0 || K < 1 || I < 0 || I_shared < 0 || H < 0) return 0;
+    const long R = static_cast<long>(T) * K;
+    size_t b = ffn_h_bytes(R, I) + ffn_h_bytes(T, I_shared) + moe::ffn_x16_bytes(T, H) + moe::ffn_xinv_bytes(T);
+    if (out_dtype != MOE_OUT_F32) b += round256(static_cast<size_t>(T) * H * 4);  // the fp32 accumulator
+    return b;
+}
+
+int moe_expert_ffn_combine(const uint16_t* x, int T, int H, int K, const moe_fp8_experts* routed,
+                           const moe_fp8_experts* shared, const int32_t* expert_offsets, const int32_t* sorted_route,
+                           const float* topk_w, void* out, int out_dtype, void* workspace, size_t workspace_bytes,
+                           int32_t* status, moe_stream_t stream) {
+    g_err.clear();
+    if (!routed) return fail(MOE_ERR_INVALID_ARG, "moe_expert_ffn_combine: routed must not be NULL");
+    const int E = routed->n_experts, I = routed->inter;
+    int rc = check_sizes(T, E, K);
+    if (rc) return rc;
+    if (out_dtype != MOE_OUT_BF16 && out_dtype != MOE_OUT_F32)
+        return fail(MOE_ERR_INVALID_ARG, "moe_expert_ffn_combine: out_dtype=%d is not BF16/F32", out_dtype);
+    if (H < 128 || H % MOE_BLOCK || H > 8192)
+        return fail(MOE_ERR_UNSUPPORTED_SHAPE, "moe_expert_ffn_combine: H=%d must be a multiple of 128 in 128..=8192",
+                    H);
+    if ((rc = check_experts(routed, H, "routed"))) return rc;
+    if (shared) {
+        if (shared->n_experts != 1)
+            return fail(MOE_ERR_INVALID_ARG, "moe_expert_ffn_combine: shared->n_experts=%d must be 1",
+                        shared->n_experts);
+        if ((rc = check_experts(shared, H, "shared"))) return rc;
+    }
+    if (!moe::ffn_prefill_supported(H, I))
+        return fail(MOE_ERR_UNSUPPORTED_SHAPE, "moe_expert_ffn_combine: H=%d, inter=%d not supported", H, I);
+    if (T == 0) return MOE_OK;
+    if (!x || !expert_offsets || !sorted_route || !topk_w || !out)
+        return fail(MOE_ERR_INVALID_ARG, "moe_expert_ffn_combine: NULL tensor pointer");
+    if (!aligned16(x) || !aligned16(expert_offsets) || !aligned16(sorted_route) || !aligned16(topk_w) ||
+        !aligned16(out) || !aligned16(workspace) || (reinterpret_cast<uintptr_t>(status) & 3))
+        return fail(MOE_ERR_MISALIGNED,
+                    "moe_expert_ffn_combine: tensor bases must be 16-byte aligned and status 4-byte aligned");
+    const long R = static_cast<long>(T) * K;
+    const int Is = shared ? shared->inter : 0;
+    const size_t need = moe_ffn_combine_workspace_bytes(T, K, H, E, I, Is, out_dtype);
+    if (workspace_bytes < need || !workspace)
+        return fail(MOE_ERR_WORKSPACE_TOO_SMALL, "moe_expert_ffn_combine: workspace of %zu bytes, need %zu",
+                    workspace_bytes, need);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    const size_t off_x16 = ffn_h_bytes(R, I) + ffn_h_bytes(T, Is);
+    const size_t off_acc = off_x16 + moe::ffn_x16_bytes(T, H) + moe::ffn_xinv_bytes(T);
+    float* acc = out_dtype == MOE_OUT_F32 ? static_cast<float*>(out) : reinterpret_cast<float*>(ws + off_acc);
+    cudaError_t e = cudaMemsetAsync(acc, 0, static_cast<size_t>(T) * H * 4, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "moe_expert_ffn_combine memset");
+    moe::FfnArgs a{};
+    a.x = x;
+    a.T = T;
+    a.H = H;
+    a.K = K;
+    a.ex = {routed->w_gate, routed->w_up, routed->w_down, routed->s_gate, routed->s_up, routed->s_down, E, I};
+    a.offsets = expert_offsets;
+    a.sorted_route = sorted_route;
+    a.topk_w = topk_w;
+    a.h = reinterpret_cast<uint16_t*>(ws);
+    a.status = status;
+    a.avg_rows = static_cast<int>((R + E - 1) / E);
+    if (shared) {
+        a.sh = {shared->w_gate, shared->w_up, shared->w_down, shared->s_gate, shared->s_up, shared->s_down, 1, Is};
+        a.h_sh = reinterpret_cast<uint16_t*>(ws + ffn_h_bytes(R, I));
+    }
+    a.x16 = reinterpret_cast<uint16_t*>(ws + off_x16);
+    a.xinv = reinterpret_cast<float*>(ws + off_x16 + moe::ffn_x16_bytes(T, H));
+    a.out_acc = acc;
+    e = moe::launch_ffn_prefill(a, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "moe_expert_ffn_combine launch");
+    if (out_dtype == MOE_OUT_BF16) {
+        e = moe::launch_acc_to_bf16(acc, static_cast<long>(T) * H, static_cast<uint16_t*>(out), stream);
+        if (e != cudaSuccess) return cuda_fail(e, "moe_expert_ffn_combine convert");
+    }
+    return MOE_OK;
+}
+
 int moe_combine(const uint16_t* y_sorted, const int32_t* inv_route, const uint16_t* y_shared, int T,
                 int K, int H, void* out, int out_dtype, int32_t* status, moe_stream_t stream) {
     g_err.clear();

@@ -57,6 +57,11 @@ def test_workspace_queries(L):
         81920 * 512 + 8192 * 512 + 8192 * 4096 * 2 + 8192 * 4
     assert L.moe_ffn_workspace_bytes(64, 8, 2048, 256, 512, 0, moe.MOE_MODE_PREFILL) == \
         512 * 512 * 2 + 64 * 2048 * 2 + 256
+    # The fused FFN + combine: no y_sorted, an fp32 accumulator for a bf16 output.
+    base = 81920 * 512 + 8192 * 512 + 8192 * 4096 * 2 + 8192 * 4
+    assert L.moe_ffn_combine_workspace_bytes(8192, 10, 4096, 512, 256, 256, moe.MOE_OUT_F32) == base
+    assert L.moe_ffn_combine_workspace_bytes(8192, 10, 4096, 512, 256, 256, moe.MOE_OUT_BF16) == \
+        base + 8192 * 4096 * 4
 
 
 def test_ffn_resolve_mode(L):

@@ -123,6 +123,25 @@ def test_pipeline(cfg):
         assert_moe_close(to_f64(out[torch.from_numpy(tk).long().cuda()]), ref, "out rows")
 
 
+def test_pipeline_fused_combine(cfg):
+    """The layer with moe_expert_ffn_combine (no y_sorted) on the workloads the
+    tensor-core form serves: every token of the 8192-token prefill, sampled
+    tokens of the large one."""
+    if cfg not in ("prefill", "prefill_large", "decode_skew"):
+        pytest.skip("the fused combine runs the tensor-core form")
+    w, dw = workload(cfg), device_workload(cfg)
+    layer = moe.MoEFFN(dw.routed, w.shape.T, w.shape.K, dw.shared, fused_combine=True)
+    out = layer(dw.x, dw.logits, dw.zero_mask)
+    torch.cuda.synchronize()
+    assert layer.status.item() == 0
+    if cfg in FULL:
+        assert_moe_close(out, oracle_full(cfg)["out"], "out")
+    else:
+        tk = sample_tokens(w.shape.T, SAMPLE_ROWS, seed=3)
+        ref = oracle.moe_tokens(w.x, w.logits, w.shape.K, w.routed, w.shared, w.zero_mask, tokens=tk)
+        assert_moe_close(to_f64(out[torch.from_numpy(tk).long().cuda()]), ref, "out rows")
+
+
 # ---------------------------------------------------------------- edge cases
 
 def _small(T, H, I, E, K, seed=0, shared_I=0, std=0.05):

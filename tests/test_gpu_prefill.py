@@ -103,3 +103,44 @@ def test_prefill_special_codes():
         out = layer(bf16_tensor(x), dev(lg))
         torch.cuda.synchronize()
         assert_moe_close(out, oracle.moe(x, lg, K, ex)["out"], "out")
+
+
+@pytest.mark.parametrize("T,H,I,E,K,Is,zf", [(300, 512, 256, 16, 4, 128, 0.05), (64, 256, 128, 8, 2, 0, 0.0),
+                                             (1000, 1024, 256, 32, 6, 256, 0.01), (193, 384, 128, 5, 2, 0, 0.0)])
+@pytest.mark.parametrize("out_dtype", [moe.MOE_OUT_BF16, moe.MOE_OUT_F32])
+def test_fused_ffn_combine(T, H, I, E, K, Is, zf, out_dtype):
+    """moe_expert_ffn_combine (the down epilogue reducing into the fp32 output
+    rows) against the oracle, with zero-weight routes and a shared expert."""
+    ex = wl.draw_experts(8, 66, E, I, H, 0.05, threads=4)
+    sh = wl.draw_experts(8, 67, 1, Is, H, 0.05, threads=1) if Is else None
+    x = wl.random_rows_bf16(T, H, seed=T + 1)
+    lg = np.random.default_rng(T + 2).standard_normal((T, E)).astype(np.float32)
+    mask = (np.random.default_rng(T + 3).random((T, K)) < zf).astype(np.uint8) if zf else None
+    layer = moe.MoEFFN(moe.Experts.from_host(ex), T, K, moe.Experts.from_host(sh) if sh else None,
+                       out_dtype=out_dtype, fused_combine=True)
+    out = layer(bf16_tensor(x), dev(lg), dev(mask) if mask is not None else None)
+    torch.cuda.synchronize()
+    assert layer.status.item() == 0
+    assert out.dtype == (torch.bfloat16 if out_dtype == moe.MOE_OUT_BF16 else torch.float32)
+    assert_moe_close(out, oracle.moe(x, lg, K, ex, sh, mask)["out"], "fused out")
+
+
+def test_fused_ffn_combine_matches_two_calls():
+    """The fused call and moe_expert_ffn + moe_combine agree to fp32 summation
+    order (same bf16 rows, different order of the fp32 additions)."""
+    T, H, I, E, K, Is = 500, 512, 256, 16, 4, 128
+    ex = wl.draw_experts(9, 68, E, I, H, 0.05, threads=4)
+    sh = wl.draw_experts(9, 69, 1, Is, H, 0.05, threads=1)
+    x = wl.random_rows_bf16(T, H, seed=9)
+    lg = np.random.default_rng(10).standard_normal((T, E)).astype(np.float32)
+    a = moe.MoEFFN(moe.Experts.from_host(ex), T, K, moe.Experts.from_host(sh), mode=moe.MOE_MODE_PREFILL,
+                   out_dtype=moe.MOE_OUT_F32)
+    b = moe.MoEFFN(moe.Experts.from_host(ex), T, K, moe.Experts.from_host(sh), out_dtype=moe.MOE_OUT_F32,
+                   fused_combine=True)
+    oa = a(bf16_tensor(x), dev(lg)).double().cpu().numpy()
+    ob = b(bf16_tensor(x), dev(lg)).double().cpu().numpy()
+    torch.cuda.synchronize()
+    ys = a.y_sorted.float().abs().cpu().numpy()
+    inv = a.inv_route.cpu().numpy().reshape(T, K)
+    bound = ys[inv].sum(axis=1) + np.abs(a.y_shared.float().cpu().numpy())
+    assert np.all(np.abs(oa - ob) <= (K + 2) * 2.0 ** -23 * bound + 1e-30)
