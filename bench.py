@@ -223,11 +223,11 @@ ARITHMETIC = {
     "decode": ("f16", "E4M3 weights taken exactly as f16 MMA operands, activations as f16 after an exact "
                       "power-of-two row scale, fp32 accumulate, fp32 block scale per 128-column partial; "
                       "bf16 h, y_sorted and out"),
-    "prefill": ("bf16", "weights decoded to bf16(e4m3 x block scale), bf16 activations, fp32 accumulate in "
-                        "TMEM; bf16 h, y_sorted and out"),
+    "prefill": ("f16+bf16", "gate/up: f16 MMA on f16(e4m3 x block scale x 2^ka) and f16(x x 2^k_t), power-of-two "
+                            "row scales undone in the epilogue; down: bf16 MMA on bf16(e4m3 x block scale) and bf16 "
+                            "h; fp32 accumulate in TMEM; bf16 h, y_sorted and out"),
     "hybrid": ("f16+bf16", "experts with few rows as the decode form (f16 MMA on exact E4M3), the others as the "
-                           "prefill form (bf16 MMA on bf16(e4m3 x scale)); fp32 accumulate; bf16 h, y_sorted "
-                           "and out"),
+                           "prefill form (f16 gate/up, bf16 down); fp32 accumulate; bf16 h, y_sorted and out"),
 }
 
 

@@ -945,6 +945,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
+    // Launched as a programmatic dependent of the weight-streaming down kernel
+    // (MOE_MODE_HYBRID), gate/up overlaps that grid's tail without reading
+    // anything it writes; waiting for it here, at the end, makes this grid's
+    // completion -- which the down GEMM and later launches wait for -- imply
+    // that grid's.  A no-op for a normal launch.
+    if (MODE == kGateUp && threadIdx.x == 0) grid_dependency_wait();
 }
 
 __global__ void __launch_bounds__(256) acc_to_bf16_kernel(const float* __restrict__ acc, long n8,
@@ -991,7 +997,7 @@ cudaError_t launch_acc_to_bf16(const float* acc, long n, uint16_t* out, cudaStre
 
 bool ffn_prefill_supported(int H, int I) { return H % 128 == 0 && I % 128 == 0 && prefill_smem(MOE_MAX_E) <= 227 * 1024; }
 
-cudaError_t launch_ffn_prefill(const FfnArgs& a, cudaStream_t stream) {
+cudaError_t launch_ffn_prefill(const FfnArgs& a, cudaStream_t stream, bool x16_done, bool gateup_after_decode) {
     if (a.identity || !a.x16 || !a.xinv) return cudaErrorInvalidValue;
     const uint64_t E = static_cast<uint64_t>(a.ex.n), I = a.ex.inter, H = a.H;
     const uint64_t R = static_cast<uint64_t>(a.T) * a.K, T = static_cast<uint64_t>(a.T);
@@ -1020,13 +1026,10 @@ cudaError_t launch_ffn_prefill(const FfnArgs& a, cudaStream_t stream) {
         err = cudaFuncSetAttribute(prefill_kernel<kDown>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (err != cudaSuccess) return err;
     const int grid = num_sms();
-    x16_kernel<<<static_cast<unsigned>((static_cast<long>(a.T) * 32 + 255) / 256), 256, 0, stream>>>(a.x, a.T, a.H,
-                                                                                                   a.x16, a.xinv);
-    err = cudaGetLastError();
-    if (err != cudaSuccess) return err;
-    prefill_kernel<kGateUp><<<grid, kThreads, smem, stream>>>(mg, a);
-    err = cudaGetLastError();
-    if (err != cudaSuccess) return err;
+    if (!x16_done) {
+        err = launch_x16(a, stream);
+        if (err != cudaSuccess) return err;
+    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(kThreads);
@@ -1036,8 +1039,19 @@ cudaError_t launch_ffn_prefill(const FfnArgs& a, cudaStream_t stream) {
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
+    // gate/up: a programmatic dependent of the preceding kernel only when that
+    // kernel is the weight-streaming down GEMM of the same call.
+    cfg.numAttrs = gateup_after_decode ? 1 : 0;
+    err = cudaLaunchKernelEx(&cfg, prefill_kernel<kGateUp>, mg, a);
+    if (err != cudaSuccess) return err;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, prefill_kernel<kDown>, md, a);
+}
+
+cudaError_t launch_x16(const FfnArgs& a, cudaStream_t stream) {
+    x16_kernel<<<static_cast<unsigned>((static_cast<long>(a.T) * 32 + 255) / 256), 256, 0, stream>>>(a.x, a.T, a.H,
+                                                                                                   a.x16, a.xinv);
+    return cudaGetLastError();
 }
 
 }  // namespace moe

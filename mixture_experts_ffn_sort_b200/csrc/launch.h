@@ -102,7 +102,13 @@ cudaError_t make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows,
 
 // ---------------------------------------------------------------- expert FFN (prefill, tcgen05)
 // Routed rows (a.identity must be false) plus the optional shared expert a.sh.
-cudaError_t launch_ffn_prefill(const FfnArgs& a, cudaStream_t stream);
+// x16_done: the f16 copy of x (launch_x16) was already launched on the stream.
+// gateup_after_decode: the preceding launch is the weight-streaming down
+// kernel of the same call, which gate/up overlaps (programmatic dependent launch).
+cudaError_t launch_ffn_prefill(const FfnArgs& a, cudaStream_t stream, bool x16_done = false,
+                               bool gateup_after_decode = false);
+// The f16 copy of x and its row scales (a.x16, a.xinv) for the tensor-core kernels.
+cudaError_t launch_x16(const FfnArgs& a, cudaStream_t stream);
 bool ffn_prefill_supported(int H, int I);
 // out[T, H] = bf16(acc[T, H]) (the last step of the fused down + combine).
 cudaError_t launch_acc_to_bf16(const float* acc, long n, uint16_t* out, cudaStream_t stream);

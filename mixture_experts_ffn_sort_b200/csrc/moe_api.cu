@@ -361,17 +361,28 @@ int moe_expert_ffn(const uint16_t* x, int T, int H, int K, const moe_fp8_experts
             a.h_sh = reinterpret_cast<uint16_t*>(ws + ffn_h_bytes(R, I));
             a.y_sh = y_shared;
         }
-        // HYBRID: the experts with more than MOE_HYBRID_ROW_SPLIT rows here, the
-        // others in the decode form below.
-        a.row_split = form == MOE_MODE_HYBRID ? MOE_HYBRID_ROW_SPLIT : 0;
         a.x16 = reinterpret_cast<uint16_t*>(ws + ffn_h_bytes(R, I) + ffn_h_bytes(T, Is));
         a.xinv = reinterpret_cast<float*>(ws + ffn_h_bytes(R, I) + ffn_h_bytes(T, Is) + moe::ffn_x16_bytes(T, H));
-        const cudaError_t e = moe::launch_ffn_prefill(a, stream);
-        if (e != cudaSuccess || form == MOE_MODE_PREFILL)
+        if (form == MOE_MODE_PREFILL) {
+            const cudaError_t e = moe::launch_ffn_prefill(a, stream);
             return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_expert_ffn launch");
-        // The decode form gets experts of at most MOE_HYBRID_ROW_SPLIT rows: its
-        // token group (8, 16 or 32 rows, from the average rows) covers them.
-        a.avg_rows = MOE_HYBRID_ROW_SPLIT / 2;
+        }
+        // HYBRID: the experts with at most MOE_HYBRID_ROW_SPLIT rows in the
+        // weight-streaming kernels (token groups of 8 rows), the others and the
+        // shared expert in the tensor-core kernels, launched after them as
+        // programmatic dependents so that they fill the SMs the weight-streaming
+        // down grid's tail leaves idle.  Each form skips the experts of the other.
+        cudaError_t e = moe::launch_x16(a, stream);
+        if (e != cudaSuccess) return cuda_fail(e, "moe_expert_ffn launch");
+        moe::FfnArgs d = a;
+        d.row_split = MOE_HYBRID_ROW_SPLIT;
+        d.avg_rows = MOE_HYBRID_ROW_SPLIT / 2;
+        d.sh = {};
+        e = moe::launch_ffn_decode(d, stream);
+        if (e != cudaSuccess) return cuda_fail(e, "moe_expert_ffn routed launch");
+        a.row_split = MOE_HYBRID_ROW_SPLIT;
+        e = moe::launch_ffn_prefill(a, stream, /*x16_done=*/true, /*gateup_after_decode=*/true);
+        return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_expert_ffn launch");
     }
     cudaError_t e = moe::launch_ffn_decode(a, stream);
     if (e != cudaSuccess) return cuda_fail(e, "moe_expert_ffn routed launch");
