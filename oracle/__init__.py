@@ -78,6 +78,14 @@ def lib():
             L.oracle_expert_rows.argtypes = [P, I, P, I, P, I, P]
             L.oracle_moe_tokens_routed.argtypes = [P, I, I, P, P, P, P, P, I, P]
             L.oracle_swiglu.argtypes = [P, P, I, P]
+            L.oracle_e4m3fn_round.restype = ctypes.c_double
+            L.oracle_e4m3fn_round.argtypes = [ctypes.c_double]
+            L.oracle_e4m3fn_round_array.argtypes = [P, I, P]
+            L.oracle_act_scale_exp.restype = I
+            L.oracle_act_scale_exp.argtypes = [ctypes.c_double]
+            L.oracle_act_quantize.argtypes = [P, I, I, P]
+            L.oracle_ffn_sorted_w8a8.argtypes = [P, I, I, I, P, P, P, P, P]
+            L.oracle_ffn_shared_w8a8.argtypes = [P, I, I, P, P]
             L.oracle_set_threads(int(os.environ.get("ORACLE_THREADS", os.cpu_count() or 1)))
             _lib = L
     return _lib
@@ -233,6 +241,52 @@ def ffn_shared(x: np.ndarray, shared) -> np.ndarray:
     ex = _ExpertsRef(shared)
     y = np.empty((T, H), np.float64)
     lib().oracle_ffn_shared(_p(x), T, H, ex.ref(), _p(y))
+    return y
+
+
+# ---------------------------------------------------------------- W8A8 form (FP8 activations)
+
+XQ_BLOCK, HQ_BLOCK = 128, 64
+
+
+def e4m3fn_round(v) -> np.ndarray:
+    """Nearest E4M3FN value (ties to even, saturating at 448) of each element."""
+    a = _c(np.atleast_1d(v), np.float64)
+    out = np.empty_like(a)
+    lib().oracle_e4m3fn_round_array(_p(a), a.size, _p(out))
+    return out.reshape(np.shape(v))
+
+
+def act_scale_exp(amax: float) -> int:
+    """k with amax * 2^k in (224, 448] (0 for amax == 0, k in [-126, 126])."""
+    return int(lib().oracle_act_scale_exp(float(amax)))
+
+
+def act_quantize(v: np.ndarray, block: int) -> np.ndarray:
+    """Blocks of `block` values -> e4m3fn(v * 2^k) * 2^-k, k from each block's largest |v|."""
+    a = _c(v, np.float64).ravel()
+    out = np.empty_like(a)
+    lib().oracle_act_quantize(_p(a), a.size, int(block), _p(out))
+    return out.reshape(np.shape(v))
+
+
+def ffn_sorted_w8a8(x: np.ndarray, K: int, experts, offsets, sorted_route, w) -> np.ndarray:
+    """ffn_sorted in the W8A8 form: x quantised per 128-column block, h per 64-feature block."""
+    x = _c(x, np.uint16)
+    T, H = x.shape
+    ex = _ExpertsRef(experts)
+    off, sr, wv = _c(offsets, np.int32), _c(sorted_route, np.int32), _c(w, np.float64).ravel()
+    y = np.zeros((T * K, H), np.float64)
+    lib().oracle_ffn_sorted_w8a8(_p(x), T, H, K, ex.ref(), _p(off), _p(sr), _p(wv), _p(y))
+    return y
+
+
+def ffn_shared_w8a8(x: np.ndarray, shared) -> np.ndarray:
+    x = _c(x, np.uint16)
+    T, H = x.shape
+    ex = _ExpertsRef(shared)
+    y = np.empty((T, H), np.float64)
+    lib().oracle_ffn_shared_w8a8(_p(x), T, H, ex.ref(), _p(y))
     return y
 
 

@@ -575,3 +575,133 @@ void oracle_expert_rows(const uint16_t* x, int H, const oracle_experts* ex, int 
 void oracle_swiglu(const double* g, const double* u, int n, double* h) {
     for (int i = 0; i < n; ++i) h[i] = (g[i] / (1.0 + exp(-g[i]))) * u[i];
 }
+
+/* ---------------------------------------------------------------- FP8 activations (W8A8) */
+
+/* The opt-in W8A8 form: the activations of both GEMMs also become E4M3FN
+ * values, in blocks with one power-of-two scale each (the FP8 activation
+ * quantisation of the NKI Library's Blockwise MM Forward MXFP8 kernel and the
+ * in-register quantisation of the hidden activation of the aiter gfx950 PR,
+ * there with MX formats; here E4M3FN with a power-of-two scale per block, the
+ * plainest reading that keeps the weights' own format).  Blocks: 128 columns
+ * of x (one weight scale block), 64 features of h. */
+#define ORACLE_XQ_BLOCK 128
+#define ORACLE_HQ_BLOCK 64
+
+/* Nearest E4M3FN value to v, ties to the even mantissa (round to nearest
+ * even), magnitudes at or above the largest finite value 448 giving 448
+ * (saturating conversion).  Subnormals are the multiples of 2^-9 below 2^-6;
+ * in the binade [2^e, 2^(e+1)) the values are the multiples of 2^(e-3). */
+double oracle_e4m3fn_round(double v) {
+    if (v != v) return NAN;
+    double a = fabs(v), q;
+    if (a >= 448.0) {
+        q = 448.0;
+    } else if (a < ldexp(1.0, -6)) {
+        q = nearbyint(ldexp(a, 9)) * ldexp(1.0, -9);
+    } else {
+        int e;
+        frexp(a, &e); /* a = f * 2^e, f in [0.5, 1): the binade is [2^(e-1), 2^e) */
+        q = ldexp(nearbyint(ldexp(a, 4 - e)), e - 4);
+    }
+    return v < 0 ? -q : q;
+}
+
+void oracle_e4m3fn_round_array(const double* v, int n, double* out) {
+    for (int i = 0; i < n; ++i) out[i] = oracle_e4m3fn_round(v[i]);
+}
+
+/* Scale exponent k of an activation block whose largest magnitude is amax:
+ * amax * 2^k lies in (224, 448] (the top binade of E4M3FN up to its largest
+ * value), k limited to [-126, 126]; 0 for an all-zero block. */
+int oracle_act_scale_exp(double amax) {
+    if (!(amax > 0.0)) return 0;
+    int e;
+    double f = frexp(amax, &e); /* amax = (2f) * 2^(e-1), 2f in [1, 2) */
+    int k = (2.0 * f <= 1.75 ? 8 : 7) - (e - 1);
+    if (k > 126) k = 126;
+    if (k < -126) k = -126;
+    return k;
+}
+
+/* v[0..n) in blocks of `block`: each block becomes e4m3fn(v * 2^k) * 2^-k
+ * with k = oracle_act_scale_exp(largest |v| of the block). */
+void oracle_act_quantize(const double* v, int n, int block, double* out) {
+    for (int b0 = 0; b0 < n; b0 += block) {
+        int b1 = b0 + block < n ? b0 + block : n;
+        double amax = 0.0;
+        for (int i = b0; i < b1; ++i) amax = fabs(v[i]) > amax ? fabs(v[i]) : amax;
+        int k = oracle_act_scale_exp(amax);
+        for (int i = b0; i < b1; ++i) out[i] = ldexp(oracle_e4m3fn_round(ldexp(v[i], k)), -k);
+    }
+}
+
+/* One expert on one row in the W8A8 form: xq = quantised x (blocks of 128
+ * columns); h = silu(Wg xq) * (Wu xq); hq = quantised h (blocks of 64
+ * features); y = Wd hq.  Every product and sum in fp64. */
+static void expert_row_w8a8(const double* x, int H, int I,
+                            const uint8_t* wg, const float* sg, const uint8_t* wu, const float* su,
+                            const uint8_t* wd, const float* sd, double* xq, double* h, double* y) {
+    oracle_act_quantize(x, H, ORACLE_XQ_BLOCK, xq);
+    for (int i = 0; i < I; ++i) {
+        double g = 0.0, u = 0.0;
+        for (int k = 0; k < H; ++k) {
+            g += weight(wg, sg, H, i, k) * xq[k];
+            u += weight(wu, su, H, i, k) * xq[k];
+        }
+        h[i] = (g / (1.0 + exp(-g))) * u;
+    }
+    oracle_act_quantize(h, I, ORACLE_HQ_BLOCK, h);
+    for (int n = 0; n < H; ++n) {
+        double acc = 0.0;
+        for (int i = 0; i < I; ++i) acc += weight(wd, sd, I, n, i) * h[i];
+        y[n] = acc;
+    }
+}
+
+/* oracle_ffn_sorted in the W8A8 form: y_sorted[p] = w[r] * FFN_e^{W8A8}(x[t]). */
+void oracle_ffn_sorted_w8a8(const uint16_t* x, int T, int H, int K, const oracle_experts* ex,
+                            const int32_t* offsets, const int32_t* sorted_route, const double* w,
+                            double* y_sorted) {
+    init_tables();
+    (void)T;
+    int E = ex->n_experts, I = ex->inter;
+    for (int e = 0; e < E; ++e) {
+        const uint8_t *wg, *wu, *wd; const float *sg, *su, *sd;
+        expert_ptrs(ex, e, H, &wg, &sg, &wu, &su, &wd, &sd);
+        int p0 = offsets[e], p1 = offsets[e + 1];
+#pragma omp parallel for num_threads(g_threads) schedule(dynamic, 1)
+        for (int p = p0; p < p1; ++p) {
+            double* xr = (double*)malloc(sizeof(double) * (size_t)H);
+            double* xq = (double*)malloc(sizeof(double) * (size_t)H);
+            double* h = (double*)malloc(sizeof(double) * (size_t)I);
+            int r = sorted_route[p];
+            load_row(x, H, r / K, xr);
+            double* y = y_sorted + (size_t)p * H;
+            expert_row_w8a8(xr, H, I, wg, sg, wu, su, wd, sd, xq, h, y);
+            for (int n = 0; n < H; ++n) y[n] *= w[r];
+            free(xr);
+            free(xq);
+            free(h);
+        }
+    }
+}
+
+/* The shared expert in the W8A8 form: y_shared[t] = FFN_s^{W8A8}(x[t]). */
+void oracle_ffn_shared_w8a8(const uint16_t* x, int T, int H, const oracle_experts* sh, double* y_shared) {
+    init_tables();
+    const uint8_t *wg, *wu, *wd; const float *sg, *su, *sd;
+    expert_ptrs(sh, 0, H, &wg, &sg, &wu, &su, &wd, &sd);
+    int I = sh->inter;
+#pragma omp parallel for num_threads(g_threads) schedule(dynamic, 1)
+    for (int t = 0; t < T; ++t) {
+        double* xr = (double*)malloc(sizeof(double) * (size_t)H);
+        double* xq = (double*)malloc(sizeof(double) * (size_t)H);
+        double* h = (double*)malloc(sizeof(double) * (size_t)I);
+        load_row(x, H, t, xr);
+        expert_row_w8a8(xr, H, I, wg, sg, wu, su, wd, sd, xq, h, y_shared + (size_t)t * H);
+        free(xr);
+        free(xq);
+        free(h);
+    }
+}

@@ -565,3 +565,135 @@ def test_router_logits_permutations_and_linearity():
     assert np.array_equal(oracle.router_logits(x, w[pe]), base[:, pe])
     x4 = wl.to_bf16_bits(oracle.bf16_array(x).astype(np.float32) * np.float32(4.0))
     assert np.array_equal(oracle.router_logits(x4, w), 4.0 * base)
+
+
+# ------------------------------------------------------------------ W8A8 form (FP8 activations)
+
+def _torch_e4m3(v32: np.ndarray) -> np.ndarray:
+    """Library rounding: torch's float32 -> float8_e4m3fn cast (round to nearest
+    even; it gives NaN at and above 464 instead of saturating)."""
+    t = torch.from_numpy(np.ascontiguousarray(v32, dtype=np.float32))
+    return t.to(torch.float8_e4m3fn).to(torch.float64).numpy()
+
+
+def test_e4m3fn_round_matches_torch_cast():
+    """Catches a wrong tie rule, a wrong binade or subnormal step, a lost sign."""
+    rng = np.random.default_rng(11)
+    mags = np.exp2(rng.uniform(-13.0, np.log2(463.0), 20000))
+    vals = (mags * rng.choice([-1.0, 1.0], mags.size)).astype(np.float32)
+    codes = torch.arange(256, dtype=torch.int32).to(torch.uint8).view(torch.float8_e4m3fn).to(torch.float64)
+    finite = np.unique(np.abs(codes.numpy()[np.isfinite(codes.numpy())]))
+    mids = ((finite[1:] + finite[:-1]) / 2).astype(np.float32)  # exact in fp32
+    for v in (vals, finite.astype(np.float32), mids, -mids):
+        np.testing.assert_array_equal(oracle.e4m3fn_round(v.astype(np.float64)), _torch_e4m3(v))
+
+
+def test_e4m3fn_round_saturates():
+    """The saturating conversion: everything at or above 448 in magnitude gives 448."""
+    r = oracle.e4m3fn_round(np.array([448.0, 463.99, 464.0, 1e9, -500.0, -448.0]))
+    np.testing.assert_array_equal(r, [448.0, 448.0, 448.0, 448.0, -448.0, -448.0])
+    assert np.isnan(oracle.e4m3fn_round(np.array([np.nan]))[0])
+
+
+def _k_by_search(amax: float) -> int:
+    """Brute force: the largest k in [-126, 126] with amax * 2^k <= 448."""
+    if amax == 0:
+        return 0
+    ks = [k for k in range(-126, 127) if amax * 2.0 ** k <= 448.0]
+    return max(ks) if ks else -126
+
+
+def test_act_scale_exp_is_the_largest_fitting_power_of_two():
+    """Catches an off-by-one exponent (a block scaled into saturation, or one
+    binade too low) and a wrong 1.75 boundary."""
+    rng = np.random.default_rng(12)
+    amaxes = list(np.exp2(rng.uniform(-40, 40, 2000))) + [1.75, np.nextafter(1.75, 2), 1.0, 2.0, 448.0,
+                                                          224.0, np.nextafter(224.0, 0), 3.5, 0.0]
+    for a in amaxes:
+        k = oracle.act_scale_exp(a)
+        assert k == _k_by_search(a), a
+        if a:
+            assert 224.0 < a * 2.0 ** k <= 448.0
+
+
+def test_act_quantize_matches_torch_blocks():
+    """Blocks of 128 (x) and 64 (h): each block scaled by its own power of two,
+    rounded with torch's cast, scaled back.  Catches a block boundary or a
+    scale taken from the wrong block."""
+    rng = np.random.default_rng(13)
+    for block in (128, 64):
+        v = rng.standard_normal(16 * block) * np.exp2(rng.integers(-20, 20, 16 * block // block).repeat(block))
+        v32 = v.astype(np.float32).astype(np.float64)  # fp32-exact inputs (as bf16 and fp32 activations are)
+        ref = np.empty_like(v32)
+        for b0 in range(0, v32.size, block):
+            blk = v32[b0:b0 + block]
+            k = _k_by_search(np.abs(blk).max())
+            ref[b0:b0 + block] = _torch_e4m3((blk * 2.0 ** k).astype(np.float32)) * 2.0 ** -k
+        np.testing.assert_array_equal(oracle.act_quantize(v32, block), ref)
+
+
+def _quant_torch(v64: np.ndarray, block: int) -> np.ndarray:
+    out = np.empty_like(v64)
+    for b0 in range(0, v64.size, block):
+        blk = v64[b0:b0 + block]
+        k = _k_by_search(np.abs(blk).max())
+        out[b0:b0 + block] = _torch_e4m3((blk * 2.0 ** k).astype(np.float32)) * 2.0 ** -k
+    return out
+
+
+def test_ffn_w8a8_matches_torch_chain():
+    """The W8A8 expert FFN against torch ops: x quantised per 128 columns
+    (torch cast), F.linear with the block-scaled FP8 weights, F.silu, h
+    quantised per 64 features, F.linear.  h passes through fp32 before torch's
+    cast, which can move a value across a rounding midpoint in rare elements,
+    so the comparison is relative-L2 at 1e-4 (the quantisation error itself is
+    about 1e-2)."""
+    E, I, H, T, K = 3, 128, 256, 6, 2
+    ex = wl.draw_experts(21, 71, E, I, H, 0.05, threads=1)
+    x = wl.random_rows_bf16(T, H, seed=22)
+    ids = np.array([[0, 1], [2, 0], [1, 2], [0, 2], [1, 0], [2, 1]], np.int32)
+    off, sr, inv, _ = oracle.sort(ids, E)
+    w = np.ones((T, K))
+    y = oracle.ffn_sorted_w8a8(x, K, ex, off, sr, w)
+    x64 = _x64(x).numpy()
+    for p, r in enumerate(sr):
+        t, e = r // K, ids.ravel()[r]
+        xq = torch.from_numpy(_quant_torch(x64[t], 128))
+        wg, wu, wd = (_fp8_dense(ex.w_gate[e], ex.s_gate[e]), _fp8_dense(ex.w_up[e], ex.s_up[e]),
+                      _fp8_dense(ex.w_down[e], ex.s_down[e]))
+        h = (F.silu(F.linear(xq, wg)) * F.linear(xq, wu)).numpy()
+        ref = F.linear(torch.from_numpy(_quant_torch(h, 64)), wd).numpy()
+        assert np.linalg.norm(y[p] - ref) <= 1e-4 * np.linalg.norm(ref)
+
+
+def test_ffn_w8a8_is_the_exact_ffn_when_quantisation_is_exact():
+    """Inputs for which both quantisations are exact, so the W8A8 FFN must
+    equal the fp64 FFN: x[t, :128] = c_t (c_t in 4..7), gate rows of E4M3FN
+    ones over those columns, so g = 128 c_t and silu(g) = g in fp64
+    (e^-g < 2^-53); x[t, 128] = d_t 2^-20 and up row i one power-of-two code
+    p_i in column 128, so u = p_i d_t 2^-20 and h = g u has at most three
+    significant bits.  The second x block is 2^-20 below the first, and the
+    two 64-feature blocks of h are 2^15 apart (codes 2^7, 2^8 against 2^-9,
+    2^-8): a scale taken from the wrong block, or h quantised in blocks of
+    128, flushes or rounds the small values and breaks the equality."""
+    E, I, H, T, K = 1, 128, 256, 4, 1
+    ex = wl.draw_experts(23, 72, E, I, H, 0.05, threads=1)
+    rng = np.random.default_rng(24)
+    ex.w_gate[:] = 0
+    ex.w_gate[0, :, :128] = 0x38  # 1.0
+    ex.s_gate[:] = 1.0
+    ex.w_up[:] = 0
+    ex.w_up[0, :64, 128] = rng.choice([0x70, 0x78], 64)  # 2^7, 2^8
+    ex.w_up[0, 64:, 128] = rng.choice([0x01, 0x02], 64)  # 2^-9, 2^-8 (subnormal codes)
+    ex.s_up[:] = 1.0
+    xs = np.zeros((T, H), np.float32)
+    xs[:, :128] = rng.integers(4, 8, (T, 1))
+    xs[:, 128:] = rng.choice([1.0, 2.0, 4.0], (T, 128)) * 2.0 ** -20
+    x = (xs.view(np.uint32) >> 16).astype(np.uint16)
+    assert np.array_equal(oracle.bf16_array(x), xs.astype(np.float64))
+    ids = np.zeros((T, K), np.int32)
+    off, sr, inv, _ = oracle.sort(ids, E)
+    w = np.ones((T, K))
+    exact = oracle.ffn_sorted(x, K, ex, off, sr, w)
+    assert np.abs(exact).max() > 0
+    np.testing.assert_allclose(oracle.ffn_sorted_w8a8(x, K, ex, off, sr, w), exact, rtol=1e-12, atol=0)
