@@ -226,6 +226,9 @@ ARITHMETIC = {
     "prefill": ("f16+bf16", "gate/up: f16 MMA on f16(e4m3 x block scale x 2^ka) and f16(x x 2^k_t), power-of-two "
                             "row scales undone in the epilogue; down: bf16 MMA on bf16(e4m3 x block scale) and bf16 "
                             "h; fp32 accumulate in TMEM; bf16 h, y_sorted and out"),
+    "w8a8": ("e4m3", "E4M3FN weights and E4M3FN activations (x in 128-column, h in 64-feature blocks with "
+                     "power-of-two scales) in m16n8k32 MMAs, fp32 accumulate, fp32 weight and activation block "
+                     "scales per partial sum; bf16 y_sorted and out"),
     "hybrid": ("f16+bf16", "experts with few rows as the decode form (f16 MMA on exact E4M3), the others as the "
                            "prefill form (f16 gate/up, bf16 down); fp32 accumulate; bf16 h, y_sorted and out"),
 }
@@ -384,7 +387,7 @@ def measure(args, shape, steps, dev, world, clk, want_e2e):
     wr = (torch.from_numpy(wl.router_weight(E, H, shape.seed).view(np.int16)).view(torch.bfloat16).to(dev)
           if args.fused_router else None)
     layer = moe.MoEFFN(routed, T, K, shared, mode=args.mode, device=dev, route_cfg=route_cfg, w_router=wr,
-                       fused_combine=args.fused_combine)
+                       fused_combine=args.fused_combine, w8a8=args.w8a8)
     stream = torch.cuda.Stream(device=dev)
 
     def run(lay, xx, ll):
@@ -423,8 +426,12 @@ def measure(args, shape, steps, dev, world, clk, want_e2e):
                                        moe.MOE_OUT_BF16, layer.status, layer.out, layer.ffn_ws)
             ev[3].record()
         else:
-            moe.moe_expert_ffn(x, K, routed, layer.offsets, layer.sorted_route, layer.topk_w, shared, args.mode,
-                               layer.status, layer.y_sorted, layer.y_shared, layer.ffn_ws)
+            if args.w8a8:
+                moe.moe_expert_ffn_w8a8(x, K, routed, layer.offsets, layer.sorted_route, layer.topk_w, shared,
+                                        layer.status, layer.y_sorted, layer.y_shared, layer.ffn_ws)
+            else:
+                moe.moe_expert_ffn(x, K, routed, layer.offsets, layer.sorted_route, layer.topk_w, shared,
+                                   args.mode, layer.status, layer.y_sorted, layer.y_shared, layer.ffn_ws)
             ev[3].record()
             moe.moe_combine(layer.y_sorted, layer.inv_route, layer.y_shared, T, K, moe.MOE_OUT_BF16, layer.out,
                             status=layer.status)
@@ -485,7 +492,8 @@ def measure(args, shape, steps, dev, world, clk, want_e2e):
     ffn_ms = statistics.median(parts["ffn"])
     R_nz = int(np.count_nonzero(layer.topk_w.cpu().numpy()))
     flops = (R_nz + (T if shape.I_shared else 0)) * 6 * H * I
-    form = moe.MOE_MODE_PREFILL if args.fused_combine else moe.moe_ffn_resolve_mode(T, K, E, args.mode)
+    form = (moe.MOE_MODE_PREFILL if args.fused_combine else
+            moe.MOE_MODE_DECODE if args.w8a8 else moe.moe_ffn_resolve_mode(T, K, E, args.mode))
     form_kind = {moe.MOE_MODE_DECODE: "decode", moe.MOE_MODE_PREFILL: "prefill",
                  moe.MOE_MODE_HYBRID: "hybrid"}[form]
     roof = ffn_roofline(shape, form_kind, touched=touched, flops=flops, ffn_ms=ffn_ms, peaks=peaks)
@@ -508,8 +516,9 @@ def measure(args, shape, steps, dev, world, clk, want_e2e):
            "window_ms_per_step": {"min": min(windows), "median": t_local, "max": max(windows)},
            "spread": (max(windows) - min(windows)) / t_local,
            "form": form_kind + ("+combine (moe_expert_ffn_combine: fp32 reductions, unordered)"
-                                if args.fused_combine else ""),
-           "dtype": ARITHMETIC[form_kind][0], "arithmetic": ARITHMETIC[form_kind][1],
+                                if args.fused_combine else " W8A8 (moe_expert_ffn_w8a8)" if args.w8a8 else ""),
+           "dtype": ARITHMETIC["w8a8" if args.w8a8 else form_kind][0],
+           "arithmetic": ARITHMETIC["w8a8" if args.w8a8 else form_kind][1],
            "l2": "inputs larger than L2 (%s expert weights %.2f GB > 126 MB)"
                  % ("touched" if form_kind != "prefill" else "all", weights_gb),
            "roofline": roof, "breakdown_ms": {k: statistics.median(v) for k, v in parts.items()},
@@ -537,7 +546,7 @@ def measure_e2e(args, w, shape, layer, routed, shared, route_cfg, wr, x, logits,
     lh = torch.from_numpy(w.logits).pin_memory()
     oh = [torch.empty((T, H), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
     layers = [layer, moe.MoEFFN(routed, T, K, shared, mode=args.mode, device=dev, route_cfg=route_cfg,
-                                w_router=wr, fused_combine=args.fused_combine)]
+                                w_router=wr, fused_combine=args.fused_combine, w8a8=args.w8a8)]
     xs, ls = [x, torch.empty_like(x)], [logits, torch.empty_like(logits)]
     h2d, d2h = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
     in_ready, in_free, out_ready, out_free = ([torch.cuda.Event(), torch.cuda.Event()] for _ in range(4))
@@ -603,6 +612,8 @@ def main():
                     help="route from x with the fused router (gate GEMM + top-K) instead of given logits")
     ap.add_argument("--eager", action="store_true",
                     help="launch every call directly instead of replaying CUDA graphs (for profilers)")
+    ap.add_argument("--w8a8", action="store_true",
+                    help="FP8 activations (moe_expert_ffn_w8a8, the opt-in W8A8 form) instead of moe_expert_ffn")
     ap.add_argument("--fused-combine", action="store_true",
                     help="expert FFN and combine in one call (moe_expert_ffn_combine; tensor-core form)")
     args = ap.parse_args()

@@ -400,6 +400,37 @@ MOE_API int moe_expert_ffn(const uint16_t* x, int T, int H, int K, const moe_fp8
                    int32_t* status, moe_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * moe_expert_ffn_w8a8 -- moe_expert_ffn with FP8 activations (opt-in W8A8 form).
+ *
+ * The activation quantisation the pages describe for their low-precision
+ * pipelines -- the NKI Library's Blockwise MM Forward MXFP8 kernel (FP8
+ * activations against FP8 weights) and the aiter gfx950 PR's in-register
+ * quantisation of the hidden activation -- applied to this library's FP8
+ * E4M3FN weights with their 128x128 fp32 block scales:
+ *   xq = quant(x) in blocks of 128 columns;  h = silu(Wg xq) * (Wu xq);
+ *   hq = quant(h) in blocks of 64 features;  y_sorted[p] = w[r] * (Wd hq),
+ * where quant(v) on a block is e4m3fn(v * 2^k) * 2^-k, with k the exponent
+ * that puts the block's largest |v| in (224, 448] (k in [-126, 126], 0 for an
+ * all-zero block), e4m3fn rounding to nearest even.  x is quantised from its
+ * bf16 values as it is staged; h from its fp32 value in the gate/up epilogue
+ * (it never exists as bf16).  Both GEMMs run as E4M3FN x E4M3FN tensor-core
+ * MMAs with fp32 accumulation, the weight block scale and the activation
+ * block scale applied to each 128-column (gate/up) or 64-column (down)
+ * partial sum.  The weight-streaming (decode) kernels run for every T; the
+ * result differs from moe_expert_ffn by the activation rounding (about 2 %
+ * relative in the library's tests; see its parity tests for the bound).
+ *   Arguments, layouts, limits and errors: those of moe_expert_ffn without
+ *   `mode`.  workspace: moe_ffn_w8a8_workspace_bytes(T, K, I, I_shared)
+ *   bytes (h as E4M3FN bytes and its block scales), any contents.
+ * ------------------------------------------------------------------------- */
+MOE_API size_t moe_ffn_w8a8_workspace_bytes(int T, int K, int I, int I_shared);
+MOE_API int moe_expert_ffn_w8a8(const uint16_t* x, int T, int H, int K, const moe_fp8_experts* routed,
+                   const moe_fp8_experts* shared, const int32_t* expert_offsets,
+                   const int32_t* sorted_route, const float* topk_w, uint16_t* y_sorted,
+                   uint16_t* y_shared, void* workspace, size_t workspace_bytes,
+                   int32_t* status, moe_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * moe_expert_ffn_combine -- the expert FFN and the combine in one call
  * (tensor-core form), without the sorted rows.
  *

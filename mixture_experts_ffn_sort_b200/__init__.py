@@ -34,7 +34,8 @@ MOE_MAX_E, MOE_MAX_K = 1024, 32
 EXPORTED = ("moe_last_error", "moe_abi_version", "moe_route", "moe_route_ex", "moe_router", "moe_sort_workspace_bytes",
             "moe_sort", "moe_selftest_bounded_wait", "moe_router_plan_check",
             "moe_sort_static_ws", "moe_ffn_resolve_mode", "moe_ffn_workspace_bytes", "moe_expert_ffn", "moe_combine",
-            "moe_ffn_combine_workspace_bytes", "moe_expert_ffn_combine")
+            "moe_ffn_combine_workspace_bytes", "moe_expert_ffn_combine", "moe_ffn_w8a8_workspace_bytes",
+            "moe_expert_ffn_w8a8")
 
 
 class MoEError(RuntimeError):
@@ -96,6 +97,10 @@ def lib() -> ctypes.CDLL:
             L.moe_ffn_combine_workspace_bytes.restype = S
             L.moe_expert_ffn_combine.argtypes = [P, I, I, I, P, P, P, P, P, P, I, P, S, P, P]
             L.moe_expert_ffn_combine.restype = I
+            L.moe_ffn_w8a8_workspace_bytes.argtypes = [I, I, I, I]
+            L.moe_ffn_w8a8_workspace_bytes.restype = S
+            L.moe_expert_ffn_w8a8.argtypes = [P, I, I, I, P, P, P, P, P, P, P, P, S, P, P]
+            L.moe_expert_ffn_w8a8.restype = I
             L.moe_combine.argtypes = [P, P, P, I, I, I, P, I, P, P]
             L.moe_combine.restype = I
             _L = L
@@ -293,6 +298,35 @@ def moe_expert_ffn(x: torch.Tensor, K: int, routed: Experts, expert_offsets: tor
     return y_sorted, (y_shared if shared is not None else None)
 
 
+def moe_ffn_w8a8_workspace_bytes(T: int, K: int, I: int, I_shared: int = 0) -> int:
+    return int(lib().moe_ffn_w8a8_workspace_bytes(T, K, I, I_shared))
+
+
+def moe_expert_ffn_w8a8(x: torch.Tensor, K: int, routed: Experts, expert_offsets: torch.Tensor,
+                        sorted_route: torch.Tensor, topk_w: torch.Tensor, shared: Optional[Experts] = None,
+                        status: Optional[torch.Tensor] = None, y_sorted=None, y_shared=None, workspace=None,
+                        stream=None):
+    """moe_expert_ffn with FP8 activations (the opt-in W8A8 form)."""
+    _need_cuda(x, expert_offsets, sorted_route, topk_w, status)
+    T, H = x.shape
+    dev = x.device
+    if y_sorted is None:
+        y_sorted = torch.empty((T * K, H), dtype=torch.bfloat16, device=dev)
+    if shared is not None and y_shared is None:
+        y_shared = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    need = moe_ffn_w8a8_workspace_bytes(T, K, routed.inter, shared.inter if shared else 0)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    rs = routed.struct()
+    ss = shared.struct() if shared is not None else None
+    _check(lib().moe_expert_ffn_w8a8(_ptr(x), T, H, K, ctypes.byref(rs),
+                                     ctypes.byref(ss) if ss is not None else None,
+                                     _ptr(expert_offsets), _ptr(sorted_route), _ptr(topk_w), _ptr(y_sorted),
+                                     _ptr(y_shared) if shared is not None else None, _ptr(workspace),
+                                     workspace.numel(), _ptr(status), _stream(stream)))
+    return y_sorted, (y_shared if shared is not None else None)
+
+
 def moe_ffn_combine_workspace_bytes(T, K, H, E, I, I_shared=0, out_dtype=MOE_OUT_BF16) -> int:
     return int(lib().moe_ffn_combine_workspace_bytes(T, K, H, E, I, I_shared, out_dtype))
 
@@ -347,14 +381,19 @@ class MoEFFN:
     moe_route.  w_router: bf16 [E, H] gate vectors for forward_fused, which
     routes with the fused router (moe_router) from x alone.  fused_combine:
     run the expert FFN and the combine as one call (moe_expert_ffn_combine:
-    tensor-core kernels, no y_sorted, fp32 reductions in no fixed order)."""
+    tensor-core kernels, no y_sorted, fp32 reductions in no fixed order).
+    w8a8: FP8 activations (moe_expert_ffn_w8a8, weight-streaming kernels);
+    `mode` is then ignored."""
 
     def __init__(self, routed: Experts, T: int, K: int, shared: Optional[Experts] = None,
                  mode: int = MOE_MODE_AUTO, out_dtype: int = MOE_OUT_BF16, device="cuda",
                  route_cfg: Optional[dict] = None, w_router: Optional[torch.Tensor] = None,
-                 fused_combine: bool = False):
+                 fused_combine: bool = False, w8a8: bool = False):
+        if fused_combine and w8a8:
+            raise ValueError("fused_combine and w8a8 are separate forms")
         self.routed, self.shared, self.T, self.K = routed, shared, T, K
         self.fused_combine = fused_combine
+        self.w8a8 = w8a8
         self.w_router = w_router
         self.route_cfg = dict(route_cfg) if route_cfg else None
         self.E, self.I, self.H = routed.n, routed.inter, routed.w_gate.shape[2]
@@ -372,9 +411,10 @@ class MoEFFN:
                 T, K, self.H, self.E, self.I, shared.inter if shared else 0, out_dtype)), dtype=torch.uint8, device=d)
             self.y_sorted, self.y_shared = None, None
         else:
-            self.ffn_ws = torch.empty(max(16, moe_ffn_workspace_bytes(T, K, self.H, self.E, self.I,
-                                                                      shared.inter if shared else 0, mode)),
-                                      dtype=torch.uint8, device=d)
+            Is = shared.inter if shared else 0
+            need = (moe_ffn_w8a8_workspace_bytes(T, K, self.I, Is) if w8a8 else
+                    moe_ffn_workspace_bytes(T, K, self.H, self.E, self.I, Is, mode))
+            self.ffn_ws = torch.empty(max(16, need), dtype=torch.uint8, device=d)
             self.y_sorted = torch.empty((R, self.H), dtype=torch.bfloat16, device=d)
             self.y_shared = torch.empty((T, self.H), dtype=torch.bfloat16, device=d) if shared else None
         dt = torch.bfloat16 if out_dtype == MOE_OUT_BF16 else torch.float32
@@ -390,7 +430,7 @@ class MoEFFN:
         if self.fused_combine:
             # f16 copy of x, gate/up, down with the reductions, fp32 -> bf16.
             return 1 + sort + 3 + (1 if self.out_dtype == MOE_OUT_BF16 else 0)
-        form = moe_ffn_resolve_mode(self.T, self.K, self.E, self.mode)
+        form = MOE_MODE_DECODE if self.w8a8 else moe_ffn_resolve_mode(self.T, self.K, self.E, self.mode)
         # The tensor-core form also launches the f16 copy of x.
         ffn = {MOE_MODE_DECODE: 2 + (2 if self.shared is not None else 0), MOE_MODE_PREFILL: 3,
                MOE_MODE_HYBRID: 5}[form]
@@ -420,8 +460,12 @@ class MoEFFN:
             return moe_expert_ffn_combine(x, self.K, self.routed, self.offsets, self.sorted_route, self.topk_w,
                                           self.shared, self.out_dtype, self.status, self.out, self.ffn_ws,
                                           stream=stream)
-        moe_expert_ffn(x, self.K, self.routed, self.offsets, self.sorted_route, self.topk_w, self.shared,
-                       self.mode, self.status, self.y_sorted, self.y_shared, self.ffn_ws, stream=stream)
+        if self.w8a8:
+            moe_expert_ffn_w8a8(x, self.K, self.routed, self.offsets, self.sorted_route, self.topk_w, self.shared,
+                                self.status, self.y_sorted, self.y_shared, self.ffn_ws, stream=stream)
+        else:
+            moe_expert_ffn(x, self.K, self.routed, self.offsets, self.sorted_route, self.topk_w, self.shared,
+                           self.mode, self.status, self.y_sorted, self.y_shared, self.ffn_ws, stream=stream)
         moe_combine(self.y_sorted, self.inv_route, self.y_shared, self.T, self.K, self.out_dtype, self.out,
                     stream=stream, status=self.status)
         return self.out

@@ -6,6 +6,7 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -183,6 +184,43 @@ __device__ __forceinline__ void mma_f16_16816(float (&d)[4], uint32_t a0, uint32
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
+
+// D += A(16x32, row) * B(32x8, col), E4M3FN inputs, fp32 accumulators.  Fragments
+// (g = lane / 4, c = lane % 4): a0 = row g, k 4c..4c+3; a1 = row g+8, the same
+// k; a2, a3 = rows g, g+8, k 16+4c..16+4c+3; b0 = column g, k 4c..4c+3;
+// b1 = column g, k 16+4c..16+4c+3 (four codes per register, lowest k in the
+// lowest byte).
+__device__ __forceinline__ void mma_e4m3_16832(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                               uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.f32.e4m3.e4m3.f32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Four fp32 values to four E4M3FN codes (v0 in the lowest byte), rounded to
+// nearest even, magnitudes beyond 448 saturating to 448.
+__device__ __forceinline__ uint32_t f32x4_to_e4m3x4(float v0, float v1, float v2, float v3) {
+    const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(v0, v1), __NV_SATFINITE, __NV_E4M3);
+    const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(v2, v3), __NV_SATFINITE, __NV_E4M3);
+    return lo | (hi << 16);
+}
+
+// Power-of-two scale exponent k of an FP8 activation block whose largest
+// magnitude has the fp32 bit pattern amax_bits: amax * 2^k lies in (224, 448]
+// (the top binade of E4M3FN up to its largest value), k limited to
+// [-126, 126]; 0 for an all-zero block.
+__device__ __forceinline__ int act_scale_exp(uint32_t amax_bits) {
+    if (amax_bits == 0) return 0;
+    const int eb = static_cast<int>(amax_bits >> 23);  // biased exponent, 0 for a subnormal
+    if (eb == 0) return 126;
+    const int k = ((amax_bits & 0x7FFFFFu) <= 0x600000u ? 8 : 7) - (eb - 127);
+    return max(-126, min(126, k));
+}
+
+// 2^k as an fp32 for -126 <= k <= 127.
+__device__ __forceinline__ float pow2_f32(int k) { return __uint_as_float(static_cast<uint32_t>(k + 127) << 23); }
 
 // ---------------------------------------------------------------- FP8 decode
 

@@ -165,6 +165,98 @@ __device__ __forceinline__ void stage_rows_f16(RowPtr row_ptr, int W, uint8_t* d
     }
 }
 
+// W8A8 form.  Activation rows in shared memory are E4M3FN codes laid out per
+// 32-byte slab (32 reduction columns) so that one 8-byte load gives the two
+// registers of an m16n8k32 B fragment: unit u (bytes 8u .. 8u+7) holds the
+// codes of columns 4u .. 4u+3 and then 16+4u .. 16+4u+3 of the slab.
+__device__ __forceinline__ uint32_t slab_offset(int col) {  // byte of column col (multiple of 4) in its row
+    const int q = col & 31;
+    return static_cast<uint32_t>((col & ~31) + 8 * ((q & 15) >> 2) + 4 * (q >> 4));
+}
+
+// Stage NG rows of W bf16 values as E4M3FN codes: each 128-column block of a
+// row is multiplied by its own power of two 2^k (act_scale_exp of the block's
+// largest magnitude; exact) and rounded to nearest even;
+// qs[q * nqb + b] = 2^-k.  row_ptr(q) gives the source row or nullptr for a
+// padding row (zeros).  Warp w handles rows w, w + 8, ...; each half-warp
+// covers one block of 16 vectors.
+template <int NG, class RowPtr>
+__device__ __forceinline__ void stage_rows_e4m3(RowPtr row_ptr, int W, uint8_t* dst, int stride, float* qs,
+                                                int nqb) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int vpr = W / 8;  // a multiple of 16: half-warps stay whole
+    for (int q = warp; q < NG; q += kConsumerWarps) {
+        const uint16_t* src = row_ptr(q);
+        uint8_t* d = dst + q * stride;
+        for (int v0 = 0; v0 < vpr; v0 += 32) {
+            const int v = v0 + lane;
+            const bool in = v < vpr;
+            const uint4 val = (src && in) ? ldg_v4(src + v * 8) : make_uint4(0, 0, 0, 0);
+            uint32_t m = absmax_bf16x8(val);
+#pragma unroll
+            for (int o = 1; o < 16; o <<= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+            const int k = act_scale_exp(m << 16);
+            if (!in) continue;
+            if ((lane & 15) == 0) qs[q * nqb + v / 16] = pow2_f32(-k);
+            const float up = pow2_f32(k);
+            const uint32_t w[4] = {val.x, val.y, val.z, val.w};
+            float f[8];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                f[2 * i] = __uint_as_float(w[i] << 16) * up;
+                f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u) * up;
+            }
+            *reinterpret_cast<uint32_t*>(d + slab_offset(8 * v)) = f32x4_to_e4m3x4(f[0], f[1], f[2], f[3]);
+            *reinterpret_cast<uint32_t*>(d + slab_offset(8 * v + 4)) = f32x4_to_e4m3x4(f[4], f[5], f[6], f[7]);
+        }
+    }
+}
+
+// Stage NG rows of W E4M3FN codes (already quantised, 16-byte vectors) into
+// the slab layout, and their nqb block scales.  row(q) gives the source row
+// index or -1 for a padding row (zeros).
+template <int NG, class RowIdx>
+__device__ __forceinline__ void stage_codes(RowIdx row, const uint8_t* codes, const float* scales, int W,
+                                            uint8_t* dst, int stride, float* qs, int nqb) {
+    const int vpr = W / 16;
+    for (int v = threadIdx.x; v < NG * vpr; v += kConsumers) {
+        const int q = v / vpr, c = v - q * vpr;
+        const long r = row(q);
+        const uint4 val = r >= 0 ? ldg_v4(codes + static_cast<size_t>(r) * W + c * 16) : make_uint4(0, 0, 0, 0);
+        uint8_t* d = dst + q * stride;
+        *reinterpret_cast<uint32_t*>(d + slab_offset(16 * c)) = val.x;
+        *reinterpret_cast<uint32_t*>(d + slab_offset(16 * c + 4)) = val.y;
+        *reinterpret_cast<uint32_t*>(d + slab_offset(16 * c + 8)) = val.z;
+        *reinterpret_cast<uint32_t*>(d + slab_offset(16 * c + 12)) = val.w;
+    }
+    for (int i = threadIdx.x; i < NG * nqb; i += kConsumers) {
+        const int q = i / nqb, b = i - q * nqb;
+        const long r = row(q);
+        qs[i] = r >= 0 ? __ldg(scales + static_cast<size_t>(r) * nqb + b) : 0.f;
+    }
+}
+
+// W8A8: one 128-column stage of one warp with FP8 activations: per 32-column
+// slab p, one ldmatrix_x4 of the weight codes is exactly the A fragment of an
+// m16n8k32 E4M3FN MMA (matrices 0/1: the 16 rows in chunk 2p, 2/3: in chunk
+// 2p+1).  SPLIT: slabs 0-1 accumulate into part[0] and slabs 2-3 into
+// part[1] (two 64-column activation scale blocks per stage).
+template <int NT, bool SPLIT>
+__device__ __forceinline__ void stage_mma_q(uint32_t tile0, uint32_t tile1, uint32_t row, uint32_t chunk_sel,
+                                            uint32_t b_addr, int stride, float (&part)[2][NT][4]) {
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+        const uint32_t chunk = 2 * p + (chunk_sel & 1);
+        uint32_t r0, r1, r2, r3;
+        ldmatrix_x4((chunk_sel & 2 ? tile1 : tile0) + sw128_offset(row, chunk & 7), r0, r1, r2, r3);
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            const uint2 b = lds64(b_addr + nt * 8 * stride + p * 32);
+            mma_e4m3_16832(part[SPLIT && p >= 2 ? 1 : 0][nt], r0, r1, r2, r3, b.x, b.y);
+        }
+    }
+}
+
 // One 128-column stage of one warp: 16 rows x 128 columns against NT token
 // tiles.  This lane's ldmatrix row is `row` of sub-tile tile0 (chunk_sel bit 1
 // clear) or tile1 (set), in chunk j (bit 0 clear) or j+1 (set) of each chunk
@@ -204,6 +296,7 @@ __device__ __forceinline__ void zero_acc(float (&a)[NT][4]) {
 
 // Shared-memory carve-up common to both kernels.
 struct Smem {
+    float* qs;        // W8A8: activation block scales [NG][nqb]
     uint8_t* ring;
     uint8_t* rows;    // staged activation rows (f16)
     uint16_t* otile;  // output tile (bf16)
@@ -217,13 +310,13 @@ struct Smem {
     int* gpre;     // [E + 1]: exclusive prefix of their token groups
 };
 
-__host__ __device__ constexpr size_t smem_bytes(int NG, int row_stride, int otile_stride, int E) {
+__host__ __device__ constexpr size_t smem_bytes(int NG, int row_stride, int otile_stride, int E, int nqb = 0) {
     return 1024 + static_cast<size_t>(kStages) * kStageBytes + static_cast<size_t>(NG) * row_stride +
            static_cast<size_t>(NG) * otile_stride * 2 + 3 * NG * 4 + 2 * kStages * 8 + 16 +
-           static_cast<size_t>(2 * E + 1) * 4;
+           static_cast<size_t>(2 * E + 1) * 4 + static_cast<size_t>(NG) * nqb * 4;
 }
 
-__device__ __forceinline__ Smem carve(uint8_t* raw, int NG, int row_stride, int otile_stride, int E) {
+__device__ __forceinline__ Smem carve(uint8_t* raw, int NG, int row_stride, int otile_stride, int E, int nqb = 0) {
     Smem s;
     uint8_t* p = align1024(raw);
     s.ring = p;
@@ -241,6 +334,7 @@ __device__ __forceinline__ Smem carve(uint8_t* raw, int NG, int row_stride, int 
     s.abort_flag = reinterpret_cast<volatile int*>(s.empty + kStages);
     s.touched = reinterpret_cast<int*>(s.empty + kStages) + 4;
     s.gpre = s.touched + E;
+    s.qs = nqb ? reinterpret_cast<float*>(s.gpre + E + 1) : nullptr;
     return s;
 }
 
@@ -361,7 +455,8 @@ __device__ __forceinline__ void init_barriers(const Smem& s) {
 
 // ------------------------------------------------------------------ gate/up + SwiGLU
 
-template <int NT>
+// Q: the W8A8 form (FP8 activations, m16n8k32 E4M3FN MMAs, h quantised in the epilogue).
+template <int NT, bool Q>
 __global__ void __launch_bounds__(kThreads, 2)
     gateup_decode_kernel(const __grid_constant__ CUtensorMap tm_gate,
                          const __grid_constant__ CUtensorMap tm_up, const FfnArgs a) {
@@ -370,9 +465,9 @@ __global__ void __launch_bounds__(kThreads, 2)
     extern __shared__ uint8_t smem_raw[];
     const int H = a.H, I = a.ex.inter;
     const int KB = H / 128;
-    const int xstride = 2 * H + 32;
+    const int xstride = Q ? H + 32 : 2 * H + 32;
     const int E = a.identity ? 1 : a.ex.n;
-    const Smem s = carve(smem_raw, NG, xstride, kGuTile, E);
+    const Smem s = carve(smem_raw, NG, xstride, kGuTile, E, Q ? KB : 0);
     init_barriers(s);
     // Items: (touched expert, token group, block of kGateUpFeat features); each
     // CTA of the persistent grid takes a contiguous, equal share.
@@ -439,12 +534,14 @@ __global__ void __launch_bounds__(kThreads, 2)
                 s.tok[threadIdx.x] = t;
             }
             named_barrier_sync(1, kConsumers);
-            stage_rows_f16<NG>(
-                [&](int q) -> const uint16_t* {
-                    const int t = s.tok[q];
-                    return t >= 0 ? a.x + static_cast<size_t>(t) * H : nullptr;
-                },
-                H, s.rows, xstride, s.inv);
+            auto x_row = [&](int q) -> const uint16_t* {
+                const int t = s.tok[q];
+                return t >= 0 ? a.x + static_cast<size_t>(t) * H : nullptr;
+            };
+            if constexpr (Q)
+                stage_rows_e4m3<NG>(x_row, H, s.rows, xstride, s.qs, KB);
+            else
+                stage_rows_f16<NG>(x_row, H, s.rows, xstride, s.inv);
             named_barrier_sync(1, kConsumers);
         }
 
@@ -452,51 +549,115 @@ __global__ void __launch_bounds__(kThreads, 2)
         zero_acc<NT>(acc);
         for (int kb = 0; kb < KB; ++kb, ++it) {
             const int st = static_cast<int>(it % kStages);
-            float part[NT][4];
-            zero_acc<NT>(part);
+            float part[2][NT][4];
+            zero_acc<NT>(part[0]);
             if (mbar_wait_or_abort(&s.full[st], static_cast<uint32_t>((it / kStages) & 1), s.abort_flag,
                                    a.status)) {
                 const uint32_t tile = ring_u32 + st * kStageBytes;
                 // chunk_sel bit 1 selects the up sub-tile (second half of the stage).
-                stage_mma<NT>(tile, tile + kStageBytes / 2, lm_row, chunk_sel, b_lane + kb * 256, xstride,
-                              part);
+                if constexpr (Q)
+                    stage_mma_q<NT, false>(tile, tile + kStageBytes / 2, lm_row, chunk_sel, b_lane + kb * 128,
+                                           xstride, part);
+                else
+                    stage_mma<NT>(tile, tile + kStageBytes / 2, lm_row, chunk_sel, b_lane + kb * 256, xstride,
+                                  part[0]);
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&s.empty[st]);
             }
             const float gs = __ldg(sg + kb), us = __ldg(su + kb);
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
-                acc[nt][0] = fmaf(part[nt][0], gs, acc[nt][0]);
-                acc[nt][1] = fmaf(part[nt][1], gs, acc[nt][1]);
-                acc[nt][2] = fmaf(part[nt][2], us, acc[nt][2]);
-                acc[nt][3] = fmaf(part[nt][3], us, acc[nt][3]);
+                // W8A8: the activation block scales of this thread's two token columns.
+                float x0 = 1.f, x1 = 1.f;
+                if constexpr (Q) {
+                    x0 = s.qs[(nt * 8 + 2 * c) * KB + kb];
+                    x1 = s.qs[(nt * 8 + 2 * c + 1) * KB + kb];
+                }
+                acc[nt][0] = fmaf(part[0][nt][0], gs * x0, acc[nt][0]);
+                acc[nt][1] = fmaf(part[0][nt][1], gs * x1, acc[nt][1]);
+                acc[nt][2] = fmaf(part[0][nt][2], us * x0, acc[nt][2]);
+                acc[nt][3] = fmaf(part[0][nt][3], us * x1, acc[nt][3]);
             }
         }
-        // SwiGLU on the true sums (undo the activation scale first).
         const int il = 8 * warp + g;
+        if constexpr (!Q) {
+            // SwiGLU on the true sums (undo the activation scale first).
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-            const int t0 = nt * 8 + 2 * c;
-            const float s0 = s.inv[t0], s1 = s.inv[t0 + 1];
-            const float h0 = silu_f32(acc[nt][0] * s0) * (acc[nt][2] * s0);
-            const float h1 = silu_f32(acc[nt][1] * s1) * (acc[nt][3] * s1);
-            s.otile[t0 * kGuTile + il] = __bfloat16_as_ushort(__float2bfloat16_rn(h0));
-            s.otile[(t0 + 1) * kGuTile + il] = __bfloat16_as_ushort(__float2bfloat16_rn(h1));
+            for (int nt = 0; nt < NT; ++nt) {
+                const int t0 = nt * 8 + 2 * c;
+                const float s0 = s.inv[t0], s1 = s.inv[t0 + 1];
+                const float h0 = silu_f32(acc[nt][0] * s0) * (acc[nt][2] * s0);
+                const float h1 = silu_f32(acc[nt][1] * s1) * (acc[nt][3] * s1);
+                s.otile[t0 * kGuTile + il] = __bfloat16_as_ushort(__float2bfloat16_rn(h0));
+                s.otile[(t0 + 1) * kGuTile + il] = __bfloat16_as_ushort(__float2bfloat16_rn(h1));
+            }
+            named_barrier_sync(1, kConsumers);
+            for (int v = threadIdx.x; v < NG * (kGateUpFeat / 8); v += kConsumers) {
+                const int q = v / (kGateUpFeat / 8), ch = v % (kGateUpFeat / 8);
+                if (q < gn && s.tok[q] >= 0)
+                    *reinterpret_cast<uint4*>(a.h + static_cast<size_t>(gp0 + q) * I + i0 + ch * 8) =
+                        *reinterpret_cast<const uint4*>(s.otile + q * kGuTile + ch * 8);
+            }
+            named_barrier_sync(1, kConsumers);
+        } else {
+            // SwiGLU, then h quantised in registers: the item's 64 features are
+            // one scale block, so each token's scale comes from the largest |h|
+            // over the eight warps (8 features each: shuffles over g, then the
+            // warps' maxima through shared memory).  Codes go through a byte
+            // tile (rows of kQRow bytes) to 16-byte stores.
+            constexpr int kQRow = kGateUpFeat + 16;
+            uint8_t* qtile = reinterpret_cast<uint8_t*>(s.otile);
+            float* wmax = reinterpret_cast<float*>(qtile + NG * kQRow);  // [NG][kConsumerWarps]
+            float hv[NT][2];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                hv[nt][0] = silu_f32(acc[nt][0]) * acc[nt][2];
+                hv[nt][1] = silu_f32(acc[nt][1]) * acc[nt][3];
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    float m = fabsf(hv[nt][j]);
+#pragma unroll
+                    for (int o = 4; o < 32; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+                    if (g == 0) wmax[(nt * 8 + 2 * c + j) * kConsumerWarps + warp] = m;
+                }
+            }
+            named_barrier_sync(1, kConsumers);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const int t = nt * 8 + 2 * c + j;
+                    float m = 0.f;
+#pragma unroll
+                    for (int w2 = 0; w2 < kConsumerWarps; ++w2) m = fmaxf(m, wmax[t * kConsumerWarps + w2]);
+                    const float up = pow2_f32(act_scale_exp(__float_as_uint(m)));
+                    qtile[t * kQRow + il] = static_cast<uint8_t>(
+                        __nv_cvt_float_to_fp8(hv[nt][j] * up, __NV_SATFINITE, __NV_E4M3));
+                }
+            named_barrier_sync(1, kConsumers);
+            uint8_t* hq = reinterpret_cast<uint8_t*>(a.h);
+            for (int v = threadIdx.x; v < NG * (kGateUpFeat / 16); v += kConsumers) {
+                const int q = v / (kGateUpFeat / 16), ch = v % (kGateUpFeat / 16);
+                if (q < gn && s.tok[q] >= 0)
+                    *reinterpret_cast<uint4*>(hq + static_cast<size_t>(gp0 + q) * I + i0 + ch * 16) =
+                        *reinterpret_cast<const uint4*>(qtile + q * kQRow + ch * 16);
+            }
+            if (threadIdx.x < NG && static_cast<int>(threadIdx.x) < gn && s.tok[threadIdx.x] >= 0) {
+                const int q = threadIdx.x;
+                float m = 0.f;
+#pragma unroll
+                for (int w2 = 0; w2 < kConsumerWarps; ++w2) m = fmaxf(m, wmax[q * kConsumerWarps + w2]);
+                a.hscale[static_cast<size_t>(gp0 + q) * (I / kGateUpFeat) + i0 / kGateUpFeat] =
+                    pow2_f32(-act_scale_exp(__float_as_uint(m)));
+            }
+            named_barrier_sync(1, kConsumers);
         }
-        named_barrier_sync(1, kConsumers);
-        for (int v = threadIdx.x; v < NG * (kGateUpFeat / 8); v += kConsumers) {
-            const int q = v / (kGateUpFeat / 8), ch = v % (kGateUpFeat / 8);
-            if (q < gn && s.tok[q] >= 0)
-                *reinterpret_cast<uint4*>(a.h + static_cast<size_t>(gp0 + q) * I + i0 + ch * 8) =
-                    *reinterpret_cast<const uint4*>(s.otile + q * kGuTile + ch * 8);
-        }
-        named_barrier_sync(1, kConsumers);
     }
 }
 
 // ------------------------------------------------------------------ down + affinity
 
-template <int NT>
+template <int NT, bool Q>
 __global__ void __launch_bounds__(kThreads, 2)
     down_decode_kernel(const __grid_constant__ CUtensorMap tm_down, const FfnArgs a) {
     constexpr int NG = 8 * NT;
@@ -506,9 +667,10 @@ __global__ void __launch_bounds__(kThreads, 2)
     extern __shared__ uint8_t smem_raw[];
     const int H = a.H, I = a.ex.inter;
     const int KB = I / 128;
-    const int hstride = 2 * I + 32;
+    const int hstride = Q ? I + 32 : 2 * I + 32;
     const int E = a.identity ? 1 : a.ex.n;
-    const Smem s = carve(smem_raw, NG, hstride, kDnTile, E);
+    const int nqb = I / kGateUpFeat;  // W8A8: h scale blocks per row
+    const Smem s = carve(smem_raw, NG, hstride, kDnTile, E, Q ? nqb : 0);
     init_barriers(s);
     // Items: (touched expert, token group, block of kDownRows output rows); each
     // CTA of the persistent grid takes a contiguous, equal share.  Offsets come
@@ -577,11 +739,16 @@ __global__ void __launch_bounds__(kThreads, 2)
                 s.wr[threadIdx.x] = wv;
             }
             named_barrier_sync(1, kConsumers);
-            stage_rows_f16<NG>(
-                [&](int q) -> const uint16_t* {
-                    return (q < gn && s.tok[q] >= 0) ? a.h + static_cast<size_t>(gp0 + q) * I : nullptr;
-                },
-                I, s.rows, hstride, s.inv);
+            if constexpr (Q)
+                stage_codes<NG>(
+                    [&](int q) -> long { return (q < gn && s.tok[q] >= 0) ? gp0 + q : -1; },
+                    reinterpret_cast<const uint8_t*>(a.h), a.hscale, I, s.rows, hstride, s.qs, nqb);
+            else
+                stage_rows_f16<NG>(
+                    [&](int q) -> const uint16_t* {
+                        return (q < gn && s.tok[q] >= 0) ? a.h + static_cast<size_t>(gp0 + q) * I : nullptr;
+                    },
+                    I, s.rows, hstride, s.inv);
             named_barrier_sync(1, kConsumers);
         }
 
@@ -589,26 +756,44 @@ __global__ void __launch_bounds__(kThreads, 2)
         zero_acc<NT>(acc);
         for (int kb = 0; kb < KB; ++kb, ++it) {
             const int st = static_cast<int>(it % kStages);
-            float part[NT][4];
-            zero_acc<NT>(part);
+            float part[2][NT][4];
+            zero_acc<NT>(part[0]);
+            if constexpr (Q) zero_acc<NT>(part[1]);
             if (mbar_wait_or_abort(&s.full[st], static_cast<uint32_t>((it / kStages) & 1), s.abort_flag,
                                    a.status)) {
                 const uint32_t tile = ring_u32 + st * kStageBytes;
-                stage_mma<NT>(tile, tile, lm_row, chunk_sel, b_lane + kb * 256, hstride, part);
+                if constexpr (Q)
+                    stage_mma_q<NT, true>(tile, tile, lm_row, chunk_sel, b_lane + kb * 128, hstride, part);
+                else
+                    stage_mma<NT>(tile, tile, lm_row, chunk_sel, b_lane + kb * 256, hstride, part[0]);
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&s.empty[st]);
             }
             const float ds = __ldg(sd + kb);
+            if constexpr (Q) {
+                // Two 64-feature scale blocks of h per 128-column stage.
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
+                for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-                for (int k = 0; k < 4; ++k) acc[nt][k] = fmaf(part[nt][k], ds, acc[nt][k]);
+                    for (int k = 0; k < 4; ++k) {
+                        const int t = nt * 8 + 2 * c + (k & 1);
+                        const float lo = s.qs[t * nqb + 2 * kb], hi = s.qs[t * nqb + 2 * kb + 1];
+                        acc[nt][k] = fmaf(fmaf(part[0][nt][k], lo, part[1][nt][k] * hi), ds, acc[nt][k]);
+                    }
+            } else {
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) acc[nt][k] = fmaf(part[0][nt][k], ds, acc[nt][k]);
+            }
         }
         const int rl = 16 * warp + g;
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
             const int t0 = nt * 8 + 2 * c;
-            const float f0 = s.inv[t0] * s.wr[t0], f1 = s.inv[t0 + 1] * s.wr[t0 + 1];
+            // The f16 form still carries each row's power-of-two scale; the W8A8
+            // form applied its block scales per stage.
+            const float f0 = (Q ? 1.f : s.inv[t0]) * s.wr[t0], f1 = (Q ? 1.f : s.inv[t0 + 1]) * s.wr[t0 + 1];
             s.otile[t0 * kDnTile + rl] = __bfloat16_as_ushort(__float2bfloat16_rn(acc[nt][0] * f0));
             s.otile[(t0 + 1) * kDnTile + rl] = __bfloat16_as_ushort(__float2bfloat16_rn(acc[nt][1] * f1));
             s.otile[t0 * kDnTile + rl + 8] = __bfloat16_as_ushort(__float2bfloat16_rn(acc[nt][2] * f0));
@@ -625,8 +810,12 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
 }
 
-size_t gateup_smem(int NT, int H, int E) { return smem_bytes(8 * NT, 2 * H + 32, kGuTile, E); }
-size_t down_smem(int NT, int I, int E) { return smem_bytes(8 * NT, 2 * I + 32, kDnTile, E); }
+size_t gateup_smem(int NT, int H, int E, bool q = false) {
+    return q ? smem_bytes(8 * NT, H + 32, kGuTile, E, H / 128) : smem_bytes(8 * NT, 2 * H + 32, kGuTile, E);
+}
+size_t down_smem(int NT, int I, int E, bool q = false) {
+    return q ? smem_bytes(8 * NT, I + 32, kDnTile, E, I / kGateUpFeat) : smem_bytes(8 * NT, 2 * I + 32, kDnTile, E);
+}
 
 int sm_count() {
     static int sms = 0;
@@ -651,20 +840,21 @@ int persistent_grid(K kernel, size_t smem, long max_items) {
 
 constexpr size_t kSmemLimit = 227 * 1024;
 
-template <int NT>
+template <int NT, bool Q>
 cudaError_t launch_nt(const FfnArgs& a, const CUtensorMap& tg, const CUtensorMap& tu,
                       const CUtensorMap& td, cudaStream_t stream) {
     const int E = a.ex.n;
-    const size_t s1 = gateup_smem(NT, a.H, E), s2 = down_smem(NT, a.ex.inter, E);
-    cudaError_t err = cudaFuncSetAttribute(gateup_decode_kernel<NT>,
+    const size_t s1 = gateup_smem(NT, a.H, E, Q), s2 = down_smem(NT, a.ex.inter, E, Q);
+    cudaError_t err = cudaFuncSetAttribute(gateup_decode_kernel<NT, Q>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(s1));
     if (err != cudaSuccess) return err;
-    err = cudaFuncSetAttribute(down_decode_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    err = cudaFuncSetAttribute(down_decode_kernel<NT, Q>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(s2));
     if (err != cudaSuccess) return err;
-    const int g1 = persistent_grid(gateup_decode_kernel<NT>, s1, static_cast<long>(E) * (a.ex.inter / kGateUpFeat));
-    const int g2 = persistent_grid(down_decode_kernel<NT>, s2, static_cast<long>(E) * (a.H / kDownRows));
-    gateup_decode_kernel<NT><<<g1, kThreads, s1, stream>>>(tg, tu, a);
+    const int g1 =
+        persistent_grid(gateup_decode_kernel<NT, Q>, s1, static_cast<long>(E) * (a.ex.inter / kGateUpFeat));
+    const int g2 = persistent_grid(down_decode_kernel<NT, Q>, s2, static_cast<long>(E) * (a.H / kDownRows));
+    gateup_decode_kernel<NT, Q><<<g1, kThreads, s1, stream>>>(tg, tu, a);
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
 
@@ -678,7 +868,7 @@ cudaError_t launch_nt(const FfnArgs& a, const CUtensorMap& tg, const CUtensorMap
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, down_decode_kernel<NT>, td, a);
+    return cudaLaunchKernelEx(&cfg, down_decode_kernel<NT, Q>, td, a);
 }
 
 }  // namespace
@@ -697,12 +887,20 @@ cudaError_t launch_ffn_decode(const FfnArgs& a, cudaStream_t stream) {
     if (err != cudaSuccess) return err;
     // Token tile: the host only knows the average rows per expert.
     int NT = a.avg_rows > 12 ? 4 : (a.avg_rows > 6 ? 2 : 1);
-    while (NT > 1 && (gateup_smem(NT, a.H, a.ex.n) > kSmemLimit || down_smem(NT, a.ex.inter, a.ex.n) > kSmemLimit))
+    while (NT > 1 && (gateup_smem(NT, a.H, a.ex.n, a.w8a8) > kSmemLimit ||
+                      down_smem(NT, a.ex.inter, a.ex.n, a.w8a8) > kSmemLimit))
         NT >>= 1;
+    if (a.w8a8) {
+        switch (NT) {
+            case 4: return launch_nt<4, true>(a, tg, tu, td, stream);
+            case 2: return launch_nt<2, true>(a, tg, tu, td, stream);
+            default: return launch_nt<1, true>(a, tg, tu, td, stream);
+        }
+    }
     switch (NT) {
-        case 4: return launch_nt<4>(a, tg, tu, td, stream);
-        case 2: return launch_nt<2>(a, tg, tu, td, stream);
-        default: return launch_nt<1>(a, tg, tu, td, stream);
+        case 4: return launch_nt<4, false>(a, tg, tu, td, stream);
+        case 2: return launch_nt<2, false>(a, tg, tu, td, stream);
+        default: return launch_nt<1, false>(a, tg, tu, td, stream);
     }
 }
 

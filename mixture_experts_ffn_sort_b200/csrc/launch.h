@@ -83,7 +83,16 @@ struct FfnArgs {
     // bf16 result (route weight applied) into out_acc[token] ([T, H] f32, zeroed
     // by the caller) with fp32 reductions instead of storing y / y_sh.
     float* out_acc;
+    // Decode form only, W8A8: the activations of both GEMMs as E4M3FN codes in
+    // blocks with power-of-two scales (x: 128 columns, quantised as it is
+    // staged; h: 64 features, quantised in the gate/up epilogue).  h then holds
+    // [rows, I] E4M3FN bytes and hscale [rows, I / 64] the inverse scales 2^-k.
+    bool w8a8;
+    float* hscale;
 };
+
+// W8A8 form: the workspace region of h holds the codes and, after them, the scales.
+inline size_t ffn_hq_codes_bytes(long rows, int I) { return (static_cast<size_t>(rows) * I + 255) & ~size_t(255); }
 
 // Bytes of the prefill form's f16 activation copy and its row scales (256-byte aligned).
 inline size_t ffn_x16_bytes(long T, int H) { return (static_cast<size_t>(T) * H * 2 + 255) & ~size_t(255); }

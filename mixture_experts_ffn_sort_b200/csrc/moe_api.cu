@@ -402,6 +402,87 @@ int moe_expert_ffn(const uint16_t* x, int T, int H, int K, const moe_fp8_experts
     return MOE_OK;
 }
 
+namespace {
+// W8A8 workspace: E4M3FN codes of h and their 64-feature block scales, routed then shared.
+size_t w8a8_part_bytes(long rows, int I) {
+    return round256(static_cast<size_t>(rows) * I) + round256(static_cast<size_t>(rows) * (I / 64) * 4);
+}
+}  // namespace
+
+size_t moe_ffn_w8a8_workspace_bytes(int T, int K, int I, int I_shared) {
+    if (T < 0 || K < 1 || I < 0 || I_shared < 0) return 0;
+    return w8a8_part_bytes(static_cast<long>(T) * K, I) + w8a8_part_bytes(T, I_shared);
+}
+
+int moe_expert_ffn_w8a8(const uint16_t* x, int T, int H, int K, const moe_fp8_experts* routed,
+                        const moe_fp8_experts* shared, const int32_t* expert_offsets, const int32_t* sorted_route,
+                        const float* topk_w, uint16_t* y_sorted, uint16_t* y_shared, void* workspace,
+                        size_t workspace_bytes, int32_t* status, moe_stream_t stream) {
+    g_err.clear();
+    if (!routed) return fail(MOE_ERR_INVALID_ARG, "moe_expert_ffn_w8a8: routed must not be NULL");
+    const int E = routed->n_experts, I = routed->inter;
+    int rc = check_sizes(T, E, K);
+    if (rc) return rc;
+    if (H < 128 || H % MOE_BLOCK || H > 8192)
+        return fail(MOE_ERR_UNSUPPORTED_SHAPE, "moe_expert_ffn_w8a8: H=%d must be a multiple of 128 in 128..=8192",
+                    H);
+    if ((rc = check_experts(routed, H, "routed"))) return rc;
+    if (shared) {
+        if (shared->n_experts != 1)
+            return fail(MOE_ERR_INVALID_ARG, "moe_expert_ffn_w8a8: shared->n_experts=%d must be 1", shared->n_experts);
+        if ((rc = check_experts(shared, H, "shared"))) return rc;
+    }
+    if (T == 0) return MOE_OK;
+    if (!x || !expert_offsets || !sorted_route || !topk_w || !y_sorted || (shared && !y_shared))
+        return fail(MOE_ERR_INVALID_ARG, "moe_expert_ffn_w8a8: NULL tensor pointer");
+    if (!aligned16(x) || !aligned16(expert_offsets) || !aligned16(sorted_route) || !aligned16(topk_w) ||
+        !aligned16(y_sorted) || (shared && !aligned16(y_shared)) || !aligned16(workspace) ||
+        (status && (reinterpret_cast<uintptr_t>(status) & 3)))
+        return fail(MOE_ERR_MISALIGNED,
+                    "moe_expert_ffn_w8a8: tensor bases must be 16-byte aligned and status 4-byte aligned");
+    const long R = static_cast<long>(T) * K;
+    const int Is = shared ? shared->inter : 0;
+    const size_t need = moe_ffn_w8a8_workspace_bytes(T, K, I, Is);
+    if (workspace_bytes < need || !workspace)
+        return fail(MOE_ERR_WORKSPACE_TOO_SMALL, "moe_expert_ffn_w8a8: workspace of %zu bytes, need %zu",
+                    workspace_bytes, need);
+
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    moe::FfnArgs a{};
+    a.x = x;
+    a.T = T;
+    a.H = H;
+    a.K = K;
+    a.ex = {routed->w_gate, routed->w_up, routed->w_down, routed->s_gate, routed->s_up, routed->s_down, E, I};
+    a.offsets = expert_offsets;
+    a.sorted_route = sorted_route;
+    a.topk_w = topk_w;
+    a.h = reinterpret_cast<uint16_t*>(ws);
+    a.hscale = reinterpret_cast<float*>(ws + round256(static_cast<size_t>(R) * I));
+    a.y = y_sorted;
+    a.status = status;
+    a.avg_rows = static_cast<int>((R + E - 1) / E);
+    a.w8a8 = true;
+    cudaError_t e = moe::launch_ffn_decode(a, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "moe_expert_ffn_w8a8 routed launch");
+    if (shared) {
+        moe::FfnArgs sa = a;
+        sa.ex = {shared->w_gate, shared->w_up, shared->w_down, shared->s_gate, shared->s_up, shared->s_down, 1, Is};
+        sa.identity = true;
+        sa.offsets = nullptr;
+        sa.sorted_route = nullptr;
+        sa.topk_w = nullptr;
+        uint8_t* sh_ws = ws + w8a8_part_bytes(R, I);
+        sa.h = reinterpret_cast<uint16_t*>(sh_ws);
+        sa.hscale = reinterpret_cast<float*>(sh_ws + round256(static_cast<size_t>(T) * Is));
+        sa.y = y_shared;
+        sa.avg_rows = T;
+        e = moe::launch_ffn_decode(sa, stream);
+        if (e != cudaSuccess) return cuda_fail(e, "moe_expert_ffn_w8a8 shared launch");
+    }
+    return MOE_OK;
+}
+
 size_t moe_ffn_combine_workspace_bytes(int T, int K, int H, int E, int I, int I_shared, int out_dtype) {
     (void)E;
     if (T < 0 || K < 1 || I < 0 || I_shared < 0 || H < 0) return 0;

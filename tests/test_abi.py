@@ -187,6 +187,35 @@ def test_expert_ffn_checks(L):
                             None, None) == moe.MOE_ERR_INVALID_ARG
 
 
+def test_expert_ffn_w8a8_checks(L):
+    ex = _experts()
+    ws = L.moe_ffn_w8a8_workspace_bytes(8, 2, 128, 0)
+    # codes (8*2*128 bytes) and 64-feature block scales (16 rows x 2 x 4 bytes), each 256-aligned
+    assert ws == 2048 + 256
+    assert L.moe_ffn_w8a8_workspace_bytes(8, 2, 128, 256) == ws + 2048 + 256
+    assert L.moe_ffn_w8a8_workspace_bytes(-1, 2, 128, 0) == 0
+    args = lambda **kw: dict(dict(x=P(16), T=8, H=256, K=2, routed=ctypes.byref(ex), shared=None,
+                                  off=P(16), sr=P(16), w=P(16), y=P(16), ys=None, ws=P(16),
+                                  wsb=ws, status=None, stream=None), **kw)
+
+    def call(**kw):
+        a = args(**kw)
+        return L.moe_expert_ffn_w8a8(a["x"], a["T"], a["H"], a["K"], a["routed"], a["shared"], a["off"], a["sr"],
+                                     a["w"], a["y"], a["ys"], a["ws"], a["wsb"], a["status"], a["stream"])
+
+    assert call(H=200) == moe.MOE_ERR_UNSUPPORTED_SHAPE
+    assert call(K=33) == moe.MOE_ERR_INVALID_ARG
+    assert call(x=P(24)) == moe.MOE_ERR_MISALIGNED
+    assert call(status=P(0x1002)) == moe.MOE_ERR_MISALIGNED
+    assert call(wsb=ws - 1) == moe.MOE_ERR_WORKSPACE_TOO_SMALL
+    assert "need" in _err(L)
+    assert call(y=None) == moe.MOE_ERR_INVALID_ARG
+    assert call(routed=None) == moe.MOE_ERR_INVALID_ARG
+    two = _experts(n=2)
+    assert call(shared=ctypes.byref(two), ys=P(16)) == moe.MOE_ERR_INVALID_ARG
+    assert call(T=0) == moe.MOE_OK
+
+
 def test_combine_checks(L):
     assert L.moe_combine(P(16), P(16), None, 4, 2, 12, P(16), 0, None, None) == moe.MOE_ERR_UNSUPPORTED_SHAPE
     assert L.moe_combine(P(16), P(16), None, 4, 2, 16, P(16), 3, None, None) == moe.MOE_ERR_INVALID_ARG

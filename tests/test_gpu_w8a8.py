@@ -1,0 +1,118 @@
+"""The opt-in W8A8 form (moe_expert_ffn_w8a8: E4M3FN activations in
+power-of-two-scaled blocks, E4M3FN tensor-core MMAs) against the oracle's
+W8A8 form, element by element, on shapes that take each token-group size of
+the weight-streaming kernels (8, 16 and 32 rows), ragged H and I (3 and 6
+scale blocks), the shared expert, zero-weight routes and every E4M3FN code;
+and its distance to the exact (fp64) FFN, which is the activation rounding."""
+import numpy as np
+import pytest
+import torch
+
+import mixture_experts_ffn_sort_b200 as moe
+import oracle
+from mixture_experts_ffn_sort_b200 import workloads as wl
+
+from _gpu_util import assert_moe_close, bf16_tensor
+
+pytestmark = pytest.mark.gpu
+
+# The activation rounding of the W8A8 form against the exact FFN: about 2 %
+# relative in these tests (E4M3FN keeps 3 mantissa bits); bounded here.
+W8A8_VS_EXACT_REL_L2 = 6e-2
+
+
+def dev(a, dtype=None):
+    t = torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    return t if dtype is None else t.to(dtype)
+
+
+def _run(x, K, ex, off, sr, wt, sh=None):
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    y, ys = moe.moe_expert_ffn_w8a8(bf16_tensor(x), K, moe.Experts.from_host(ex), dev(off), dev(sr),
+                                    dev(wt, torch.float32), moe.Experts.from_host(sh) if sh else None,
+                                    status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0, status.item()
+    return y, ys
+
+
+def _rel(a, b):
+    return float(np.linalg.norm(a - b) / np.linalg.norm(b))
+
+
+# (T, H, I, E, K, I_shared): about 2, 10 and 40 rows per expert (token groups
+# of 8, 16 and 32 rows), ragged 384-wide H and I, and a shared expert.
+SHAPES = [(16, 512, 256, 8, 1, 0), (40, 512, 256, 8, 2, 128), (160, 256, 128, 4, 1, 0),
+          (64, 384, 384, 16, 4, 0), (33, 1024, 512, 32, 8, 256), (300, 512, 256, 16, 4, 128)]
+
+
+@pytest.mark.parametrize("T,H,I,E,K,Is", SHAPES)
+def test_w8a8_matches_w8a8_oracle(T, H, I, E, K, Is):
+    ex = wl.draw_experts(31, 81, E, I, H, 0.05, threads=4)
+    sh = wl.draw_experts(31, 82, 1, Is, H, 0.05, threads=1) if Is else None
+    x = wl.random_rows_bf16(T, H, seed=T + H)
+    lg = np.random.default_rng(T).standard_normal((T, E)).astype(np.float32)
+    ids, wt = oracle.route(lg, K)
+    off, sr, inv, _ = oracle.sort(ids, E)
+    wt32 = wt.astype(np.float32).astype(np.float64)
+    y, ys = _run(x, K, ex, off, sr, wt32, sh)
+    ref = oracle.ffn_sorted_w8a8(x, K, ex, off, sr, wt32)
+    assert_moe_close(y, ref, "y_sorted")
+    assert _rel(y.double().cpu().numpy(), oracle.ffn_sorted(x, K, ex, off, sr, wt32)) <= W8A8_VS_EXACT_REL_L2
+    if sh:
+        assert_moe_close(ys, oracle.ffn_shared_w8a8(x, sh), "y_shared")
+
+
+def test_w8a8_special_codes_and_zero_weights():
+    T, H, I, E, K = 48, 256, 128, 2, 1
+    for ex in (wl.subnormal_experts(E, I, H, seed=41), wl.all_code_experts(E, I, H, seed=42)):
+        x = wl.random_rows_bf16(T, H, seed=43)
+        ids = (np.arange(T) % E).astype(np.int32).reshape(T, K)
+        off, sr, inv, _ = oracle.sort(ids, E)
+        wt = np.where(np.arange(T) % 5 == 0, 0.0, 1.0).reshape(T, K)
+        y, _ = _run(x, K, ex, off, sr, wt)
+        assert_moe_close(y, oracle.ffn_sorted_w8a8(x, K, ex, off, sr, wt), "y_sorted")
+        yz = y.double().cpu().numpy()[inv.reshape(T, K)[wt == 0.0]]
+        assert np.all(yz == 0.0)
+
+
+def test_w8a8_rows_of_very_different_scale():
+    """Tokens 2^-30 and 2^+20 apart, and one 128-column block of each row
+    2^-12 below the rest: every block takes its own scale."""
+    T, H, I, E, K = 24, 512, 256, 4, 2
+    ex = wl.draw_experts(44, 83, E, I, H, 0.05, threads=2)
+    xs = np.random.default_rng(45).standard_normal((T, H)).astype(np.float32)
+    xs *= np.exp2(np.random.default_rng(46).integers(-30, 21, (T, 1))).astype(np.float32)
+    xs[:, 128:256] *= 2.0 ** -12
+    x = (xs.view(np.uint32) >> 16).astype(np.uint16)
+    lg = np.random.default_rng(47).standard_normal((T, E)).astype(np.float32)
+    ids, wt = oracle.route(lg, K)
+    off, sr, inv, _ = oracle.sort(ids, E)
+    wt32 = wt.astype(np.float32).astype(np.float64)
+    y, _ = _run(x, K, ex, off, sr, wt32)
+    ref = oracle.ffn_sorted_w8a8(x, K, ex, off, sr, wt32)
+    # Rows differ by up to 2^50 in magnitude: compare each row to its own scale.
+    yg = y.double().cpu().numpy()
+    for p in range(T * K):
+        n = np.linalg.norm(ref[p])
+        if n > 0:
+            assert np.linalg.norm(yg[p] - ref[p]) <= 5e-3 * n, p
+
+
+def test_w8a8_layer_pipeline():
+    """MoEFFN(w8a8=True): route, sort, the W8A8 FFN and the combine, against the
+    oracle's W8A8 rows combined in fp64."""
+    T, H, I, E, K, Is = 64, 512, 256, 16, 4, 128
+    ex = wl.draw_experts(48, 84, E, I, H, 0.05, threads=4)
+    sh = wl.draw_experts(48, 85, 1, Is, H, 0.05, threads=1)
+    x = wl.random_rows_bf16(T, H, seed=49)
+    lg = np.random.default_rng(50).standard_normal((T, E)).astype(np.float32)
+    layer = moe.MoEFFN(moe.Experts.from_host(ex), T, K, moe.Experts.from_host(sh), w8a8=True)
+    out = layer(bf16_tensor(x), dev(lg))
+    torch.cuda.synchronize()
+    assert layer.status.item() == 0
+    ids, wt = oracle.route(lg, K)
+    off, sr, inv, _ = oracle.sort(ids, E)
+    ys = oracle.ffn_sorted_w8a8(x, K, ex, off, sr, wt)
+    ref = oracle.combine(ys, inv, oracle.ffn_shared_w8a8(x, sh), T, K)
+    assert_moe_close(out, ref, "out")
