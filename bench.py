@@ -71,6 +71,7 @@ def profile_traffic(workload, kind, root=ROOT):
 
 
 FFN_SOURCES = {"decode": ("ffn_decode.cu", "device_common.cuh", "launch.h"),
+               "w8a8": ("ffn_decode.cu", "device_common.cuh", "launch.h"),
                "prefill": ("ffn_prefill.cu", "device_common.cuh", "launch.h"),
                "hybrid": ("ffn_decode.cu", "ffn_prefill.cu", "device_common.cuh", "launch.h")}
 
@@ -193,7 +194,7 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm), "source": self.source}
 
 
-def ffn_roofline(shape, form_kind, touched, flops, ffn_ms, peaks, root=ROOT):
+def ffn_roofline(shape, form_kind, touched, flops, ffn_ms, peaks, root=ROOT, profile_kind=None):
     """The roofline object of the FFN call: touched-expert bytes against HBM
     for the weight-streaming and hybrid forms (form_kind "decode" / "hybrid"),
     bf16 FLOPs against the tensor cores for the prefill form.  The FFN time is
@@ -205,7 +206,7 @@ def ffn_roofline(shape, form_kind, touched, flops, ffn_ms, peaks, root=ROOT):
         algo = touched * expert_bytes(H, I) + (expert_bytes(H, shape.I_shared) if shape.I_shared else 0)
         ach = algo / (ffn_ms * 1e-3) / 1e9
         return {"bound": "hbm", "achieved": ach, "peak": peaks["hbm"], "unit": "GB/s",
-                "frac": ach / peaks["hbm"], "traffic": profile_traffic(shape.name, form_kind, root),
+                "frac": ach / peaks["hbm"], "traffic": profile_traffic(shape.name, profile_kind or form_kind, root),
                 "kernel": "moe_expert_ffn (gate/up + down kernels)", "algorithmic_bytes": algo,
                 "touched_experts": touched, "peak_source": peaks["src"] + " copy bandwidth",
                 "spec_peak": SPEC_HBM_GBS, "frac_of_spec": ach / SPEC_HBM_GBS}
@@ -496,7 +497,8 @@ def measure(args, shape, steps, dev, world, clk, want_e2e):
             moe.MOE_MODE_DECODE if args.w8a8 else moe.moe_ffn_resolve_mode(T, K, E, args.mode))
     form_kind = {moe.MOE_MODE_DECODE: "decode", moe.MOE_MODE_PREFILL: "prefill",
                  moe.MOE_MODE_HYBRID: "hybrid"}[form]
-    roof = ffn_roofline(shape, form_kind, touched=touched, flops=flops, ffn_ms=ffn_ms, peaks=peaks)
+    roof = ffn_roofline(shape, form_kind, touched=touched, flops=flops, ffn_ms=ffn_ms, peaks=peaks,
+                        profile_kind="w8a8" if args.w8a8 else None)
     if form_kind == "hybrid":
         # The tensor-core share of the same call, for reference.
         roof["flops"] = flops
