@@ -302,8 +302,12 @@ size_t sort_workspace_bytes(long R, int E) {
 cudaError_t launch_sort(const int32_t* ids, long R, int E, int32_t* offsets, int32_t* sorted_route,
                         int32_t* inv_route, void* ws, int32_t* status, cudaStream_t stream) {
     if (R <= kSortSmallMaxRoutes) {
-        // As many warps as 32-route slices, up to what shared memory holds.
-        const int nw = static_cast<int>(std::min<long>(small_sort_warps(E), std::max<long>(1, (R + 31) / 32)));
+        // A warp per 128 routes (at least four warps, and no more than 32-route
+        // slices), up to what shared memory holds: the per-warp histograms and
+        // their scan grow with the warps, so fewer, fuller warps win until the
+        // block is too narrow to hide its load latency.
+        const long want = std::min<long>((R + 31) / 32, std::max<long>(4, (R + 127) / 128));
+        const int nw = static_cast<int>(std::min<long>(small_sort_warps(E), std::max<long>(1, want)));
         const size_t smem = (static_cast<size_t>(nw) * E + 32) * sizeof(int32_t);
         const long per = ((R + nw - 1) / nw + 31) / 32;  // ids per lane of a warp's chunk
 #define MOE_SORT_SMALL(P) \
