@@ -44,7 +44,8 @@
  *    back.  The first call of a process also does one-time host set-up (kernel
  *    attributes, driver entry points); make one call before capturing a CUDA
  *    graph, after which moe_route, moe_route_ex, moe_router, moe_sort,
- *    moe_expert_ffn and moe_combine may be captured.
+ *    moe_expert_ffn, moe_expert_ffn_w8a8, moe_expert_ffn_combine and
+ *    moe_combine may be captured.
  *  - Return value: MOE_OK (0) or a negative moe_status.  On error nothing has
  *    been launched and moe_last_error() holds a message (thread-local, valid
  *    until the next call on the same thread).  MOE_ERR_CUDA reports a launch
