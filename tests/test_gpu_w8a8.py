@@ -116,3 +116,24 @@ def test_w8a8_layer_pipeline():
     ys = oracle.ffn_sorted_w8a8(x, K, ex, off, sr, wt)
     ref = oracle.combine(ys, inv, oracle.ffn_shared_w8a8(x, sh), T, K)
     assert_moe_close(out, ref, "out")
+
+
+def test_w8a8_layer_replays_from_a_cuda_graph():
+    """After one eager call, a captured forward replays to the same bits."""
+    T, H, I, E, K = 64, 512, 256, 16, 4
+    ex = wl.draw_experts(51, 86, E, I, H, 0.05, threads=4)
+    x = bf16_tensor(wl.random_rows_bf16(T, H, seed=52))
+    lg = dev(np.random.default_rng(53).standard_normal((T, E)).astype(np.float32))
+    layer = moe.MoEFFN(moe.Experts.from_host(ex), T, K, w8a8=True)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        eager = layer(x, lg).clone()
+    s.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        layer(x, lg)
+    layer.out.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    assert layer.status.item() == 0
+    assert torch.equal(layer.out.view(torch.int16), eager.view(torch.int16))
