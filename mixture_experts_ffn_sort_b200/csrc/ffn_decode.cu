@@ -40,6 +40,12 @@
 //  * The down kernel is a programmatic dependent launch: its producer starts
 //    streaming weights while the gate/up grid drains, and its consumers wait
 //    (griddepcontrol.wait) before reading h.
+//  * W8A8 (moe_expert_ffn_w8a8, template flag Q): the activations become
+//    E4M3FN codes in blocks with power-of-two scales -- x per 128 columns as
+//    it is staged, h per 64 features in the gate/up epilogue -- and both GEMMs
+//    run as m16n8k32 E4M3FN MMAs whose A fragment is one ldmatrix of the
+//    weight codes (no conversion); the weight and activation block scales
+//    multiply each fp32 partial.
 #include <algorithm>
 
 #include "device_common.cuh"
