@@ -837,11 +837,12 @@ int sm_count() {
 // Persistent grid: every CTA the GPU holds at once, but no more than the items
 // of the call could use.
 template <class K>
-int persistent_grid(K kernel, size_t smem, long max_items) {
+int persistent_grid(K kernel, size_t smem, long max_items, int sm_limit) {
     int per_sm = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kThreads, smem) != cudaSuccess || per_sm < 1)
         per_sm = 1;
-    return static_cast<int>(std::max(1L, std::min(static_cast<long>(per_sm) * sm_count(), max_items)));
+    const int sms = sm_limit > 0 ? std::min(sm_limit, sm_count()) : sm_count();
+    return static_cast<int>(std::max(1L, std::min(static_cast<long>(per_sm) * sms, max_items)));
 }
 
 constexpr size_t kSmemLimit = 227 * 1024;
@@ -858,8 +859,9 @@ cudaError_t launch_nt(const FfnArgs& a, const CUtensorMap& tg, const CUtensorMap
                                static_cast<int>(s2));
     if (err != cudaSuccess) return err;
     const int g1 =
-        persistent_grid(gateup_decode_kernel<NT, Q>, s1, static_cast<long>(E) * (a.ex.inter / kGateUpFeat));
-    const int g2 = persistent_grid(down_decode_kernel<NT, Q>, s2, static_cast<long>(E) * (a.H / kDownRows));
+        persistent_grid(gateup_decode_kernel<NT, Q>, s1, static_cast<long>(E) * (a.ex.inter / kGateUpFeat), a.sm_limit);
+    const int g2 =
+        persistent_grid(down_decode_kernel<NT, Q>, s2, static_cast<long>(E) * (a.H / kDownRows), a.sm_limit);
     gateup_decode_kernel<NT, Q><<<g1, kThreads, s1, stream>>>(tg, tu, a);
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;

@@ -62,6 +62,7 @@
 // Every mbarrier wait is bounded; an expired wait sets a CTA-wide abort flag
 // and every role runs to the end without waiting, so the CTA always reaches
 // the TMEM de-allocation.
+#include <algorithm>
 #include <cstring>
 
 #include "device_common.cuh"
@@ -1025,7 +1026,7 @@ cudaError_t launch_ffn_prefill(const FfnArgs& a, cudaStream_t stream, bool x16_d
     if (err == cudaSuccess)
         err = cudaFuncSetAttribute(prefill_kernel<kDown>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (err != cudaSuccess) return err;
-    const int grid = num_sms();
+    const int grid = a.sm_limit > 0 ? std::min(a.sm_limit, num_sms()) : num_sms();
     if (!x16_done) {
         err = launch_x16(a, stream);
         if (err != cudaSuccess) return err;

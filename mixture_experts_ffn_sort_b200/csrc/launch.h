@@ -89,6 +89,9 @@ struct FfnArgs {
     // [rows, I] E4M3FN bytes and hscale [rows, I / 64] the inverse scales 2^-k.
     bool w8a8;
     float* hscale;
+    // > 0: the persistent grids use at most this many SMs (MOE_MODE_HYBRID runs
+    // the two forms side by side on disjoint SMs).
+    int sm_limit;
 };
 
 // W8A8 form: the workspace region of h holds the codes and, after them, the scales.

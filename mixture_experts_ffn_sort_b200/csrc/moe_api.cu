@@ -8,6 +8,7 @@
 #include <stdarg.h>
 #include <stdio.h>
 
+#include <mutex>
 #include <string>
 
 #include "../../include/moe_ffn.h"
@@ -78,6 +79,43 @@ int check_experts(const moe_fp8_experts* ex, int H, const char* which) {
 }
 
 size_t ffn_h_bytes(long R, int I) { return round256(static_cast<size_t>(R) * I * 2); }
+
+// The hybrid form's second stream and its fork/join events, one set per
+// device, created by the first hybrid call on that device (host set-up, like
+// the kernels' attributes).
+struct SideStream {
+    int device = -1;
+    cudaStream_t stream = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+};
+
+cudaError_t side_stream(SideStream* out) {
+    static std::mutex mu;
+    static SideStream table[64];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    SideStream& t = table[dev];
+    if (t.device != dev) {
+        e = cudaStreamCreateWithFlags(&t.stream, cudaStreamNonBlocking);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&t.fork, cudaEventDisableTiming);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&t.join, cudaEventDisableTiming);
+        if (e != cudaSuccess) return e;
+        t.device = dev;
+    }
+    *out = t;
+    return cudaSuccess;
+}
+
+int device_sms() {
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        sms <= 0)
+        sms = 148;
+    return sms;
+}
 
 }  // namespace
 
@@ -369,20 +407,35 @@ int moe_expert_ffn(const uint16_t* x, int T, int H, int K, const moe_fp8_experts
         }
         // HYBRID: the experts with at most MOE_HYBRID_ROW_SPLIT rows in the
         // weight-streaming kernels (token groups of 8 rows), the others and the
-        // shared expert in the tensor-core kernels, launched after them as
-        // programmatic dependents so that they fill the SMs the weight-streaming
-        // down grid's tail leaves idle.  Each form skips the experts of the other.
-        cudaError_t e = moe::launch_x16(a, stream);
+        // shared expert in the tensor-core kernels.  The two forms run at the
+        // same time on disjoint SMs: the tensor-core grids (one CTA per SM,
+        // launched first) on 7/10 of them, the weight-streaming grids (two CTAs
+        // per SM) on the rest, from a second stream forked from and joined back
+        // to `stream` with events.  Each form skips the experts of the other.
+        // (The share is a measured optimum on a skewed 512-token batch: 1/2,
+        // 3/5, 13/20, 7/10, 3/4, 4/5 and 17/20 of the SMs gave 164, 135, 131,
+        // 125-127, 133, 141 and 137 us against 129-131 us for the two forms
+        // one after the other.)
+        SideStream side;
+        cudaError_t e = side_stream(&side);
+        if (e != cudaSuccess) return cuda_fail(e, "moe_expert_ffn side stream");
+        e = moe::launch_x16(a, stream);
+        if (e == cudaSuccess) e = cudaEventRecord(side.fork, stream);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(side.stream, side.fork, 0);
+        if (e != cudaSuccess) return cuda_fail(e, "moe_expert_ffn launch");
+        const int sms = device_sms(), tc_sms = (7 * sms + 9) / 10;
+        a.row_split = MOE_HYBRID_ROW_SPLIT;
+        a.sm_limit = tc_sms;
+        e = moe::launch_ffn_prefill(a, stream, /*x16_done=*/true);
         if (e != cudaSuccess) return cuda_fail(e, "moe_expert_ffn launch");
         moe::FfnArgs d = a;
-        d.row_split = MOE_HYBRID_ROW_SPLIT;
         d.avg_rows = MOE_HYBRID_ROW_SPLIT / 2;
         d.sh = {};
-        e = moe::launch_ffn_decode(d, stream);
-        if (e != cudaSuccess) return cuda_fail(e, "moe_expert_ffn routed launch");
-        a.row_split = MOE_HYBRID_ROW_SPLIT;
-        e = moe::launch_ffn_prefill(a, stream, /*x16_done=*/true, /*gateup_after_decode=*/true);
-        return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_expert_ffn launch");
+        d.sm_limit = sms - tc_sms;
+        e = moe::launch_ffn_decode(d, side.stream);
+        if (e == cudaSuccess) e = cudaEventRecord(side.join, side.stream);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(stream, side.join, 0);
+        return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_expert_ffn routed launch");
     }
     cudaError_t e = moe::launch_ffn_decode(a, stream);
     if (e != cudaSuccess) return cuda_fail(e, "moe_expert_ffn routed launch");
