@@ -364,8 +364,10 @@ int moe_expert_ffn(const uint16_t* x, int T, int H, int K, const moe_fp8_experts
     if (!x || !expert_offsets || !sorted_route || !topk_w || !y_sorted || (shared && !y_shared))
         return fail(MOE_ERR_INVALID_ARG, "moe_expert_ffn: NULL tensor pointer");
     if (!aligned16(x) || !aligned16(expert_offsets) || !aligned16(sorted_route) || !aligned16(topk_w) ||
-        !aligned16(y_sorted) || (shared && !aligned16(y_shared)) || !aligned16(workspace))
-        return fail(MOE_ERR_MISALIGNED, "moe_expert_ffn: tensor bases must be 16-byte aligned");
+        !aligned16(y_sorted) || (shared && !aligned16(y_shared)) || !aligned16(workspace) ||
+        (status && (reinterpret_cast<uintptr_t>(status) & 3)))
+        return fail(MOE_ERR_MISALIGNED,
+                    "moe_expert_ffn: tensor bases must be 16-byte aligned and status 4-byte aligned");
     const long R = static_cast<long>(T) * K;
     const int Is = shared ? shared->inter : 0;
     const size_t need = moe_ffn_workspace_bytes(T, K, H, E, I, Is, mode);

@@ -176,6 +176,7 @@ def test_expert_ffn_checks(L):
     assert call(mode=7) == moe.MOE_ERR_INVALID_ARG
     assert call(K=33) == moe.MOE_ERR_INVALID_ARG
     assert call(x=P(24)) == moe.MOE_ERR_MISALIGNED
+    assert call(status=P(0x1002)) == moe.MOE_ERR_MISALIGNED
     assert call(wsb=ws - 1) == moe.MOE_ERR_WORKSPACE_TOO_SMALL
     assert call(y=None) == moe.MOE_ERR_INVALID_ARG
     bad_inter = _experts(inter=192)
