@@ -383,7 +383,12 @@ MOE_API int moe_ffn_resolve_mode(int T, int K, int E, int mode);
  *   mode           MOE_MODE_AUTO | MOE_MODE_DECODE | MOE_MODE_PREFILL |
  *                  MOE_MODE_HYBRID (AUTO as moe_ffn_resolve_mode resolves it;
  *                  HYBRID launches both forms, each skipping the experts the
- *                  other takes, so every row is written exactly once)
+ *                  other takes, so every row is written exactly once; they
+ *                  run side by side on disjoint SMs, the weight-streaming pair
+ *                  on a library-owned second stream (created by the first
+ *                  HYBRID call on a device) forked from `stream` and joined
+ *                  back to it with events, so the call stays ordered on
+ *                  `stream` and can be captured like the other forms)
  *   workspace      moe_ffn_workspace_bytes(...) bytes of device scratch
  *   status         optional device int32: MOE_STATUS_BAD_MAP is OR-ed in when
  *                  offsets or route ids are out of range (those rows skipped)
