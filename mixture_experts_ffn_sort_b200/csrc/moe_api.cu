@@ -82,16 +82,20 @@ size_t ffn_h_bytes(long R, int I) { return round256(static_cast<size_t>(R) * I *
 
 // The hybrid form's second stream and its fork/join events, one set per
 // device, created by the first hybrid call on that device (host set-up, like
-// the kernels' attributes).
+// the kernels' attributes).  `mu` serialises the enqueue of a fork ... join
+// sequence, so that calls from several host threads never interleave their
+// event records.
 struct SideStream {
     int device = -1;
     cudaStream_t stream = nullptr;
     cudaEvent_t fork = nullptr, join = nullptr;
+    std::mutex* mu = nullptr;
 };
 
 cudaError_t side_stream(SideStream* out) {
     static std::mutex mu;
     static SideStream table[64];
+    static std::mutex enqueue_mu[64];
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
@@ -103,6 +107,7 @@ cudaError_t side_stream(SideStream* out) {
         if (e == cudaSuccess) e = cudaEventCreateWithFlags(&t.fork, cudaEventDisableTiming);
         if (e == cudaSuccess) e = cudaEventCreateWithFlags(&t.join, cudaEventDisableTiming);
         if (e != cudaSuccess) return e;
+        t.mu = &enqueue_mu[dev];
         t.device = dev;
     }
     *out = t;
@@ -421,6 +426,7 @@ int moe_expert_ffn(const uint16_t* x, int T, int H, int K, const moe_fp8_experts
         SideStream side;
         cudaError_t e = side_stream(&side);
         if (e != cudaSuccess) return cuda_fail(e, "moe_expert_ffn side stream");
+        std::lock_guard<std::mutex> enqueue(*side.mu);
         e = moe::launch_x16(a, stream);
         if (e == cudaSuccess) e = cudaEventRecord(side.fork, stream);
         if (e == cudaSuccess) e = cudaStreamWaitEvent(side.stream, side.fork, 0);
