@@ -68,6 +68,12 @@ def test_ffn_roofline_objects(tmp_path):
     skew = wl.SHAPES["decode_skew"]
     r = bench.ffn_roofline(skew, "hybrid", touched=106, flops=0, ffn_ms=0.143, peaks=peaks, root=str(tmp_path))
     assert r["bound"] == "hbm" and r["traffic"] == 1.5e9
+    # The W8A8 form reads its own summary (same workload, profile kind "w8a8").
+    (prof / "ffn_w8a8_decode.md").write_text("traffic_bytes_per_call: 7.0e8\nsources_sha256: %s\n"
+                                              % bench.sources_hash("w8a8"))
+    r = bench.ffn_roofline(dec, "decode", touched=222, flops=0, ffn_ms=0.123, peaks=peaks, root=str(tmp_path),
+                           profile_kind="w8a8")
+    assert r["bound"] == "hbm" and r["traffic"] == 7.0e8
     # A summary taken on other kernel sources gives no traffic.
     (prof / "ffn_decode_decode.md").write_text("traffic_bytes_per_call: 1.5e9\nsources_sha256: 0123abcd\n")
     r = bench.ffn_roofline(dec, "decode", touched=222, flops=0, ffn_ms=0.119, peaks=peaks, root=str(tmp_path))
