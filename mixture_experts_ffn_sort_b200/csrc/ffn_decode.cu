@@ -667,8 +667,8 @@ template <int NT, bool Q>
 __global__ void __launch_bounds__(kThreads, 2)
     down_decode_kernel(const __grid_constant__ CUtensorMap tm_down, const FfnArgs a) {
     constexpr int NG = 8 * NT;
-    // A following tensor-core gate/up launch of the same call (MOE_MODE_HYBRID)
-    // may start on the SMs this grid leaves idle.
+    // A following programmatic-dependent launch (a tensor-core gate/up grid
+    // chained after this one) may start on the SMs this grid leaves idle.
     if (threadIdx.x == 0) grid_dependency_launch();
     extern __shared__ uint8_t smem_raw[];
     const int H = a.H, I = a.ex.inter;

@@ -946,11 +946,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
-    // Launched as a programmatic dependent of the weight-streaming down kernel
-    // (MOE_MODE_HYBRID), gate/up overlaps that grid's tail without reading
-    // anything it writes; waiting for it here, at the end, makes this grid's
-    // completion -- which the down GEMM and later launches wait for -- imply
-    // that grid's.  A no-op for a normal launch.
+    // When launched as a programmatic dependent of the weight-streaming down
+    // kernel on the same stream (launch_ffn_prefill's gateup_after_decode),
+    // gate/up overlaps that grid's tail without reading anything it writes;
+    // waiting for it here, at the end, makes this grid's completion -- which
+    // the down GEMM and later launches wait for -- imply that grid's.  A no-op
+    // for a normal launch (the hybrid form now runs the two forms on two
+    // streams instead).
     if (MODE == kGateUp && threadIdx.x == 0) grid_dependency_wait();
 }
 
@@ -1040,8 +1042,9 @@ cudaError_t launch_ffn_prefill(const FfnArgs& a, cudaStream_t stream, bool x16_d
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    // gate/up: a programmatic dependent of the preceding kernel only when that
-    // kernel is the weight-streaming down GEMM of the same call.
+    // gate/up: a programmatic dependent of the preceding kernel only when the
+    // caller asks for it (the preceding kernel being the weight-streaming down
+    // GEMM of the same call).
     cfg.numAttrs = gateup_after_decode ? 1 : 0;
     err = cudaLaunchKernelEx(&cfg, prefill_kernel<kGateUp>, mg, a);
     if (err != cudaSuccess) return err;

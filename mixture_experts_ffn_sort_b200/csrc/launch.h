@@ -116,7 +116,8 @@ cudaError_t make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows,
 // Routed rows (a.identity must be false) plus the optional shared expert a.sh.
 // x16_done: the f16 copy of x (launch_x16) was already launched on the stream.
 // gateup_after_decode: the preceding launch is the weight-streaming down
-// kernel of the same call, which gate/up overlaps (programmatic dependent launch).
+// kernel of the same call, which gate/up overlaps (programmatic dependent
+// launch); the hybrid form runs the forms on two streams and does not use it.
 cudaError_t launch_ffn_prefill(const FfnArgs& a, cudaStream_t stream, bool x16_done = false,
                                bool gateup_after_decode = false);
 // The f16 copy of x and its row scales (a.x16, a.xinv) for the tensor-core kernels.
