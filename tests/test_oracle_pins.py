@@ -697,3 +697,15 @@ def test_ffn_w8a8_is_the_exact_ffn_when_quantisation_is_exact():
     exact = oracle.ffn_sorted(x, K, ex, off, sr, w)
     assert np.abs(exact).max() > 0
     np.testing.assert_allclose(oracle.ffn_sorted_w8a8(x, K, ex, off, sr, w), exact, rtol=1e-12, atol=0)
+
+
+def test_ffn_shared_w8a8_is_the_routed_form_with_every_token_on_one_expert():
+    """The shared expert's W8A8 rows equal the routed W8A8 rows of a one-expert
+    layer where every token is routed to that expert with weight 1."""
+    T, H, I = 5, 256, 128
+    sh = wl.draw_experts(25, 73, 1, I, H, 0.05, threads=1)
+    x = wl.random_rows_bf16(T, H, seed=26)
+    ids = np.zeros((T, 1), np.int32)
+    off, sr, inv, _ = oracle.sort(ids, 1)
+    routed = oracle.ffn_sorted_w8a8(x, 1, sh, off, sr, np.ones((T, 1)))
+    np.testing.assert_array_equal(oracle.ffn_shared_w8a8(x, sh), routed[inv])
